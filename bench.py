@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark of one MONA / Muon optimizer step on B200 (one JSON line).
+
+A step is one call of muon_step_batched over every matrix of the workload:
+the fused MONA pre-pass with the Frobenius norms, 5 quintic Newton-Schulz
+steps on tensor cores (grouped by shape), and the weight update fused into
+the last step.  Inputs are synthetic (seeded; shapes of the named model).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+value = Newton-Schulz TFLOP/s over all ranks (algorithmic flops: symmetric
+products count the half they need), timed with CUDA events on the step's
+stream between barriers, max over ranks.  Under torchrun each rank steps its
+own copy of the workload (weak scaling, no collective on the data path).
+--impl reference times the fp64 CPU oracle on a bounded sample instead.
+"""
+import argparse
+import ctypes
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Muon step ms & Newton-Schulz TFLOP/s on 1 B200; % of bf16 tensor / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="gpt2_small")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ns-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def ns_flops(shapes, ns_steps):
+    """Algorithmic flops of the iteration: per step s^2 l (X X^T, half) + s^3 (A A, half) + 2 s^2 l (B X)."""
+    tot = 0.0
+    for r, c in shapes:
+        s, l = min(r, c), max(r, c)
+        tot += ns_steps * (3.0 * s * s * l + float(s) ** 3)
+    return tot
+
+
+def describe(name, w):
+    from collections import Counter
+    cnt = Counter((min(r, c), max(r, c)) for r, c in w["shapes"])
+    groups = " + ".join(f"{n} x {s}x{l}" for (s, l), n in sorted(cnt.items()))
+    nel = sum(r * c for r, c in w["shapes"])
+    return groups, nel
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline and reference arm)
+
+def oracle_sample_run(w, shapes, seed_base=0):
+    """One full MONA/Muon step in fp64 on the given shapes; returns seconds."""
+    import numpy as np
+    import oracle
+    from muon_family_optimizer_b200 import synthetic as syn
+    arrays = []
+    for j, (r, c) in enumerate(shapes):
+        W = syn.initial_weight(w["name"], j, r, c).double().numpy()
+        G = syn.gradient(w["name"], j, seed_base, r, c).double().numpy()
+        Gp = syn.gradient(w["name"], j, seed_base + 8, r, c).double().numpy()
+        arrays.append((W, G, Gp, np.zeros_like(W), np.zeros_like(W)))
+    hp = w["hp"]
+    t0 = time.perf_counter()
+    for W, G, Gp, A, M in arrays:
+        oracle.muon_step(W, G, Gp, A, M, mu=hp["mu"], eta=hp["eta"], lam=hp["lambda"], gamma=hp["gamma"],
+                         beta_a=hp["beta_a"], alpha=hp["alpha"], coeffs=[tuple(syn.QUINTIC)] * 5)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, ns_steps):
+    import oracle
+    seen, sample = set(), []
+    for r, c in w["shapes"]:
+        key = (min(r, c), max(r, c))
+        if key not in seen:
+            seen.add(key)
+            sample.append((r, c))
+    secs = oracle_sample_run(w, sample)
+    fl = ns_flops(sample, ns_steps)
+    full = ns_flops(w["shapes"], ns_steps)
+    return {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"one matrix per shape group ({', '.join(f'{r}x{c}' for r, c in sample)}): full "
+                      f"fp64 MONA step with {ns_steps} quintic steps, {secs:.2f} s",
+            "ms_per_step_extrapolated": secs * full / fl * 1e3}
+
+
+def run_reference(args, w, ns_steps):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    shapes_by_group = []
+    seen = set()
+    for r, c in w["shapes"]:
+        key = (min(r, c), max(r, c))
+        if key not in seen:
+            seen.add(key)
+            shapes_by_group.append((r, c))
+    # one matrix per step, cycling through the shape groups, smallest first
+    shapes_by_group.sort(key=lambda rc: rc[0] * rc[1])
+    for i in range(args.warmup):
+        oracle_sample_run(w, [shapes_by_group[i % len(shapes_by_group)]], seed_base=i)
+    fl = secs = 0.0
+    steps = 0
+    budget = 150.0
+    t_start = time.perf_counter()
+    for i in range(args.steps):
+        sh = shapes_by_group[i % len(shapes_by_group)]
+        secs += oracle_sample_run(w, [sh], seed_base=i)
+        fl += ns_flops([sh], ns_steps)
+        steps += 1
+        if time.perf_counter() - t_start > budget:
+            break
+    value = fl / secs / 1e12
+    full = ns_flops(w["shapes"], ns_steps)
+    ms_step = secs / fl * full * 1e3
+    groups, nel = describe(args.workload, w)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: {groups}", "elements": nel, "ns_steps": ns_steps},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{steps} timed steps, each one full fp64 MONA step of one matrix "
+                                       "(cycling through the shape groups); ms_per_step extrapolated"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def main():
+    args = parse()
+    from muon_family_optimizer_b200 import synthetic as syn
+    w = dict(syn.WORKLOADS[args.workload])
+    w["name"] = args.workload
+    ns_steps = args.ns_steps
+    if args.impl == "reference":
+        return run_reference(args, w, ns_steps)
+
+    import torch
+    import torch.distributed as dist
+    import muon_family_optimizer_b200 as mo
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w_dt, ns_dt = w["w_dtype"], w["ns_dtype"]
+    shapes = w["shapes"]
+    # ---- state (each rank its own copy); gradients live in one buffer per set
+    nel = sum(r * c for r, c in shapes)
+    esz = torch.empty((), dtype=w_dt).element_size()
+    gbuf = [torch.empty(nel, dtype=w_dt, device=dev) for _ in range(2)]
+    params = [[], []]
+    off = 0
+    torch.manual_seed(1234 + rank)
+    cache = {}
+    for j, (r, c) in enumerate(shapes):
+        key = (r, c)
+        if key not in cache:
+            cache[key] = [syn.gradient(args.workload, j, t, r, c, device=dev) for t in range(2)]
+        W = syn.initial_weight(args.workload, j, r, c, device=dev).to(w_dt)
+        Gp = cache[key][1].to(w_dt).contiguous()
+        A = torch.zeros(r, c, dtype=torch.float32, device=dev)
+        M = torch.zeros(r, c, dtype=torch.float32, device=dev)
+        for t in range(2):
+            g = gbuf[t][off:off + r * c].view(r, c)
+            sign = torch.randint(0, 2, (1, c), device=dev, dtype=torch.int8).float() * 2 - 1
+            g.copy_(cache[key][t] * sign)
+            params[t].append(dict(W=W, G=g, G_prev=Gp, A=A, M=M))
+        off += r * c
+    del cache
+    arrs = [mo.make_params(p) for p in params]
+    sched = mo.quintic_schedule(ns_steps)
+    ws = torch.empty(mo.muon_workspace_size(arrs[0], mo._dtype_code(ns_dt)), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    wcode, ncode = mo._dtype_code(w_dt), mo._dtype_code(ns_dt)
+
+    def step(i):
+        mo.muon_step_batched(arrs[i % 2], wcode, ncode, w["hp"], sched, ws, d_status=status, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after warm-up")
+
+    # ---- timed region (device time, CUDA events on the step's stream)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    mo.muon_trace_enable(True)
+    mo.muon_trace_read()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    mo.muon_trace_enable(False)
+    recs = mo.muon_trace_read()
+    clk = clocks.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    fl_step = ns_flops(shapes, ns_steps)
+    value = world * fl_step * args.steps / (ms_total / 1e3) / 1e12
+
+    # ---- per-kernel figures from the trace (same timed region)
+    per = {}
+    for kind, work, ms in recs:
+        d = per.setdefault(mo.KERNEL_NAMES[kind], {"launches": 0, "work": 0.0, "ms": 0.0})
+        d["launches"] += 1
+        d["work"] += work
+        d["ms"] += ms
+    pk, pk_src = peaks()
+    dom = max(per.items(), key=lambda kv: kv[1]["ms"])[0] if per else None
+    roofline = None
+    if dom:
+        d = per[dom]
+        if dom in ("prepass", "other"):
+            ach, peak, unit, bound = d["work"] / (d["ms"] / 1e3) / 1e9, pk["hbm_gbs"], "GB/s", "hbm"
+        else:
+            sustained = ms_total > 1000.0
+            peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+            ach, unit, bound = d["work"] / (d["ms"] / 1e3) / 1e12, "TFLOP/s", "tensor"
+        roofline = {"bound": bound, "kernel": dom, "achieved": ach, "peak": peak, "unit": unit,
+                    "frac": ach / peak, "traffic": None,
+                    "peak_source": f"{pk_src} ({'sustained' if bound == 'tensor' and ms_total > 1000 else 'burst' if bound == 'tensor' else 'copy'})"}
+    kernels = {}
+    for name, d in per.items():
+        rate = d["work"] / (d["ms"] / 1e3)
+        kernels[name] = {"launches": d["launches"], "ms_total": round(d["ms"], 4),
+                         "share": round(d["ms"] / max(1e-9, sum(x["ms"] for x in per.values())), 4),
+                         ("GB/s" if name in ("prepass", "other") else "TFLOP/s"):
+                             round(rate / 1e9, 1) if name in ("prepass", "other") else round(rate / 1e12, 1)}
+
+    # ---- end to end through the public API: H2D of the step's gradients from
+    # pinned host memory, the step, D2H of the step's status word
+    e2e = None
+    if not args.no_e2e:
+        host_g = [gbuf[t].cpu().pin_memory() for t in range(2)]
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        k = max(3, min(args.steps, 50))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(k):
+            gbuf[i % 2].copy_(host_g[i % 2], non_blocking=True)
+            step(i)
+            st = int(status.item())       # D2H read of the step's result
+            if st != 0:
+                raise RuntimeError(f"device status {st}")
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * fl_step * k / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": nel * esz, "d2h_bytes_per_step": 4, "ms_per_step": e_ms / k}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, ns_steps)
+
+    if rank == 0:
+        groups, _ = describe(args.workload, w)
+        state_bytes = nel * (3 * esz + 8)
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": {torch.bfloat16: "bf16", torch.float16: "fp16",
+                                               torch.float32: "fp32"}[ns_dt],
+                "data": "synthetic (seeded; shapes of the named model, random values)",
+                "config": {"workload": f"{args.workload}: {groups} (wide view s x l)", "elements": nel,
+                           "ns_steps": ns_steps, "w_dtype": str(w_dt).replace("torch.", ""),
+                           "state_bytes": state_bytes,
+                           "l2": f"inputs larger than L2: {state_bytes / 1e9:.2f} GB of state per step",
+                           "parallelism": f"{world} replica(s), each rank steps its own copy"},
+                "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": len(recs), "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

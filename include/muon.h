@@ -1,0 +1,222 @@
+/*
+ * muon.h -- C ABI of the B200 (sm_100a) Muon / MONA optimizer step.
+ *
+ * The method (sources):
+ *   [MONA]  "MONA - Muon-optimizer met Nesterov-versnelling" (gist.science,
+ *           paper 2605.26842), section 2 "Methodologie: MONA", Kernalgoritme
+ *           steps 1-4:
+ *             D = G - G_prev;  A = beta_a A + (1 - beta_a) D;  Gt = G + alpha A;
+ *             M = mu M + Gt;   O = Newton-Schulz(M);
+ *             W = W - eta (gamma O + lambda W).
+ *           "Ontwerprichtlijnen": the acceleration term is applied before the
+ *           orthogonalisation, never after.
+ *   [POLAR] quant_prune_distill post 677 (tgviewer.app): the Muon step
+ *           substitutes the polar factor polar(X) = U V^T (X = U S V^T) of the
+ *           momentum; it is found by Newton-Schulz.  Gram route:
+ *           polar(X) = X (X^T X)^{-1/2} with the inverse square root also found
+ *           by Newton-Schulz on the small Gram matrix, half of every symmetric
+ *           product computed and mirrored, restarts, and a division by
+ *           1.02-1.05 so that the eigenvalues stay inside [0, 1].
+ *
+ * Iteration used by every entry point (readings of the pages, which name
+ * Newton-Schulz but print no coefficients): on the wide view X (s x l,
+ * s = min(rows, cols); a matrix with rows > cols is iterated transposed,
+ * polar(X^T) = polar(X)^T) start from X0 = M / ((||M||_F + eps) f) and, for
+ * k = 0 .. n_steps-1 with (a, b, c) = coeffs[k]:
+ *     A = X X^T;   B = b A + c A A;   X = a X + B X
+ * At every step k > 0 listed in `restarts` X is divided by f once more before
+ * the step.  The Gram route evaluates the same polynomial through
+ * R = X X^T:  h = a I + b R + c R^2,  Q <- h Q,  R <- h R h, and at a restart
+ * k > 0: Xb <- Q Xb / f, R <- Xb Xb^T, Q <- I;  finally X = Q Xb.
+ *
+ * Conventions common to all entry points:
+ *   - Every pointer named d_* or documented as "device" is CUDA device memory
+ *     of the current device, owned by the caller.  Host arrays (schedule
+ *     coefficients, restarts, parameter descriptors) are read during the call
+ *     only and may be freed as soon as it returns.
+ *   - The library allocates no memory.  Scratch space is the caller-provided
+ *     `workspace` (device, >= the size returned by the matching *_size query,
+ *     256-byte aligned).  Its contents need no initialisation and are
+ *     clobbered.
+ *   - Matrices are dense, row-major and contiguous (row stride = cols).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.  Argument errors
+ *     are returned before anything is enqueued.  Faults seen on the device
+ *     (non-finite norm, a wait that ran out) are OR-ed into *d_status
+ *     (MUON_FLAG_* bits) when d_status is not NULL; the caller reads it after
+ *     synchronising.  d_status is never cleared by the library.
+ *   - Calls that share a workspace must be ordered on the GPU (same stream,
+ *     or events); concurrent calls on one workspace race.
+ */
+#ifndef MUON_B200_H
+#define MUON_B200_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* muon_stream_t;
+
+typedef enum {
+    MUON_OK = 0,
+    MUON_ERR_INVALID_ARG = 1,   /* NULL pointer, bad size, bad enum, bad schedule */
+    MUON_ERR_UNSUPPORTED = 2,   /* valid request this build cannot run (no sm_100 device, shape limits) */
+    MUON_ERR_WORKSPACE = 3,     /* workspace NULL, misaligned or smaller than the size query */
+    MUON_ERR_NONFINITE = 4,     /* host-side name for MUON_FLAG_NONFINITE */
+    MUON_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed (see cudaGetLastError) */
+    MUON_ERR_TIMEOUT = 6        /* host-side name for MUON_FLAG_TIMEOUT */
+} muon_status;
+
+/* Bits OR-ed into *d_status by the device. */
+#define MUON_FLAG_NONFINITE 1   /* a matrix had a non-finite Frobenius norm; its W was left unchanged */
+#define MUON_FLAG_TIMEOUT   2   /* a kernel's internal wait ran out (about 4 s); its output is invalid */
+
+typedef enum {
+    MUON_BF16 = 0,
+    MUON_FP16 = 1,
+    MUON_FP32 = 2
+} muon_dtype;
+
+/* One Newton-Schulz step X <- a X + (b A + c A^2) X. */
+typedef struct {
+    float a, b, c;
+} muon_ns_coeff;
+
+typedef struct {
+    int n_steps;                 /* >= 1, <= 64 */
+    const muon_ns_coeff* coeffs; /* host array of n_steps entries */
+    float eps;                   /* added to ||M||_F before dividing; >= 0 (1e-7 is the usual choice) */
+    const int* restarts;         /* host array of step indices (0 allowed, ignored); may be NULL if n_restarts == 0 */
+    int n_restarts;              /* >= 0, <= 64 */
+    float scale_f;               /* >= 1: extra divisor at the start and at every restart (1.02-1.05 on the Gram route) */
+} muon_schedule;
+
+/* Hyper-parameters of [MONA] section 2. */
+typedef struct {
+    float mu;       /* momentum */
+    float eta;      /* learning rate */
+    float lambda;   /* decoupled weight decay */
+    float gamma;    /* scale of the orthogonalised update */
+    float beta_a;   /* EMA factor of the acceleration buffer */
+    float alpha;    /* weight of the acceleration term */
+} muon_hparams;
+
+/* One matrix parameter and its optimizer state (all device memory). */
+typedef struct {
+    int rows, cols;    /* >= 1 */
+    void* W;           /* rows x cols, w_dtype, updated in place */
+    const void* G;     /* rows x cols, w_dtype, this step's gradient (read only) */
+    void* G_prev;      /* rows x cols, w_dtype, previous gradient; receives G */
+    float* A;          /* rows x cols, fp32 acceleration buffer, updated in place */
+    float* M;          /* rows x cols, fp32 momentum, updated in place */
+    float gamma;       /* per-matrix gamma; NaN means "use hparams.gamma" */
+    float* O_out;      /* optional rows x cols fp32: receives O (the orthogonalised momentum); NULL to skip */
+} muon_param;
+
+/*
+ * Bytes of workspace muon_step_batched needs for these parameters.
+ * params: host array of n descriptors (only rows/cols are read).
+ * Returns MUON_ERR_INVALID_ARG for n < 1, NULL pointers or non-positive sizes.
+ */
+MUON_API muon_status muon_workspace_size(const muon_param* params, int n, muon_dtype ns_dtype,
+                                size_t* bytes);
+
+/*
+ * One optimizer step ([MONA] section 2, steps 1-4) for n matrix parameters.
+ *   1. One fused pass over every element: A, M, G_prev updated in place as in
+ *      steps 1-4, the Frobenius norm of the new M accumulated per matrix, and
+ *      M written in ns_dtype (wide view) to the workspace.
+ *   2. The quintic iteration above on every matrix (matrices with the same
+ *      (short side, long side) are batched together).
+ *   3. W <- W - eta (gamma O + lambda W), fused into the last iteration step;
+ *      O never reaches memory unless O_out is given.
+ * w_dtype: element type of W, G and G_prev (MUON_BF16, MUON_FP16 or MUON_FP32).
+ * ns_dtype: arithmetic of the iteration: MUON_BF16 / MUON_FP16 (tensor cores,
+ *   fp32 accumulation, 16-bit operands) or MUON_FP32 (CUDA-core fp32).
+ * hp: host struct.  sched: host struct (restarts divide by scale_f as above).
+ * A matrix whose norm is not finite keeps its W and sets MUON_FLAG_NONFINITE.
+ * W, G, G_prev, A, M of one parameter may not overlap another parameter's.
+ */
+MUON_API muon_status muon_step_batched(const muon_param* params, int n, muon_dtype w_dtype,
+                              muon_dtype ns_dtype, const muon_hparams* hp,
+                              const muon_schedule* sched, void* workspace, size_t ws_bytes,
+                              int* d_status, muon_stream_t stream);
+
+/*
+ * Bytes of workspace ns_polar / gram_polar need for a batch of rows x cols
+ * matrices in `dtype`.
+ */
+MUON_API muon_status ns_polar_workspace_size(int batch, int rows, int cols, muon_dtype dtype,
+                                    size_t* bytes);
+MUON_API muon_status gram_polar_workspace_size(int batch, int rows, int cols, muon_dtype dtype,
+                                      size_t* bytes);
+
+/*
+ * Orthogonalise a batch of matrices with the direct iteration ([POLAR]
+ * Newton-Schulz).  X_in: device, batch matrices of rows x cols in `dtype`,
+ * matrix i at X_in + i * batch_stride elements (batch_stride >= rows*cols).
+ * X_out: device, same layout and dtype; may equal X_in.
+ * dtype MUON_BF16 / MUON_FP16 run on tensor cores, MUON_FP32 on CUDA cores.
+ */
+MUON_API muon_status ns_polar(const void* X_in, void* X_out, int batch, int rows, int cols,
+                     long long batch_stride, muon_dtype dtype, const muon_schedule* sched,
+                     void* workspace, size_t ws_bytes, int* d_status, muon_stream_t stream);
+
+/*
+ * The same result through the Gram route ([POLAR] X (X^T X)^{-1/2}): all
+ * iteration steps work on s x s symmetric matrices (upper tiles computed and
+ * mirrored); the s x l operand is touched only at the start, at restarts and
+ * at the end.  Arguments as ns_polar; sched->restarts and sched->scale_f
+ * select the restart steps and the divisor f.
+ */
+MUON_API muon_status gram_polar(const void* X_in, void* X_out, int batch, int rows, int cols,
+                       long long batch_stride, muon_dtype dtype, const muon_schedule* sched,
+                       void* workspace, size_t ws_bytes, int* d_status, muon_stream_t stream);
+
+/*
+ * Tracing aid (optional).  While enabled, every kernel the library launches
+ * is bracketed by two CUDA events recorded on the launch stream, and the
+ * launch's algorithmic work is noted: floating-point operations for the
+ * Newton-Schulz products (a symmetric product counts the half it needs,
+ * n*n*k; a full product 2*m*n*k) or bytes moved for the elementwise pass.
+ * Events come from a fixed host-side pool created on first use (up to
+ * MUON_TRACE_CAPACITY launches; later launches are not recorded).
+ * muon_trace_read synchronises on the recorded events, copies up to `max`
+ * records (oldest first) to `out` (host array), clears the log and returns
+ * the number of records copied (or -1 on a CUDA error).
+ */
+#define MUON_TRACE_CAPACITY 8192
+typedef enum {
+    MUON_KERNEL_PREPASS = 0,   /* fused MONA pre-pass / input copy + norms (work = bytes) */
+    MUON_KERNEL_SYM = 1,       /* tcgen05 symmetric product X X^T, A A, ... (work = flops) */
+    MUON_KERNEL_UPD = 2,       /* tcgen05 update product X <- aX + BX, Q Xb (work = flops) */
+    MUON_KERNEL_SIMT = 3,      /* fp32 CUDA-core product (work = flops) */
+    MUON_KERNEL_OTHER = 4      /* identity fill (work = bytes) */
+} muon_kernel_kind;
+
+typedef struct {
+    int kind;        /* muon_kernel_kind */
+    double work;     /* algorithmic flops or bytes of this launch */
+    float ms;        /* device time between the bracketing events */
+} muon_trace_record;
+
+MUON_API muon_status muon_trace_enable(int enable);
+MUON_API int muon_trace_read(muon_trace_record* out, int max);
+
+/* Static, NUL-terminated description of a status code. */
+MUON_API const char* muon_status_string(muon_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_B200_H */

@@ -1,0 +1,238 @@
+"""Python binding of the sm_100a Muon / MONA optimizer library (libmuon_b200.so).
+
+Argument marshalling only: every step of the optimizer runs in the CUDA
+kernels behind the C ABI of ``include/muon.h``.  PyTorch is used for device
+memory and streams.  There is no fallback: if the shared library is missing
+or cannot be loaded, every call raises.
+
+Names follow the C ABI: :func:`muon_step_batched`, :func:`ns_polar`,
+:func:`gram_polar`, :func:`muon_workspace_size`, :func:`ns_polar_workspace_size`,
+:func:`gram_polar_workspace_size`, :func:`muon_status_string`.
+"""
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmuon_b200.so")
+
+BF16, FP16, FP32 = 0, 1, 2
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_NONFINITE, ERR_CUDA, ERR_TIMEOUT = range(7)
+FLAG_NONFINITE, FLAG_TIMEOUT = 1, 2
+
+# the fixed quintic coefficients (a, b, c) of the Muon iteration
+QUINTIC = (3.4445, -4.7750, 2.0315)
+# cubic Newton-Schulz for the polar factor (converges for 0 < sigma < sqrt(3))
+CUBIC = (1.5, -0.5, 0.0)
+
+
+class MuonError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {muon_status_string(status)} (status {status})")
+
+
+class NsCoeff(ctypes.Structure):
+    _fields_ = [("a", ctypes.c_float), ("b", ctypes.c_float), ("c", ctypes.c_float)]
+
+
+class Schedule(ctypes.Structure):
+    _fields_ = [("n_steps", ctypes.c_int), ("coeffs", ctypes.POINTER(NsCoeff)),
+                ("eps", ctypes.c_float), ("restarts", ctypes.POINTER(ctypes.c_int)),
+                ("n_restarts", ctypes.c_int), ("scale_f", ctypes.c_float)]
+
+
+class HParams(ctypes.Structure):
+    _fields_ = [("mu", ctypes.c_float), ("eta", ctypes.c_float), ("lambda_", ctypes.c_float),
+                ("gamma", ctypes.c_float), ("beta_a", ctypes.c_float), ("alpha", ctypes.c_float)]
+
+
+class Param(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("cols", ctypes.c_int), ("W", ctypes.c_void_p),
+                ("G", ctypes.c_void_p), ("G_prev", ctypes.c_void_p), ("A", ctypes.c_void_p),
+                ("M", ctypes.c_void_p), ("gamma", ctypes.c_float), ("O_out", ctypes.c_void_p)]
+
+
+KERNEL_PREPASS, KERNEL_SYM, KERNEL_UPD, KERNEL_SIMT, KERNEL_OTHER = range(5)
+KERNEL_NAMES = {KERNEL_PREPASS: "prepass", KERNEL_SYM: "tc_sym", KERNEL_UPD: "tc_upd",
+                KERNEL_SIMT: "simt", KERNEL_OTHER: "other"}
+TRACE_CAPACITY = 8192
+
+
+class TraceRecord(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("work", ctypes.c_double), ("ms", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libmuon_b200.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m muon_family_optimizer_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        st = ctypes.c_int
+        vp = ctypes.c_void_p
+        sz = ctypes.POINTER(ctypes.c_size_t)
+        L.muon_status_string.restype = ctypes.c_char_p
+        L.muon_status_string.argtypes = [st]
+        L.muon_workspace_size.restype = st
+        L.muon_workspace_size.argtypes = [ctypes.POINTER(Param), ctypes.c_int, ctypes.c_int, sz]
+        L.muon_step_batched.restype = st
+        L.muon_step_batched.argtypes = [ctypes.POINTER(Param), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.POINTER(HParams), ctypes.POINTER(Schedule), vp,
+                                        ctypes.c_size_t, vp, vp]
+        for name in ("ns_polar_workspace_size", "gram_polar_workspace_size"):
+            f = getattr(L, name)
+            f.restype = st
+            f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, sz]
+        for name in ("ns_polar", "gram_polar"):
+            f = getattr(L, name)
+            f.restype = st
+            f.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
+                          ctypes.c_int, ctypes.POINTER(Schedule), vp, ctypes.c_size_t, vp, vp]
+        L.muon_trace_enable.restype = st
+        L.muon_trace_enable.argtypes = [ctypes.c_int]
+        L.muon_trace_read.restype = ctypes.c_int
+        L.muon_trace_read.argtypes = [ctypes.POINTER(TraceRecord), ctypes.c_int]
+        _lib = L
+    return _lib
+
+
+def muon_status_string(status):
+    return lib().muon_status_string(int(status)).decode()
+
+
+def _check(status, where):
+    if status != OK:
+        raise MuonError(status, where)
+
+
+def make_schedule(coeffs, eps=1e-7, restarts=(), scale_f=1.0):
+    """Build a C schedule; the returned object keeps its arrays alive."""
+    coeffs = [tuple(c) for c in coeffs]
+    arr = (NsCoeff * len(coeffs))(*[NsCoeff(*c) for c in coeffs])
+    rs = list(restarts)
+    rarr = (ctypes.c_int * max(1, len(rs)))(*rs) if rs else None
+    s = Schedule(len(coeffs), arr, eps, rarr, len(rs), scale_f)
+    s._keep = (arr, rarr)
+    return s
+
+
+def quintic_schedule(n_steps=5, eps=1e-7, scale_f=1.0):
+    return make_schedule([QUINTIC] * n_steps, eps=eps, scale_f=scale_f)
+
+
+def _dtype_code(t):
+    import torch
+    return {torch.bfloat16: BF16, torch.float16: FP16, torch.float32: FP32}[t]
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def make_params(params):
+    """params: list of dicts with torch tensors W, G, G_prev, A, M (+ optional gamma, O_out)."""
+    arr = (Param * len(params))()
+    for i, p in enumerate(params):
+        W = p["W"]
+        rows, cols = W.shape
+        for k in ("W", "G", "G_prev", "A", "M"):
+            t = p[k]
+            if tuple(t.shape) != (rows, cols) or not t.is_contiguous():
+                raise ValueError(f"param {i}: {k} must be a contiguous {rows}x{cols} tensor")
+        arr[i] = Param(rows, cols, W.data_ptr(), p["G"].data_ptr(), p["G_prev"].data_ptr(),
+                       p["A"].data_ptr(), p["M"].data_ptr(), float(p.get("gamma", math.nan)),
+                       p["O_out"].data_ptr() if p.get("O_out") is not None else None)
+    return arr
+
+
+def muon_workspace_size(params, ns_dtype):
+    arr = params if isinstance(params, ctypes.Array) else make_params(params)
+    out = ctypes.c_size_t(0)
+    _check(lib().muon_workspace_size(arr, len(arr), int(ns_dtype), ctypes.byref(out)),
+           "muon_workspace_size")
+    return out.value
+
+
+def muon_step_batched(params, w_dtype, ns_dtype, hp, schedule, workspace, d_status=None, stream=None):
+    """One MONA/Muon step on every parameter (see include/muon.h).
+
+    params: list of dicts (see make_params) or a ctypes Param array.
+    hp: dict with mu, eta, lambda, gamma, beta_a, alpha.  schedule: make_schedule(...).
+    workspace: a CUDA uint8 tensor of at least muon_workspace_size(...) bytes.
+    """
+    arr = params if isinstance(params, ctypes.Array) else make_params(params)
+    h = HParams(hp["mu"], hp["eta"], hp["lambda"], hp["gamma"], hp["beta_a"], hp["alpha"])
+    _check(lib().muon_step_batched(arr, len(arr), int(w_dtype), int(ns_dtype), ctypes.byref(h),
+                                   ctypes.byref(schedule), _ptr(workspace), workspace.numel(),
+                                   _ptr(d_status), _stream_ptr(stream)), "muon_step_batched")
+
+
+def ns_polar_workspace_size(batch, rows, cols, dtype):
+    out = ctypes.c_size_t(0)
+    _check(lib().ns_polar_workspace_size(batch, rows, cols, int(dtype), ctypes.byref(out)),
+           "ns_polar_workspace_size")
+    return out.value
+
+
+def gram_polar_workspace_size(batch, rows, cols, dtype):
+    out = ctypes.c_size_t(0)
+    _check(lib().gram_polar_workspace_size(batch, rows, cols, int(dtype), ctypes.byref(out)),
+           "gram_polar_workspace_size")
+    return out.value
+
+
+def _polar(fn, X_in, X_out, schedule, workspace, d_status, stream):
+    if X_in.dim() == 2:
+        batch, (rows, cols) = 1, X_in.shape
+    else:
+        batch, rows, cols = X_in.shape
+    if not X_in.is_contiguous() or not X_out.is_contiguous() or X_out.shape != X_in.shape \
+            or X_out.dtype != X_in.dtype:
+        raise ValueError("X_in / X_out must be contiguous tensors of the same shape and dtype")
+    _check(fn(_ptr(X_in), _ptr(X_out), batch, rows, cols, rows * cols, _dtype_code(X_in.dtype),
+              ctypes.byref(schedule), _ptr(workspace), workspace.numel(), _ptr(d_status),
+              _stream_ptr(stream)), fn.__name__)
+
+
+def ns_polar(X_in, X_out, schedule, workspace, d_status=None, stream=None):
+    """Direct Newton-Schulz orthogonalisation of a (batch of) matrices."""
+    _polar(lib().ns_polar, X_in, X_out, schedule, workspace, d_status, stream)
+
+
+def gram_polar(X_in, X_out, schedule, workspace, d_status=None, stream=None):
+    """The same iteration through the Gram matrix (restarts, divisor scale_f)."""
+    _polar(lib().gram_polar, X_in, X_out, schedule, workspace, d_status, stream)
+
+
+def converged_schedule(eps=1e-7):
+    """8 quintic + 6 cubic steps, restarts before steps 3, 5 and 7, divisor 1.05.
+
+    Converges to the polar factor for condition numbers up to about 1e3; the
+    restarts keep the Gram route stable in 16-bit arithmetic."""
+    return make_schedule([QUINTIC] * 8 + [CUBIC] * 6, eps=eps, restarts=(3, 5, 7), scale_f=1.05)
+
+
+def muon_trace_enable(enable=True):
+    _check(lib().muon_trace_enable(1 if enable else 0), "muon_trace_enable")
+
+
+def muon_trace_read():
+    """List of (kind, work, ms) for the launches recorded since the last read."""
+    buf = (TraceRecord * TRACE_CAPACITY)()
+    n = lib().muon_trace_read(buf, TRACE_CAPACITY)
+    if n < 0:
+        raise MuonError(ERR_CUDA, "muon_trace_read")
+    return [(buf[i].kind, buf[i].work, buf[i].ms) for i in range(n)]

@@ -1,0 +1,68 @@
+// gemm.h -- host-side description of one batched GEMM problem of the
+// Newton-Schulz iteration and the two back ends that run it.
+#pragma once
+
+#include "epilogue.cuh"
+
+namespace muon {
+
+// D = A B^T (sym = 1: B given as N x K rows, result symmetric, upper tiles
+// computed and mirrored) or D = A B (sym = 0: B given as K x N row-major),
+// for `count` matrices; strides and leading dimensions in elements.
+struct GemmOp {
+    int sym;
+    // Operand stored as a symmetric matrix of which only the tiles on or above
+    // the diagonal (128 x 128) are valid (tensor-core path): blocks left of the
+    // diagonal tile are read transposed from the stored upper tile.
+    int a_sym, b_sym;
+    int count, M, N, K;
+    const void* A; long long lda, strideA;
+    const void* B; long long ldb, strideB;
+    Epilogue epi;
+};
+
+namespace tc {
+// tcgen05 back end for 16-bit operands (dt = DT_BF16 or DT_FP16); all ops of
+// one call must have the same `sym` and are run by one launch.
+muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, const FinalEntry* fin,
+                   int nfin, cudaStream_t stream);
+}
+namespace simt {
+// CUDA-core fp32 back end (dt = DT_FP32): one launch per op.
+muon_status simt_run(const GemmOp* ops, int nops, const FinalCtx& fc, const FinalEntry* fin, int nfin,
+                     cudaStream_t stream);
+}
+
+// Fused elementwise passes ahead of the iteration (prepass.cu).
+constexpr int kMaxPrep = 64;
+
+struct PrepEntry {
+    const void* G; void* Gp; float* A; float* M;   // MONA mode: this parameter's state
+    const void* X; long long x_stride;             // COPY mode: batch input
+    void* X0; long long x0_stride, ld;             // wide-view destination
+    int rows, cols, count, transposed, vec_ok;
+    int sumsq_index;
+    int tiles_c;
+    long long tiles_per_mat, tile_begin;
+};
+
+struct PrepParams {
+    PrepEntry e[kMaxPrep];
+    int n;
+    long long total_tiles;
+    int in_dt, x0_dt, mode;   // mode 0 = MONA pre-pass, 1 = copy (normalisation input of ns/gram_polar)
+    float beta_a, alpha, mu;
+    double* sumsq;
+};
+
+muon_status prep_run(PrepParams& prm, cudaStream_t stream);
+
+// Launch tracing (trace.cu): no-ops unless muon_trace_enable(1) was called.
+void trace_begin(int kind, double work, cudaStream_t stream);
+void trace_end(cudaStream_t stream);
+
+// Small helpers (prepass.cu)
+muon_status fill_identity(void* D, int dt, int count, int s, long long ld, long long stride,
+                          cudaStream_t stream);
+
+}  // namespace muon

@@ -1,0 +1,644 @@
+// gemm_tc.cu -- batched, grouped tcgen05 GEMMs for the Newton-Schulz steps.
+//
+// [POLAR] (quant_prune_distill post 677): the Muon step replaces the momentum
+// by its polar factor, computed by Newton-Schulz; products of symmetric
+// matrices need only half of their elements.  Every product of one iteration
+// step is one of two shapes:
+//   SYM:  D = A B^T with a symmetric result: X X^T, A A (A symmetric), and on
+//         the Gram route R R, h Q, h R, (h R) h (polynomials in one symmetric
+//         matrix commute, so each product is symmetric).  Only the 128 x 128
+//         tiles on or above the diagonal are computed and stored; nothing is
+//         mirrored.  A consumer that needs a block left of the diagonal tile
+//         reads the stored block above the diagonal transposed (MN-major
+//         operand layout), chosen per 64-deep k-block.
+//   UPD:  D = A X with A (s x s) symmetric and X (s x l) row-major, i.e. the
+//         B operand is MN-major: X <- (a I + b A + c A^2) X, Xb <- Q Xb.
+//
+// Kernel shape (one CTA per SM, persistent over a flattened tile list that
+// spans every matrix of up to four shape groups):
+//   warp 0      TMA producer: 128-byte-swizzled boxes of A and B into a ring
+//               of shared-memory stages (no multicast: every CTA loads its own
+//               tiles);
+//   warp 1      allocates tensor memory; one thread issues tcgen05.mma
+//               (kind::f16, fp32 accumulate, 128 x BN x 16) and commits stage
+//               releases and accumulator hand-offs to mbarriers;
+//   warps 2-9   epilogue, two warps per tensor-memory lane quadrant (each takes
+//               half of the columns): tcgen05.ld of the fp32 accumulator,
+//               scale / combine, round to 16 bits into a per-warp 128B-swizzled
+//               staging box (32 rows x 64 columns) and a TMA bulk store of the
+//               box; the final step writes the caller's layout directly.
+// Two accumulator buffers in tensor memory let the epilogue of tile t overlap
+// the main loop of tile t+1.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "epilogue.cuh"
+#include "gemm.h"
+
+namespace muon {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;    // 64 16-bit elements = one 128-byte swizzle row
+constexpr int kEpiWarps = 8;    // two per tensor-memory lane quadrant, each takes half the columns
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+
+template <int BN>
+struct Cfg {
+    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kABytes = BM * BK * 2;
+    static constexpr int kBBytes = BN * BK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kTmemCols = 2 * BN;
+    static constexpr int kStgBytes = 32 * 64 * 2;              // one 32 x 64 16-bit box per epilogue warp
+    static constexpr int kFinBytes = 32 * 33 * 4;              // final steps: one padded 32 x 32 fp32 box per warp
+    static constexpr int kStgOffset = kStages * kStageBytes;
+    static constexpr int kBarOffset = kStgOffset + kEpiWarps * kFinBytes;   // kFinBytes > kStgBytes
+    static constexpr int kBarBytes = 256;
+    static constexpr int kSmemBytes = 1024 + kBarOffset + kBarBytes;
+};
+
+struct TcProblem {
+    CUtensorMap mapA;    // A rows, K-major boxes 64 (K) x 128 (M)
+    CUtensorMap mapAt;   // A symmetric: transposed reads, boxes 64 (M) x 64 (K)
+    CUtensorMap mapB;    // SYM: B rows, boxes 64 (K) x 128 (N); UPD: X panel, boxes 64 (N) x 64 (K)
+    CUtensorMap mapBt;   // B symmetric: transposed reads, boxes 64 (N) x 64 (K)
+    CUtensorMap mapD;    // output stores, boxes 64 (N) x 32 (M)
+    int count, M, N, K;
+    int tiles_m, tiles_n, tiles_per_mat, sym, a_sym, b_sym;
+    long long tile_begin;
+    Epilogue epi;
+};
+
+struct TcParams {
+    TcProblem prob[kMaxProblems];
+    int nprob;
+    long long total_tiles;
+    FinalCtx fc;
+    FinalEntry fin[kMaxFinal];
+};
+
+__device__ __forceinline__ void decode_tile(const TcParams& p, long long t, int& pi, int& m,
+                                            int& ti, int& tj) {
+    pi = 0;
+    while (pi + 1 < p.nprob && t >= p.prob[pi + 1].tile_begin) ++pi;
+    const TcProblem& P = p.prob[pi];
+    long long local = t - P.tile_begin;
+    m = (int)(local / P.tiles_per_mat);
+    int r = (int)(local - (long long)m * P.tiles_per_mat);
+    if (P.sym) {
+        int nt = P.tiles_m, i = 0;
+        while (r >= nt - i) { r -= nt - i; ++i; }
+        ti = i;
+        tj = i + r;
+    } else {
+        ti = r % P.tiles_m;
+        tj = r / P.tiles_m;
+    }
+}
+
+// Previous-operand values of one chunk (row gi, columns gj0..gj0+31) as raw
+// 16-bit data in four 16-byte words; issued ahead of use to hide its latency.
+template <typename T>
+__device__ __forceinline__ void cin_fetch(const Epilogue& E, int m, int gi, int gj0, int M, int N,
+                                          uint4 (&c)[4]) {
+    if (gi >= M || gj0 >= N) return;
+    const T* src = static_cast<const T*>(E.Cin) + (size_t)m * E.strideC + (size_t)gi * E.ldc + gj0;
+    if (gj0 + 32 <= N) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) c[q] = reinterpret_cast<const uint4*>(src)[q];
+    } else {
+        T* e = reinterpret_cast<T*>(c);
+        for (int q = 0; q < 32; ++q) e[q] = gj0 + q < N ? src[q] : from_float<T>(0.f);
+    }
+}
+
+// Final step for one 32 x 32 block of the wide view (rows gi0..gi0+31 held by
+// the warp's lanes, columns gj0..gj0+31), already staged in `fs` (padded
+// [32][33] fp32, row = wide row).  Writes the caller's output (FIN_OUT) or
+// applies W <- W - eta (gamma O + lambda W) (FIN_WUPD) in the parameter's own
+// orientation: each lane moves 8 consecutive elements of one parameter row,
+// four lanes per 32-element row segment, so every global access is a
+// coalesced 16-byte (or 32-byte) access whichever way the parameter is stored.
+template <typename TW>
+__device__ __forceinline__ void final_block(const Epilogue& E, const FinalCtx& fc, int m, int M, int N,
+                                            int gi0, int gj0, const float* fs, int lane) {
+    constexpr int kDt = sizeof(TW) == 4 ? DT_FP32 : (IsBf16<TW>::value ? DT_BF16 : DT_FP16);
+    TW* W;
+    float* O_out = nullptr;
+    float g = 0.f;
+    int tr, vec;
+    const bool wupd = E.fin == FIN_WUPD;
+    if (!wupd) {
+        W = reinterpret_cast<TW*>(static_cast<char*>(fc.out) + (size_t)m * fc.out_stride * sizeof(TW));
+        tr = fc.out_transposed; vec = fc.out_vec;
+    } else {
+        const FinalEntry& fe = fc.fin[E.fin_base + m];
+        W = static_cast<TW*>(fe.W); O_out = fe.O_out; g = fe.gamma; tr = fe.transposed; vec = fe.vec_ok;
+    }
+    // parameter extent: tr ? (N rows x M cols) : (M rows x N cols)
+    const int prow_n = tr ? N : M, pcol_n = tr ? M : N;
+    const int prow0 = tr ? gj0 : gi0, pcol0 = tr ? gi0 : gj0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int rr = 8 * k + (lane >> 2);       // parameter row inside the block
+        const int cc = (lane & 3) * 8;            // first of 8 parameter columns inside the block
+        const int prow = prow0 + rr, pcol = pcol0 + cc;
+        if (prow >= prow_n || pcol >= pcol_n) continue;
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = tr ? fs[(cc + e) * 33 + rr] : fs[rr * 33 + cc + e];
+        TW* wp = W + (size_t)prow * pcol_n + pcol;
+        const bool full = vec && pcol + 8 <= pcol_n;
+        if (wupd) {
+            float w[8];
+            if (full) {
+                load8_dt(wp, 0, kDt, true, 8, w);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) w[e] = pcol + e < pcol_n ? to_float(wp[e]) : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = w[e] - fc.eta * (g * o[e] + fc.lambda * w[e]);
+            if (full) {
+                store8_dt(wp, 0, kDt, true, 8, w);
+                if (O_out) store8_dt(O_out + (size_t)prow * pcol_n + pcol, 0, DT_FP32, true, 8, o);
+            } else {
+                for (int e = 0; e < 8 && pcol + e < pcol_n; ++e) {
+                    wp[e] = from_float<TW>(w[e]);
+                    if (O_out) O_out[(size_t)prow * pcol_n + pcol + e] = o[e];
+                }
+            }
+        } else if (full) {
+            store8_dt(wp, 0, kDt, true, 8, o);
+        } else {
+            for (int e = 0; e < 8 && pcol + e < pcol_n; ++e) wp[e] = from_float<TW>(o[e]);
+        }
+    }
+}
+
+// Stage the warp's 32 x 32 block (this lane: wide row gi0 + lane) and write it out.
+__device__ __forceinline__ void final_chunk_dispatch(const Epilogue& E, const FinalCtx& fc, int m, int M,
+                                                     int N, int gi0, int gj0, const float (&v)[32],
+                                                     float* fs, int lane) {
+    __syncwarp();                       // the previous block's reads of fs are done
+#pragma unroll
+    for (int q = 0; q < 32; ++q) fs[lane * 33 + q] = v[q];
+    __syncwarp();
+    const int dt = E.fin == FIN_OUT ? fc.out_dt : fc.w_dt;
+    if (dt == DT_BF16) final_block<__nv_bfloat16>(E, fc, m, M, N, gi0, gj0, fs, lane);
+    else if (dt == DT_FP16) final_block<__half>(E, fc, m, M, N, gi0, gj0, fs, lane);
+    else final_block<float>(E, fc, m, M, N, gi0, gj0, fs, lane);
+}
+
+// Combine one 32-column chunk of the accumulator (row gi, columns
+// gj0..gj0+31) with the scale, the previous operand (`c`, when beta != 0) and
+// the diagonal shift.
+template <typename T>
+__device__ __forceinline__ void epi_combine(const Epilogue& E, int gi, int gj0, float sc, float (&v)[32],
+                                            const uint4 (&c)[4]) {
+    if (E.beta != 0.f) {
+        const T* ce = reinterpret_cast<const T*>(c);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) v[q] = sc * (E.alpha * v[q] + E.beta * to_float(ce[q]));
+    } else {
+        const float s = sc * E.alpha;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) v[q] *= s;
+    }
+    if (E.diag != 0.f && gi >= gj0 && gi < gj0 + 32) v[gi - gj0] += E.diag;
+}
+
+// Write 32 values (row `r` of the warp's 32 x 64 staging box, 16-byte chunks
+// c16 .. c16+3) in the 128-byte swizzle the store's tensor map expects:
+// chunk c of row r lives at r * 128 + ((c ^ (r % 8)) * 16).
+template <typename T>
+__device__ __forceinline__ void stage32(uint8_t* stg, int r, int c16, const float (&v)[32]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 u;
+        T* e = reinterpret_cast<T*>(&u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) e[i] = from_float<T>(v[8 * q + i]);
+        *reinterpret_cast<uint4*>(stg + r * 128 + (((c16 + q) ^ (r & 7)) * 16)) = u;
+    }
+}
+
+// Barrier over the epilogue warps only (named barrier 1).
+__device__ __forceinline__ void epi_bar() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+}
+
+// Byte offset of element (r, c) (r < 32, c < 64) in a 32 x 64 16-bit staging box.
+__device__ __forceinline__ int stg_off(int r, int c) {
+    return r * 128 + (((c >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
+}
+
+// Diagonal tile of a symmetric result: the eight epilogue warps hold the whole
+// 128 x 128 tile in their staging boxes (box quad + 4 * half: rows 32*quad..,
+// columns 64*half..).  Overwrite this thread's elements below the diagonal
+// (local row i, column j < i) with the element (j, i) above it, so the stored
+// tile is exactly symmetric.  Reads touch only positions above the diagonal,
+// writes only positions below it.
+template <typename T>
+__device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int half, int lane) {
+    const int i = quad * 32 + lane;
+    uint8_t* mine = stg_base + (quad + 4 * half) * (32 * 64 * 2);
+    for (int q = 0; q < 64; ++q) {
+        const int j = half * 64 + q;
+        if (j >= i) break;
+        const uint8_t* ob = stg_base + ((j >> 5) + 4 * (i >> 6)) * (32 * 64 * 2);
+        const T x = *reinterpret_cast<const T*>(ob + stg_off(j & 31, i & 63));
+        *reinterpret_cast<T*>(mine + stg_off(lane, q)) = x;
+    }
+}
+
+template <int BN, bool B_MN, typename T>
+__global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
+    using C = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+    uint64_t* empty_bar = full_bar + C::kStages;
+    uint64_t* tfull_bar = empty_bar + C::kStages;
+    uint64_t* tempty_bar = tfull_bar + 2;
+    uint64_t* drain_bar = tempty_bar + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    int* d_status = p.fc.d_status;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], kEpiThreads);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < p.nprob; ++i) {
+            prefetch_tensormap(&p.prob[i].mapA);
+            prefetch_tensormap(&p.prob[i].mapB);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t armed = 0;          // bit s: stage s has been armed at least once
+            uint32_t armed_parity = 0;   // bit s: parity of the phase stage s was last armed in
+            for (long long t = blockIdx.x; t < p.total_tiles && !*abort_flag; t += gridDim.x) {
+                int pi, m, ti, tj;
+                decode_tile(p, t, pi, m, ti, tj);
+                const TcProblem& P = p.prob[pi];
+                const int nkb = (P.K + BK - 1) / BK;
+                int nchunk = BN / 64;
+                if (B_MN) {
+                    const int rem = P.N - tj * BN;
+                    nchunk = min(BN / 64, (rem + 63) / 64);
+                }
+                const uint32_t bytes = C::kABytes + (B_MN ? nchunk * 64 * BK * 2 : C::kBBytes);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, d_status)) break;
+                    uint8_t* sa = smem + stage * C::kStageBytes;
+                    uint8_t* sb = sa + C::kABytes;
+                    mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                    if (P.a_sym && (kb >> 1) < ti) {
+                        // rows ti*128.. of a symmetric A, k-block left of the diagonal
+                        // tile: read the stored block above the diagonal, transposed
+                        tma_load_3d(&P.mapAt, &full_bar[stage], sa, ti * BM, kb * BK, m);
+                        tma_load_3d(&P.mapAt, &full_bar[stage], sa + 64 * BK * 2, ti * BM + 64, kb * BK, m);
+                    } else {
+                        tma_load_3d(&P.mapA, &full_bar[stage], sa, kb * BK, ti * BM, m);
+                    }
+                    if (B_MN) {
+                        for (int c = 0; c < nchunk; ++c)
+                            tma_load_3d(&P.mapB, &full_bar[stage], sb + c * (64 * BK * 2), tj * BN + c * 64, kb * BK, m);
+                    } else if (P.b_sym && (kb >> 1) < tj) {
+                        for (int c = 0; c < BN / 64; ++c)
+                            tma_load_3d(&P.mapBt, &full_bar[stage], sb + c * (64 * BK * 2), tj * BN + c * 64, kb * BK, m);
+                    } else {
+                        tma_load_3d(&P.mapB, &full_bar[stage], sb, kb * BK, tj * BN, m);
+                    }
+                    armed |= 1u << stage;
+                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (*abort_flag) {
+                // wind down: every armed stage's copies must land before the CTA exits
+                const unsigned long long t0 = global_ns();
+                for (int s = 0; s < C::kStages; ++s) {
+                    if (!(armed >> s & 1u)) continue;
+                    const uint32_t par = armed_parity >> s & 1u;
+                    while (!mbar_try_wait(&full_bar[s], par) && global_ns() - t0 < kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc0 = make_idesc_f16(IsBf16<T>::value ? 1 : 0, 0, BM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            for (long long t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x, ++it) {
+                int pi, m, ti, tj;
+                decode_tile(p, t, pi, m, ti, tj);
+                const TcProblem& P = p.prob[pi];
+                const int nkb = (P.K + BK - 1) / BK;
+                const int buf = it & 1;
+                const uint32_t tphase = (it >> 1) & 1;
+                if (!mbar_wait(&tempty_bar[buf], tphase ^ 1, abort_flag, d_status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, abort_flag, d_status)) { ok = false; break; }
+                    tc_fence_after();
+                    const bool at = P.a_sym && (kb >> 1) < ti;                 // A block read transposed
+                    const bool bm = B_MN || (P.b_sym && (kb >> 1) < tj);       // B block MN-major
+                    const uint32_t idesc = idesc0 | (at ? 1u << 15 : 0u) | (bm ? 1u << 16 : 0u);
+                    const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+                    const uint32_t sb = sa + C::kABytes;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        // K-major: the k-th 16-element slice sits 32 bytes further in each
+                        // swizzled 128-byte row; MN-major: 16 rows of 128 bytes further,
+                        // 64-element MN chunks 64 x BK x 2 bytes apart.
+                        const uint64_t ad = at ? smem_desc_sw128(sa + k * 2048, 64 * BK * 2, 1024)
+                                               : smem_desc_sw128(sa + k * 32, 16, 1024);
+                        const uint64_t bd = bm ? smem_desc_sw128(sb + k * 2048, 64 * BK * 2, 1024)
+                                               : smem_desc_sw128(sb + k * 32, 16, 1024);
+                        tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty_bar[stage]);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(&tfull_bar[buf]);
+            }
+            // make sure no MMA is still writing tensor memory before it is freed
+            tc_commit(drain_bar);
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try_wait(drain_bar, 0) && global_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        // No warp leaves this loop early: diagonal tiles of symmetric results
+        // synchronise the eight epilogue warps, so every warp walks every tile
+        // and attends those barriers; a warp whose wait failed (abort) only
+        // skips the work.
+        const int ew = warp - 2;              // 0..7
+        const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
+        const int half = ew >> 2;             // which half of the tile's columns
+        const int row = quad * 32 + lane;
+        constexpr int kPairs = BN / 128;      // 64-column boxes per half
+        uint8_t* stg_base = smem + C::kStgOffset;
+        uint8_t* stg = stg_base + (quad + 4 * half) * C::kStgBytes;   // box of rows 32*quad.., columns 64*half..
+        bool stg_busy = false;                // a bulk store may still be reading stg
+        bool dead = false;
+        FinalCtx fc = p.fc;
+        fc.fin = p.fin;
+        int it = 0;
+        for (long long t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
+            int pi, m, ti, tj;
+            decode_tile(p, t, pi, m, ti, tj);
+            const TcProblem& P = p.prob[pi];
+            const Epilogue& E = P.epi;
+            const int buf = it & 1;
+            const uint32_t tphase = (it >> 1) & 1;
+            const int gi = ti * BM + row;
+            const int col0 = tj * BN + half * (BN / 2);
+            const bool has_cin = E.beta != 0.f;
+            const bool diag_sym = P.sym && ti == tj && E.fin == FIN_STORE;   // uniform over the CTA
+            uint4 c0[4] = {}, c1[4] = {};
+            if (!dead) {
+                if (has_cin) {   // independent of the accumulator: fetch before waiting for it
+                    cin_fetch<T>(E, m, gi, col0, P.M, P.N, c0);
+                    cin_fetch<T>(E, m, gi, col0 + 32, P.M, P.N, c1);
+                }
+                // warp-uniform outcome: tcgen05.ld below is warp-collective
+                const bool ok = mbar_wait(&tfull_bar[buf], tphase, abort_flag, d_status);
+                dead = !__all_sync(0xffffffffu, ok);
+                if (!dead) tc_fence_after();
+            }
+            const float sc = epi_scale(E, m);
+            bool skip = false;
+            if (!dead && E.fin != FIN_STORE && !epi_finite(E, m, sc)) {
+                skip = E.fin == FIN_WUPD;   // keep W; a FIN_OUT result carries the NaN
+                if (row == 0 && half == 0 && tj == 0 && ti == 0 && d_status)
+                    atomicOr(d_status, MUON_FLAG_NONFINITE);
+            }
+#pragma unroll 1
+            for (int pr = 0; pr < kPairs; ++pr) {
+                const int gj0 = col0 + pr * 64;
+                const bool work = !dead && gj0 < P.N;       // warp-uniform
+                float v0[32], v1[32];
+                if (work) {
+                    if (has_cin && pr > 0) {
+                        cin_fetch<T>(E, m, gi, gj0, P.M, P.N, c0);
+                        cin_fetch<T>(E, m, gi, gj0 + 32, P.M, P.N, c1);
+                    }
+                    const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                          (uint32_t)(buf * BN + half * (BN / 2) + pr * 64);
+                    tmem_ld_32x32b_x32(tcol, v0);
+                    tmem_ld_32x32b_x32(tcol + 32, v1);
+                    if (!skip) {
+                        epi_combine<T>(E, gi, gj0, sc, v0, c0);
+                        epi_combine<T>(E, gi, gj0 + 32, sc, v1, c1);
+                    }
+                }
+                if (E.fin == FIN_STORE) {
+                    // 32 rows x 64 columns -> staging box -> one bulk tensor store
+                    if (work) {
+                        if (stg_busy) {
+                            if (lane == 0) bulk_wait_read0();
+                            __syncwarp();
+                        }
+                        stage32<T>(stg, lane, 0, v0);
+                        stage32<T>(stg, lane, 4, v1);
+                    }
+                    if (diag_sym) {          // BN == 128 here: the eight boxes cover the tile
+                        epi_bar();
+                        if (work) fix_lower<T>(stg_base, quad, half, lane);
+                        epi_bar();
+                    }
+                    if (work && ti * BM + quad * 32 < P.M) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&P.mapD, stg, gj0, ti * BM + quad * 32, m);
+                            bulk_commit();
+                        }
+                        stg_busy = true;
+                    }
+                } else if (work && !skip && ti * BM + quad * 32 < P.M) {
+                    float* fs = reinterpret_cast<float*>(stg_base + (quad + 4 * half) * C::kFinBytes);
+                    const int gi0 = ti * BM + quad * 32;
+                    final_chunk_dispatch(E, fc, m, P.M, P.N, gi0, gj0, v0, fs, lane);
+                    if (gj0 + 32 < P.N) final_chunk_dispatch(E, fc, m, P.M, P.N, gi0, gj0 + 32, v1, fs, lane);
+                }
+            }
+            if (!dead) {
+                tc_fence_before();
+                mbar_arrive(&tempty_bar[buf]);
+            }
+        }
+        if (lane == 0) bulk_wait0();   // stores complete before the CTA's shared memory goes away
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Host side
+// ----------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 3-D map over `count` matrices of `rows` x `inner` 16-bit elements with row
+// stride `ld` and matrix stride `mstride` (elements); box = box_inner x box_rows x 1.
+static bool encode_map(CUtensorMap* map, int dt, const void* base, long long inner, long long rows,
+                       long long count, long long ld, long long mstride, int box_inner, int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)count};
+    cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)mstride * 2};
+    cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, dt == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN, bool B_MN, typename T>
+static cudaError_t launch_one(const TcParams& prm, int grid, cudaStream_t stream) {
+    using C = Cfg<BN>;
+    auto kern = tc_gemm_kernel<BN, B_MN, T>;
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured_dev = dev;
+    }
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, const FinalEntry* fin,
+                   int nfin, cudaStream_t stream) {
+    if (nops <= 0) return MUON_OK;
+    if (nops > kMaxProblems || nfin > kMaxFinal) return MUON_ERR_UNSUPPORTED;
+    const int sym = ops[0].sym;
+    const int BN = sym ? 128 : 256;
+    // the final-step staging boxes overlap the store boxes: one kind per launch
+    for (int i = 1; i < nops; ++i)
+        if ((ops[i].epi.fin == FIN_STORE) != (ops[0].epi.fin == FIN_STORE)) return MUON_ERR_INVALID_ARG;
+    static TcParams prm_storage;   // large: keep off the stack; filled and consumed within this call
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    TcParams& prm = prm_storage;
+    memset(&prm, 0, sizeof(prm));
+    long long tiles = 0;
+    for (int i = 0; i < nops; ++i) {
+        const GemmOp& o = ops[i];
+        if (o.sym != sym) return MUON_ERR_INVALID_ARG;
+        TcProblem& P = prm.prob[i];
+        P.count = o.count; P.M = o.M; P.N = o.N; P.K = o.K; P.sym = sym;
+        P.tiles_m = (o.M + BM - 1) / BM;
+        P.tiles_n = (o.N + BN - 1) / BN;
+        P.tiles_per_mat = sym ? P.tiles_m * (P.tiles_m + 1) / 2 : P.tiles_m * P.tiles_n;
+        P.tile_begin = tiles;
+        tiles += (long long)P.tiles_per_mat * o.count;
+        P.epi = o.epi;
+        P.a_sym = o.a_sym;
+        P.b_sym = sym ? o.b_sym : 0;
+        // A operand: M rows x K (K contiguous); a symmetric A is also read transposed
+        if (!encode_map(&P.mapA, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, BK, BM)) return MUON_ERR_CUDA;
+        if (o.a_sym && !encode_map(&P.mapAt, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, 64, BK))
+            return MUON_ERR_CUDA;
+        if (sym) {
+            if (!encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK, BN)) return MUON_ERR_CUDA;
+            if (o.b_sym && !encode_map(&P.mapBt, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, 64, BK))
+                return MUON_ERR_CUDA;
+        } else {
+            // X panel: K rows x N (N contiguous); boxes of 64 (N) x BK (K)
+            if (!encode_map(&P.mapB, dt, o.B, o.N, o.K, o.count, o.ldb, o.strideB, 64, BK)) return MUON_ERR_CUDA;
+        }
+        if (o.epi.fin == FIN_STORE &&
+            !encode_map(&P.mapD, dt, o.epi.D, o.N, o.M, o.count, o.epi.ldd, o.epi.strideD, 64, 32))
+            return MUON_ERR_CUDA;
+    }
+    prm.nprob = nops;
+    prm.total_tiles = tiles;
+    prm.fc = fc;
+    for (int i = 0; i < nfin; ++i) prm.fin[i] = fin[i];
+    prm.fc.fin = nullptr;   // the kernel points it at its own copy of the table
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = (int)(tiles < nsm ? tiles : nsm);
+    if (grid <= 0) return MUON_OK;
+    double work = 0.0;   // algorithmic flops: half of a symmetric product, all of a full one
+    for (int i = 0; i < nops; ++i)
+        work += sym ? (double)ops[i].count * ops[i].N * ops[i].N * ops[i].K
+                    : 2.0 * ops[i].count * ops[i].M * ops[i].N * ops[i].K;
+    trace_begin(sym ? MUON_KERNEL_SYM : MUON_KERNEL_UPD, work, stream);
+    cudaError_t e;
+    if (dt == DT_BF16) {
+        e = sym ? launch_one<128, false, __nv_bfloat16>(prm, grid, stream)
+                : launch_one<256, true, __nv_bfloat16>(prm, grid, stream);
+    } else {
+        e = sym ? launch_one<128, false, __half>(prm, grid, stream)
+                : launch_one<256, true, __half>(prm, grid, stream);
+    }
+    trace_end(stream);
+    return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+}
+
+}  // namespace tc
+}  // namespace muon

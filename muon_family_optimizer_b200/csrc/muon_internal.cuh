@@ -1,0 +1,312 @@
+// muon_internal.cuh -- device helpers and launch descriptors shared by the
+// kernels of the sm_100a Muon library (not part of the public ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "muon.h"
+
+namespace muon {
+
+// ----------------------------------------------------------------------------
+// Element types
+// ----------------------------------------------------------------------------
+enum Dt : int { DT_BF16 = MUON_BF16, DT_FP16 = MUON_FP16, DT_FP32 = MUON_FP32 };
+
+__host__ __device__ inline int dt_size(int dt) { return dt == DT_FP32 ? 4 : 2; }
+
+template <typename T> struct IsBf16 { static constexpr bool value = false; };
+template <> struct IsBf16<__nv_bfloat16> { static constexpr bool value = true; };
+
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_float(__half x) { return __half2float(x); }
+__device__ __forceinline__ float to_float(float x) { return x; }
+
+template <typename T> __device__ __forceinline__ T from_float(float x);
+template <> __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+template <> __device__ __forceinline__ __half from_float<__half>(float x) { return __float2half_rn(x); }
+template <> __device__ __forceinline__ float from_float<float>(float x) { return x; }
+
+__device__ __forceinline__ float ld_elem(const void* p, long long i, int dt) {
+    if (dt == DT_FP32) return static_cast<const float*>(p)[i];
+    if (dt == DT_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+    return __half2float(static_cast<const __half*>(p)[i]);
+}
+
+__device__ __forceinline__ void st_elem(void* p, long long i, int dt, float v) {
+    if (dt == DT_FP32) static_cast<float*>(p)[i] = v;
+    else if (dt == DT_BF16) static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+    else static_cast<__half*>(p)[i] = __float2half_rn(v);
+}
+
+// 8 consecutive elements of runtime type dt at base[idx..idx+7]: one or two
+// 16-byte accesses when `vec` (caller guarantees 16-byte alignment), else
+// the first nvalid elements one by one (the rest read as 0).
+__device__ __forceinline__ void load8_dt(const void* base, long long idx, int dt, bool vec, int nvalid,
+                                         float* out) {
+    if (vec) {
+        if (dt == DT_FP32) {
+            const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
+            float4 a = p[0], b = p[1];
+            out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+            out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+        } else {
+            uint4 u = *reinterpret_cast<const uint4*>(static_cast<const char*>(base) + idx * 2);
+            if (dt == DT_BF16) {
+                const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) out[i] = __bfloat162float(e[i]);
+            } else {
+                const __half* e = reinterpret_cast<const __half*>(&u);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) out[i] = __half2float(e[i]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) out[i] = i < nvalid ? ld_elem(base, idx + i, dt) : 0.f;
+    }
+}
+
+__device__ __forceinline__ void store8_dt(void* base, long long idx, int dt, bool vec, int nvalid,
+                                          const float* v) {
+    if (vec) {
+        if (dt == DT_FP32) {
+            float4* p = reinterpret_cast<float4*>(static_cast<float*>(base) + idx);
+            p[0] = make_float4(v[0], v[1], v[2], v[3]);
+            p[1] = make_float4(v[4], v[5], v[6], v[7]);
+        } else {
+            uint4 u;
+            if (dt == DT_BF16) {
+                __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&u);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) e[i] = __float2bfloat16_rn(v[i]);
+            } else {
+                __half* e = reinterpret_cast<__half*>(&u);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) e[i] = __float2half_rn(v[i]);
+            }
+            *reinterpret_cast<uint4*>(static_cast<char*>(base) + idx * 2) = u;
+        }
+    } else {
+        for (int i = 0; i < nvalid; ++i) st_elem(base, idx + i, dt, v[i]);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Bounded waits: every spin in this library gives up after kWaitLimitNs,
+// records MUON_FLAG_TIMEOUT and lets the kernel wind down.
+// ----------------------------------------------------------------------------
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;   // 4 s
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ----------------------------------------------------------------------------
+// mbarrier
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete.  Returns false when
+// the CTA-wide abort flag is raised or the time limit is reached (which
+// raises the flag and reports MUON_FLAG_TIMEOUT).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* d_status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    unsigned long long t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (global_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                if (d_status) atomicOr(d_status, MUON_FLAG_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------
+// TMA (tiled, no multicast): 3-D box load into shared memory, completion
+// counted on an mbarrier.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* smem_dst,
+                                            int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cta.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+          "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// 3-D box store from shared memory (bulk-group completion).  Elements of
+// the box outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until the shared-memory source of every committed store has been read
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until every committed store has completed
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// make this thread's generic-proxy shared-memory writes visible to the async (TMA) proxy
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ----------------------------------------------------------------------------
+// tcgen05 (5th-generation tensor cores, accumulators in tensor memory)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(slot_smem)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 / fp16 in, fp32 accumulate)
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on an mbarrier once all previously issued tcgen05 operations of this thread complete.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+// 32 lanes x 32 columns of 32-bit accumulator: thread t of the warp gets row (lane base + t).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor (sm_100 layout): start address, leading and
+// stride byte offsets (all >> 4), version 1, layout type 2 = 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;   // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;   // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor for kind::f16: fp32 accumulator, A/B type (0 = f16,
+// 1 = bf16), K-major A, B major-ness, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t make_idesc_f16(int ab_bf16, int b_mn_major, int M, int N) {
+    return (1u << 4) | ((uint32_t)ab_bf16 << 7) | ((uint32_t)ab_bf16 << 10) |
+           ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ----------------------------------------------------------------------------
+// Launch descriptors (host builds them, kernels read them as __grid_constant__)
+// ----------------------------------------------------------------------------
+
+// What the epilogue of one GEMM problem does with the accumulator `acc` of
+// output element (i, j) of matrix m:
+//   v = sc(m) * (alpha * acc + beta * Cin[i][j]) + (i == j ? diag : 0)
+// with sc(m) = sc_mul * (sqrt(sumsq[m]) + eps)^(-sc_pow) when sumsq != NULL,
+// else sc_mul.  Then, by `fin`:
+//   FIN_STORE : D[i][j] = v  (symmetric problems store the upper triangle and
+//               mirror it, so D is exactly symmetric)
+//   FIN_OUT   : user output (param orientation, out_dt) = v
+//   FIN_WUPD  : W = W - eta (gamma v + lambda W) on the param (orientation
+//               and pointer from the final table); O_out (fp32) = v if given.
+enum Fin : int { FIN_STORE = 0, FIN_OUT = 1, FIN_WUPD = 2 };
+
+struct FinalEntry {
+    void* W;          // FIN_WUPD: the parameter; FIN_OUT: output matrix
+    float* O_out;     // optional fp32 copy of O (param orientation)
+    float gamma;
+    int transposed;   // 1: param is rows > cols, stored as the transpose of the wide view
+    int vec_ok;       // W (and O_out) 16-byte aligned with cols % 8 == 0: 16-byte accesses allowed
+};
+
+struct Epilogue {
+    const void* Cin; long long ldc, strideC;     // element type = problem type
+    void* D; long long ldd, strideD;
+    float alpha, beta, diag, sc_mul;
+    const double* sumsq; float eps; int sc_pow;
+    const double* check;   // final steps: per-matrix sums of squares whose finiteness gates the output
+    int fin;
+    int fin_base;      // first FinalEntry of this problem (matrix m uses fin_base + m)
+};
+
+constexpr int kMaxProblems = 4;
+constexpr int kMaxFinal = 128;
+
+}  // namespace muon

@@ -1,0 +1,131 @@
+"""The C ABI library loads, exports every entry point include/muon.h declares,
+and its host-side checks behave -- no GPU needed (no compute is launched).
+
+The ctypes structures of the Python binding are checked against the C
+header's layout by compiling a probe with gcc that prints sizeof/offsetof.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import muon_family_optimizer_b200 as mo
+from muon_family_optimizer_b200 import build as mbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "muon.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mbuild.build()
+    return mo.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"MUON_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) >= {"muon_step_batched", "ns_polar", "gram_polar", "muon_workspace_size",
+                          "muon_status_string"}
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", mo.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(names) <= exported
+
+
+def test_library_links_no_cuda_runtime_dynamically(lib):
+    out = subprocess.run(["ldd", mo.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcudart" not in out and "libtorch" not in out
+
+
+PROBE = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "muon.h"
+#define P(T, f) printf(#T "." #f " %zu\n", offsetof(T, f));
+int main(void) {
+  printf("muon_param %zu\n", sizeof(muon_param));
+  printf("muon_schedule %zu\n", sizeof(muon_schedule));
+  printf("muon_hparams %zu\n", sizeof(muon_hparams));
+  printf("muon_ns_coeff %zu\n", sizeof(muon_ns_coeff));
+  P(muon_param, rows) P(muon_param, cols) P(muon_param, W) P(muon_param, G) P(muon_param, G_prev)
+  P(muon_param, A) P(muon_param, M) P(muon_param, gamma) P(muon_param, O_out)
+  P(muon_schedule, n_steps) P(muon_schedule, coeffs) P(muon_schedule, eps)
+  P(muon_schedule, restarts) P(muon_schedule, n_restarts) P(muon_schedule, scale_f)
+  P(muon_hparams, mu) P(muon_hparams, eta) P(muon_hparams, lambda) P(muon_hparams, gamma)
+  P(muon_hparams, beta_a) P(muon_hparams, alpha)
+  return 0;
+}
+"""
+
+
+def test_binding_struct_layout_matches_header(tmp_path):
+    src = tmp_path / "probe.c"
+    src.write_text(PROBE)
+    exe = tmp_path / "probe"
+    subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    got = dict(line.rsplit(" ", 1) for line in subprocess.check_output([str(exe)], text=True).splitlines())
+    assert int(got["muon_param"]) == ctypes.sizeof(mo.Param)
+    assert int(got["muon_schedule"]) == ctypes.sizeof(mo.Schedule)
+    assert int(got["muon_hparams"]) == ctypes.sizeof(mo.HParams)
+    assert int(got["muon_ns_coeff"]) == ctypes.sizeof(mo.NsCoeff)
+    py = {"muon_param": mo.Param, "muon_schedule": mo.Schedule, "muon_hparams": mo.HParams}
+    for key, val in got.items():
+        if "." not in key:
+            continue
+        struct, field = key.split(".")
+        field = "lambda_" if field == "lambda" else field
+        assert getattr(py[struct], field).offset == int(val), key
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = mo.muon_status_string(code)
+        assert s and s != "unknown status"
+    assert mo.muon_status_string(99) == "unknown status"
+
+
+def test_workspace_size_queries_are_host_only(lib):
+    arr = (mo.Param * 3)()
+    for i, (r, c) in enumerate([(768, 768), (768, 3072), (3072, 768)]):
+        arr[i].rows, arr[i].cols = r, c
+    n16 = mo.muon_workspace_size(arr, mo.BF16)
+    n32 = mo.muon_workspace_size(arr, mo.FP32)
+    assert n16 > 0 and n32 > n16
+    # the two 768x3072 orientations share a group: 2 X buffers of 2 x 768 x 3072,
+    # 2 square buffers of 2 x 768 x 768, plus 768x768 group -- in bf16
+    lower = 2 * (2 * 768 * 3072 * 2) + 2 * (2 * 768 * 768 * 2) + 4 * (768 * 768 * 2)
+    assert lower <= n16 <= lower + 64 * 1024
+    assert mo.ns_polar_workspace_size(4, 100, 300, mo.BF16) < mo.gram_polar_workspace_size(4, 100, 300, mo.BF16)
+
+
+def test_invalid_arguments_are_rejected_before_any_launch(lib):
+    L = lib
+    sched = mo.quintic_schedule(5)
+    bad = mo.make_schedule([(1, 0, 0)], restarts=[5])        # restart beyond n_steps
+    sz = ctypes.c_size_t(0)
+    assert L.ns_polar_workspace_size(0, 4, 4, mo.BF16, ctypes.byref(sz)) == mo.ERR_INVALID_ARG
+    assert L.ns_polar_workspace_size(1, 4, 4, 7, ctypes.byref(sz)) == mo.ERR_INVALID_ARG
+    assert L.ns_polar(None, None, 1, 4, 4, 16, mo.BF16, ctypes.byref(sched), None, 0, None, None) == \
+        mo.ERR_INVALID_ARG
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    assert L.ns_polar(p, p, 1, 4, 4, 16, mo.BF16, ctypes.byref(bad), p, 64, None, None) == mo.ERR_INVALID_ARG
+    # workspace too small is reported as such (still before any device call)
+    assert L.ns_polar(p, p, 1, 4, 4, 16, mo.BF16, ctypes.byref(sched), p, 1, None, None) == mo.ERR_WORKSPACE
+    nan_sched = mo.make_schedule([(float("nan"), 0, 0)])
+    assert L.gram_polar(p, p, 1, 4, 4, 16, mo.BF16, ctypes.byref(nan_sched), p, 1 << 20, None, None) == \
+        mo.ERR_INVALID_ARG
+    arr = (mo.Param * 1)()
+    arr[0].rows, arr[0].cols = 4, 4
+    hp = mo.HParams(0.9, 0.02, 0.0, 1.0, 0.9, 0.5)
+    # W/G/... NULL
+    assert L.muon_step_batched(arr, 1, mo.BF16, mo.BF16, ctypes.byref(hp), ctypes.byref(sched), p, 1 << 20,
+                               None, None) == mo.ERR_INVALID_ARG
