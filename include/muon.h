@@ -183,6 +183,33 @@ MUON_API muon_status gram_polar(const void* X_in, void* X_out, int batch, int ro
                        void* workspace, size_t ws_bytes, int* d_status, muon_stream_t stream);
 
 /*
+ * ns_polar without a workspace argument, for callers that cannot allocate
+ * device memory when they need the orthogonalisation: code running during CUDA
+ * graph capture, runtimes whose allocators forbid outside allocations, and
+ * plugins that only receive pointers to existing buffers.  The pages describe
+ * no such entry point; it exists for this library's users.
+ *
+ * It runs exactly the ns_polar iteration with a fixed scratch array compiled
+ * into the library: ns_polar_noalloc_capacity() bytes (32 MiB) of device
+ * memory that every GPU loading the library keeps until the process exits.
+ * A request whose ns_polar_workspace_size exceeds that capacity returns
+ * MUON_ERR_WORKSPACE without launching anything.  Nothing is allocated: no
+ * cudaMalloc, cudaFree or allocating library routine is called.
+ *   - The first call on each device looks up the scratch array's device
+ *     address (cudaGetSymbolAddress, with that device current); make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the scratch, which keeps the previous
+ *     call's contents (each call clears what must start at zero).  Calls that
+ *     overlap on the GPU (unordered streams) race: order them.
+ * Arguments and results are those of ns_polar.
+ */
+MUON_API muon_status ns_polar_noalloc(const void* X_in, void* X_out, int batch, int rows, int cols,
+                                      long long batch_stride, muon_dtype dtype,
+                                      const muon_schedule* sched, int* d_status, muon_stream_t stream);
+/* Bytes of the fixed scratch behind ns_polar_noalloc. */
+MUON_API size_t ns_polar_noalloc_capacity(void);
+
+/*
  * Tracing aid (optional).  While enabled, every kernel the library launches
  * is bracketed by two CUDA events recorded on the launch stream, and the
  * launch's algorithmic work is noted: floating-point operations for the

@@ -94,6 +94,11 @@ def lib():
             f.restype = st
             f.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
                           ctypes.c_int, ctypes.POINTER(Schedule), vp, ctypes.c_size_t, vp, vp]
+        L.ns_polar_noalloc.restype = st
+        L.ns_polar_noalloc.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
+                                       ctypes.c_int, ctypes.POINTER(Schedule), vp, vp]
+        L.ns_polar_noalloc_capacity.restype = ctypes.c_size_t
+        L.ns_polar_noalloc_capacity.argtypes = []
         L.muon_trace_enable.restype = st
         L.muon_trace_enable.argtypes = [ctypes.c_int]
         L.muon_trace_read.restype = ctypes.c_int
@@ -205,6 +210,26 @@ def _polar(fn, X_in, X_out, schedule, workspace, d_status, stream):
     _check(fn(_ptr(X_in), _ptr(X_out), batch, rows, cols, rows * cols, _dtype_code(X_in.dtype),
               ctypes.byref(schedule), _ptr(workspace), workspace.numel(), _ptr(d_status),
               _stream_ptr(stream)), fn.__name__)
+
+
+def ns_polar_noalloc(X_in, X_out, schedule, d_status=None, stream=None):
+    """ns_polar on the library's fixed device scratch, for callers that cannot
+    allocate a workspace (e.g. during CUDA graph capture).  The first call on a
+    device should come before any capture; calls on one device must not overlap."""
+    if X_in.dim() == 2:
+        batch, (rows, cols) = 1, X_in.shape
+    else:
+        batch, rows, cols = X_in.shape
+    if not X_in.is_contiguous() or not X_out.is_contiguous() or X_out.shape != X_in.shape \
+            or X_out.dtype != X_in.dtype:
+        raise ValueError("X_in / X_out must be contiguous tensors of the same shape and dtype")
+    _check(lib().ns_polar_noalloc(_ptr(X_in), _ptr(X_out), batch, rows, cols, rows * cols,
+                                  _dtype_code(X_in.dtype), ctypes.byref(schedule), _ptr(d_status),
+                                  _stream_ptr(stream)), "ns_polar_noalloc")
+
+
+def ns_polar_noalloc_capacity():
+    return lib().ns_polar_noalloc_capacity()
 
 
 def ns_polar(X_in, X_out, schedule, workspace, d_status=None, stream=None):
