@@ -15,6 +15,9 @@ struct GemmOp {
     // the diagonal (128 x 128) are valid (tensor-core path): blocks left of the
     // diagonal tile are read transposed from the stored upper tile.
     int a_sym, b_sym;
+    // Symmetric result that an update product will read on CTA pairs: also
+    // store the first tile below the diagonal (exact mirror of the one above).
+    int band;
     int count, M, N, K;
     const void* A; long long lda, strideA;
     const void* B; long long ldb, strideB;

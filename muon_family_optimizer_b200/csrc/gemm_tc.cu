@@ -31,6 +31,9 @@
 // the main loop of tile t+1.
 #include <cudaTypedefs.h>
 
+#include <stdlib.h>
+#include <string.h>
+
 #include <mutex>
 
 #include "epilogue.cuh"
@@ -45,11 +48,13 @@ constexpr int kEpiWarps = 8;    // two per tensor-memory lane quadrant, each tak
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 
-template <int BN>
+// Per-CTA configuration.  PAIR: two CTAs share each MMA (cta_group::2): the
+// pair computes a 256 x BN tile, each CTA loads its 128 rows of A and BN/2 of B.
+template <int BN, bool PAIR>
 struct Cfg {
-    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kStages = (PAIR || BN == 128) ? 6 : 4;
     static constexpr int kABytes = BM * BK * 2;
-    static constexpr int kBBytes = BN * BK * 2;
+    static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * BK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kTmemCols = 2 * BN;
     static constexpr int kStgBytes = 32 * 64 * 2;              // one 32 x 64 16-bit box per epilogue warp
@@ -58,6 +63,7 @@ struct Cfg {
     static constexpr int kBarOffset = kStgOffset + kEpiWarps * kFinBytes;   // kFinBytes > kStgBytes
     static constexpr int kBarBytes = 256;
     static constexpr int kSmemBytes = 1024 + kBarOffset + kBarBytes;
+    static constexpr int kRows = PAIR ? 2 * BM : BM;           // output rows per tile
 };
 
 struct TcProblem {
@@ -66,8 +72,9 @@ struct TcProblem {
     CUtensorMap mapB;    // SYM: B rows, boxes 64 (K) x 128 (N); UPD: X panel, boxes 64 (N) x 64 (K)
     CUtensorMap mapBt;   // B symmetric: transposed reads, boxes 64 (N) x 64 (K)
     CUtensorMap mapD;    // output stores, boxes 64 (N) x 32 (M)
+    CUtensorMap mapDt;   // band: transposed stores, boxes 32 (M) x 64 (N), no swizzle
     int count, M, N, K;
-    int tiles_m, tiles_n, tiles_per_mat, sym, a_sym, b_sym;
+    int tiles_m, tiles_n, tiles_per_mat, sym, a_sym, b_sym, band;
     long long tile_begin;
     Epilogue epi;
 };
@@ -141,10 +148,25 @@ __device__ __forceinline__ void final_block(const Epilogue& E, const FinalCtx& f
     // parameter extent: tr ? (N rows x M cols) : (M rows x N cols)
     const int prow_n = tr ? N : M, pcol_n = tr ? M : N;
     const int prow0 = tr ? gj0 : gi0, pcol0 = tr ? gi0 : gj0;
+    const int cc = (lane & 3) * 8;                // first of 8 parameter columns inside the block
+    // pass 1: issue every load of W first (four independent 16/32-byte loads per lane)
+    float w[4][8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int prow = prow0 + 8 * k + (lane >> 2), pcol = pcol0 + cc;
+        if (!wupd || prow >= prow_n || pcol >= pcol_n) continue;
+        const TW* wp = W + (size_t)prow * pcol_n + pcol;
+        if (vec && pcol + 8 <= pcol_n) {
+            load8_dt(wp, 0, kDt, true, 8, w[k]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[k][e] = pcol + e < pcol_n ? to_float(wp[e]) : 0.f;
+        }
+    }
+    // pass 2: combine with the staged result and store
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int rr = 8 * k + (lane >> 2);       // parameter row inside the block
-        const int cc = (lane & 3) * 8;            // first of 8 parameter columns inside the block
         const int prow = prow0 + rr, pcol = pcol0 + cc;
         if (prow >= prow_n || pcol >= pcol_n) continue;
         float o[8];
@@ -153,21 +175,14 @@ __device__ __forceinline__ void final_block(const Epilogue& E, const FinalCtx& f
         TW* wp = W + (size_t)prow * pcol_n + pcol;
         const bool full = vec && pcol + 8 <= pcol_n;
         if (wupd) {
-            float w[8];
-            if (full) {
-                load8_dt(wp, 0, kDt, true, 8, w);
-            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) w[e] = pcol + e < pcol_n ? to_float(wp[e]) : 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = w[e] - fc.eta * (g * o[e] + fc.lambda * w[e]);
+            for (int e = 0; e < 8; ++e) w[k][e] = w[k][e] - fc.eta * (g * o[e] + fc.lambda * w[k][e]);
             if (full) {
-                store8_dt(wp, 0, kDt, true, 8, w);
+                store8_dt(wp, 0, kDt, true, 8, w[k]);
                 if (O_out) store8_dt(O_out + (size_t)prow * pcol_n + pcol, 0, DT_FP32, true, 8, o);
             } else {
                 for (int e = 0; e < 8 && pcol + e < pcol_n; ++e) {
-                    wp[e] = from_float<TW>(w[e]);
+                    wp[e] = from_float<TW>(w[k][e]);
                     if (O_out) O_out[(size_t)prow * pcol_n + pcol + e] = o[e];
                 }
             }
@@ -179,18 +194,22 @@ __device__ __forceinline__ void final_block(const Epilogue& E, const FinalCtx& f
     }
 }
 
-// Stage the warp's 32 x 32 block (this lane: wide row gi0 + lane) and write it out.
-__device__ __forceinline__ void final_chunk_dispatch(const Epilogue& E, const FinalCtx& fc, int m, int M,
-                                                     int N, int gi0, int gj0, const float (&v)[32],
-                                                     float* fs, int lane) {
-    __syncwarp();                       // the previous block's reads of fs are done
-#pragma unroll
-    for (int q = 0; q < 32; ++q) fs[lane * 33 + q] = v[q];
-    __syncwarp();
+// Write out the warp's staged 32 x 32 block (kept out of line: only the
+// final step takes this path, and inlining it would crowd the hot loop).
+__device__ __noinline__ void final_write(const Epilogue& E, const FinalCtx& fc, int m, int M, int N,
+                                         int gi0, int gj0, const float* fs, int lane) {
     const int dt = E.fin == FIN_OUT ? fc.out_dt : fc.w_dt;
     if (dt == DT_BF16) final_block<__nv_bfloat16>(E, fc, m, M, N, gi0, gj0, fs, lane);
     else if (dt == DT_FP16) final_block<__half>(E, fc, m, M, N, gi0, gj0, fs, lane);
     else final_block<float>(E, fc, m, M, N, gi0, gj0, fs, lane);
+}
+
+// Stage 32 values of this lane's row into the warp's padded final box.
+__device__ __forceinline__ void final_stage(float* fs, int lane, const float (&v)[32]) {
+    __syncwarp();                       // the previous block's reads of fs are done
+#pragma unroll
+    for (int q = 0; q < 32; ++q) fs[lane * 33 + q] = v[q];
+    __syncwarp();
 }
 
 // Combine one 32-column chunk of the accumulator (row gi, columns
@@ -200,15 +219,26 @@ template <typename T>
 __device__ __forceinline__ void epi_combine(const Epilogue& E, int gi, int gj0, float sc, float (&v)[32],
                                             const uint4 (&c)[4]) {
     if (E.beta != 0.f) {
-        const T* ce = reinterpret_cast<const T*>(c);
+        const float a = sc * E.alpha, b = sc * E.beta;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = sc * (E.alpha * v[q] + E.beta * to_float(ce[q]));
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t w[4] = {c[q].x, c[q].y, c[q].z, c[q].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                v[8 * q + 2 * h] = a * v[8 * q + 2 * h] + b * unpack_lo<T>(w[h]);
+                v[8 * q + 2 * h + 1] = a * v[8 * q + 2 * h + 1] + b * unpack_hi<T>(w[h]);
+            }
+        }
     } else {
         const float s = sc * E.alpha;
 #pragma unroll
         for (int q = 0; q < 32; ++q) v[q] *= s;
     }
-    if (E.diag != 0.f && gi >= gj0 && gi < gj0 + 32) v[gi - gj0] += E.diag;
+    if (E.diag != 0.f) {   // static indices only: keeps v in registers
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+            if (gi == gj0 + q) v[q] += E.diag;
+    }
 }
 
 // Write 32 values (row `r` of the warp's 32 x 64 staging box, 16-byte chunks
@@ -219,11 +249,23 @@ __device__ __forceinline__ void stage32(uint8_t* stg, int r, int c16, const floa
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         uint4 u;
-        T* e = reinterpret_cast<T*>(&u);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) e[i] = from_float<T>(v[8 * q + i]);
+        u.x = pack2<T>(v[8 * q + 0], v[8 * q + 1]);
+        u.y = pack2<T>(v[8 * q + 2], v[8 * q + 3]);
+        u.z = pack2<T>(v[8 * q + 4], v[8 * q + 5]);
+        u.w = pack2<T>(v[8 * q + 6], v[8 * q + 7]);
         *reinterpret_cast<uint4*>(stg + r * 128 + (((c16 + q) ^ (r & 7)) * 16)) = u;
     }
+}
+
+// Transpose of 32 columns (c0..c0+31) of the warp's 32 x 64 block into the
+// staging box taken as a dense 64 x 32 box (row c = block column c, 64 bytes
+// per row, no swizzle): lane r writes column r, so the warp's 32 lanes fill
+// one 64-byte row per element.
+template <typename T>
+__device__ __forceinline__ void stage_transposed(uint8_t* stg, int lane, int c0, const float (&v)[32]) {
+    T* box = reinterpret_cast<T*>(stg);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) box[(c0 + c) * 32 + lane] = from_float<T>(v[c]);
 }
 
 // Barrier over the epilogue warps only (named barrier 1).
@@ -255,9 +297,10 @@ __device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int half,
     }
 }
 
-template <int BN, bool B_MN, typename T>
+template <int BN, bool B_MN, bool PAIR, typename T>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
-    using C = Cfg<BN>;
+    static_assert(!PAIR || (B_MN && BN == 256), "CTA pairs are used for the update product only");
+    using C = Cfg<BN, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
@@ -271,6 +314,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     int* d_status = p.fc.d_status;
+    // CTA pairs: rank 0 (leader) issues the MMAs for both CTAs of the cluster
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const long long unit = PAIR ? (blockIdx.x >> 1) : blockIdx.x;
+    const long long nunits = PAIR ? (gridDim.x >> 1) : gridDim.x;
+    constexpr uint32_t kTemptyCount = kEpiWarps * (PAIR ? 2 : 1);   // one arrival per epilogue warp
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -279,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull_bar[b], 1);
-            mbar_init(&tempty_bar[b], kEpiThreads);
+            mbar_init(&tempty_bar[b], kTemptyCount);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -292,11 +340,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         }
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, C::kTmemCols);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(tmem_slot, C::kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, C::kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    if (PAIR) cluster_sync(); else __syncthreads();   // barriers of both CTAs initialised
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -307,38 +361,56 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             uint32_t phase = 0;
             uint32_t armed = 0;          // bit s: stage s has been armed at least once
             uint32_t armed_parity = 0;   // bit s: parity of the phase stage s was last armed in
-            for (long long t = blockIdx.x; t < p.total_tiles && !*abort_flag; t += gridDim.x) {
+            for (long long t = unit; t < p.total_tiles && !*abort_flag; t += nunits) {
                 int pi, m, ti, tj;
                 decode_tile(p, t, pi, m, ti, tj);
                 const TcProblem& P = p.prob[pi];
                 const int nkb = (P.K + BK - 1) / BK;
-                int nchunk = BN / 64;
-                if (B_MN) {
-                    const int rem = P.N - tj * BN;
-                    nchunk = min(BN / 64, (rem + 63) / 64);
-                }
-                const uint32_t bytes = C::kABytes + (B_MN ? nchunk * 64 * BK * 2 : C::kBBytes);
+                const int rows0 = ti * C::kRows + (int)rank * BM;   // this CTA's rows of A
+                // this CTA's columns of B (MN-major panel) and the 64-wide boxes they span
+                constexpr int kBCols = PAIR ? BN / 2 : BN;
+                const int bcol0 = tj * BN + (int)rank * kBCols;
+                auto chunks = [&](int c0) { return max(0, min(kBCols / 64, (P.N - c0 + 63) / 64)); };
+                const int nchunk = B_MN ? chunks(bcol0) : kBCols / 64;
+                uint32_t bytes = C::kABytes + (B_MN ? nchunk * 64 * BK * 2 : C::kBBytes);
+                if (PAIR) bytes = 2 * C::kABytes + (chunks(tj * BN) + chunks(tj * BN + kBCols)) * 64 * BK * 2;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, d_status)) break;
                     uint8_t* sa = smem + stage * C::kStageBytes;
                     uint8_t* sb = sa + C::kABytes;
-                    mbar_arrive_expect_tx(&full_bar[stage], bytes);
-                    if (P.a_sym && (kb >> 1) < ti) {
-                        // rows ti*128.. of a symmetric A, k-block left of the diagonal
-                        // tile: read the stored block above the diagonal, transposed
-                        tma_load_3d(&P.mapAt, &full_bar[stage], sa, ti * BM, kb * BK, m);
-                        tma_load_3d(&P.mapAt, &full_bar[stage], sa + 64 * BK * 2, ti * BM + 64, kb * BK, m);
-                    } else {
-                        tma_load_3d(&P.mapA, &full_bar[stage], sa, kb * BK, ti * BM, m);
-                    }
-                    if (B_MN) {
+                    // A block left of the diagonal of a symmetric A: read the stored
+                    // block above the diagonal transposed.  For a pair the decision is
+                    // taken on the pair's first 128-row block, so both halves agree
+                    // (the first sub-diagonal tile is stored for such operands).
+                    const bool at = P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti);
+                    if (PAIR) {
+                        const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+                        if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                        if (at) {
+                            tma_load_3d_pair(&P.mapAt, fb, sa, rows0, kb * BK, m);
+                            tma_load_3d_pair(&P.mapAt, fb, sa + 64 * BK * 2, rows0 + 64, kb * BK, m);
+                        } else {
+                            tma_load_3d_pair(&P.mapA, fb, sa, kb * BK, rows0, m);
+                        }
                         for (int c = 0; c < nchunk; ++c)
-                            tma_load_3d(&P.mapB, &full_bar[stage], sb + c * (64 * BK * 2), tj * BN + c * 64, kb * BK, m);
-                    } else if (P.b_sym && (kb >> 1) < tj) {
-                        for (int c = 0; c < BN / 64; ++c)
-                            tma_load_3d(&P.mapBt, &full_bar[stage], sb + c * (64 * BK * 2), tj * BN + c * 64, kb * BK, m);
+                            tma_load_3d_pair(&P.mapB, fb, sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK, m);
                     } else {
-                        tma_load_3d(&P.mapB, &full_bar[stage], sb, kb * BK, tj * BN, m);
+                        mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                        if (at) {
+                            tma_load_3d(&P.mapAt, &full_bar[stage], sa, rows0, kb * BK, m);
+                            tma_load_3d(&P.mapAt, &full_bar[stage], sa + 64 * BK * 2, rows0 + 64, kb * BK, m);
+                        } else {
+                            tma_load_3d(&P.mapA, &full_bar[stage], sa, kb * BK, rows0, m);
+                        }
+                        if (B_MN) {
+                            for (int c = 0; c < nchunk; ++c)
+                                tma_load_3d(&P.mapB, &full_bar[stage], sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK, m);
+                        } else if (P.b_sym && (kb >> 1) < tj) {
+                            for (int c = 0; c < BN / 64; ++c)
+                                tma_load_3d(&P.mapBt, &full_bar[stage], sb + c * (64 * BK * 2), tj * BN + c * 64, kb * BK, m);
+                        } else {
+                            tma_load_3d(&P.mapB, &full_bar[stage], sb, kb * BK, tj * BN, m);
+                        }
                     }
                     armed |= 1u << stage;
                     armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -346,25 +418,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 }
             }
             if (*abort_flag) {
-                // wind down: every armed stage's copies must land before the CTA exits
+                // wind down: every copy this CTA started must land before it exits
                 const unsigned long long t0 = global_ns();
-                for (int s = 0; s < C::kStages; ++s) {
-                    if (!(armed >> s & 1u)) continue;
-                    const uint32_t par = armed_parity >> s & 1u;
-                    while (!mbar_try_wait(&full_bar[s], par) && global_ns() - t0 < kWaitLimitNs) {
+                if (!PAIR || rank == 0) {
+                    for (int s = 0; s < C::kStages; ++s) {
+                        if (!(armed >> s & 1u)) continue;
+                        const uint32_t par = armed_parity >> s & 1u;
+                        while (!mbar_try_wait(&full_bar[s], par) && global_ns() - t0 < kWaitLimitNs) {
+                        }
+                    }
+                } else {
+                    // the second CTA of a pair counts its copies on the leader's
+                    // barriers: give them a fixed time to land
+                    while (global_ns() - t0 < 200000ull) {
                     }
                 }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc0 = make_idesc_f16(IsBf16<T>::value ? 1 : 0, 0, BM, BN);
+            constexpr uint32_t idesc0 = make_idesc_f16(IsBf16<T>::value ? 1 : 0, 0, C::kRows, BN);
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
             bool ok = true;
-            for (long long t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x, ++it) {
+            for (long long t = unit; ok && t < p.total_tiles; t += nunits, ++it) {
                 int pi, m, ti, tj;
                 decode_tile(p, t, pi, m, ti, tj);
                 const TcProblem& P = p.prob[pi];
@@ -377,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, abort_flag, d_status)) { ok = false; break; }
                     tc_fence_after();
-                    const bool at = P.a_sym && (kb >> 1) < ti;                 // A block read transposed
-                    const bool bm = B_MN || (P.b_sym && (kb >> 1) < tj);       // B block MN-major
+                    const bool at = P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti);   // A block read transposed
+                    const bool bm = B_MN || (P.b_sym && (kb >> 1) < tj);          // B block MN-major
                     const uint32_t idesc = idesc0 | (at ? 1u << 15 : 0u) | (bm ? 1u << 16 : 0u);
                     const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t sb = sa + C::kABytes;
@@ -391,16 +470,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                                : smem_desc_sw128(sa + k * 32, 16, 1024);
                         const uint64_t bd = bm ? smem_desc_sw128(sb + k * 2048, 64 * BK * 2, 1024)
                                                : smem_desc_sw128(sb + k * 32, 16, 1024);
-                        tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+                        if (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+                        else tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
                     }
-                    tc_commit(&empty_bar[stage]);
+                    if (PAIR) {   // release the stage in both CTAs
+                        tc_commit_pair(smem_u32(&empty_bar[stage]));
+                        tc_commit_pair(mapa_shared(smem_u32(&empty_bar[stage]), 1));
+                    } else {
+                        tc_commit(&empty_bar[stage]);
+                    }
                     if (++stage == C::kStages) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                tc_commit(&tfull_bar[buf]);
+                if (PAIR) {       // accumulators ready in both CTAs
+                    tc_commit_pair(smem_u32(&tfull_bar[buf]));
+                    tc_commit_pair(mapa_shared(smem_u32(&tfull_bar[buf]), 1));
+                } else {
+                    tc_commit(&tfull_bar[buf]);
+                }
             }
             // make sure no MMA is still writing tensor memory before it is freed
-            tc_commit(drain_bar);
+            if (PAIR) tc_commit_pair(smem_u32(drain_bar)); else tc_commit(drain_bar);
             const unsigned long long t0 = global_ns();
             while (!mbar_try_wait(drain_bar, 0) && global_ns() - t0 < kWaitLimitNs) {
             }
@@ -423,14 +513,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         FinalCtx fc = p.fc;
         fc.fin = p.fin;
         int it = 0;
-        for (long long t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
+        for (long long t = unit; t < p.total_tiles; t += nunits, ++it) {
             int pi, m, ti, tj;
             decode_tile(p, t, pi, m, ti, tj);
             const TcProblem& P = p.prob[pi];
             const Epilogue& E = P.epi;
             const int buf = it & 1;
             const uint32_t tphase = (it >> 1) & 1;
-            const int gi = ti * BM + row;
+            const int row0 = ti * C::kRows + (int)rank * BM;   // first output row of this CTA
+            const int gi = row0 + row;
             const int col0 = tj * BN + half * (BN / 2);
             const bool has_cin = E.beta != 0.f;
             const bool diag_sym = P.sym && ti == tj && E.fin == FIN_STORE;   // uniform over the CTA
@@ -449,62 +540,92 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             bool skip = false;
             if (!dead && E.fin != FIN_STORE && !epi_finite(E, m, sc)) {
                 skip = E.fin == FIN_WUPD;   // keep W; a FIN_OUT result carries the NaN
-                if (row == 0 && half == 0 && tj == 0 && ti == 0 && d_status)
+                if (row == 0 && half == 0 && tj == 0 && ti == 0 && rank == 0 && d_status)
                     atomicOr(d_status, MUON_FLAG_NONFINITE);
             }
 #pragma unroll 1
             for (int pr = 0; pr < kPairs; ++pr) {
                 const int gj0 = col0 + pr * 64;
                 const bool work = !dead && gj0 < P.N;       // warp-uniform
-                float v0[32], v1[32];
-                if (work) {
-                    if (has_cin && pr > 0) {
-                        cin_fetch<T>(E, m, gi, gj0, P.M, P.N, c0);
-                        cin_fetch<T>(E, m, gi, gj0 + 32, P.M, P.N, c1);
-                    }
-                    const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) +
-                                          (uint32_t)(buf * BN + half * (BN / 2) + pr * 64);
-                    tmem_ld_32x32b_x32(tcol, v0);
-                    tmem_ld_32x32b_x32(tcol + 32, v1);
-                    if (!skip) {
-                        epi_combine<T>(E, gi, gj0, sc, v0, c0);
-                        epi_combine<T>(E, gi, gj0 + 32, sc, v1, c1);
-                    }
+                const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                      (uint32_t)(buf * BN + half * (BN / 2) + pr * 64);
+                if (work && has_cin && pr > 0) {
+                    cin_fetch<T>(E, m, gi, gj0, P.M, P.N, c0);
+                    cin_fetch<T>(E, m, gi, gj0 + 32, P.M, P.N, c1);
                 }
                 if (E.fin == FIN_STORE) {
-                    // 32 rows x 64 columns -> staging box -> one bulk tensor store
+                    // 32 rows x 64 columns -> staging box -> one bulk tensor store;
+                    // one 32-column chunk in registers at a time
                     if (work) {
                         if (stg_busy) {
                             if (lane == 0) bulk_wait_read0();
                             __syncwarp();
                         }
-                        stage32<T>(stg, lane, 0, v0);
-                        stage32<T>(stg, lane, 4, v1);
+                        float v[32];
+                        tmem_ld_32x32b_x32(tcol, v);
+                        epi_combine<T>(E, gi, gj0, sc, v, c0);
+                        stage32<T>(stg, lane, 0, v);
+                        tmem_ld_32x32b_x32(tcol + 32, v);
+                        epi_combine<T>(E, gi, gj0 + 32, sc, v, c1);
+                        stage32<T>(stg, lane, 4, v);
                     }
                     if (diag_sym) {          // BN == 128 here: the eight boxes cover the tile
                         epi_bar();
                         if (work) fix_lower<T>(stg_base, quad, half, lane);
                         epi_bar();
                     }
-                    if (work && ti * BM + quad * 32 < P.M) {
+                    if (work && row0 + quad * 32 < P.M) {
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_3d(&P.mapD, stg, gj0, ti * BM + quad * 32, m);
+                            tma_store_3d(&P.mapD, stg, gj0, row0 + quad * 32, m);
                             bulk_commit();
                         }
                         stg_busy = true;
+                        if (P.band && tj == ti + 1) {
+                            // first tile right of the diagonal: also store its transpose
+                            // (the tile below the diagonal), exactly mirrored; the values
+                            // are formed again from the accumulator, still in TMEM
+                            if (lane == 0) bulk_wait_read0();
+                            __syncwarp();
+                            float v[32];
+                            tmem_ld_32x32b_x32(tcol, v);
+                            epi_combine<T>(E, gi, gj0, sc, v, c0);
+                            stage_transposed<T>(stg, lane, 0, v);
+                            tmem_ld_32x32b_x32(tcol + 32, v);
+                            epi_combine<T>(E, gi, gj0 + 32, sc, v, c1);
+                            stage_transposed<T>(stg, lane, 32, v);
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_3d(&P.mapDt, stg, row0 + quad * 32, gj0, m);
+                                bulk_commit();
+                            }
+                        }
                     }
-                } else if (work && !skip && ti * BM + quad * 32 < P.M) {
+                } else if (work && !skip && row0 + quad * 32 < P.M) {
                     float* fs = reinterpret_cast<float*>(stg_base + (quad + 4 * half) * C::kFinBytes);
-                    const int gi0 = ti * BM + quad * 32;
-                    final_chunk_dispatch(E, fc, m, P.M, P.N, gi0, gj0, v0, fs, lane);
-                    if (gj0 + 32 < P.N) final_chunk_dispatch(E, fc, m, P.M, P.N, gi0, gj0 + 32, v1, fs, lane);
+                    const int gi0 = row0 + quad * 32;
+                    float v[32];
+                    tmem_ld_32x32b_x32(tcol, v);
+                    epi_combine<T>(E, gi, gj0, sc, v, c0);
+                    final_stage(fs, lane, v);
+                    final_write(E, fc, m, P.M, P.N, gi0, gj0, fs, lane);
+                    if (gj0 + 32 < P.N) {
+                        tmem_ld_32x32b_x32(tcol + 32, v);
+                        epi_combine<T>(E, gi, gj0 + 32, sc, v, c1);
+                        final_stage(fs, lane, v);
+                        final_write(E, fc, m, P.M, P.N, gi0, gj0 + 32, fs, lane);
+                    }
                 }
             }
             if (!dead) {
                 tc_fence_before();
-                mbar_arrive(&tempty_bar[buf]);
+                __syncwarp();
+                if (lane == 0) {
+                    if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+                    else mbar_arrive(&tempty_bar[buf]);
+                }
             }
         }
         if (lane == 0) bulk_wait0();   // stores complete before the CTA's shared memory goes away
@@ -512,10 +633,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     }
 
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    if (PAIR) cluster_sync(); else __syncthreads();   // neither CTA of a pair leaves while the other works
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+        if (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+        else tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 
@@ -539,7 +662,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 // 3-D map over `count` matrices of `rows` x `inner` 16-bit elements with row
 // stride `ld` and matrix stride `mstride` (elements); box = box_inner x box_rows x 1.
 static bool encode_map(CUtensorMap* map, int dt, const void* base, long long inner, long long rows,
-                       long long count, long long ld, long long mstride, int box_inner, int box_rows) {
+                       long long count, long long ld, long long mstride, int box_inner, int box_rows,
+                       bool swizzle = true) {
     auto enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)count};
@@ -548,15 +672,16 @@ static bool encode_map(CUtensorMap* map, int dt, const void* base, long long inn
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, dt == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool B_MN, typename T>
+template <int BN, bool B_MN, bool PAIR, typename T>
 static cudaError_t launch_one(const TcParams& prm, int grid, cudaStream_t stream) {
-    using C = Cfg<BN>;
-    auto kern = tc_gemm_kernel<BN, B_MN, T>;
+    using C = Cfg<BN, PAIR>;
+    auto kern = tc_gemm_kernel<BN, B_MN, PAIR, T>;
     static thread_local int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -565,7 +690,22 @@ static cudaError_t launch_one(const TcParams& prm, int grid, cudaStream_t stream
         if (e != cudaSuccess) return e;
         configured_dev = dev;
     }
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(prm);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -575,6 +715,14 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
     if (nops > kMaxProblems || nfin > kMaxFinal) return MUON_ERR_UNSUPPORTED;
     const int sym = ops[0].sym;
     const int BN = sym ? 128 : 256;
+    // update products run on CTA pairs (cta_group::2, 256 x 256 tiles) unless
+    // MUON_UPDATE_KERNEL=single selects one CTA per 128 x 256 tile
+    static const bool pair_ok = [] {
+        const char* v = getenv("MUON_UPDATE_KERNEL");
+        return !(v && strcmp(v, "single") == 0);
+    }();
+    const bool pair = !sym && pair_ok;
+    const int rows_per_tile = pair ? 2 * BM : BM;
     // the final-step staging boxes overlap the store boxes: one kind per launch
     for (int i = 1; i < nops; ++i)
         if ((ops[i].epi.fin == FIN_STORE) != (ops[0].epi.fin == FIN_STORE)) return MUON_ERR_INVALID_ARG;
@@ -589,7 +737,7 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         if (o.sym != sym) return MUON_ERR_INVALID_ARG;
         TcProblem& P = prm.prob[i];
         P.count = o.count; P.M = o.M; P.N = o.N; P.K = o.K; P.sym = sym;
-        P.tiles_m = (o.M + BM - 1) / BM;
+        P.tiles_m = (o.M + rows_per_tile - 1) / rows_per_tile;
         P.tiles_n = (o.N + BN - 1) / BN;
         P.tiles_per_mat = sym ? P.tiles_m * (P.tiles_m + 1) / 2 : P.tiles_m * P.tiles_n;
         P.tile_begin = tiles;
@@ -597,6 +745,7 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         P.epi = o.epi;
         P.a_sym = o.a_sym;
         P.b_sym = sym ? o.b_sym : 0;
+        P.band = sym ? o.band : 0;
         // A operand: M rows x K (K contiguous); a symmetric A is also read transposed
         if (!encode_map(&P.mapA, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, BK, BM)) return MUON_ERR_CUDA;
         if (o.a_sym && !encode_map(&P.mapAt, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, 64, BK))
@@ -612,6 +761,10 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         if (o.epi.fin == FIN_STORE &&
             !encode_map(&P.mapD, dt, o.epi.D, o.N, o.M, o.count, o.epi.ldd, o.epi.strideD, 64, 32))
             return MUON_ERR_CUDA;
+        if (P.band && (o.epi.fin != FIN_STORE ||
+                       !encode_map(&P.mapDt, dt, o.epi.D, o.N, o.M, o.count, o.epi.ldd, o.epi.strideD, 32, 64,
+                                   false)))
+            return MUON_ERR_CUDA;
     }
     prm.nprob = nops;
     prm.total_tiles = tiles;
@@ -621,7 +774,8 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
     int dev = 0, nsm = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = (int)(tiles < nsm ? tiles : nsm);
+    const long long units = pair ? nsm / 2 : nsm;   // persistent CTAs (pairs)
+    const int grid = (int)((tiles < units ? tiles : units) * (pair ? 2 : 1));
     if (grid <= 0) return MUON_OK;
     double work = 0.0;   // algorithmic flops: half of a symmetric product, all of a full one
     for (int i = 0; i < nops; ++i)
@@ -630,11 +784,13 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
     trace_begin(sym ? MUON_KERNEL_SYM : MUON_KERNEL_UPD, work, stream);
     cudaError_t e;
     if (dt == DT_BF16) {
-        e = sym ? launch_one<128, false, __nv_bfloat16>(prm, grid, stream)
-                : launch_one<256, true, __nv_bfloat16>(prm, grid, stream);
+        e = sym ? launch_one<128, false, false, __nv_bfloat16>(prm, grid, stream)
+                : pair ? launch_one<256, true, true, __nv_bfloat16>(prm, grid, stream)
+                       : launch_one<256, true, false, __nv_bfloat16>(prm, grid, stream);
     } else {
-        e = sym ? launch_one<128, false, __half>(prm, grid, stream)
-                : launch_one<256, true, __half>(prm, grid, stream);
+        e = sym ? launch_one<128, false, false, __half>(prm, grid, stream)
+                : pair ? launch_one<256, true, true, __half>(prm, grid, stream)
+                       : launch_one<256, true, false, __half>(prm, grid, stream);
     }
     trace_end(stream);
     return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;

@@ -179,9 +179,9 @@ Epilogue epi_store(void* D, long long ldd, long long strideD) {
 // D = A B^T, symmetric result; a_sym / b_sym: the operand itself is a stored
 // symmetric matrix (only its upper tiles are valid on the tensor-core path).
 GemmOp sym_op(int count, int n, int k, const void* A, long long lda, long long sA, const void* B,
-              long long ldb, long long sB, const Epilogue& e, int a_sym = 0, int b_sym = 0) {
+              long long ldb, long long sB, const Epilogue& e, int a_sym = 0, int b_sym = 0, int band = 0) {
     GemmOp o;
-    o.sym = 1; o.a_sym = a_sym; o.b_sym = b_sym; o.count = count; o.M = n; o.N = n; o.K = k;
+    o.sym = 1; o.a_sym = a_sym; o.b_sym = b_sym; o.band = band; o.count = count; o.M = n; o.N = n; o.K = k;
     o.A = A; o.lda = lda; o.strideA = sA;
     o.B = B; o.ldb = ldb; o.strideB = sB;
     o.epi = e;
@@ -192,7 +192,7 @@ GemmOp sym_op(int count, int n, int k, const void* A, long long lda, long long s
 GemmOp upd_op(int count, int s, int l, const void* A, long long lda, long long sA, const void* X,
               long long ldx, long long sX, const Epilogue& e) {
     GemmOp o;
-    o.sym = 0; o.a_sym = 1; o.b_sym = 0; o.count = count; o.M = s; o.N = l; o.K = s;
+    o.sym = 0; o.a_sym = 1; o.b_sym = 0; o.band = 0; o.count = count; o.M = s; o.N = l; o.K = s;
     o.A = A; o.lda = lda; o.strideA = sA;
     o.B = X; o.ldb = ldx; o.strideB = sX;
     o.epi = e;
@@ -233,7 +233,7 @@ muon_status run_direct(Runner& R, const Layout& L, void* ws, const muon_schedule
             Epilogue e = epi_store(at(ws, g.sq[1]), g.lds, ss);
             e.alpha = c.c; e.beta = c.b; e.diag = c.a;
             e.Cin = at(ws, g.sq[0]); e.ldc = g.lds; e.strideC = ss;
-            ops.push_back(sym_op(cnt, g.s, g.s, at(ws, g.sq[0]), g.lds, ss, at(ws, g.sq[0]), g.lds, ss, e, 1, 1));
+            ops.push_back(sym_op(cnt, g.s, g.s, at(ws, g.sq[0]), g.lds, ss, at(ws, g.sq[0]), g.lds, ss, e, 1, 1, 1));
         }
         st = R.run(ops, {});
         if (st != MUON_OK) return st;
@@ -325,7 +325,7 @@ muon_status run_gram(Runner& R, const Layout& L, void* ws, const muon_schedule* 
             Epilogue e = epi_store(sq(iH), g.lds, ss);
             e.alpha = c.c; e.beta = c.b; e.diag = c.a;
             e.Cin = sq(iR); e.ldc = g.lds; e.strideC = ss;
-            st = R.run({sym_op(cnt, g.s, g.s, sq(iR), g.lds, ss, sq(iR), g.lds, ss, e, 1, 1)}, {});
+            st = R.run({sym_op(cnt, g.s, g.s, sq(iR), g.lds, ss, sq(iR), g.lds, ss, e, 1, 1, 1)}, {});
             if (st != MUON_OK) return st;
         }
         const bool need_r = k + 1 < sch->n_steps && !is_restart(sch, k + 1);
@@ -333,7 +333,7 @@ muon_status run_gram(Runner& R, const Layout& L, void* ws, const muon_schedule* 
         std::vector<GemmOp> ops;
         if (!q_identity)
             ops.push_back(sym_op(cnt, g.s, g.s, sq(iH), g.lds, ss, sq(iQ), g.lds, ss, epi_store(sq(iQn), g.lds, ss),
-                                 1, 1));
+                                 1, 1, 1));
         if (need_r)
             ops.push_back(sym_op(cnt, g.s, g.s, sq(iH), g.lds, ss, sq(iR), g.lds, ss, epi_store(sq(iT), g.lds, ss),
                                  1, 1));
