@@ -50,17 +50,22 @@ constexpr int kEpiThreads = 32 * kEpiWarps;
 
 // Per-CTA configuration.  PAIR: two CTAs share each MMA (cta_group::2): the
 // pair computes a 256 x BN tile, each CTA loads its 128 rows of A and BN/2 of B.
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool B_MN>
 struct Cfg {
-    static constexpr int kStages = (PAIR || BN == 128) ? 6 : 4;
+    // symmetric products on CTA pairs stage a whole 128 x 256 output (16 boxes)
+    static constexpr bool kSymPair = PAIR && !B_MN;
+    static constexpr int kStages = kSymPair ? 5 : ((PAIR || BN == 128) ? 6 : 4);
     static constexpr int kABytes = BM * BK * 2;
     static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * BK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kTmemCols = 2 * BN;
-    static constexpr int kStgBytes = 32 * 64 * 2;              // one 32 x 64 16-bit box per epilogue warp
+    static constexpr int kStgBytes = 32 * 64 * 2;              // one 32 x 64 16-bit box
     static constexpr int kFinBytes = 32 * 33 * 4;              // final steps: one padded 32 x 32 fp32 box per warp
+    static constexpr int kBoxes = kSymPair ? 16 : kEpiWarps;   // staging boxes
+    static constexpr int kStgRegion = kBoxes * kStgBytes > kEpiWarps * kFinBytes ? kBoxes * kStgBytes
+                                                                                 : kEpiWarps * kFinBytes;
     static constexpr int kStgOffset = kStages * kStageBytes;
-    static constexpr int kBarOffset = kStgOffset + kEpiWarps * kFinBytes;   // kFinBytes > kStgBytes
+    static constexpr int kBarOffset = kStgOffset + kStgRegion;
     static constexpr int kBarBytes = 256;
     static constexpr int kSmemBytes = 1024 + kBarOffset + kBarBytes;
     static constexpr int kRows = PAIR ? 2 * BM : BM;           // output rows per tile
@@ -278,20 +283,21 @@ __device__ __forceinline__ int stg_off(int r, int c) {
     return r * 128 + (((c >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
 }
 
-// Diagonal tile of a symmetric result: the eight epilogue warps hold the whole
-// 128 x 128 tile in their staging boxes (box quad + 4 * half: rows 32*quad..,
-// columns 64*half..).  Overwrite this thread's elements below the diagonal
-// (local row i, column j < i) with the element (j, i) above it, so the stored
-// tile is exactly symmetric.  Reads touch only positions above the diagonal,
-// writes only positions below it.
+// Diagonal 128 x 128 block of a symmetric result, held in staging boxes
+// (box (q, c): rows 32q.., columns 64c.. of the CTA's tile; the block is box
+// columns cb0, cb0 + 1).  Overwrite this thread's elements of its box
+// (q = quad, c = cown) that lie below the diagonal (block row i, column j < i)
+// with element (j, i) above it, so the stored block is exactly symmetric.
+// Reads touch only positions above the diagonal, writes only positions below.
 template <typename T>
-__device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int half, int lane) {
+__device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int cb0, int cown, int lane) {
     const int i = quad * 32 + lane;
-    uint8_t* mine = stg_base + (quad + 4 * half) * (32 * 64 * 2);
+    uint8_t* mine = stg_base + (quad + 4 * cown) * (32 * 64 * 2);
+    const int jbase = (cown - cb0) * 64;
     for (int q = 0; q < 64; ++q) {
-        const int j = half * 64 + q;
+        const int j = jbase + q;
         if (j >= i) break;
-        const uint8_t* ob = stg_base + ((j >> 5) + 4 * (i >> 6)) * (32 * 64 * 2);
+        const uint8_t* ob = stg_base + ((j >> 5) + 4 * (cb0 + (i >> 6))) * (32 * 64 * 2);
         const T x = *reinterpret_cast<const T*>(ob + stg_off(j & 31, i & 63));
         *reinterpret_cast<T*>(mine + stg_off(lane, q)) = x;
     }
@@ -299,8 +305,8 @@ __device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int half,
 
 template <int BN, bool B_MN, bool PAIR, typename T>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
-    static_assert(!PAIR || (B_MN && BN == 256), "CTA pairs are used for the update product only");
-    using C = Cfg<BN, PAIR>;
+    static_assert(!PAIR || BN == 256, "CTA pairs compute 256 x 256 tiles");
+    using C = Cfg<BN, PAIR, B_MN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
@@ -367,50 +373,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 const TcProblem& P = p.prob[pi];
                 const int nkb = (P.K + BK - 1) / BK;
                 const int rows0 = ti * C::kRows + (int)rank * BM;   // this CTA's rows of A
-                // this CTA's columns of B (MN-major panel) and the 64-wide boxes they span
+                // this CTA's columns of the result (rows of a K-major B, columns of an
+                // MN-major B panel) and, for a panel, the 64-wide boxes they span
                 constexpr int kBCols = PAIR ? BN / 2 : BN;
                 const int bcol0 = tj * BN + (int)rank * kBCols;
                 auto chunks = [&](int c0) { return max(0, min(kBCols / 64, (P.N - c0 + 63) / 64)); };
                 const int nchunk = B_MN ? chunks(bcol0) : kBCols / 64;
                 uint32_t bytes = C::kABytes + (B_MN ? nchunk * 64 * BK * 2 : C::kBBytes);
-                if (PAIR) bytes = 2 * C::kABytes + (chunks(tj * BN) + chunks(tj * BN + kBCols)) * 64 * BK * 2;
+                if (PAIR) {   // the leader's barrier counts both CTAs' boxes
+                    bytes = B_MN ? 2 * C::kABytes + (chunks(tj * BN) + chunks(tj * BN + kBCols)) * 64 * BK * 2
+                                 : 2 * (C::kABytes + C::kBBytes);
+                }
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, d_status)) break;
                     uint8_t* sa = smem + stage * C::kStageBytes;
                     uint8_t* sb = sa + C::kABytes;
-                    // A block left of the diagonal of a symmetric A: read the stored
-                    // block above the diagonal transposed.  For a pair the decision is
-                    // taken on the pair's first 128-row block, so both halves agree
-                    // (the first sub-diagonal tile is stored for such operands).
+                    // Blocks left of the diagonal of a stored symmetric operand are read
+                    // transposed from the block above the diagonal.  On a pair the
+                    // decision is taken on the pair's first 128-row (128-column) block,
+                    // so both halves agree (such operands also store the first tile
+                    // below the diagonal).
                     const bool at = P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti);
-                    if (PAIR) {
-                        const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
-                        if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], bytes);
-                        if (at) {
-                            tma_load_3d_pair(&P.mapAt, fb, sa, rows0, kb * BK, m);
-                            tma_load_3d_pair(&P.mapAt, fb, sa + 64 * BK * 2, rows0 + 64, kb * BK, m);
-                        } else {
-                            tma_load_3d_pair(&P.mapA, fb, sa, kb * BK, rows0, m);
-                        }
-                        for (int c = 0; c < nchunk; ++c)
-                            tma_load_3d_pair(&P.mapB, fb, sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK, m);
+                    const bool bt = !B_MN && P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj);
+                    const uint32_t fb = PAIR ? mapa_shared(smem_u32(&full_bar[stage]), 0) : 0u;
+                    auto load = [&](const CUtensorMap* map, void* dst, int x, int y) {
+                        if (PAIR) tma_load_3d_pair(map, fb, dst, x, y, m);
+                        else tma_load_3d(map, &full_bar[stage], dst, x, y, m);
+                    };
+                    if (!PAIR || rank == 0) mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                    if (at) {
+                        load(&P.mapAt, sa, rows0, kb * BK);
+                        load(&P.mapAt, sa + 64 * BK * 2, rows0 + 64, kb * BK);
                     } else {
-                        mbar_arrive_expect_tx(&full_bar[stage], bytes);
-                        if (at) {
-                            tma_load_3d(&P.mapAt, &full_bar[stage], sa, rows0, kb * BK, m);
-                            tma_load_3d(&P.mapAt, &full_bar[stage], sa + 64 * BK * 2, rows0 + 64, kb * BK, m);
-                        } else {
-                            tma_load_3d(&P.mapA, &full_bar[stage], sa, kb * BK, rows0, m);
-                        }
-                        if (B_MN) {
-                            for (int c = 0; c < nchunk; ++c)
-                                tma_load_3d(&P.mapB, &full_bar[stage], sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK, m);
-                        } else if (P.b_sym && (kb >> 1) < tj) {
-                            for (int c = 0; c < BN / 64; ++c)
-                                tma_load_3d(&P.mapBt, &full_bar[stage], sb + c * (64 * BK * 2), tj * BN + c * 64, kb * BK, m);
-                        } else {
-                            tma_load_3d(&P.mapB, &full_bar[stage], sb, kb * BK, tj * BN, m);
-                        }
+                        load(&P.mapA, sa, kb * BK, rows0);
+                    }
+                    if (B_MN) {
+                        for (int c = 0; c < nchunk; ++c) load(&P.mapB, sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK);
+                    } else if (bt) {
+                        for (int c = 0; c < kBCols / 64; ++c)
+                            load(&P.mapBt, sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK);
+                    } else {
+                        load(&P.mapB, sb, kb * BK, bcol0);
                     }
                     armed |= 1u << stage;
                     armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -457,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     if (!mbar_wait(&full_bar[stage], phase, abort_flag, d_status)) { ok = false; break; }
                     tc_fence_after();
                     const bool at = P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti);   // A block read transposed
-                    const bool bm = B_MN || (P.b_sym && (kb >> 1) < tj);          // B block MN-major
+                    const bool bm = B_MN || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj));   // B block MN-major
                     const uint32_t idesc = idesc0 | (at ? 1u << 15 : 0u) | (bm ? 1u << 16 : 0u);
                     const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t sb = sa + C::kABytes;
@@ -543,6 +546,95 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 if (row == 0 && half == 0 && tj == 0 && ti == 0 && rank == 0 && d_status)
                     atomicOr(d_status, MUON_FLAG_NONFINITE);
             }
+            if constexpr (C::kSymPair) {
+                // Symmetric result on a CTA pair: this CTA holds rows row0.. of a
+                // 256-column tile; box (q, c) = rows 32q.., columns 64c..; this warp
+                // owns box columns 2*half and 2*half + 1.  Both boxes are staged
+                // before anything is stored, so a diagonal block (tile on the
+                // diagonal: this CTA's block column `rank`) can be made exactly
+                // symmetric across the warps first.  In a diagonal tile the second
+                // CTA's first block column lies below the diagonal and is not stored
+                // (its exact mirror comes from the first CTA's band store).
+                const bool diag_pair = ti == tj;
+                bool have[2] = {false, false};
+                if (!dead && stg_busy) {
+                    if (lane == 0) bulk_wait_read0();
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int pr = 0; pr < 2; ++pr) {
+                    const int cbox = 2 * half + pr;
+                    const int gj0 = tj * BN + cbox * 64;
+                    have[pr] = !dead && gj0 < P.N;
+                    if (!have[pr]) continue;
+                    if (has_cin && pr > 0) {
+                        cin_fetch<T>(E, m, gi, gj0, P.M, P.N, c0);
+                        cin_fetch<T>(E, m, gi, gj0 + 32, P.M, P.N, c1);
+                    }
+                    const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                          (uint32_t)(buf * BN + cbox * 64);
+                    uint8_t* box = stg_base + (quad + 4 * cbox) * C::kStgBytes;
+                    float v[32];
+                    tmem_ld_32x32b_x32(tcol, v);
+                    epi_combine<T>(E, gi, gj0, sc, v, c0);
+                    stage32<T>(box, lane, 0, v);
+                    tmem_ld_32x32b_x32(tcol + 32, v);
+                    epi_combine<T>(E, gi, gj0 + 32, sc, v, c1);
+                    stage32<T>(box, lane, 4, v);
+                }
+                if (diag_pair) {     // uniform over the CTA: every epilogue warp attends
+                    epi_bar();
+                    if (half == (int)rank) {
+#pragma unroll
+                        for (int pr = 0; pr < 2; ++pr)
+                            if (have[pr]) fix_lower<T>(stg_base, quad, 2 * (int)rank, 2 * half + pr, lane);
+                    }
+                    epi_bar();
+                }
+                const bool rows_ok = row0 + quad * 32 < P.M;
+                const bool lower = diag_pair && rank == 1 && half == 0;   // below the diagonal
+#pragma unroll
+                for (int pr = 0; pr < 2; ++pr) {
+                    if (!have[pr] || !rows_ok || lower) continue;
+                    const int cbox = 2 * half + pr;
+                    const int gj0 = tj * BN + cbox * 64;
+                    uint8_t* box = stg_base + (quad + 4 * cbox) * C::kStgBytes;
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&P.mapD, box, gj0, row0 + quad * 32, m);
+                        bulk_commit();
+                    }
+                    stg_busy = true;
+                    // 128-block (bi, bj) of this box; the first block right of the
+                    // diagonal is also stored transposed (exact mirror)
+                    const int bi = 2 * ti + (int)rank, bj = 2 * tj + half;
+                    if (P.band && bj == bi + 1) {
+                        if (lane == 0) bulk_wait_read0();
+                        __syncwarp();
+                        uint4 d0[4] = {}, d1[4] = {};
+                        if (has_cin) {
+                            cin_fetch<T>(E, m, gi, gj0, P.M, P.N, d0);
+                            cin_fetch<T>(E, m, gi, gj0 + 32, P.M, P.N, d1);
+                        }
+                        const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                              (uint32_t)(buf * BN + cbox * 64);
+                        float v[32];
+                        tmem_ld_32x32b_x32(tcol, v);
+                        epi_combine<T>(E, gi, gj0, sc, v, d0);
+                        stage_transposed<T>(box, lane, 0, v);
+                        tmem_ld_32x32b_x32(tcol + 32, v);
+                        epi_combine<T>(E, gi, gj0 + 32, sc, v, d1);
+                        stage_transposed<T>(box, lane, 32, v);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&P.mapDt, box, row0 + quad * 32, gj0, m);
+                            bulk_commit();
+                        }
+                    }
+                }
+            } else {
 #pragma unroll 1
             for (int pr = 0; pr < kPairs; ++pr) {
                 const int gj0 = col0 + pr * 64;
@@ -571,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     }
                     if (diag_sym) {          // BN == 128 here: the eight boxes cover the tile
                         epi_bar();
-                        if (work) fix_lower<T>(stg_base, quad, half, lane);
+                        if (work) fix_lower<T>(stg_base, quad, 0, half, lane);
                         epi_bar();
                     }
                     if (work && row0 + quad * 32 < P.M) {
@@ -619,6 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     }
                 }
             }
+            }   // kSymPair
             if (!dead) {
                 tc_fence_before();
                 __syncwarp();
@@ -680,7 +773,7 @@ static bool encode_map(CUtensorMap* map, int dt, const void* base, long long inn
 
 template <int BN, bool B_MN, bool PAIR, typename T>
 static cudaError_t launch_one(const TcParams& prm, int grid, cudaStream_t stream) {
-    using C = Cfg<BN, PAIR>;
+    using C = Cfg<BN, PAIR, B_MN>;
     auto kern = tc_gemm_kernel<BN, B_MN, PAIR, T>;
     static thread_local int configured_dev = -1;
     int dev = 0;
@@ -714,14 +807,15 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
     if (nops <= 0) return MUON_OK;
     if (nops > kMaxProblems || nfin > kMaxFinal) return MUON_ERR_UNSUPPORTED;
     const int sym = ops[0].sym;
-    const int BN = sym ? 128 : 256;
-    // update products run on CTA pairs (cta_group::2, 256 x 256 tiles) unless
-    // MUON_UPDATE_KERNEL=single selects one CTA per 128 x 256 tile
-    static const bool pair_ok = [] {
-        const char* v = getenv("MUON_UPDATE_KERNEL");
-        return !(v && strcmp(v, "single") == 0);
+    // Products run on CTA pairs (cta_group::2, 256 x 256 tiles) unless
+    // MUON_CTA_PAIRS=0 selects one CTA per tile (128 x 128 symmetric, 128 x 256
+    // update).  On pairs every symmetric result also stores its first tile below
+    // the diagonal, which pair consumers need.
+    static const bool pair = [] {
+        const char* v = getenv("MUON_CTA_PAIRS");
+        return !(v && strcmp(v, "0") == 0);
     }();
-    const bool pair = !sym && pair_ok;
+    const int BN = (sym && !pair) ? 128 : 256;
     const int rows_per_tile = pair ? 2 * BM : BM;
     // the final-step staging boxes overlap the store boxes: one kind per launch
     for (int i = 1; i < nops; ++i)
@@ -745,13 +839,15 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         P.epi = o.epi;
         P.a_sym = o.a_sym;
         P.b_sym = sym ? o.b_sym : 0;
-        P.band = sym ? o.band : 0;
+        P.band = sym ? (pair ? 1 : o.band) : 0;
         // A operand: M rows x K (K contiguous); a symmetric A is also read transposed
         if (!encode_map(&P.mapA, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, BK, BM)) return MUON_ERR_CUDA;
         if (o.a_sym && !encode_map(&P.mapAt, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, 64, BK))
             return MUON_ERR_CUDA;
         if (sym) {
-            if (!encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK, BN)) return MUON_ERR_CUDA;
+            // each CTA of a pair loads half of the tile's B rows
+            if (!encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK, pair ? BN / 2 : BN))
+                return MUON_ERR_CUDA;
             if (o.b_sym && !encode_map(&P.mapBt, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, 64, BK))
                 return MUON_ERR_CUDA;
         } else {
@@ -784,13 +880,15 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
     trace_begin(sym ? MUON_KERNEL_SYM : MUON_KERNEL_UPD, work, stream);
     cudaError_t e;
     if (dt == DT_BF16) {
-        e = sym ? launch_one<128, false, false, __nv_bfloat16>(prm, grid, stream)
-                : pair ? launch_one<256, true, true, __nv_bfloat16>(prm, grid, stream)
-                       : launch_one<256, true, false, __nv_bfloat16>(prm, grid, stream);
+        if (sym) e = pair ? launch_one<256, false, true, __nv_bfloat16>(prm, grid, stream)
+                          : launch_one<128, false, false, __nv_bfloat16>(prm, grid, stream);
+        else e = pair ? launch_one<256, true, true, __nv_bfloat16>(prm, grid, stream)
+                      : launch_one<256, true, false, __nv_bfloat16>(prm, grid, stream);
     } else {
-        e = sym ? launch_one<128, false, false, __half>(prm, grid, stream)
-                : pair ? launch_one<256, true, true, __half>(prm, grid, stream)
-                       : launch_one<256, true, false, __half>(prm, grid, stream);
+        if (sym) e = pair ? launch_one<256, false, true, __half>(prm, grid, stream)
+                          : launch_one<128, false, false, __half>(prm, grid, stream);
+        else e = pair ? launch_one<256, true, true, __half>(prm, grid, stream)
+                      : launch_one<256, true, false, __half>(prm, grid, stream);
     }
     trace_end(stream);
     return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
