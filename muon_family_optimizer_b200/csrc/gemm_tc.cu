@@ -50,20 +50,20 @@ constexpr int kEpiThreads = 32 * kEpiWarps;
 
 // Per-CTA configuration.  PAIR: two CTAs share each MMA (cta_group::2): the
 // pair computes a 256 x BN tile, each CTA loads its 128 rows of A and BN/2 of B.
-template <int BN, bool PAIR, bool B_MN>
+template <int BN, bool PAIR, bool B_MN, bool FIN>
 struct Cfg {
-    // symmetric products on CTA pairs stage a whole 128 x 256 output (16 boxes)
+    // symmetric products on CTA pairs stage a whole 128 x 256 output (16 boxes);
+    // the final step keeps two 32 x 32 blocks of the target per epilogue warp
     static constexpr bool kSymPair = PAIR && !B_MN;
-    static constexpr int kStages = kSymPair ? 5 : ((PAIR || BN == 128) ? 6 : 4);
+    static constexpr int kStages = FIN ? (PAIR ? 4 : 3) : kSymPair ? 5 : ((PAIR || BN == 128) ? 6 : 4);
     static constexpr int kABytes = BM * BK * 2;
     static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * BK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kTmemCols = 2 * BN;
     static constexpr int kStgBytes = 32 * 64 * 2;              // one 32 x 64 16-bit box
-    static constexpr int kFinBytes = 32 * 33 * 4;              // final steps: one padded 32 x 32 fp32 box per warp
     static constexpr int kBoxes = kSymPair ? 16 : kEpiWarps;   // staging boxes
-    static constexpr int kStgRegion = kBoxes * kStgBytes > kEpiWarps * kFinBytes ? kBoxes * kStgBytes
-                                                                                 : kEpiWarps * kFinBytes;
+    static constexpr int kFinBlock = 32 * 32 * 4;               // one 32 x 32 block of the target (up to fp32)
+    static constexpr int kStgRegion = FIN ? kEpiWarps * 2 * kFinBlock : kBoxes * kStgBytes;
     static constexpr int kStgOffset = kStages * kStageBytes;
     static constexpr int kBarOffset = kStgOffset + kStgRegion;
     static constexpr int kBarBytes = 256;
@@ -127,94 +127,197 @@ __device__ __forceinline__ void cin_fetch(const Epilogue& E, int m, int gi, int 
     }
 }
 
-// Final step for one 32 x 32 block of the wide view (rows gi0..gi0+31 held by
-// the warp's lanes, columns gj0..gj0+31), already staged in `fs` (padded
-// [32][33] fp32, row = wide row).  Writes the caller's output (FIN_OUT) or
-// applies W <- W - eta (gamma O + lambda W) (FIN_WUPD) in the parameter's own
-// orientation: each lane moves 8 consecutive elements of one parameter row,
-// four lanes per 32-element row segment, so every global access is a
-// coalesced 16-byte (or 32-byte) access whichever way the parameter is stored.
-template <typename TW>
-__device__ __forceinline__ void final_block(const Epilogue& E, const FinalCtx& fc, int m, int M, int N,
-                                            int gi0, int gj0, const float* fs, int lane) {
-    constexpr int kDt = sizeof(TW) == 4 ? DT_FP32 : (IsBf16<TW>::value ? DT_BF16 : DT_FP16);
-    TW* W;
-    float* O_out = nullptr;
-    float g = 0.f;
-    int tr, vec;
-    const bool wupd = E.fin == FIN_WUPD;
-    if (!wupd) {
-        W = reinterpret_cast<TW*>(static_cast<char*>(fc.out) + (size_t)m * fc.out_stride * sizeof(TW));
-        tr = fc.out_transposed; vec = fc.out_vec;
+// ---------------------------------------------------------------------------
+// Final step (FIN_WUPD: W <- W - eta (gamma O + lambda W); FIN_OUT: the
+// caller's output), one warp at a time: wide rows gi0..gi0+31 (one per lane)
+// and 32-column blocks of wide columns.  Each block of the target matrix is
+// moved between global and shared memory in its own orientation with
+// coalesced 16-byte accesses (W prefetched with cp.async one block ahead),
+// updated in shared memory by the lane that owns the row of O, and written
+// back.  Block layout in shared memory (param rows of 32 * sizeof(TW) bytes):
+//   wide view (!tr): row = wide row, 16-byte chunks XOR-swizzled by row;
+//   transposed (tr): row = wide column, unswizzled (lanes then touch
+//   consecutive elements of one row).
+// ---------------------------------------------------------------------------
+struct FinalTarget {
+    void* W;
+    float* O_out;
+    float g;
+    int tr, vec, dt;
+    bool wupd;
+};
+
+__device__ __forceinline__ FinalTarget final_target(const Epilogue& E, const FinalCtx& fc, int m) {
+    FinalTarget F;
+    F.wupd = E.fin == FIN_WUPD;
+    if (!F.wupd) {
+        F.W = static_cast<char*>(fc.out) + (size_t)m * fc.out_stride * dt_size(fc.out_dt);
+        F.O_out = nullptr; F.g = 0.f; F.tr = fc.out_transposed; F.vec = fc.out_vec; F.dt = fc.out_dt;
     } else {
         const FinalEntry& fe = fc.fin[E.fin_base + m];
-        W = static_cast<TW*>(fe.W); O_out = fe.O_out; g = fe.gamma; tr = fe.transposed; vec = fe.vec_ok;
+        F.W = fe.W; F.O_out = fe.O_out; F.g = fe.gamma; F.tr = fe.transposed; F.vec = fe.vec_ok; F.dt = fc.w_dt;
     }
-    // parameter extent: tr ? (N rows x M cols) : (M rows x N cols)
-    const int prow_n = tr ? N : M, pcol_n = tr ? M : N;
-    const int prow0 = tr ? gj0 : gi0, pcol0 = tr ? gi0 : gj0;
-    const int cc = (lane & 3) * 8;                // first of 8 parameter columns inside the block
-    // pass 1: issue every load of W first (four independent 16/32-byte loads per lane)
-    float w[4][8];
+    return F;
+}
+
+template <typename TW>
+__device__ __forceinline__ int wb_off(int prow, int chunk, bool swz) {
+    constexpr int kRowBytes = 32 * (int)sizeof(TW);
+    const int c = !swz ? chunk : (sizeof(TW) == 2 ? chunk ^ ((prow >> 1) & 3) : chunk ^ (prow & 7));
+    return prow * kRowBytes + c * 16;
+}
+
+// Copy the target's block (wide rows gi0.., wide columns gj0..) into `buf`
+// (to_smem) or back from it; chunks outside the matrix are zero-filled on the
+// way in and skipped on the way out.
+template <typename TW, bool kIn>
+__device__ __forceinline__ void final_move(const FinalTarget& F, int M, int N, int gi0, int gj0, uint8_t* buf,
+                                           int lane) {
+    constexpr int kEpc = 16 / (int)sizeof(TW);       // elements per 16-byte chunk
+    constexpr int kChunks = 32 / kEpc;               // chunks per block row
+    const int prow_n = F.tr ? N : M, pcol_n = F.tr ? M : N;
+    const int prow0 = F.tr ? gj0 : gi0, pcol0 = F.tr ? gi0 : gj0;
+    TW* W = static_cast<TW*>(F.W);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int prow = prow0 + 8 * k + (lane >> 2), pcol = pcol0 + cc;
-        if (!wupd || prow >= prow_n || pcol >= pcol_n) continue;
-        const TW* wp = W + (size_t)prow * pcol_n + pcol;
-        if (vec && pcol + 8 <= pcol_n) {
-            load8_dt(wp, 0, kDt, true, 8, w[k]);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w[k][e] = pcol + e < pcol_n ? to_float(wp[e]) : 0.f;
+    for (int k = 0; k < kChunks; ++k) {
+        const int id = lane + 32 * k;
+        const int pr = id / kChunks, ch = id % kChunks;
+        const int prow = prow0 + pr, pcol = pcol0 + ch * kEpc;
+        const bool in = prow < prow_n && pcol < pcol_n;
+        uint8_t* sp = buf + wb_off<TW>(pr, ch, !F.tr);
+        if (kIn) {
+            cp_async16(sp, in ? W + (size_t)prow * pcol_n + pcol : W, in ? 16u : 0u);
+        } else if (in) {
+            *reinterpret_cast<uint4*>(W + (size_t)prow * pcol_n + pcol) = *reinterpret_cast<const uint4*>(sp);
         }
     }
-    // pass 2: combine with the staged result and store
+}
+
+// Apply the final step to this lane's row of the staged block.
+template <typename TW>
+__device__ __forceinline__ void final_apply(const FinalTarget& F, const FinalCtx& fc, uint8_t* buf,
+                                            const float (&v)[32], int lane) {
+    constexpr int kEpc = 16 / (int)sizeof(TW);
+    if (!F.tr) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int rr = 8 * k + (lane >> 2);       // parameter row inside the block
-        const int prow = prow0 + rr, pcol = pcol0 + cc;
-        if (prow >= prow_n || pcol >= pcol_n) continue;
-        float o[8];
+        for (int ch = 0; ch < 32 / kEpc; ++ch) {
+            uint4* p = reinterpret_cast<uint4*>(buf + wb_off<TW>(lane, ch, true));
+            uint4 u = *p;
+            uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = tr ? fs[(cc + e) * 33 + rr] : fs[rr * 33 + cc + e];
-        TW* wp = W + (size_t)prow * pcol_n + pcol;
-        const bool full = vec && pcol + 8 <= pcol_n;
-        if (wupd) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w[k][e] = w[k][e] - fc.eta * (g * o[e] + fc.lambda * w[k][e]);
-            if (full) {
-                store8_dt(wp, 0, kDt, true, 8, w[k]);
-                if (O_out) store8_dt(O_out + (size_t)prow * pcol_n + pcol, 0, DT_FP32, true, 8, o);
-            } else {
-                for (int e = 0; e < 8 && pcol + e < pcol_n; ++e) {
-                    wp[e] = from_float<TW>(w[k][e]);
-                    if (O_out) O_out[(size_t)prow * pcol_n + pcol + e] = o[e];
+            for (int h = 0; h < 4; ++h) {
+                if constexpr (sizeof(TW) == 4) {
+                    const float o = v[ch * 4 + h];
+                    const float w = __uint_as_float(w4[h]);
+                    w4[h] = __float_as_uint(F.wupd ? w - fc.eta * (F.g * o + fc.lambda * w) : o);
+                } else {
+                    const float o0 = v[ch * 8 + 2 * h], o1 = v[ch * 8 + 2 * h + 1];
+                    float a = o0, b = o1;
+                    if (F.wupd) {
+                        const float w0 = unpack_lo<TW>(w4[h]), w1 = unpack_hi<TW>(w4[h]);
+                        a = w0 - fc.eta * (F.g * o0 + fc.lambda * w0);
+                        b = w1 - fc.eta * (F.g * o1 + fc.lambda * w1);
+                    }
+                    w4[h] = pack2<TW>(a, b);
                 }
             }
-        } else if (full) {
-            store8_dt(wp, 0, kDt, true, 8, o);
-        } else {
-            for (int e = 0; e < 8 && pcol + e < pcol_n; ++e) wp[e] = from_float<TW>(o[e]);
+            u.x = w4[0]; u.y = w4[1]; u.z = w4[2]; u.w = w4[3];
+            *p = u;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            TW* p = reinterpret_cast<TW*>(buf + (q * 32 + lane) * (int)sizeof(TW));
+            if (F.wupd) {
+                const float w = to_float(*p);
+                *p = from_float<TW>(w - fc.eta * (F.g * v[q] + fc.lambda * w));
+            } else {
+                *p = from_float<TW>(v[q]);
+            }
         }
     }
 }
 
-// Write out the warp's staged 32 x 32 block (kept out of line: only the
-// final step takes this path, and inlining it would crowd the hot loop).
-__device__ __noinline__ void final_write(const Epilogue& E, const FinalCtx& fc, int m, int M, int N,
-                                         int gi0, int gj0, const float* fs, int lane) {
-    const int dt = E.fin == FIN_OUT ? fc.out_dt : fc.w_dt;
-    if (dt == DT_BF16) final_block<__nv_bfloat16>(E, fc, m, M, N, gi0, gj0, fs, lane);
-    else if (dt == DT_FP16) final_block<__half>(E, fc, m, M, N, gi0, gj0, fs, lane);
-    else final_block<float>(E, fc, m, M, N, gi0, gj0, fs, lane);
+// Unaligned or ragged target: element by element from and to global memory.
+template <typename TW>
+__device__ __forceinline__ void final_scalar(const FinalTarget& F, const FinalCtx& fc, int M, int N, int gi,
+                                             int gj0, const float (&v)[32]) {
+    if (gi >= M) return;
+    TW* W = static_cast<TW*>(F.W);
+    float w[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+        const int j = gj0 + q;
+        const size_t idx = F.tr ? (size_t)j * M + gi : (size_t)gi * N + j;
+        w[q] = (F.wupd && j < N) ? to_float(W[idx]) : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+        const int j = gj0 + q;
+        if (j >= N) continue;
+        const size_t idx = F.tr ? (size_t)j * M + gi : (size_t)gi * N + j;
+        W[idx] = from_float<TW>(F.wupd ? w[q] - fc.eta * (F.g * v[q] + fc.lambda * w[q]) : v[q]);
+    }
 }
 
-// Stage 32 values of this lane's row into the warp's padded final box.
-__device__ __forceinline__ void final_stage(float* fs, int lane, const float (&v)[32]) {
-    __syncwarp();                       // the previous block's reads of fs are done
+// Optional fp32 copy of O in the parameter's orientation.
+__device__ __forceinline__ void final_o_out(const FinalTarget& F, int M, int N, int gi, int gj0,
+                                            const float (&v)[32]) {
+    if (!F.O_out || gi >= M) return;
 #pragma unroll
-    for (int q = 0; q < 32; ++q) fs[lane * 33 + q] = v[q];
-    __syncwarp();
+    for (int q = 0; q < 32; ++q) {
+        const int j = gj0 + q;
+        if (j < N) F.O_out[F.tr ? (size_t)j * M + gi : (size_t)gi * N + j] = v[q];
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void epi_combine(const Epilogue& E, int gi, int gj0, float sc, float (&v)[32],
+                                            const uint4 (&c)[4]);
+
+// The final step for the warp's wide rows gi0.. and its BN/2 wide columns
+// from col0: four 32-column blocks, block b's target data in wbuf[b % 2].
+// Block 0's copy may already be in flight (pf_issued).
+template <typename T, typename TW, int BN>
+__device__ __forceinline__ void final_tile(const FinalTarget& F, const Epilogue& E, const FinalCtx& fc, int m,
+                                           const TcProblem& P, int gi0, int col0, int gi, float sc, uint32_t tcol0,
+                                           uint8_t* wbuf, int lane, bool pf_issued) {
+    constexpr int kBlocks = BN / 64;                 // 32-column blocks per warp
+    constexpr int kBlockBytes = 32 * 32 * 4;
+    const bool staged = F.vec;                      // aligned target: go through shared memory
+    const uint4 none[4] = {};
+#pragma unroll 1
+    for (int b = 0; b < kBlocks; ++b) {
+        const int gj0 = col0 + 32 * b;
+        if (gj0 >= P.N) break;                       // warp-uniform
+        uint8_t* cur = wbuf + (b & 1) * kBlockBytes;
+        if (staged && F.wupd) {
+            if (b == 0 && !pf_issued) {
+                final_move<TW, true>(F, P.M, P.N, gi0, gj0, cur, lane);
+                cp_async_commit();
+            }
+            if (b + 1 < kBlocks && gj0 + 32 < P.N) {  // next block's copy in flight during this one
+                final_move<TW, true>(F, P.M, P.N, gi0, gj0 + 32, wbuf + ((b + 1) & 1) * kBlockBytes, lane);
+                cp_async_commit();
+            }
+        }
+        float v[32];
+        tmem_ld_32x32b_x32(tcol0 + 32 * b, v);
+        epi_combine<T>(E, gi, gj0, sc, v, none);
+        final_o_out(F, P.M, P.N, gi, gj0, v);
+        if (!staged) {
+            final_scalar<TW>(F, fc, P.M, P.N, gi, gj0, v);
+            continue;
+        }
+        if (F.wupd) {
+            if (b + 1 < kBlocks && gj0 + 32 < P.N) cp_async_wait<1>(); else cp_async_wait<0>();
+        }
+        __syncwarp();                                // this block's copy visible to every lane
+        final_apply<TW>(F, fc, cur, v, lane);
+        __syncwarp();
+        final_move<TW, false>(F, P.M, P.N, gi0, gj0, cur, lane);
+        __syncwarp();                                // cur free for the block after next
+    }
 }
 
 // Combine one 32-column chunk of the accumulator (row gi, columns
@@ -303,10 +406,11 @@ __device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int cb0, 
     }
 }
 
-template <int BN, bool B_MN, bool PAIR, typename T>
+template <int BN, bool B_MN, bool PAIR, bool FIN, typename T>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
     static_assert(!PAIR || BN == 256, "CTA pairs compute 256 x 256 tiles");
-    using C = Cfg<BN, PAIR, B_MN>;
+    static_assert(!FIN || B_MN, "the final step is an update product");
+    using C = Cfg<BN, PAIR, B_MN, FIN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
@@ -511,6 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         constexpr int kPairs = BN / 128;      // 64-column boxes per half
         uint8_t* stg_base = smem + C::kStgOffset;
         uint8_t* stg = stg_base + (quad + 4 * half) * C::kStgBytes;   // box of rows 32*quad.., columns 64*half..
+        uint8_t* wbuf = stg_base + (quad + 4 * half) * 2 * C::kFinBlock;   // final step: two target blocks
         bool stg_busy = false;                // a bulk store may still be reading stg
         bool dead = false;
         FinalCtx fc = p.fc;
@@ -529,6 +634,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             const bool has_cin = E.beta != 0.f;
             const bool diag_sym = P.sym && ti == tj && E.fin == FIN_STORE;   // uniform over the CTA
             uint4 c0[4] = {}, c1[4] = {};
+            bool pf_issued = false;
+            if constexpr (FIN) {
+                // the target's first block is independent of the accumulator: prefetch it
+                if (!dead && row0 + quad * 32 < P.M) {
+                    const FinalTarget F = final_target(E, fc, m);
+                    if (F.wupd && F.vec && col0 < P.N) {
+                        if (F.dt == DT_BF16) final_move<__nv_bfloat16, true>(F, P.M, P.N, row0 + quad * 32, col0, wbuf, lane);
+                        else if (F.dt == DT_FP16) final_move<__half, true>(F, P.M, P.N, row0 + quad * 32, col0, wbuf, lane);
+                        else final_move<float, true>(F, P.M, P.N, row0 + quad * 32, col0, wbuf, lane);
+                        cp_async_commit();
+                        pf_issued = true;
+                    }
+                }
+            }
             if (!dead) {
                 if (has_cin) {   // independent of the accumulator: fetch before waiting for it
                     cin_fetch<T>(E, m, gi, col0, P.M, P.N, c0);
@@ -546,7 +665,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 if (row == 0 && half == 0 && tj == 0 && ti == 0 && rank == 0 && d_status)
                     atomicOr(d_status, MUON_FLAG_NONFINITE);
             }
-            if constexpr (C::kSymPair) {
+            if constexpr (FIN) {
+                // final step: W update (or the caller's output) block by block,
+                // the target's next block prefetched while this one is applied
+                if (!dead && !skip && row0 + quad * 32 < P.M) {
+                    const FinalTarget F = final_target(E, fc, m);
+                    if (F.dt == DT_BF16) final_tile<T, __nv_bfloat16, BN>(F, E, fc, m, P, row0 + quad * 32, col0, gi, sc,
+                                                                        tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                                                            (uint32_t)(buf * BN + half * (BN / 2)),
+                                                                        wbuf, lane, pf_issued);
+                    else if (F.dt == DT_FP16) final_tile<T, __half, BN>(F, E, fc, m, P, row0 + quad * 32, col0, gi, sc,
+                                                                      tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                                                          (uint32_t)(buf * BN + half * (BN / 2)),
+                                                                      wbuf, lane, pf_issued);
+                    else final_tile<T, float, BN>(F, E, fc, m, P, row0 + quad * 32, col0, gi, sc,
+                                                  tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                                      (uint32_t)(buf * BN + half * (BN / 2)),
+                                                  wbuf, lane, pf_issued);
+                }
+                cp_async_wait<0>();   // nothing of this tile stays in flight
+                __syncwarp();
+            } else if constexpr (C::kSymPair) {
                 // Symmetric result on a CTA pair: this CTA holds rows row0.. of a
                 // 256-column tile; box (q, c) = rows 32q.., columns 64c..; this warp
                 // owns box columns 2*half and 2*half + 1.  Both boxes are staged
@@ -695,20 +834,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                             }
                         }
                     }
-                } else if (work && !skip && row0 + quad * 32 < P.M) {
-                    float* fs = reinterpret_cast<float*>(stg_base + (quad + 4 * half) * C::kFinBytes);
-                    const int gi0 = row0 + quad * 32;
-                    float v[32];
-                    tmem_ld_32x32b_x32(tcol, v);
-                    epi_combine<T>(E, gi, gj0, sc, v, c0);
-                    final_stage(fs, lane, v);
-                    final_write(E, fc, m, P.M, P.N, gi0, gj0, fs, lane);
-                    if (gj0 + 32 < P.N) {
-                        tmem_ld_32x32b_x32(tcol + 32, v);
-                        epi_combine<T>(E, gi, gj0 + 32, sc, v, c1);
-                        final_stage(fs, lane, v);
-                        final_write(E, fc, m, P.M, P.N, gi0, gj0 + 32, fs, lane);
-                    }
                 }
             }
             }   // kSymPair
@@ -771,10 +896,10 @@ static bool encode_map(CUtensorMap* map, int dt, const void* base, long long inn
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool B_MN, bool PAIR, typename T>
+template <int BN, bool B_MN, bool PAIR, bool FIN, typename T>
 static cudaError_t launch_one(const TcParams& prm, int grid, cudaStream_t stream) {
-    using C = Cfg<BN, PAIR, B_MN>;
-    auto kern = tc_gemm_kernel<BN, B_MN, PAIR, T>;
+    using C = Cfg<BN, PAIR, B_MN, FIN>;
+    auto kern = tc_gemm_kernel<BN, B_MN, PAIR, FIN, T>;
     static thread_local int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -879,16 +1004,21 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
                     : 2.0 * ops[i].count * ops[i].M * ops[i].N * ops[i].K;
     trace_begin(sym ? MUON_KERNEL_SYM : MUON_KERNEL_UPD, work, stream);
     cudaError_t e;
+    const bool final_step = ops[0].epi.fin != FIN_STORE;
     if (dt == DT_BF16) {
-        if (sym) e = pair ? launch_one<256, false, true, __nv_bfloat16>(prm, grid, stream)
-                          : launch_one<128, false, false, __nv_bfloat16>(prm, grid, stream);
-        else e = pair ? launch_one<256, true, true, __nv_bfloat16>(prm, grid, stream)
-                      : launch_one<256, true, false, __nv_bfloat16>(prm, grid, stream);
+        if (sym) e = pair ? launch_one<256, false, true, false, __nv_bfloat16>(prm, grid, stream)
+                          : launch_one<128, false, false, false, __nv_bfloat16>(prm, grid, stream);
+        else if (final_step) e = pair ? launch_one<256, true, true, true, __nv_bfloat16>(prm, grid, stream)
+                               : launch_one<256, true, false, true, __nv_bfloat16>(prm, grid, stream);
+        else e = pair ? launch_one<256, true, true, false, __nv_bfloat16>(prm, grid, stream)
+                      : launch_one<256, true, false, false, __nv_bfloat16>(prm, grid, stream);
     } else {
-        if (sym) e = pair ? launch_one<256, false, true, __half>(prm, grid, stream)
-                          : launch_one<128, false, false, __half>(prm, grid, stream);
-        else e = pair ? launch_one<256, true, true, __half>(prm, grid, stream)
-                      : launch_one<256, true, false, __half>(prm, grid, stream);
+        if (sym) e = pair ? launch_one<256, false, true, false, __half>(prm, grid, stream)
+                          : launch_one<128, false, false, false, __half>(prm, grid, stream);
+        else if (final_step) e = pair ? launch_one<256, true, true, true, __half>(prm, grid, stream)
+                               : launch_one<256, true, false, true, __half>(prm, grid, stream);
+        else e = pair ? launch_one<256, true, true, false, __half>(prm, grid, stream)
+                      : launch_one<256, true, false, false, __half>(prm, grid, stream);
     }
     trace_end(stream);
     return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
