@@ -37,7 +37,7 @@ muon_status simt_run(const GemmOp* ops, int nops, const FinalCtx& fc, const Fina
 }
 
 // Fused elementwise passes ahead of the iteration (prepass.cu).
-constexpr int kMaxPrep = 64;
+constexpr int kMaxPrep = 128;
 
 struct PrepEntry {
     const void* G; void* Gp; float* A; float* M;   // MONA mode: this parameter's state

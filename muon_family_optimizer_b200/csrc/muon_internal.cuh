@@ -118,7 +118,9 @@ __device__ __forceinline__ void store8_dt(void* base, long long idx, int dt, boo
             *reinterpret_cast<uint4*>(static_cast<char*>(base) + idx * 2) = u;
         }
     } else {
-        for (int i = 0; i < nvalid; ++i) st_elem(base, idx + i, dt, v[i]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)   // fixed trip count: keeps v in registers
+            if (i < nvalid) st_elem(base, idx + i, dt, v[i]);
     }
 }
 

@@ -12,11 +12,13 @@
 //
 // Traffic per element (bf16 G/G_prev, fp32 A/M, bf16 copy): 12 bytes read,
 // 12 bytes written; the norm costs no extra bytes.  Tiles of 32 rows x 64
-// columns; 256 threads, 8 consecutive elements each (16-byte loads of
-// 16-bit data, 2 x 16-byte loads of fp32).  Transposed copies go through a
-// shared-memory tile so both the reads and the writes stay coalesced.
-// Blocks own contiguous runs of tiles and flush the per-matrix sum once per
-// run (warp shuffles, then one double atomic per block and matrix).
+// columns; 256 threads, each 8 consecutive elements of one row (16-byte loads
+// of 16-bit data, 2 x 16-byte loads of fp32), all loads of a tile issued
+// before any use; at most 64 registers so that four blocks share an SM.  The
+// gradient is read once (streaming loads).  Transposed copies go through a
+// shared-memory tile so both the reads and the writes stay coalesced.  Blocks own contiguous runs
+// of tiles and flush the per-matrix sum once per run (warp shuffles, then one
+// double atomic per block and matrix).
 #include "gemm.h"
 
 namespace muon {
@@ -38,14 +40,38 @@ __device__ __forceinline__ double block_sum(double x, double* red) {
     return t;
 }
 
-__global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepParams p) {
+// 8 consecutive 16-bit elements, read once: no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+    uint4 u;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "l"(p));
+    return u;
+}
+
+template <int dt>
+__device__ __forceinline__ void load8_in(const void* base, long long idx, bool vec, int nvalid, float* out) {
+    if (vec && dt != DT_FP32) {
+        const uint4 u = ld_stream16(static_cast<const char*>(base) + idx * 2);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            out[2 * h] = dt == DT_BF16 ? unpack_lo<__nv_bfloat16>(w[h]) : unpack_lo<__half>(w[h]);
+            out[2 * h + 1] = dt == DT_BF16 ? unpack_hi<__nv_bfloat16>(w[h]) : unpack_hi<__half>(w[h]);
+        }
+    } else {
+        load8_dt(base, idx, dt, vec, nvalid, out);
+    }
+}
+
+template <int IN_DT, int X0_DT>
+__global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ PrepParams p) {
     __shared__ float stile[TC][TR + 1];
     __shared__ double red[8];
     const long long T = p.total_tiles;
     const long long per = (T + gridDim.x - 1) / gridDim.x;
     const long long t_begin = (long long)blockIdx.x * per;
     const long long t_end = min(T, t_begin + per);
-    const int r = threadIdx.x >> 3;          // row inside the tile
+    const int r = threadIdx.x >> 3;          // row r of the tile
     const int c8 = (threadIdx.x & 7) * 8;    // first of 8 columns inside the tile
     int cur = -1;
     double acc = 0.0;
@@ -66,58 +92,81 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
             cur = key;
             acc = 0.0;
         }
-        const int gr = tr * TR + r;
         const int gc0 = tc * TC + c8;
-        const int nvalid = gr < E.rows ? max(0, min(8, E.cols - gc0)) : 0;
-        const bool vec = E.vec_ok && nvalid == 8;
-        const long long idx = (long long)gr * E.cols + gc0;
-        float x[8];
-        if (p.mode == 0) {
-            float g[8], gp[8], a[8], mm[8];
-            load8_dt(E.G, idx, p.in_dt, vec, nvalid, g);
-            load8_dt(E.Gp, idx, p.in_dt, vec, nvalid, gp);
-            load8_dt(E.A, idx, DT_FP32, vec, nvalid, a);
-            load8_dt(E.M, idx, DT_FP32, vec, nvalid, mm);
+        constexpr int H = TR / 32;           // rows per thread
+        int gr[H], nvalid[H];
+        bool vec[H];
+        long long idx[H];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float d = g[i] - gp[i];                                   // step 1
-                const float an = p.beta_a * a[i] + (1.f - p.beta_a) * d;        // step 2
-                const float gt = g[i] + p.alpha * an;                            // step 3
-                const float mn = p.mu * mm[i] + gt;                              // step 4
-                a[i] = an;
-                x[i] = mn;
+        for (int h = 0; h < H; ++h) {
+            gr[h] = tr * TR + r + 32 * h;
+            nvalid[h] = gr[h] < E.rows ? max(0, min(8, E.cols - gc0)) : 0;
+            vec[h] = E.vec_ok && nvalid[h] == 8;
+            idx[h] = (long long)gr[h] * E.cols + gc0;
+        }
+        float x[H][8];
+        if (p.mode == 0) {
+            float g[H][8], gp[H][8], a[H][8], mm[H][8];
+#pragma unroll
+            for (int h = 0; h < H; ++h) {        // every load of the tile first
+                load8_in<IN_DT>(E.G, idx[h], vec[h], nvalid[h], g[h]);
+                load8_in<IN_DT>(E.Gp, idx[h], vec[h], nvalid[h], gp[h]);
+                load8_dt(E.A, idx[h], DT_FP32, vec[h], nvalid[h], a[h]);
+                load8_dt(E.M, idx[h], DT_FP32, vec[h], nvalid[h], mm[h]);
             }
-            store8_dt(E.A, idx, DT_FP32, vec, nvalid, a);
-            store8_dt(E.M, idx, DT_FP32, vec, nvalid, x);
-            store8_dt(E.Gp, idx, p.in_dt, vec, nvalid, g);
+#pragma unroll
+            for (int h = 0; h < H; ++h) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float d = g[h][i] - gp[h][i];                            // step 1
+                    const float an = p.beta_a * a[h][i] + (1.f - p.beta_a) * d;    // step 2
+                    const float gt = g[h][i] + p.alpha * an;                        // step 3
+                    const float mn = p.mu * mm[h][i] + gt;                          // step 4
+                    a[h][i] = an;
+                    x[h][i] = mn;
+                }
+                store8_dt(E.A, idx[h], DT_FP32, vec[h], nvalid[h], a[h]);
+                store8_dt(E.M, idx[h], DT_FP32, vec[h], nvalid[h], x[h]);
+                store8_dt(E.Gp, idx[h], IN_DT, vec[h], nvalid[h], g[h]);
+            }
         } else {
-            const void* X = static_cast<const char*>(E.X) + (size_t)b * E.x_stride * dt_size(p.in_dt);
-            load8_dt(X, idx, p.in_dt, vec, nvalid, x);
+            const void* X = static_cast<const char*>(E.X) + (size_t)b * E.x_stride * dt_size(IN_DT);
+#pragma unroll
+            for (int h = 0; h < H; ++h) load8_in<IN_DT>(X, idx[h], vec[h], nvalid[h], x[h]);
         }
         float part = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) part += x[i] * x[i];
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) part += x[h][i] * x[h][i];
         acc += (double)part;
 
-        void* X0 = static_cast<char*>(E.X0) + (size_t)b * E.x0_stride * dt_size(p.x0_dt);
+        void* X0 = static_cast<char*>(E.X0) + (size_t)b * E.x0_stride * dt_size(X0_DT);
         if (!E.transposed) {
             // wide view = the matrix itself; X0 rows are 16-byte aligned (ld % 8 == 0)
-            store8_dt(X0, (long long)gr * E.ld + gc0, p.x0_dt, nvalid == 8, nvalid, x);
-        } else {
-            // wide view = transpose: X0[c][r] = M[r][c]
 #pragma unroll
-            for (int i = 0; i < 8; ++i) stile[c8 + i][r] = x[i];
+            for (int h = 0; h < H; ++h)
+                store8_dt(X0, (long long)gr[h] * E.ld + gc0, X0_DT, nvalid[h] == 8, nvalid[h], x[h]);
+        } else {
+            // wide view = transpose: X0[c][r] = M[r][c], written as TR-row column segments
+#pragma unroll
+            for (int h = 0; h < H; ++h)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) stile[c8 + i][r + 32 * h] = x[h][i];
             __syncthreads();
             const int cc = threadIdx.x >> 2;          // tile column -> X0 row
-            const int rr0 = (threadIdx.x & 3) * 8;    // 8 tile rows -> X0 columns
+            const int rr0 = (threadIdx.x & 3) * (TR / 4);   // TR/4 tile rows -> X0 columns
             const int xrow = tc * TC + cc;
-            const int xcol0 = tr * TR + rr0;
             if (xrow < E.cols) {
-                float y[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) y[i] = stile[cc][rr0 + i];
-                const int nv = max(0, min(8, E.rows - xcol0));
-                store8_dt(X0, (long long)xrow * E.ld + xcol0, p.x0_dt, nv == 8, nv, y);
+                for (int h = 0; h < H; ++h) {
+                    const int xcol0 = tr * TR + rr0 + 8 * h;
+                    float y[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) y[i] = stile[cc][rr0 + 8 * h + i];
+                    const int nv = max(0, min(8, E.rows - xcol0));
+                    store8_dt(X0, (long long)xrow * E.ld + xcol0, X0_DT, nv == 8, nv, y);
+                }
             }
             __syncthreads();
         }
@@ -156,7 +205,12 @@ muon_status prep_run(PrepParams& prm, cudaStream_t stream) {
     int dev = 0, nsm = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    const long long want = (long long)nsm * 8;
+    // one wave of resident blocks: each block owns a contiguous run of tiles
+    static int occ = 0;
+    if (occ <= 0 && cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prep_kernel<DT_BF16, DT_BF16>, 256, 0) !=
+                        cudaSuccess)
+        occ = 1;
+    const long long want = (long long)nsm * (occ > 0 ? occ : 1);
     const int grid = (int)(tiles < want ? tiles : want);
     double elems = 0.0;
     for (int i = 0; i < prm.n; ++i) elems += (double)prm.e[i].rows * prm.e[i].cols * prm.e[i].count;
@@ -164,7 +218,13 @@ muon_status prep_run(PrepParams& prm, cudaStream_t stream) {
     // MONA: read G, G_prev, A, M; write A, M, G_prev, X0.  COPY: read X, write X0.
     const double per = prm.mode == 0 ? 3.0 * isz + 16.0 + xsz : (double)(isz + xsz);
     trace_begin(MUON_KERNEL_PREPASS, elems * per, stream);
-    prep_kernel<<<grid, 256, 0, stream>>>(prm);
+    // element types are compile-time in the kernel: loads and stores stay in registers
+#define MUON_PREP(I, X)                                                   \
+    if (prm.in_dt == I && prm.x0_dt == X) prep_kernel<I, X><<<grid, 256, 0, stream>>>(prm);
+    MUON_PREP(DT_BF16, DT_BF16) else MUON_PREP(DT_BF16, DT_FP16) else MUON_PREP(DT_BF16, DT_FP32)
+    else MUON_PREP(DT_FP16, DT_BF16) else MUON_PREP(DT_FP16, DT_FP16) else MUON_PREP(DT_FP16, DT_FP32)
+    else MUON_PREP(DT_FP32, DT_BF16) else MUON_PREP(DT_FP32, DT_FP16) else MUON_PREP(DT_FP32, DT_FP32)
+#undef MUON_PREP
     trace_end(stream);
     return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
