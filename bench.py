@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--ns-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--launch", default="graph", choices=["graph", "eager"],
+                    help="replay each step as a captured CUDA graph (default) or launch it eagerly")
     return ap.parse_args()
 
 
@@ -261,8 +263,9 @@ def main():
     stream = torch.cuda.current_stream(dev)
     wcode, ncode = mo._dtype_code(w_dt), mo._dtype_code(ns_dt)
 
-    def step(i):
-        mo.muon_step_batched(arrs[i % 2], wcode, ncode, w["hp"], sched, ws, d_status=status, stream=stream)
+    def step(i, st=None):
+        mo.muon_step_batched(arrs[i % 2], wcode, ncode, w["hp"], sched, ws, d_status=status,
+                             stream=st if st is not None else stream)
 
     for i in range(args.warmup):
         step(i)
@@ -270,25 +273,42 @@ def main():
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} after warm-up")
 
+    # One step per gradient set captured as a CUDA graph (the library's launches
+    # are plain stream work: capturable once its one-time set-up ran above).
+    graphs = None
+    if args.launch == "graph":
+        graphs = []
+        cap = torch.cuda.Stream(dev)
+        for i in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                step(i, torch.cuda.current_stream(dev))
+            graphs.append(g)
+        for i in range(max(2, args.warmup)):
+            graphs[i % 2].replay()
+        torch.cuda.synchronize(dev)
+
+    def run(i):
+        if graphs is not None:
+            graphs[i % 2].replay()
+        else:
+            step(i)
+
     # ---- timed region (device time, CUDA events on the step's stream)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    mo.muon_trace_enable(True)
-    mo.muon_trace_read()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for i in range(args.steps):
-        step(i)
+        run(i)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    mo.muon_trace_enable(False)
-    recs = mo.muon_trace_read()
     clk = clocks.stop()
     ms_total = ev0.elapsed_time(ev1)
     if world > 1:
@@ -299,7 +319,16 @@ def main():
     fl_step = ns_flops(shapes, ns_steps)
     value = world * fl_step * args.steps / (ms_total / 1e3) / 1e12
 
-    # ---- per-kernel figures from the trace (same timed region)
+    # ---- per-kernel device times: the same steps launched eagerly with every
+    # launch of the library bracketed by CUDA events on its stream
+    ktrace = min(args.steps, 50)
+    mo.muon_trace_enable(True)
+    mo.muon_trace_read()
+    for i in range(ktrace):
+        step(i)
+    torch.cuda.synchronize(dev)
+    mo.muon_trace_enable(False)
+    recs = mo.muon_trace_read()
     per = {}
     for kind, work, ms in recs:
         d = per.setdefault(mo.KERNEL_NAMES[kind], {"launches": 0, "work": 0.0, "ms": 0.0})
@@ -323,37 +352,56 @@ def main():
     kernels = {}
     for name, d in per.items():
         rate = d["work"] / (d["ms"] / 1e3)
-        kernels[name] = {"launches": d["launches"], "ms_total": round(d["ms"], 4),
+        kernels[name] = {"launches": d["launches"], "ms_per_step": round(d["ms"] / ktrace, 4),
                          "share": round(d["ms"] / max(1e-9, sum(x["ms"] for x in per.values())), 4),
                          ("GB/s" if name in ("prepass", "other") else "TFLOP/s"):
                              round(rate / 1e9, 1) if name in ("prepass", "other") else round(rate / 1e12, 1)}
+    launches_per_step = len(recs) / max(1, ktrace)
 
-    # ---- end to end through the public API: H2D of the step's gradients from
-    # pinned host memory, the step, D2H of the step's status word
+    # ---- end to end through the public API: each step's gradients copied from
+    # pinned host memory (on a copy stream, overlapping the previous step),
+    # the step, then a device->host read of the step's status word
     e2e = None
     if not args.no_e2e:
         host_g = [gbuf[t].cpu().pin_memory() for t in range(2)]
+        host_status = torch.zeros(1, dtype=torch.int32).pin_memory()
+        s_copy = torch.cuda.Stream(dev)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        used = [torch.cuda.Event() for _ in range(2)]
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         k = max(3, min(args.steps, 50))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+
+        def issue_copy(i):
+            with torch.cuda.stream(s_copy):
+                s_copy.wait_event(used[i % 2])          # buffer no longer read by step i-2
+                gbuf[i % 2].copy_(host_g[i % 2], non_blocking=True)
+                copied[i % 2].record(s_copy)
+
+        for e in used:
+            e.record(stream)
+        t0 = time.perf_counter()
+        issue_copy(0)
         for i in range(k):
-            gbuf[i % 2].copy_(host_g[i % 2], non_blocking=True)
-            step(i)
-            st = int(status.item())       # D2H read of the step's result
-            if st != 0:
-                raise RuntimeError(f"device status {st}")
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e_ms = e0.elapsed_time(e1)
+            if i + 1 < k:
+                issue_copy(i + 1)
+            stream.wait_event(copied[i % 2])
+            run(i)
+            used[i % 2].record(stream)
+            host_status.copy_(status, non_blocking=True)   # D2H read of the step's result
+            stream.synchronize()
+            if int(host_status.item()) != 0:
+                raise RuntimeError(f"device status {int(host_status.item())}")
+        e_s = time.perf_counter() - t0
+        e_ms = e_s * 1e3
         if world > 1:
             t = torch.tensor([e_ms], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
         e2e = {"value": world * fl_step * k / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": nel * esz, "d2h_bytes_per_step": 4, "ms_per_step": e_ms / k}
+               "h2d_bytes_per_step": nel * esz, "d2h_bytes_per_step": 4, "ms_per_step": e_ms / k,
+               "timing": "wall clock over the loop, H2D of step i+1 overlapped with step i"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -373,7 +421,10 @@ def main():
                            "l2": f"inputs larger than L2: {state_bytes / 1e9:.2f} GB of state per step",
                            "parallelism": f"{world} replica(s), each rank steps its own copy"},
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": len(recs), "clocks": clk}
+                "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clk,
+                "launch": args.launch + (" (one CUDA graph per step)" if graphs is not None else ""),
+                "kernel_timing": f"per-kernel device time from {ktrace} eagerly launched steps, each launch "
+                                 "bracketed by CUDA events on its stream"}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
