@@ -55,6 +55,47 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# Sources whose change invalidates a recorded DRAM-traffic figure.
+TRAFFIC_SOURCES = ("muon_family_optimizer_b200/csrc/gemm_tc.cu", "muon_family_optimizer_b200/csrc/muon_internal.cuh",
+                   "muon_family_optimizer_b200/csrc/epilogue.cuh", "muon_family_optimizer_b200/csrc/muon_api.cu",
+                   "muon_family_optimizer_b200/csrc/prepass.cu")
+
+
+def sources_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, ns_steps):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+    ``kernel`` from the ncu summaries under profiles/: a line
+    ``traffic-record: {json}`` written when the counters were taken.  None when
+    no record matches the workload or the kernel sources changed since."""
+    d = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(d):
+        return None, None
+    digest = sources_digest()
+    for name in sorted(os.listdir(d)):
+        if not name.endswith(".md"):
+            continue
+        with open(os.path.join(d, name)) as fh:
+            for line in fh:
+                if not line.startswith("traffic-record:"):
+                    continue
+                try:
+                    rec = json.loads(line.split(":", 1)[1])
+                except ValueError:
+                    continue
+                if (rec.get("kernel") == kernel and rec.get("workload") == workload
+                        and rec.get("ns_steps") == ns_steps and rec.get("sources") == digest):
+                    return float(rec["bytes_per_launch"]), f"profiles/{name}"
+    return None, None
+
+
 def ns_flops(shapes, ns_steps):
     """Algorithmic flops of the iteration: per step s^2 l (X X^T, half) + s^3 (A A, half) + 2 s^2 l (B X)."""
     tot = 0.0
@@ -346,8 +387,10 @@ def main():
             sustained = ms_total > 1000.0
             peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
             ach, unit, bound = d["work"] / (d["ms"] / 1e3) / 1e12, "TFLOP/s", "tensor"
+        traffic, traffic_src = recorded_traffic(dom, args.workload, ns_steps)
         roofline = {"bound": bound, "kernel": dom, "achieved": ach, "peak": peak, "unit": unit,
-                    "frac": ach / peak, "traffic": None,
+                    "frac": ach / peak, "traffic": traffic,
+                    "traffic_source": traffic_src or "no ncu record for the current kernel sources",
                     "peak_source": f"{pk_src} ({'sustained' if bound == 'tensor' and ms_total > 1000 else 'burst' if bound == 'tensor' else 'copy'})"}
     kernels = {}
     for name, d in per.items():

@@ -376,6 +376,17 @@ __device__ __forceinline__ void stage_transposed(uint8_t* stg, int lane, int c0,
     for (int c = 0; c < 32; ++c) box[(c0 + c) * 32 + lane] = from_float<T>(v[c]);
 }
 
+// One 32-column chunk of a symmetric result's box: accumulator -> epilogue ->
+// staging box (16-byte chunks c16..c16+3).
+template <typename T>
+__device__ __forceinline__ void sym_chunk(const Epilogue& E, int gi, int gj0, float sc, uint32_t tcol, uint8_t* box,
+                                          int lane, int c16, const uint4 (&c)[4]) {
+    float v[32];
+    tmem_ld_32x32b_x32(tcol, v);
+    epi_combine<T>(E, gi, gj0, sc, v, c);
+    stage32<T>(box, lane, c16, v);
+}
+
 // Barrier over the epilogue warps only (named barrier 1).
 __device__ __forceinline__ void epi_bar() {
     asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
@@ -384,6 +395,44 @@ __device__ __forceinline__ void epi_bar() {
 // Byte offset of element (r, c) (r < 32, c < 64) in a 32 x 64 16-bit staging box.
 __device__ __forceinline__ int stg_off(int r, int c) {
     return r * 128 + (((c >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
+}
+
+// The mirror of a staged 32 x 64 box of a symmetric result (rows gi0.., columns
+// gj0..): element (gi0 + i, gj0 + c) is written to (gj0 + c, gi0 + i).  Lane l
+// takes box columns l and l + 32; a column's 32 elements are read from shared
+// memory (for one i the warp reads 64 bytes of one 128-byte row: no bank
+// conflict) and written as 64 contiguous bytes of the destination row.
+template <typename T>
+__device__ __forceinline__ void mirror_box(const Epilogue& E, int m, int gi0, int gj0, int M, int N,
+                                           const uint8_t* box, int lane) {
+    T* base = static_cast<T*>(E.D) + (size_t)m * E.strideD;
+    const bool full_rows = gi0 + 32 <= M;
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+        const int c = lane + 32 * h;
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t lo = *reinterpret_cast<const uint16_t*>(box + stg_off(2 * i, c));
+            const uint32_t hi = *reinterpret_cast<const uint16_t*>(box + stg_off(2 * i + 1, c));
+            w[i] = lo | (hi << 16);
+        }
+        if (gj0 + c >= N) continue;
+        T* dst = base + (size_t)(gj0 + c) * E.ldd + gi0;
+        if (full_rows && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (gi0 + i < M) {
+                    const uint16_t e = (uint16_t)(i & 1 ? w[i >> 1] >> 16 : w[i >> 1] & 0xFFFFu);
+                    reinterpret_cast<uint16_t*>(dst)[i] = e;
+                }
+            }
+        }
+    }
 }
 
 // Diagonal 128 x 128 block of a symmetric result, held in staging boxes
@@ -634,6 +683,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             const bool has_cin = E.beta != 0.f;
             const bool diag_sym = P.sym && ti == tj && E.fin == FIN_STORE;   // uniform over the CTA
             uint4 c0[4] = {}, c1[4] = {};
+            uint4 c2[4] = {}, c3[4] = {};   // symmetric pair tiles: the second box's columns
+            bool released = false;          // accumulator buffer handed back early
             bool pf_issued = false;
             if constexpr (FIN) {
                 // the target's first block is independent of the accumulator: prefetch it
@@ -652,6 +703,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 if (has_cin) {   // independent of the accumulator: fetch before waiting for it
                     cin_fetch<T>(E, m, gi, col0, P.M, P.N, c0);
                     cin_fetch<T>(E, m, gi, col0 + 32, P.M, P.N, c1);
+                    if constexpr (C::kSymPair) {
+                        cin_fetch<T>(E, m, gi, col0 + 64, P.M, P.N, c2);
+                        cin_fetch<T>(E, m, gi, col0 + 96, P.M, P.N, c3);
+                    }
                 }
                 // warp-uniform outcome: tcgen05.ld below is warp-collective
                 const bool ok = mbar_wait(&tfull_bar[buf], tphase, abort_flag, d_status);
@@ -688,90 +743,66 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             } else if constexpr (C::kSymPair) {
                 // Symmetric result on a CTA pair: this CTA holds rows row0.. of a
                 // 256-column tile; box (q, c) = rows 32q.., columns 64c..; this warp
-                // owns box columns 2*half and 2*half + 1.  Both boxes are staged
-                // before anything is stored, so a diagonal block (tile on the
-                // diagonal: this CTA's block column `rank`) can be made exactly
-                // symmetric across the warps first.  In a diagonal tile the second
-                // CTA's first block column lies below the diagonal and is not stored
-                // (its exact mirror comes from the first CTA's band store).
+                // owns box columns 2*half and 2*half + 1, i.e. the 128-block
+                // (bi, bj) below.  Both boxes are staged before anything is stored,
+                // so a diagonal block (tile on the diagonal: this CTA's block column
+                // `rank`) can be made exactly symmetric across the warps first.  In a
+                // diagonal tile the second CTA's first block column lies below the
+                // diagonal and is not stored: its exact mirror is written by the
+                // warps holding the first block right of the diagonal (bj = bi + 1),
+                // straight from the registers that fill their staging boxes.  The
+                // accumulator buffer is handed back as soon as it has been read.
                 const bool diag_pair = ti == tj;
-                bool have[2] = {false, false};
+                const int bi = 2 * ti + (int)rank, bj = 2 * tj + half;
+                const bool mirror = P.band && bj == bi + 1;
+                const int gjb = tj * BN + 2 * half * 64;   // first column of box 2*half
+                const bool have0 = !dead && gjb < P.N;
+                const bool have1 = !dead && gjb + 64 < P.N;
                 if (!dead && stg_busy) {
                     if (lane == 0) bulk_wait_read0();
                     __syncwarp();
                 }
-#pragma unroll
-                for (int pr = 0; pr < 2; ++pr) {
-                    const int cbox = 2 * half + pr;
-                    const int gj0 = tj * BN + cbox * 64;
-                    have[pr] = !dead && gj0 < P.N;
-                    if (!have[pr]) continue;
-                    if (has_cin && pr > 0) {
-                        cin_fetch<T>(E, m, gi, gj0, P.M, P.N, c0);
-                        cin_fetch<T>(E, m, gi, gj0 + 32, P.M, P.N, c1);
-                    }
-                    const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) +
-                                          (uint32_t)(buf * BN + cbox * 64);
-                    uint8_t* box = stg_base + (quad + 4 * cbox) * C::kStgBytes;
-                    float v[32];
-                    tmem_ld_32x32b_x32(tcol, v);
-                    epi_combine<T>(E, gi, gj0, sc, v, c0);
-                    stage32<T>(box, lane, 0, v);
-                    tmem_ld_32x32b_x32(tcol + 32, v);
-                    epi_combine<T>(E, gi, gj0 + 32, sc, v, c1);
-                    stage32<T>(box, lane, 4, v);
+                const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN + 2 * half * 64);
+                uint8_t* box0 = stg_base + (quad + 4 * (2 * half)) * C::kStgBytes;
+                uint8_t* box1 = stg_base + (quad + 4 * (2 * half + 1)) * C::kStgBytes;
+                if (have0) {
+                    sym_chunk<T>(E, gi, gjb, sc, tcol, box0, lane, 0, c0);
+                    sym_chunk<T>(E, gi, gjb + 32, sc, tcol + 32, box0, lane, 4, c1);
+                }
+                if (have1) {
+                    sym_chunk<T>(E, gi, gjb + 64, sc, tcol + 64, box1, lane, 0, c2);
+                    sym_chunk<T>(E, gi, gjb + 96, sc, tcol + 96, box1, lane, 4, c3);
+                }
+                if (!dead) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+                    released = true;
                 }
                 if (diag_pair) {     // uniform over the CTA: every epilogue warp attends
                     epi_bar();
                     if (half == (int)rank) {
-#pragma unroll
-                        for (int pr = 0; pr < 2; ++pr)
-                            if (have[pr]) fix_lower<T>(stg_base, quad, 2 * (int)rank, 2 * half + pr, lane);
+                        if (have0) fix_lower<T>(stg_base, quad, 2 * (int)rank, 2 * half, lane);
+                        if (have1) fix_lower<T>(stg_base, quad, 2 * (int)rank, 2 * half + 1, lane);
                     }
                     epi_bar();
                 }
                 const bool rows_ok = row0 + quad * 32 < P.M;
                 const bool lower = diag_pair && rank == 1 && half == 0;   // below the diagonal
-#pragma unroll
-                for (int pr = 0; pr < 2; ++pr) {
-                    if (!have[pr] || !rows_ok || lower) continue;
-                    const int cbox = 2 * half + pr;
-                    const int gj0 = tj * BN + cbox * 64;
-                    uint8_t* box = stg_base + (quad + 4 * cbox) * C::kStgBytes;
+                if (rows_ok && !lower && (have0 || have1)) {
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_3d(&P.mapD, box, gj0, row0 + quad * 32, m);
+                        if (have0) tma_store_3d(&P.mapD, box0, gjb, row0 + quad * 32, m);
+                        if (have1) tma_store_3d(&P.mapD, box1, gjb + 64, row0 + quad * 32, m);
                         bulk_commit();
                     }
                     stg_busy = true;
-                    // 128-block (bi, bj) of this box; the first block right of the
-                    // diagonal is also stored transposed (exact mirror)
-                    const int bi = 2 * ti + (int)rank, bj = 2 * tj + half;
-                    if (P.band && bj == bi + 1) {
-                        if (lane == 0) bulk_wait_read0();
-                        __syncwarp();
-                        uint4 d0[4] = {}, d1[4] = {};
-                        if (has_cin) {
-                            cin_fetch<T>(E, m, gi, gj0, P.M, P.N, d0);
-                            cin_fetch<T>(E, m, gi, gj0 + 32, P.M, P.N, d1);
-                        }
-                        const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) +
-                                              (uint32_t)(buf * BN + cbox * 64);
-                        float v[32];
-                        tmem_ld_32x32b_x32(tcol, v);
-                        epi_combine<T>(E, gi, gj0, sc, v, d0);
-                        stage_transposed<T>(box, lane, 0, v);
-                        tmem_ld_32x32b_x32(tcol + 32, v);
-                        epi_combine<T>(E, gi, gj0 + 32, sc, v, d1);
-                        stage_transposed<T>(box, lane, 32, v);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_3d(&P.mapDt, box, row0 + quad * 32, gj0, m);
-                            bulk_commit();
-                        }
-                    }
+                }
+                if (mirror && rows_ok) {   // off-diagonal block: the staged boxes are final
+                    __syncwarp();
+                    if (have0) mirror_box<T>(E, m, row0 + quad * 32, gjb, P.M, P.N, box0, lane);
+                    if (have1) mirror_box<T>(E, m, row0 + quad * 32, gjb + 64, P.M, P.N, box1, lane);
                 }
             } else {
 #pragma unroll 1
@@ -837,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 }
             }
             }   // kSymPair
-            if (!dead) {
+            if (!dead && !released) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
