@@ -80,6 +80,7 @@ struct TcProblem {
     CUtensorMap mapDt;   // band: transposed stores, boxes 32 (M) x 64 (N), no swizzle
     int count, M, N, K;
     int tiles_m, tiles_n, tiles_per_mat, sym, a_sym, b_sym, band;
+    int same_ab;         // A and B are one operand: a diagonal tile loads one panel for both
     long long tile_begin;
     Epilogue epi;
 };
@@ -275,23 +276,53 @@ template <typename T>
 __device__ __forceinline__ void epi_combine(const Epilogue& E, int gi, int gj0, float sc, float (&v)[32],
                                             const uint4 (&c)[4]);
 
+// Start the copies of the target's blocks for the warp's wide rows gi0.. and
+// BN/2 wide columns from col0.  16-bit targets: all four 2 KB blocks (one
+// cp.async group each, empty groups past the matrix edge); 32-bit: block 0.
+template <typename TW, int BN>
+__device__ __forceinline__ void final_prefetch(const FinalTarget& F, int M, int N, int gi0, int col0, uint8_t* wbuf,
+                                               int lane) {
+    constexpr int kBlocks = BN / 64;
+    if constexpr (sizeof(TW) == 2) {
+#pragma unroll 1
+        for (int b = 0; b < kBlocks; ++b) {
+            if (col0 + 32 * b < N) final_move<TW, true>(F, M, N, gi0, col0 + 32 * b, wbuf + b * 2048, lane);
+            cp_async_commit();
+        }
+    } else {
+        final_move<TW, true>(F, M, N, gi0, col0, wbuf, lane);
+        cp_async_commit();
+    }
+}
+
+__device__ __forceinline__ void cp_async_wait_upto(int n) {   // at most n groups still pending
+    if (n <= 0) cp_async_wait<0>();
+    else if (n == 1) cp_async_wait<1>();
+    else if (n == 2) cp_async_wait<2>();
+    else cp_async_wait<3>();
+}
+
 // The final step for the warp's wide rows gi0.. and its BN/2 wide columns
-// from col0: four 32-column blocks, block b's target data in wbuf[b % 2].
-// Block 0's copy may already be in flight (pf_issued).
+// from col0: four 32-column blocks.  16-bit targets: block b's data in
+// wbuf + 2 KB * b, all copies started by final_prefetch (pf_issued);
+// 32-bit: wbuf[b % 2], block b + 1's copy started while block b is applied
+// (block 0's possibly by final_prefetch).
 template <typename T, typename TW, int BN>
 __device__ __forceinline__ void final_tile(const FinalTarget& F, const Epilogue& E, const FinalCtx& fc, int m,
                                            const TcProblem& P, int gi0, int col0, int gi, float sc, uint32_t tcol0,
                                            uint8_t* wbuf, int lane, bool pf_issued) {
     constexpr int kBlocks = BN / 64;                 // 32-column blocks per warp
-    constexpr int kBlockBytes = 32 * 32 * 4;
+    constexpr bool kAll = sizeof(TW) == 2;          // every block's copy started up front
+    constexpr int kBlockBytes = kAll ? 32 * 32 * 2 : 32 * 32 * 4;
     const bool staged = F.vec;                      // aligned target: go through shared memory
     const uint4 none[4] = {};
+    if (kAll && staged && F.wupd && !pf_issued) final_prefetch<TW, BN>(F, P.M, P.N, gi0, col0, wbuf, lane);
 #pragma unroll 1
     for (int b = 0; b < kBlocks; ++b) {
         const int gj0 = col0 + 32 * b;
         if (gj0 >= P.N) break;                       // warp-uniform
-        uint8_t* cur = wbuf + (b & 1) * kBlockBytes;
-        if (staged && F.wupd) {
+        uint8_t* cur = wbuf + (kAll ? b : (b & 1)) * kBlockBytes;
+        if (!kAll && staged && F.wupd) {
             if (b == 0 && !pf_issued) {
                 final_move<TW, true>(F, P.M, P.N, gi0, gj0, cur, lane);
                 cp_async_commit();
@@ -310,7 +341,9 @@ __device__ __forceinline__ void final_tile(const FinalTarget& F, const Epilogue&
             continue;
         }
         if (F.wupd) {
-            if (b + 1 < kBlocks && gj0 + 32 < P.N) cp_async_wait<1>(); else cp_async_wait<0>();
+            if (kAll) cp_async_wait_upto(kBlocks - 1 - b);
+            else if (b + 1 < kBlocks && gj0 + 32 < P.N) cp_async_wait<1>();
+            else cp_async_wait<0>();
         }
         __syncwarp();                                // this block's copy visible to every lane
         final_apply<TW>(F, fc, cur, v, lane);
@@ -520,6 +553,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             uint32_t phase = 0;
             uint32_t armed = 0;          // bit s: stage s has been armed at least once
             uint32_t armed_parity = 0;   // bit s: parity of the phase stage s was last armed in
+            constexpr int kBCols = PAIR ? BN / 2 : BN;
+            auto chunks_of = [&](int N, int c0) { return max(0, min(kBCols / 64, (N - c0 + 63) / 64)); };
             for (long long t = unit; t < p.total_tiles && !*abort_flag; t += nunits) {
                 int pi, m, ti, tj;
                 decode_tile(p, t, pi, m, ti, tj);
@@ -528,14 +563,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 const int rows0 = ti * C::kRows + (int)rank * BM;   // this CTA's rows of A
                 // this CTA's columns of the result (rows of a K-major B, columns of an
                 // MN-major B panel) and, for a panel, the 64-wide boxes they span
-                constexpr int kBCols = PAIR ? BN / 2 : BN;
                 const int bcol0 = tj * BN + (int)rank * kBCols;
-                auto chunks = [&](int c0) { return max(0, min(kBCols / 64, (P.N - c0 + 63) / 64)); };
+                auto chunks = [&](int c0) { return chunks_of(P.N, c0); };
                 const int nchunk = B_MN ? chunks(bcol0) : kBCols / 64;
-                uint32_t bytes = C::kABytes + (B_MN ? nchunk * 64 * BK * 2 : C::kBBytes);
+                // A diagonal tile of a product whose operands are one matrix (X X^T,
+                // S S) needs the same rows as A and as B: one panel serves both.
+                const bool one_panel = !B_MN && P.same_ab && ti == tj;
+                uint32_t bytes = C::kABytes + (B_MN ? nchunk * 64 * BK * 2 : (one_panel ? 0 : C::kBBytes));
                 if (PAIR) {   // the leader's barrier counts both CTAs' boxes
                     bytes = B_MN ? 2 * C::kABytes + (chunks(tj * BN) + chunks(tj * BN + kBCols)) * 64 * BK * 2
-                                 : 2 * (C::kABytes + C::kBBytes);
+                                 : 2 * (C::kABytes + (one_panel ? 0 : C::kBBytes));
                 }
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, d_status)) break;
@@ -562,6 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     }
                     if (B_MN) {
                         for (int c = 0; c < nchunk; ++c) load(&P.mapB, sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK);
+                    } else if (one_panel) {
+                        // B is the A panel just loaded
                     } else if (bt) {
                         for (int c = 0; c < kBCols / 64; ++c)
                             load(&P.mapBt, sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK);
@@ -609,6 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 if (!mbar_wait(&tempty_bar[buf], tphase ^ 1, abort_flag, d_status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+                const bool one_panel = !B_MN && P.same_ab && ti == tj;   // B read from the A panel
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, abort_flag, d_status)) { ok = false; break; }
                     tc_fence_after();
@@ -616,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     const bool bm = B_MN || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj));   // B block MN-major
                     const uint32_t idesc = idesc0 | (at ? 1u << 15 : 0u) | (bm ? 1u << 16 : 0u);
                     const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
-                    const uint32_t sb = sa + C::kABytes;
+                    const uint32_t sb = one_panel ? sa : sa + C::kABytes;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
                         // K-major: the k-th 16-element slice sits 32 bytes further in each
@@ -691,10 +731,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 if (!dead && row0 + quad * 32 < P.M) {
                     const FinalTarget F = final_target(E, fc, m);
                     if (F.wupd && F.vec && col0 < P.N) {
-                        if (F.dt == DT_BF16) final_move<__nv_bfloat16, true>(F, P.M, P.N, row0 + quad * 32, col0, wbuf, lane);
-                        else if (F.dt == DT_FP16) final_move<__half, true>(F, P.M, P.N, row0 + quad * 32, col0, wbuf, lane);
-                        else final_move<float, true>(F, P.M, P.N, row0 + quad * 32, col0, wbuf, lane);
-                        cp_async_commit();
+                        if (F.dt == DT_BF16) final_prefetch<__nv_bfloat16, BN>(F, P.M, P.N, row0 + quad * 32, col0, wbuf, lane);
+                        else if (F.dt == DT_FP16) final_prefetch<__half, BN>(F, P.M, P.N, row0 + quad * 32, col0, wbuf, lane);
+                        else final_prefetch<float, BN>(F, P.M, P.N, row0 + quad * 32, col0, wbuf, lane);
                         pf_issued = true;
                     }
                 }
@@ -996,6 +1035,7 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         P.a_sym = o.a_sym;
         P.b_sym = sym ? o.b_sym : 0;
         P.band = sym ? (pair ? 1 : o.band) : 0;
+        P.same_ab = sym && o.A == o.B && o.lda == o.ldb && o.strideA == o.strideB && o.a_sym == o.b_sym;
         // A operand: M rows x K (K contiguous); a symmetric A is also read transposed
         if (!encode_map(&P.mapA, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, BK, BM)) return MUON_ERR_CUDA;
         if (o.a_sym && !encode_map(&P.mapAt, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, 64, BK))
