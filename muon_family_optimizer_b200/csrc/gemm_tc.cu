@@ -721,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             const int gi = row0 + row;
             const int col0 = tj * BN + half * (BN / 2);
             const bool has_cin = E.beta != 0.f;
-            const bool diag_sym = P.sym && ti == tj && E.fin == FIN_STORE;   // uniform over the CTA
+            const bool diag_sym = P.sym && !P.same_ab && ti == tj && E.fin == FIN_STORE;   // uniform over the CTA
             uint4 c0[4] = {}, c1[4] = {};
             uint4 c2[4] = {}, c3[4] = {};   // symmetric pair tiles: the second box's columns
             bool released = false;          // accumulator buffer handed back early
@@ -818,7 +818,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
                     released = true;
                 }
-                if (diag_pair) {     // uniform over the CTA: every epilogue warp attends
+                // A product of one operand with itself (X X^T, S S with S stored exactly
+                // symmetric) is formed at (i, j) and (j, i) from the same products in the
+                // same order, so its diagonal block is already exactly symmetric; a
+                // product of two matrices (h Q, (h R) h) is symmetrised here.
+                if (diag_pair && !P.same_ab) {     // uniform over the CTA: every epilogue warp attends
                     epi_bar();
                     if (half == (int)rank) {
                         if (have0) fix_lower<T>(stg_base, quad, 2 * (int)rank, 2 * half, lane);

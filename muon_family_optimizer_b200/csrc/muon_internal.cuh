@@ -309,13 +309,6 @@ __device__ __forceinline__ void cluster_sync() {
 }
 // Box load into this CTA's shared memory whose completion is counted on an
 // mbarrier of the pair's leader CTA (`bar_cluster`: shared::cluster address).
-// L2 prefetch of one box of a tiled tensor map (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
-                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z)
-                 : "memory");
-}
-
 __device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap* map, uint32_t bar_cluster, void* smem_dst,
                                                  int x, int y, int z) {
     asm volatile(
