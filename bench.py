@@ -105,6 +105,15 @@ def ns_flops(shapes, ns_steps):
     return tot
 
 
+def ns_flops_dense(shapes, ns_steps):
+    """Dense-equivalent flops: both symmetric products counted in full, 4 s^2 l + 2 s^3 per step."""
+    tot = 0.0
+    for r, c in shapes:
+        s, l = min(r, c), max(r, c)
+        tot += ns_steps * (4.0 * s * s * l + 2.0 * float(s) ** 3)
+    return tot
+
+
 def describe(name, w):
     from collections import Counter
     cnt = Counter((min(r, c), max(r, c)) for r, c in w["shapes"])
@@ -463,6 +472,8 @@ def main():
                            "state_bytes": state_bytes,
                            "l2": f"inputs larger than L2: {state_bytes / 1e9:.2f} GB of state per step",
                            "parallelism": f"{world} replica(s), each rank steps its own copy"},
+                "dense_equivalent": {"value": world * ns_flops_dense(shapes, ns_steps) * args.steps / (ms_total / 1e3) / 1e12,
+                                     "unit": "TFLOP/s", "note": "symmetric products counted in full (not the headline)"},
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clk,
                 "launch": args.launch + (" (one CUDA graph per step)" if graphs is not None else ""),
