@@ -63,6 +63,13 @@ def configure(L):
                                    ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                    ctypes.c_int, _D, ctypes.c_double, ctypes.c_double,
                                    ctypes.c_int]
+    L.oracle_mona_lite.argtypes = [ctypes.c_longlong, _D, _D, _D, ctypes.c_double, ctypes.c_double,
+                                   ctypes.c_double, ctypes.c_int]
+    L.oracle_muon_lite_step.argtypes = [ctypes.c_int, ctypes.c_int, _D, _D, _D, _D, _D,
+                                        ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                        ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                        ctypes.c_int, _D, ctypes.c_double, ctypes.c_double,
+                                        ctypes.c_int, ctypes.c_int]
     return L
 
 
@@ -202,3 +209,27 @@ def muon_step(W, G, Gp, A, M, *, mu, eta, lam, gamma, beta_a, alpha,
                            mu, eta, lam, gamma, beta_a, alpha, n, _p(c), eps, f,
                            int(round_to))
     return {"W": W, "G_prev": Gp, "A": A, "M": M, "O": O}
+
+
+def mona_lite(G, B, M, beta_a, alpha, mu, round_b=True):
+    """MONA-Lite elementwise pass (one buffer B instead of G_prev and A, B in
+    bfloat16 when round_b); returns (B', M') as new arrays."""
+    G = _f64(G)
+    B, M = _f64(B).copy(), _f64(M).copy()
+    assert G.shape == B.shape == M.shape
+    lib().oracle_mona_lite(G.size, _p(G), _p(B), _p(M), beta_a, alpha, mu, 1 if round_b else 0)
+    return B, M
+
+
+def muon_lite_step(W, G, B, M, *, mu, eta, lam, gamma, beta_a, alpha,
+                   coeffs, eps=1e-7, f=1.0, round_to=ROUND_NONE, round_b=True):
+    """One MONA-Lite step for one matrix; returns dict of new W, B, M and O."""
+    W, B, M = (_f64(v).copy() for v in (W, B, M))
+    G = _f64(G)
+    rows, cols = W.shape
+    O = np.empty_like(W)
+    c, n = _coeffs(coeffs)
+    lib().oracle_muon_lite_step(rows, cols, _p(W), _p(G), _p(B), _p(M), _p(O),
+                                mu, eta, lam, gamma, beta_a, alpha, n, _p(c), eps, f,
+                                int(round_to), 1 if round_b else 0)
+    return {"W": W, "B": B, "M": M, "O": O}

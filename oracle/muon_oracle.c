@@ -400,6 +400,34 @@ void oracle_orthogonalise(const double* M, int rows, int cols, double* O,
 }
 
 /* ------------------------------------------------------------------------ */
+/* MONA-Lite, [MONA] section "Efficientie en Implementatie": the auxiliary   */
+/* state is kept in bfloat16 and the gradient difference is formed in place  */
+/* instead of from a stored previous gradient.  Reading taken (the page     */
+/* gives no formulas): step 2 rewritten with the one buffer                 */
+/*   B_{k-1} = beta_a A_{k-1} - (1-beta_a) G_{k-1}                           */
+/* so that                                                                   */
+/*   A_k  = B_{k-1} + (1-beta_a) G_k          (= step 2 exactly)             */
+/*   Gt   = G_k + alpha A_k                   (step 3)                       */
+/*   M_k  = mu M_{k-1} + Gt                   (step 4)                       */
+/*   B_k  = beta_a A_k - (1-beta_a) G_k       (for the next step)            */
+/* B starts at 0 (A_0 = G_prev = 0).  round_b != 0 stores B rounded to       */
+/* bfloat16 (RNE), the page's precision for the auxiliary state; with      */
+/* round_b == 0 the sequence of M equals oracle_mona's exactly (algebra).   */
+/* ------------------------------------------------------------------------ */
+void oracle_mona_lite(long long n, const double* G, double* B, double* M,
+                      double beta_a, double alpha, double mu, int round_b)
+{
+    for (long long i = 0; i < n; ++i) {
+        double An = B[i] + (1.0 - beta_a) * G[i];
+        double Gt = G[i] + alpha * An;
+        double Mn = mu * M[i] + Gt;
+        double Bn = beta_a * An - (1.0 - beta_a) * G[i];
+        M[i] = Mn;
+        B[i] = round_b ? oracle_round_bf16(Bn) : Bn;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* One full MONA/Muon step for one matrix parameter, [MONA] section 2:       */
 /* elementwise pre-pass, orthogonalisation of M', decoupled weight update.   */
 /* W, Gp, A, M are updated in place; O (rows x cols) receives the            */
@@ -415,6 +443,24 @@ void oracle_muon_step(int rows, int cols, double* W, const double* G, double* Gp
 {
     long long n = (long long)rows * cols;
     oracle_mona(n, G, Gp, A, M, beta_a, alpha, mu);
+    oracle_orthogonalise(M, rows, cols, O, 0, n_steps, coeffs, NULL, 0, f, eps, round_kind);
+    oracle_weight_update(n, W, O, eta, gamma, lambda);
+}
+
+/* ------------------------------------------------------------------------ */
+/* One MONA-Lite step for one matrix parameter: oracle_mona_lite (B in      */
+/* bfloat16 when round_b), then the same orthogonalisation and update as     */
+/* oracle_muon_step.                                                         */
+/* ------------------------------------------------------------------------ */
+void oracle_muon_lite_step(int rows, int cols, double* W, const double* G, double* B,
+                           double* M, double* O,
+                           double mu, double eta, double lambda, double gamma,
+                           double beta_a, double alpha,
+                           int n_steps, const double* coeffs, double eps, double f,
+                           int round_kind, int round_b)
+{
+    long long n = (long long)rows * cols;
+    oracle_mona_lite(n, G, B, M, beta_a, alpha, mu, round_b);
     oracle_orthogonalise(M, rows, cols, O, 0, n_steps, coeffs, NULL, 0, f, eps, round_kind);
     oracle_weight_update(n, W, O, eta, gamma, lambda);
 }

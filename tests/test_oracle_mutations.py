@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+import test_oracle_lite as lite
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "muon_oracle.c")
@@ -26,7 +27,8 @@ MUTATIONS = [
      "mat_mul(X, X, A, s, s, s);", [lambda: pins.test_ns_poly_closed_form_through_svd((8, 8))]),
     ("mona_difference_sign", "double D = G[i] - Gp[i];", "double D = Gp[i] - G[i];",
      [pins.test_mona_hand_example]),
-    ("mona_uses_old_buffer", "double Gt = G[i] + alpha * An;", "double Gt = G[i] + alpha * A[i];",
+    ("mona_uses_old_buffer", "(1.0 - beta_a) * D;\n        double Gt = G[i] + alpha * An;",
+     "(1.0 - beta_a) * D;\n        double Gt = G[i] + alpha * A[i];",
      [pins.test_mona_hand_example]),
     ("decay_sign", "W[i] = W[i] - eta * (gamma * O[i] + lambda * W[i]);",
      "W[i] = W[i] - eta * (gamma * O[i] - lambda * W[i]);", [pins.test_weight_update_hand_example]),
@@ -38,6 +40,11 @@ MUTATIONS = [
      [lambda: pins.test_polar_matches_lapack_svd((16, 32))]),
     ("orientation_not_transposed_back", "else transpose(X, O, cols, rows);",
      "else memcpy(O, X, sizeof(double) * sl);", [pins.test_orthogonalise_orientation_and_scale]),
+    ("lite_b_update_sign", "double Bn = beta_a * An - (1.0 - beta_a) * G[i];",
+     "double Bn = beta_a * An + (1.0 - beta_a) * G[i];", [lite.test_mona_lite_hand_example]),
+    ("lite_difference_weight", "double An = B[i] + (1.0 - beta_a) * G[i];",
+     "double An = B[i] + beta_a * G[i];",
+     [lambda: lite.test_mona_lite_equals_mona_without_rounding(0.9, 0.5, 0.95)]),
     ("bf16_precision", "return round_to_format(x, 8, -126, 0x1.fep127);",
      "return round_to_format(x, 7, -126, 0x1.fep127);",
      [pins.test_round_bf16_matches_torch_on_float32_values]),
