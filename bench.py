@@ -43,6 +43,11 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--launch", default="graph", choices=["graph", "eager"],
                     help="replay each step as a captured CUDA graph (default) or launch it eagerly")
+    ap.add_argument("--variant", default="mona", choices=["mona", "lite"],
+                    help="mona: G_prev and A state (default); lite: MONA-Lite, one bfloat16 buffer B")
+    ap.add_argument("--route", default="step", choices=["step", "gram", "direct"],
+                    help="step: the optimizer step (default); gram / direct: the orthogonalisation alone "
+                         "(gram_polar / ns_polar, converged schedule) of the workload's matrices, one batch per shape")
     return ap.parse_args()
 
 
@@ -259,6 +264,82 @@ def run_reference(args, w, ns_steps):
 
 # ------------------------------------------------------------------ GPU arm
 
+def run_polar_route(args, w):
+    """Time gram_polar (Gram route with restarts and the 1.05 divisor) or ns_polar
+    with the same converged schedule on the workload's matrices (log-spaced
+    spectra, condition numbers 1e1..1e3), one call per shape batch per step.
+    Work is the library's own algorithmic flop count of the launches."""
+    import torch
+    import muon_family_optimizer_b200 as mo
+    from collections import OrderedDict
+    from muon_family_optimizer_b200 import synthetic as syn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    dt = w["ns_dtype"]
+    groups = OrderedDict()
+    for j, (r, c) in enumerate(w["shapes"]):
+        groups.setdefault((r, c), []).append(j)
+    kappas = [1e1, 1e2, 1e3]
+    batches = []
+    for (r, c), idx in groups.items():
+        X = torch.stack([syn.log_spectrum(r, c, kappas[i % 3], 4000 + j, device=dev) for i, j in enumerate(idx)])
+        X = X.to(dt).contiguous()
+        size = (mo.gram_polar_workspace_size if args.route == "gram" else mo.ns_polar_workspace_size)(
+            len(idx), r, c, mo._dtype_code(dt))
+        batches.append((X, torch.empty_like(X), torch.empty(size, dtype=torch.uint8, device=dev)))
+    sched = mo.converged_schedule()
+    fn = mo.gram_polar if args.route == "gram" else mo.ns_polar
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(st=None):
+        for X, out, ws in batches:
+            fn(X, out, sched, ws, d_status=status, stream=st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after warm-up")
+    mo.muon_trace_enable(True)
+    mo.muon_trace_read()
+    step()
+    torch.cuda.synchronize(dev)
+    mo.muon_trace_enable(False)
+    recs = mo.muon_trace_read()
+    work = sum(wk for k, wk, ms in recs if k in (mo.KERNEL_SYM, mo.KERNEL_UPD))
+    stream = torch.cuda.current_stream(dev)
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    with torch.cuda.graph(g, stream=cap):
+        step(torch.cuda.current_stream(dev))
+    for _ in range(max(2, args.warmup)):
+        g.replay()
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    groups_desc = " + ".join(f"{len(v)} x {r}x{c}" for (r, c), v in groups.items())
+    line = {"metric": METRIC, "value": work / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": {torch.bfloat16: "bf16", torch.float16: "fp16", torch.float32: "fp32"}[dt],
+            "data": "synthetic (log-spaced spectra, condition numbers 1e1, 1e2, 1e3)",
+            "config": {"workload": f"{w['name']}: {groups_desc}, {'gram_polar' if args.route == 'gram' else 'ns_polar'}"
+                                   " with the converged schedule (8 quintic + 6 cubic, restarts 3/5/7, divisor 1.05)",
+                       "route": args.route, "launches_per_step": len(recs), "work_flops_per_step": work},
+            "gpu_launches": len(recs) * args.steps, "clocks": clk, "launch": "graph (one CUDA graph per step)"}
+    print(json.dumps(line), flush=True)
+    del g
+
+
 def main():
     args = parse()
     from muon_family_optimizer_b200 import synthetic as syn
@@ -267,6 +348,8 @@ def main():
     ns_steps = args.ns_steps
     if args.impl == "reference":
         return run_reference(args, w, ns_steps)
+    if args.route != "step":
+        return run_polar_route(args, w)
 
     import torch
     import torch.distributed as dist
@@ -296,26 +379,33 @@ def main():
         if key not in cache:
             cache[key] = [syn.gradient(args.workload, j, t, r, c, device=dev) for t in range(2)]
         W = syn.initial_weight(args.workload, j, r, c, device=dev).to(w_dt)
-        Gp = cache[key][1].to(w_dt).contiguous()
-        A = torch.zeros(r, c, dtype=torch.float32, device=dev)
         M = torch.zeros(r, c, dtype=torch.float32, device=dev)
+        if args.variant == "lite":
+            B = (cache[key][1] * -0.01).to(torch.bfloat16).contiguous()
+        else:
+            Gp = cache[key][1].to(w_dt).contiguous()
+            A = torch.zeros(r, c, dtype=torch.float32, device=dev)
         for t in range(2):
             g = gbuf[t][off:off + r * c].view(r, c)
             sign = torch.randint(0, 2, (1, c), device=dev, dtype=torch.int8).float() * 2 - 1
             g.copy_(cache[key][t] * sign)
-            params[t].append(dict(W=W, G=g, G_prev=Gp, A=A, M=M))
+            params[t].append(dict(W=W, G=g, B=B, M=M) if args.variant == "lite" else
+                             dict(W=W, G=g, G_prev=Gp, A=A, M=M))
         off += r * c
     del cache
-    arrs = [mo.make_params(p) for p in params]
+    lite = args.variant == "lite"
+    arrs = [(mo.make_lite_params if lite else mo.make_params)(p) for p in params]
     sched = mo.quintic_schedule(ns_steps)
-    ws = torch.empty(mo.muon_workspace_size(arrs[0], mo._dtype_code(ns_dt)), dtype=torch.uint8, device=dev)
+    ws = torch.empty((mo.muon_lite_workspace_size if lite else mo.muon_workspace_size)(arrs[0], mo._dtype_code(ns_dt)),
+                     dtype=torch.uint8, device=dev)
+    step_fn = mo.muon_lite_step_batched if lite else mo.muon_step_batched
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     wcode, ncode = mo._dtype_code(w_dt), mo._dtype_code(ns_dt)
 
     def step(i, st=None):
-        mo.muon_step_batched(arrs[i % 2], wcode, ncode, w["hp"], sched, ws, d_status=status,
-                             stream=st if st is not None else stream)
+        step_fn(arrs[i % 2], wcode, ncode, w["hp"], sched, ws, d_status=status,
+                stream=st if st is not None else stream)
 
     for i in range(args.warmup):
         step(i)
@@ -461,13 +551,15 @@ def main():
 
     if rank == 0:
         groups, _ = describe(args.workload, w)
-        state_bytes = nel * (3 * esz + 8)
+        # W, G, G_prev (w dtype), A, M (fp32); MONA-Lite: W, G, B (bf16), M
+        state_bytes = nel * (2 * esz + 2 + 4) if lite else nel * (3 * esz + 8)
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": {torch.bfloat16: "bf16", torch.float16: "fp16",
                                                torch.float32: "fp32"}[ns_dt],
                 "data": "synthetic (seeded; shapes of the named model, random values)",
-                "config": {"workload": f"{args.workload}: {groups} (wide view s x l)", "elements": nel,
+                "config": {"workload": f"{args.workload}{' (MONA-Lite)' if lite else ''}: {groups} (wide view s x l)",
+                           "variant": args.variant, "elements": nel,
                            "ns_steps": ns_steps, "w_dtype": str(w_dt).replace("torch.", ""),
                            "state_bytes": state_bytes,
                            "l2": f"inputs larger than L2: {state_bytes / 1e9:.2f} GB of state per step",

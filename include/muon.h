@@ -152,6 +152,43 @@ MUON_API muon_status muon_step_batched(const muon_param* params, int n, muon_dty
                               int* d_status, muon_stream_t stream);
 
 /*
+ * MONA-Lite ([MONA] section "Efficientie en Implementatie"): the auxiliary
+ * state kept in bfloat16 and the gradient difference formed in place, without
+ * a stored previous gradient.  One buffer per parameter replaces G_prev and A:
+ *     B = beta_a A - (1 - beta_a) G      (of the previous step; 0 at the start)
+ * so that step 2 reads A_k = B + (1 - beta_a) G_k, and after step 4
+ *     B <- beta_a A_k - (1 - beta_a) G_k   (rounded to bfloat16, RNE).
+ * Unrounded this is exactly steps 1-4; the state shrinks from G_prev + A to
+ * one bfloat16 matrix and the fused pass from 24 to 16 bytes per element
+ * (bf16 W/G, fp32 M, 16-bit copy).
+ */
+typedef struct {
+    int rows, cols;    /* >= 1 */
+    void* W;           /* rows x cols, w_dtype, updated in place */
+    const void* G;     /* rows x cols, w_dtype, this step's gradient (read only) */
+    void* B;           /* rows x cols, bfloat16 auxiliary buffer, updated in place (zero initially) */
+    float* M;          /* rows x cols, fp32 momentum, updated in place */
+    float gamma;       /* per-matrix gamma; NaN means "use hparams.gamma" */
+    float* O_out;      /* optional rows x cols fp32: receives O; NULL to skip */
+} muon_lite_param;
+
+/* Bytes of workspace muon_lite_step_batched needs (only rows/cols are read). */
+MUON_API muon_status muon_lite_workspace_size(const muon_lite_param* params, int n, muon_dtype ns_dtype,
+                                     size_t* bytes);
+
+/*
+ * One MONA-Lite optimizer step for n matrix parameters: the fused pass above
+ * (B and M updated in place, the norm of the new M, its 16-bit wide view),
+ * then the same iteration and fused weight update as muon_step_batched, with
+ * the same arguments, errors and ownership rules (B takes the place of G_prev
+ * and A).
+ */
+MUON_API muon_status muon_lite_step_batched(const muon_lite_param* params, int n, muon_dtype w_dtype,
+                                   muon_dtype ns_dtype, const muon_hparams* hp,
+                                   const muon_schedule* sched, void* workspace, size_t ws_bytes,
+                                   int* d_status, muon_stream_t stream);
+
+/*
  * Bytes of workspace ns_polar / gram_polar need for a batch of rows x cols
  * matrices in `dtype`.
  */

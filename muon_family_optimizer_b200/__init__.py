@@ -53,6 +53,12 @@ class Param(ctypes.Structure):
                 ("M", ctypes.c_void_p), ("gamma", ctypes.c_float), ("O_out", ctypes.c_void_p)]
 
 
+class LiteParam(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("cols", ctypes.c_int), ("W", ctypes.c_void_p),
+                ("G", ctypes.c_void_p), ("B", ctypes.c_void_p), ("M", ctypes.c_void_p),
+                ("gamma", ctypes.c_float), ("O_out", ctypes.c_void_p)]
+
+
 KERNEL_PREPASS, KERNEL_SYM, KERNEL_UPD, KERNEL_SIMT, KERNEL_OTHER = range(5)
 KERNEL_NAMES = {KERNEL_PREPASS: "prepass", KERNEL_SYM: "tc_sym", KERNEL_UPD: "tc_upd",
                 KERNEL_SIMT: "simt", KERNEL_OTHER: "other"}
@@ -85,6 +91,12 @@ def lib():
         L.muon_step_batched.argtypes = [ctypes.POINTER(Param), ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.POINTER(HParams), ctypes.POINTER(Schedule), vp,
                                         ctypes.c_size_t, vp, vp]
+        L.muon_lite_workspace_size.restype = st
+        L.muon_lite_workspace_size.argtypes = [ctypes.POINTER(LiteParam), ctypes.c_int, ctypes.c_int, sz]
+        L.muon_lite_step_batched.restype = st
+        L.muon_lite_step_batched.argtypes = [ctypes.POINTER(LiteParam), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.POINTER(HParams), ctypes.POINTER(Schedule), vp,
+                                             ctypes.c_size_t, vp, vp]
         for name in ("ns_polar_workspace_size", "gram_polar_workspace_size"):
             f = getattr(L, name)
             f.restype = st
@@ -183,6 +195,43 @@ def muon_step_batched(params, w_dtype, ns_dtype, hp, schedule, workspace, d_stat
     _check(lib().muon_step_batched(arr, len(arr), int(w_dtype), int(ns_dtype), ctypes.byref(h),
                                    ctypes.byref(schedule), _ptr(workspace), workspace.numel(),
                                    _ptr(d_status), _stream_ptr(stream)), "muon_step_batched")
+
+
+def make_lite_params(params):
+    """params: list of dicts with torch tensors W, G, B (bfloat16), M (+ optional gamma, O_out)."""
+    import torch
+    arr = (LiteParam * len(params))()
+    for i, p in enumerate(params):
+        W = p["W"]
+        rows, cols = W.shape
+        for k in ("W", "G", "B", "M"):
+            t = p[k]
+            if tuple(t.shape) != (rows, cols) or not t.is_contiguous():
+                raise ValueError(f"param {i}: {k} must be a contiguous {rows}x{cols} tensor")
+        if p["B"].dtype != torch.bfloat16 or p["M"].dtype != torch.float32:
+            raise ValueError(f"param {i}: B must be bfloat16 and M float32")
+        arr[i] = LiteParam(rows, cols, W.data_ptr(), p["G"].data_ptr(), p["B"].data_ptr(), p["M"].data_ptr(),
+                           float(p.get("gamma", math.nan)),
+                           p["O_out"].data_ptr() if p.get("O_out") is not None else None)
+    return arr
+
+
+def muon_lite_workspace_size(params, ns_dtype):
+    arr = params if isinstance(params, ctypes.Array) else make_lite_params(params)
+    out = ctypes.c_size_t(0)
+    _check(lib().muon_lite_workspace_size(arr, len(arr), int(ns_dtype), ctypes.byref(out)),
+           "muon_lite_workspace_size")
+    return out.value
+
+
+def muon_lite_step_batched(params, w_dtype, ns_dtype, hp, schedule, workspace, d_status=None, stream=None):
+    """One MONA-Lite step on every parameter (see include/muon.h): B (bfloat16)
+    replaces G_prev and A."""
+    arr = params if isinstance(params, ctypes.Array) else make_lite_params(params)
+    h = HParams(hp["mu"], hp["eta"], hp["lambda"], hp["gamma"], hp["beta_a"], hp["alpha"])
+    _check(lib().muon_lite_step_batched(arr, len(arr), int(w_dtype), int(ns_dtype), ctypes.byref(h),
+                                        ctypes.byref(schedule), _ptr(workspace), workspace.numel(),
+                                        _ptr(d_status), _stream_ptr(stream)), "muon_lite_step_batched")
 
 
 def ns_polar_workspace_size(batch, rows, cols, dtype):

@@ -53,7 +53,8 @@ struct PrepParams {
     PrepEntry e[kMaxPrep];
     int n;
     long long total_tiles;
-    int in_dt, x0_dt, mode;   // mode 0 = MONA pre-pass, 1 = copy (normalisation input of ns/gram_polar)
+    int in_dt, x0_dt, mode;   // mode 0 = MONA pre-pass, 1 = copy (normalisation input of ns/gram_polar),
+                              // 2 = MONA-Lite (Gp holds the bfloat16 buffer B, A unused)
     float beta_a, alpha, mu;
     double* sumsq;
 };

@@ -399,14 +399,15 @@ muon_status muon_workspace_size(const muon_param* params, int n, muon_dtype ns_d
     return MUON_OK;
 }
 
-muon_status muon_step_batched(const muon_param* params, int n, muon_dtype w_dtype, muon_dtype ns_dtype,
-                              const muon_hparams* hp, const muon_schedule* sched, void* workspace,
-                              size_t ws_bytes, int* d_status, muon_stream_t stream) {
+// lite: MONA-Lite state (G_prev holds the bfloat16 buffer B, A is unused).
+static muon_status step_common(const muon_param* params, int n, muon_dtype w_dtype, muon_dtype ns_dtype,
+                               const muon_hparams* hp, const muon_schedule* sched, void* workspace,
+                               size_t ws_bytes, int* d_status, muon_stream_t stream, bool lite) {
     if (!valid_dtype(w_dtype) || !valid_dtype(ns_dtype) || !hp) return MUON_ERR_INVALID_ARG;
     muon_status st = check_params(params, n);
     if (st != MUON_OK) return st;
     for (int i = 0; i < n; ++i)
-        if (!params[i].W || !params[i].G || !params[i].G_prev || !params[i].A || !params[i].M)
+        if (!params[i].W || !params[i].G || !params[i].G_prev || (!lite && !params[i].A) || !params[i].M)
             return MUON_ERR_INVALID_ARG;
     st = check_schedule(sched);
     if (st != MUON_OK) return st;
@@ -426,7 +427,7 @@ muon_status muon_step_batched(const muon_param* params, int n, muon_dtype w_dtyp
     // 1. fused MONA pre-pass + norms + wide-view copies
     PrepParams pp;
     memset(&pp, 0, sizeof(pp));
-    pp.in_dt = w_dtype; pp.x0_dt = ns_dtype; pp.mode = 0;
+    pp.in_dt = w_dtype; pp.x0_dt = ns_dtype; pp.mode = lite ? 2 : 0;
     pp.beta_a = hp->beta_a; pp.alpha = hp->alpha; pp.mu = hp->mu;
     pp.sumsq = sumsq;
     const size_t in_sz = dt_size(w_dtype);
@@ -481,6 +482,38 @@ muon_status muon_step_batched(const muon_param* params, int n, muon_dtype w_dtyp
         fins.push_back(f);
     }
     return run_direct(R, L, workspace, sched, fins, FIN_WUPD);
+}
+
+muon_status muon_step_batched(const muon_param* params, int n, muon_dtype w_dtype, muon_dtype ns_dtype,
+                              const muon_hparams* hp, const muon_schedule* sched, void* workspace,
+                              size_t ws_bytes, int* d_status, muon_stream_t stream) {
+    return step_common(params, n, w_dtype, ns_dtype, hp, sched, workspace, ws_bytes, d_status, stream, false);
+}
+
+// MONA-Lite descriptors as the common path's (B in the G_prev slot, no A).
+static std::vector<muon_param> lite_as_params(const muon_lite_param* lp, int n) {
+    std::vector<muon_param> out(n > 0 ? n : 0);
+    for (int i = 0; i < n; ++i) {
+        muon_param& p = out[i];
+        p.rows = lp[i].rows; p.cols = lp[i].cols;
+        p.W = lp[i].W; p.G = lp[i].G; p.G_prev = lp[i].B; p.A = nullptr; p.M = lp[i].M;
+        p.gamma = lp[i].gamma; p.O_out = lp[i].O_out;
+    }
+    return out;
+}
+
+muon_status muon_lite_workspace_size(const muon_lite_param* params, int n, muon_dtype ns_dtype, size_t* bytes) {
+    if (!params || n < 1) return MUON_ERR_INVALID_ARG;
+    std::vector<muon_param> p = lite_as_params(params, n);
+    return muon_workspace_size(p.data(), n, ns_dtype, bytes);
+}
+
+muon_status muon_lite_step_batched(const muon_lite_param* params, int n, muon_dtype w_dtype, muon_dtype ns_dtype,
+                                   const muon_hparams* hp, const muon_schedule* sched, void* workspace,
+                                   size_t ws_bytes, int* d_status, muon_stream_t stream) {
+    if (!params || n < 1) return MUON_ERR_INVALID_ARG;
+    std::vector<muon_param> p = lite_as_params(params, n);
+    return step_common(p.data(), n, w_dtype, ns_dtype, hp, sched, workspace, ws_bytes, d_status, stream, true);
 }
 
 static muon_status check_batch(const void* X_in, void* X_out, int batch, int rows, int cols,

@@ -129,6 +129,27 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
                 store8_dt(E.M, idx[h], DT_FP32, vec[h], nvalid[h], x[h]);
                 store8_dt(E.Gp, idx[h], IN_DT, vec[h], nvalid[h], g[h]);
             }
+        } else if (p.mode == 2) {
+            // MONA-Lite: B = beta_a A - (1 - beta_a) G of the previous step, bfloat16
+            float g[H][8], bb[H][8], mm[H][8];
+#pragma unroll
+            for (int h = 0; h < H; ++h) {
+                load8_in<IN_DT>(E.G, idx[h], vec[h], nvalid[h], g[h]);
+                load8_in<DT_BF16>(E.Gp, idx[h], vec[h], nvalid[h], bb[h]);
+                load8_dt(E.M, idx[h], DT_FP32, vec[h], nvalid[h], mm[h]);
+            }
+#pragma unroll
+            for (int h = 0; h < H; ++h) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float an = bb[h][i] + (1.f - p.beta_a) * g[h][i];       // step 2 (= A_k)
+                    const float gt = g[h][i] + p.alpha * an;                         // step 3
+                    x[h][i] = p.mu * mm[h][i] + gt;                                  // step 4
+                    bb[h][i] = p.beta_a * an - (1.f - p.beta_a) * g[h][i];           // next step's B
+                }
+                store8_dt(E.M, idx[h], DT_FP32, vec[h], nvalid[h], x[h]);
+                store8_dt(E.Gp, idx[h], DT_BF16, vec[h], nvalid[h], bb[h]);
+            }
         } else {
             const void* X = static_cast<const char*>(E.X) + (size_t)b * E.x_stride * dt_size(IN_DT);
 #pragma unroll
@@ -216,7 +237,9 @@ muon_status prep_run(PrepParams& prm, cudaStream_t stream) {
     for (int i = 0; i < prm.n; ++i) elems += (double)prm.e[i].rows * prm.e[i].cols * prm.e[i].count;
     const int isz = dt_size(prm.in_dt), xsz = dt_size(prm.x0_dt);
     // MONA: read G, G_prev, A, M; write A, M, G_prev, X0.  COPY: read X, write X0.
-    const double per = prm.mode == 0 ? 3.0 * isz + 16.0 + xsz : (double)(isz + xsz);
+    // MONA-Lite: read G, B, M; write B, M, X0.
+    const double per = prm.mode == 0 ? 3.0 * isz + 16.0 + xsz
+                     : prm.mode == 2 ? isz + 12.0 + xsz : (double)(isz + xsz);
     trace_begin(MUON_KERNEL_PREPASS, elems * per, stream);
     // element types are compile-time in the kernel: loads and stores stay in registers
 #define MUON_PREP(I, X)                                                   \

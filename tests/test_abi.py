@@ -55,6 +55,9 @@ int main(void) {
   printf("muon_schedule %zu\n", sizeof(muon_schedule));
   printf("muon_hparams %zu\n", sizeof(muon_hparams));
   printf("muon_ns_coeff %zu\n", sizeof(muon_ns_coeff));
+  printf("muon_lite_param %zu\n", sizeof(muon_lite_param));
+  P(muon_lite_param, rows) P(muon_lite_param, cols) P(muon_lite_param, W) P(muon_lite_param, G)
+  P(muon_lite_param, B) P(muon_lite_param, M) P(muon_lite_param, gamma) P(muon_lite_param, O_out)
   P(muon_param, rows) P(muon_param, cols) P(muon_param, W) P(muon_param, G) P(muon_param, G_prev)
   P(muon_param, A) P(muon_param, M) P(muon_param, gamma) P(muon_param, O_out)
   P(muon_schedule, n_steps) P(muon_schedule, coeffs) P(muon_schedule, eps)
@@ -76,7 +79,9 @@ def test_binding_struct_layout_matches_header(tmp_path):
     assert int(got["muon_schedule"]) == ctypes.sizeof(mo.Schedule)
     assert int(got["muon_hparams"]) == ctypes.sizeof(mo.HParams)
     assert int(got["muon_ns_coeff"]) == ctypes.sizeof(mo.NsCoeff)
-    py = {"muon_param": mo.Param, "muon_schedule": mo.Schedule, "muon_hparams": mo.HParams}
+    assert int(got["muon_lite_param"]) == ctypes.sizeof(mo.LiteParam)
+    py = {"muon_param": mo.Param, "muon_schedule": mo.Schedule, "muon_hparams": mo.HParams,
+          "muon_lite_param": mo.LiteParam}
     for key, val in got.items():
         if "." not in key:
             continue
@@ -129,3 +134,29 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     # W/G/... NULL
     assert L.muon_step_batched(arr, 1, mo.BF16, mo.BF16, ctypes.byref(hp), ctypes.byref(sched), p, 1 << 20,
                                None, None) == mo.ERR_INVALID_ARG
+
+
+def test_lite_entry_points_host_checks(lib):
+    L = lib
+    shapes = [(768, 768), (768, 3072), (3072, 768)]
+    arr = (mo.Param * 3)()
+    lite = (mo.LiteParam * 3)()
+    for i, (r, c) in enumerate(shapes):
+        arr[i].rows, arr[i].cols = r, c
+        lite[i].rows, lite[i].cols = r, c
+    # same iteration workspace as the full step
+    assert mo.muon_lite_workspace_size(lite, mo.BF16) == mo.muon_workspace_size(arr, mo.BF16)
+    sz = ctypes.c_size_t(0)
+    assert L.muon_lite_workspace_size(None, 1, mo.BF16, ctypes.byref(sz)) == mo.ERR_INVALID_ARG
+    assert L.muon_lite_workspace_size(lite, 0, mo.BF16, ctypes.byref(sz)) == mo.ERR_INVALID_ARG
+    sched = mo.quintic_schedule(5)
+    hp = mo.HParams(0.9, 0.02, 0.0, 1.0, 0.9, 0.5)
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    # NULL W / G / B / M
+    assert L.muon_lite_step_batched(lite, 1, mo.BF16, mo.BF16, ctypes.byref(hp), ctypes.byref(sched), p,
+                                    1 << 20, None, None) == mo.ERR_INVALID_ARG
+    one = (mo.LiteParam * 1)()
+    one[0] = mo.LiteParam(4, 4, p.value, p.value, None, p.value, float("nan"), None)
+    assert L.muon_lite_step_batched(one, 1, mo.BF16, mo.BF16, ctypes.byref(hp), ctypes.byref(sched), p,
+                                    1 << 20, None, None) == mo.ERR_INVALID_ARG
