@@ -46,6 +46,7 @@ struct PrepEntry {
     int rows, cols, count, transposed, vec_ok;
     int sumsq_index;
     int tiles_c;
+    int flat;          // set by prep_run: processed as one contiguous array
     long long tiles_per_mat, tile_begin;
 };
 

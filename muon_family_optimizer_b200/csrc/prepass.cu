@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
         const long long local = t - E.tile_begin;
         const int b = (int)(local / E.tiles_per_mat);
         const long long tt = local - (long long)b * E.tiles_per_mat;
-        const int tr = (int)(tt / E.tiles_c), tc = (int)(tt % E.tiles_c);
+        const int tr = E.flat ? 0 : (int)(tt / E.tiles_c), tc = E.flat ? 0 : (int)(tt % E.tiles_c);
         const int key = E.sumsq_index + b;
         if (key != cur) {   // uniform over the block
             if (cur >= 0) {
@@ -97,12 +97,23 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
         int gr[H], nvalid[H];
         bool vec[H];
         long long idx[H];
+        static_assert(H == 1, "the contiguous layout below gives each thread one group of 8");
+        if (E.flat) {
+            // contiguous run of TR*TC elements: thread i takes elements 8i..8i+7
+            const long long e0 = tt * (TR * TC) + (long long)threadIdx.x * 8;
+            const long long n = (long long)E.rows * E.cols;
+            gr[0] = 0;
+            nvalid[0] = (int)max(0LL, min(8LL, n - e0));
+            vec[0] = E.vec_ok && nvalid[0] == 8;
+            idx[0] = e0;
+        } else {
 #pragma unroll
-        for (int h = 0; h < H; ++h) {
-            gr[h] = tr * TR + r + 32 * h;
-            nvalid[h] = gr[h] < E.rows ? max(0, min(8, E.cols - gc0)) : 0;
-            vec[h] = E.vec_ok && nvalid[h] == 8;
-            idx[h] = (long long)gr[h] * E.cols + gc0;
+            for (int h = 0; h < H; ++h) {
+                gr[h] = tr * TR + r + 32 * h;
+                nvalid[h] = gr[h] < E.rows ? max(0, min(8, E.cols - gc0)) : 0;
+                vec[h] = E.vec_ok && nvalid[h] == 8;
+                idx[h] = (long long)gr[h] * E.cols + gc0;
+            }
         }
         float x[H][8];
         if (p.mode == 0) {
@@ -167,7 +178,7 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
             // wide view = the matrix itself; X0 rows are 16-byte aligned (ld % 8 == 0)
 #pragma unroll
             for (int h = 0; h < H; ++h)
-                store8_dt(X0, (long long)gr[h] * E.ld + gc0, X0_DT, nvalid[h] == 8, nvalid[h], x[h]);
+                store8_dt(X0, E.flat ? idx[h] : (long long)gr[h] * E.ld + gc0, X0_DT, nvalid[h] == 8, nvalid[h], x[h]);
         } else {
             // wide view = transpose: X0[c][r] = M[r][c], written as TR-row column segments
 #pragma unroll
@@ -218,6 +229,11 @@ muon_status prep_run(PrepParams& prm, cudaStream_t stream) {
         const int tiles_r = (E.rows + TR - 1) / TR;
         E.tiles_c = (E.cols + TC - 1) / TC;
         E.tiles_per_mat = (long long)tiles_r * E.tiles_c;
+        // not transposed and X0 rows unpadded: every buffer of the matrix is one
+        // contiguous array, processed in runs of TR*TC elements (long coalesced
+        // streams per array instead of TR separate row segments)
+        E.flat = !E.transposed && E.ld == E.cols;
+        if (E.flat) E.tiles_per_mat = ((long long)E.rows * E.cols + TR * TC - 1) / (TR * TC);
         E.tile_begin = tiles;
         tiles += E.tiles_per_mat * E.count;
     }
