@@ -63,6 +63,8 @@ def configure(L):
                                    ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                    ctypes.c_int, _D, ctypes.c_double, ctypes.c_double,
                                    ctypes.c_int]
+    L.oracle_adamw.argtypes = [ctypes.c_longlong, _D, _D, _D, _D, ctypes.c_double, ctypes.c_double,
+                               ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_int]
     L.oracle_mona_lite.argtypes = [ctypes.c_longlong, _D, _D, _D, ctypes.c_double, ctypes.c_double,
                                    ctypes.c_double, ctypes.c_int]
     L.oracle_muon_lite_step.argtypes = [ctypes.c_int, ctypes.c_int, _D, _D, _D, _D, _D,
@@ -233,3 +235,12 @@ def muon_lite_step(W, G, B, M, *, mu, eta, lam, gamma, beta_a, alpha,
                                 mu, eta, lam, gamma, beta_a, alpha, n, _p(c), eps, f,
                                 int(round_to), 1 if round_b else 0)
     return {"W": W, "B": B, "M": M, "O": O}
+
+
+def adamw(W, G, m, v, *, lr, beta1, beta2, eps, weight_decay, step):
+    """AdamW (bias-corrected, decoupled decay) on flat arrays; returns (W', m', v')."""
+    W, m, v = _f64(W).copy(), _f64(m).copy(), _f64(v).copy()
+    G = _f64(G)
+    assert W.shape == G.shape == m.shape == v.shape
+    lib().oracle_adamw(W.size, _p(W), _p(G), _p(m), _p(v), lr, beta1, beta2, eps, weight_decay, int(step))
+    return W, m, v

@@ -464,3 +464,26 @@ void oracle_muon_lite_step(int rows, int cols, double* W, const double* G, doubl
     oracle_orthogonalise(M, rows, cols, O, 0, n_steps, coeffs, NULL, 0, f, eps, round_kind);
     oracle_weight_update(n, W, O, eta, gamma, lambda);
 }
+
+/* ------------------------------------------------------------------------ */
+/* AdamW for vector-valued parameters (embeddings, biases): the MONA page,  */
+/* section 2 ("Ontwerprichtlijnen"), keeps Muon's convention of standard    */
+/* AdamW for them and prints no formulas.  Reading: Adam with bias          */
+/* correction and decoupled weight decay (Loshchilov and Hutter), step t>=1:*/
+/*   m' = b1 m + (1-b1) g        v' = b2 v + (1-b2) g^2                      */
+/*   W' = W - lr ( (m'/(1-b1^t)) / (sqrt(v'/(1-b2^t)) + eps) + wd W )        */
+/* ------------------------------------------------------------------------ */
+void oracle_adamw(long long n, double* W, const double* G, double* m, double* v,
+                  double lr, double b1, double b2, double eps, double wd, int t)
+{
+    const double c1 = 1.0 - pow(b1, (double)t);
+    const double c2 = 1.0 - pow(b2, (double)t);
+    for (long long i = 0; i < n; ++i) {
+        const double mn = b1 * m[i] + (1.0 - b1) * G[i];
+        const double vn = b2 * v[i] + (1.0 - b2) * G[i] * G[i];
+        const double upd = (mn / c1) / (sqrt(vn / c2) + eps);
+        W[i] = W[i] - lr * (upd + wd * W[i]);
+        m[i] = mn;
+        v[i] = vn;
+    }
+}

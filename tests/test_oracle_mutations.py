@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+import test_oracle_adamw as adamw
 import test_oracle_lite as lite
 import test_oracle_pins as pins
 
@@ -45,6 +46,12 @@ MUTATIONS = [
     ("lite_difference_weight", "double An = B[i] + (1.0 - beta_a) * G[i];",
      "double An = B[i] + beta_a * G[i];",
      [lambda: lite.test_mona_lite_equals_mona_without_rounding(0.9, 0.5, 0.95)]),
+    ("adamw_bias_correction_step", "const double c1 = 1.0 - pow(b1, (double)t);",
+     "const double c1 = 1.0 - pow(b1, (double)(t + 1));", [adamw.test_adamw_hand_example_two_steps]),
+    ("adamw_no_sqrt", "const double upd = (mn / c1) / (sqrt(vn / c2) + eps);",
+     "const double upd = (mn / c1) / ((vn / c2) + eps);", [adamw.test_adamw_hand_example_two_steps]),
+    ("adamw_coupled_decay", "W[i] = W[i] - lr * (upd + wd * W[i]);", "W[i] = W[i] - lr * upd;",
+     [adamw.test_adamw_zero_gradient_is_pure_decay]),
     ("bf16_precision", "return round_to_format(x, 8, -126, 0x1.fep127);",
      "return round_to_format(x, 7, -126, 0x1.fep127);",
      [pins.test_round_bf16_matches_torch_on_float32_values]),
