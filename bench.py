@@ -45,9 +45,10 @@ def parse():
                     help="replay each step as a captured CUDA graph (default) or launch it eagerly")
     ap.add_argument("--variant", default="mona", choices=["mona", "lite"],
                     help="mona: G_prev and A state (default); lite: MONA-Lite, one bfloat16 buffer B")
-    ap.add_argument("--route", default="step", choices=["step", "gram", "direct"],
+    ap.add_argument("--route", default="step", choices=["step", "gram", "direct", "adamw"],
                     help="step: the optimizer step (default); gram / direct: the orthogonalisation alone "
-                         "(gram_polar / ns_polar, converged schedule) of the workload's matrices, one batch per shape")
+                         "(gram_polar / ns_polar, converged schedule) of the workload's matrices, one batch per shape; "
+                         "adamw: the AdamW step of the model's vector-valued parameters")
     return ap.parse_args()
 
 
@@ -264,6 +265,62 @@ def run_reference(args, w, ns_steps):
 
 # ------------------------------------------------------------------ GPU arm
 
+def run_adamw_route(args, w):
+    """Time adamw_step_batched on the model family's vector-valued parameters
+    (bf16 W and G, fp32 moments): a streaming pass, 22 bytes per element."""
+    import torch
+    import muon_family_optimizer_b200 as mo
+    from muon_family_optimizer_b200 import synthetic as syn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    shapes = syn.VECTOR_SHAPES[w["name"]]
+    g = torch.Generator(device=dev).manual_seed(77)
+    params = []
+    for sh in shapes:
+        params.append(dict(W=(torch.randn(sh, generator=g, device=dev) * 0.02).to(torch.bfloat16),
+                           G=torch.randn(sh, generator=g, device=dev).to(torch.bfloat16),
+                           m=torch.zeros(sh, device=dev), v=torch.zeros(sh, device=dev)))
+    arr = mo.make_vec_params(params)
+    hp = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    nel = sum(p["W"].numel() for p in params)
+    for t in range(1, args.warmup + 1):
+        mo.adamw_step_batched(arr, mo.BF16, hp, t, d_status=status)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    with torch.cuda.graph(graph, stream=cap):
+        mo.adamw_step_batched(arr, mo.BF16, hp, args.warmup + 1, d_status=status,
+                              stream=torch.cuda.current_stream(dev))
+    for _ in range(3):
+        graph.replay()
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    gbs = nel * 22.0 / (ms / 1e3) / 1e9
+    pk, src = peaks()
+    line = {"metric": "AdamW step of the vector-valued parameters, GB/s", "value": gbs, "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 W/G, fp32 moments", "data": "synthetic",
+            "config": {"workload": f"{w['name']} vector parameters: {len(shapes)} tensors, {nel} elements",
+                       "bytes_per_element": 22, "l2": f"inputs larger than L2: {nel * 22 / 1e9:.2f} GB per step"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None, "peak_source": f"{src} (copy)"},
+            "gpu_launches": args.steps, "clocks": clk, "launch": "graph (one CUDA graph per step)"}
+    print(json.dumps(line), flush=True)
+    del graph
+
+
 def run_polar_route(args, w):
     """Time gram_polar (Gram route with restarts and the 1.05 divisor) or ns_polar
     with the same converged schedule on the workload's matrices (log-spaced
@@ -348,6 +405,8 @@ def main():
     ns_steps = args.ns_steps
     if args.impl == "reference":
         return run_reference(args, w, ns_steps)
+    if args.route == "adamw":
+        return run_adamw_route(args, w)
     if args.route != "step":
         return run_polar_route(args, w)
 

@@ -189,6 +189,38 @@ MUON_API muon_status muon_lite_step_batched(const muon_lite_param* params, int n
                                    int* d_status, muon_stream_t stream);
 
 /*
+ * AdamW for vector-valued parameters ([MONA] section 2, "Ontwerprichtlijnen":
+ * embeddings and biases keep standard AdamW, as in Muon; the page gives no
+ * formulas, read as Adam with bias correction and decoupled weight decay):
+ *     m <- beta1 m + (1 - beta1) g          v <- beta2 v + (1 - beta2) g^2
+ *     W <- W - lr ( (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps) + weight_decay W )
+ * evaluated in fp32 per element.  One streaming launch per 128 parameters.
+ */
+typedef struct {
+    long long n;       /* elements (>= 1); any shape, contiguous */
+    void* W;           /* n elements, w_dtype, updated in place */
+    const void* G;     /* n elements, w_dtype (read only) */
+    float* m;          /* n fp32 first moments, updated in place (zero initially) */
+    float* v;          /* n fp32 second moments, updated in place (zero initially) */
+} muon_vec_param;
+
+typedef struct {
+    float lr, beta1, beta2, eps, weight_decay;   /* 0 <= beta < 1, eps >= 0 */
+} muon_adamw_hparams;
+
+/*
+ * One AdamW step (t = step >= 1, the bias-correction count) on n vector
+ * parameters, asynchronous on `stream`.  Argument errors return before any
+ * launch (MUON_ERR_INVALID_ARG: NULL pointers, n < 1, step < 1, non-finite or
+ * out-of-range hyper-parameters).  An element whose gradient is not finite
+ * keeps its W, m and v, and MUON_FLAG_NONFINITE is OR-ed into *d_status
+ * (when given).  No workspace.
+ */
+MUON_API muon_status adamw_step_batched(const muon_vec_param* params, int n, muon_dtype w_dtype,
+                               const muon_adamw_hparams* hp, int step, int* d_status,
+                               muon_stream_t stream);
+
+/*
  * Bytes of workspace ns_polar / gram_polar need for a batch of rows x cols
  * matrices in `dtype`.
  */
@@ -264,7 +296,8 @@ typedef enum {
     MUON_KERNEL_SYM = 1,       /* tcgen05 symmetric product X X^T, A A, ... (work = flops) */
     MUON_KERNEL_UPD = 2,       /* tcgen05 update product X <- aX + BX, Q Xb (work = flops) */
     MUON_KERNEL_SIMT = 3,      /* fp32 CUDA-core product (work = flops) */
-    MUON_KERNEL_OTHER = 4      /* identity fill (work = bytes) */
+    MUON_KERNEL_OTHER = 4,     /* identity fill (work = bytes) */
+    MUON_KERNEL_ADAMW = 5      /* AdamW streaming pass over vector parameters (work = bytes) */
 } muon_kernel_kind;
 
 typedef struct {

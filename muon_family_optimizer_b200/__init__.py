@@ -59,8 +59,18 @@ class LiteParam(ctypes.Structure):
                 ("gamma", ctypes.c_float), ("O_out", ctypes.c_void_p)]
 
 
-KERNEL_PREPASS, KERNEL_SYM, KERNEL_UPD, KERNEL_SIMT, KERNEL_OTHER = range(5)
-KERNEL_NAMES = {KERNEL_PREPASS: "prepass", KERNEL_SYM: "tc_sym", KERNEL_UPD: "tc_upd",
+class VecParam(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_longlong), ("W", ctypes.c_void_p), ("G", ctypes.c_void_p),
+                ("m", ctypes.c_void_p), ("v", ctypes.c_void_p)]
+
+
+class AdamWHParams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float)]
+
+
+KERNEL_PREPASS, KERNEL_SYM, KERNEL_UPD, KERNEL_SIMT, KERNEL_OTHER, KERNEL_ADAMW = range(6)
+KERNEL_NAMES = {KERNEL_PREPASS: "prepass", KERNEL_SYM: "tc_sym", KERNEL_UPD: "tc_upd", KERNEL_ADAMW: "adamw",
                 KERNEL_SIMT: "simt", KERNEL_OTHER: "other"}
 TRACE_CAPACITY = 8192
 
@@ -97,6 +107,9 @@ def lib():
         L.muon_lite_step_batched.argtypes = [ctypes.POINTER(LiteParam), ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.POINTER(HParams), ctypes.POINTER(Schedule), vp,
                                              ctypes.c_size_t, vp, vp]
+        L.adamw_step_batched.restype = st
+        L.adamw_step_batched.argtypes = [ctypes.POINTER(VecParam), ctypes.c_int, ctypes.c_int,
+                                         ctypes.POINTER(AdamWHParams), ctypes.c_int, vp, vp]
         for name in ("ns_polar_workspace_size", "gram_polar_workspace_size"):
             f = getattr(L, name)
             f.restype = st
@@ -232,6 +245,30 @@ def muon_lite_step_batched(params, w_dtype, ns_dtype, hp, schedule, workspace, d
     _check(lib().muon_lite_step_batched(arr, len(arr), int(w_dtype), int(ns_dtype), ctypes.byref(h),
                                         ctypes.byref(schedule), _ptr(workspace), workspace.numel(),
                                         _ptr(d_status), _stream_ptr(stream)), "muon_lite_step_batched")
+
+
+def make_vec_params(params):
+    """params: list of dicts with torch tensors W, G (same dtype), m, v (float32), any shape, contiguous."""
+    import torch
+    arr = (VecParam * len(params))()
+    for i, p in enumerate(params):
+        n = p["W"].numel()
+        for k in ("W", "G", "m", "v"):
+            if p[k].numel() != n or not p[k].is_contiguous():
+                raise ValueError(f"vector param {i}: {k} must be contiguous with {n} elements")
+        if p["m"].dtype != torch.float32 or p["v"].dtype != torch.float32 or p["G"].dtype != p["W"].dtype:
+            raise ValueError(f"vector param {i}: m and v must be float32 and G of W's dtype")
+        arr[i] = VecParam(n, p["W"].data_ptr(), p["G"].data_ptr(), p["m"].data_ptr(), p["v"].data_ptr())
+    return arr
+
+
+def adamw_step_batched(params, w_dtype, hp, step, d_status=None, stream=None):
+    """One AdamW step (see include/muon.h) on vector parameters.
+    hp: dict with lr, beta1, beta2, eps, weight_decay; step: t >= 1."""
+    arr = params if isinstance(params, ctypes.Array) else make_vec_params(params)
+    h = AdamWHParams(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    _check(lib().adamw_step_batched(arr, len(arr), int(w_dtype), ctypes.byref(h), int(step), _ptr(d_status),
+                                    _stream_ptr(stream)), "adamw_step_batched")
 
 
 def ns_polar_workspace_size(batch, rows, cols, dtype):

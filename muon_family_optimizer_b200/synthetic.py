@@ -106,6 +106,18 @@ WORKLOADS = {
 }
 
 
+# Vector-valued parameters of the model families (updated with AdamW, not the
+# orthogonalised step): embeddings, layer-norm weights and biases, biases.
+def _gpt2_vectors():
+    out = [(50257, 768), (1024, 768)]                       # token, position embeddings
+    for _ in range(12):
+        out += [(768,), (768,), (2304,), (768,), (768,), (768,), (3072,), (768,)]
+    return out + [(768,), (768,)]                           # final layer norm
+
+
+VECTOR_SHAPES = {"gpt2_small": _gpt2_vectors()}
+
+
 def gradient(workload, j, t, rows, cols, device="cpu", kappa=1e3):
     """Gradient of matrix j at step t for a workload (fp32)."""
     w = WORKLOADS[workload]

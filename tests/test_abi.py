@@ -56,6 +56,11 @@ int main(void) {
   printf("muon_hparams %zu\n", sizeof(muon_hparams));
   printf("muon_ns_coeff %zu\n", sizeof(muon_ns_coeff));
   printf("muon_lite_param %zu\n", sizeof(muon_lite_param));
+  printf("muon_vec_param %zu\n", sizeof(muon_vec_param));
+  printf("muon_adamw_hparams %zu\n", sizeof(muon_adamw_hparams));
+  P(muon_vec_param, n) P(muon_vec_param, W) P(muon_vec_param, G) P(muon_vec_param, m) P(muon_vec_param, v)
+  P(muon_adamw_hparams, lr) P(muon_adamw_hparams, beta1) P(muon_adamw_hparams, beta2) P(muon_adamw_hparams, eps)
+  P(muon_adamw_hparams, weight_decay)
   P(muon_lite_param, rows) P(muon_lite_param, cols) P(muon_lite_param, W) P(muon_lite_param, G)
   P(muon_lite_param, B) P(muon_lite_param, M) P(muon_lite_param, gamma) P(muon_lite_param, O_out)
   P(muon_param, rows) P(muon_param, cols) P(muon_param, W) P(muon_param, G) P(muon_param, G_prev)
@@ -80,8 +85,11 @@ def test_binding_struct_layout_matches_header(tmp_path):
     assert int(got["muon_hparams"]) == ctypes.sizeof(mo.HParams)
     assert int(got["muon_ns_coeff"]) == ctypes.sizeof(mo.NsCoeff)
     assert int(got["muon_lite_param"]) == ctypes.sizeof(mo.LiteParam)
+    assert int(got["muon_vec_param"]) == ctypes.sizeof(mo.VecParam)
+    assert int(got["muon_adamw_hparams"]) == ctypes.sizeof(mo.AdamWHParams)
     py = {"muon_param": mo.Param, "muon_schedule": mo.Schedule, "muon_hparams": mo.HParams,
-          "muon_lite_param": mo.LiteParam}
+          "muon_lite_param": mo.LiteParam, "muon_vec_param": mo.VecParam,
+          "muon_adamw_hparams": mo.AdamWHParams}
     for key, val in got.items():
         if "." not in key:
             continue
@@ -160,3 +168,22 @@ def test_lite_entry_points_host_checks(lib):
     one[0] = mo.LiteParam(4, 4, p.value, p.value, None, p.value, float("nan"), None)
     assert L.muon_lite_step_batched(one, 1, mo.BF16, mo.BF16, ctypes.byref(hp), ctypes.byref(sched), p,
                                     1 << 20, None, None) == mo.ERR_INVALID_ARG
+
+
+def test_adamw_argument_checks(lib):
+    L = lib
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.cast(buf, ctypes.c_void_p).value
+    good = mo.AdamWHParams(1e-3, 0.9, 0.999, 1e-8, 0.01)
+    one = (mo.VecParam * 1)(mo.VecParam(4, p, p, p, p))
+    assert L.adamw_step_batched(None, 1, mo.BF16, ctypes.byref(good), 1, None, None) == mo.ERR_INVALID_ARG
+    assert L.adamw_step_batched(one, 0, mo.BF16, ctypes.byref(good), 1, None, None) == mo.ERR_INVALID_ARG
+    assert L.adamw_step_batched(one, 1, mo.BF16, ctypes.byref(good), 0, None, None) == mo.ERR_INVALID_ARG
+    assert L.adamw_step_batched(one, 1, 9, ctypes.byref(good), 1, None, None) == mo.ERR_INVALID_ARG
+    for bad in (mo.AdamWHParams(1e-3, 1.0, 0.999, 1e-8, 0.0), mo.AdamWHParams(1e-3, 0.9, -0.1, 1e-8, 0.0),
+                mo.AdamWHParams(float("nan"), 0.9, 0.999, 1e-8, 0.0), mo.AdamWHParams(1e-3, 0.9, 0.999, -1.0, 0.0)):
+        assert L.adamw_step_batched(one, 1, mo.BF16, ctypes.byref(bad), 1, None, None) == mo.ERR_INVALID_ARG
+    nul = (mo.VecParam * 1)(mo.VecParam(4, p, None, p, p))
+    assert L.adamw_step_batched(nul, 1, mo.BF16, ctypes.byref(good), 1, None, None) == mo.ERR_INVALID_ARG
+    empty = (mo.VecParam * 1)(mo.VecParam(0, p, p, p, p))
+    assert L.adamw_step_batched(empty, 1, mo.BF16, ctypes.byref(good), 1, None, None) == mo.ERR_INVALID_ARG
