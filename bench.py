@@ -61,16 +61,20 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# Sources whose change invalidates a recorded DRAM-traffic figure.
-TRAFFIC_SOURCES = ("muon_family_optimizer_b200/csrc/gemm_tc.cu", "muon_family_optimizer_b200/csrc/muon_internal.cuh",
-                   "muon_family_optimizer_b200/csrc/epilogue.cuh", "muon_family_optimizer_b200/csrc/muon_api.cu",
-                   "muon_family_optimizer_b200/csrc/prepass.cu")
+# Sources whose change invalidates a recorded DRAM-traffic figure, per kernel.
+_COMMON = ("muon_family_optimizer_b200/csrc/muon_internal.cuh", "muon_family_optimizer_b200/csrc/gemm.h",
+           "muon_family_optimizer_b200/csrc/muon_api.cu")
+TRAFFIC_SOURCES = {
+    "tc_sym": _COMMON + ("muon_family_optimizer_b200/csrc/gemm_tc.cu", "muon_family_optimizer_b200/csrc/epilogue.cuh"),
+    "tc_upd": _COMMON + ("muon_family_optimizer_b200/csrc/gemm_tc.cu", "muon_family_optimizer_b200/csrc/epilogue.cuh"),
+    "prepass": _COMMON + ("muon_family_optimizer_b200/csrc/prepass.cu",),
+}
 
 
-def sources_digest():
+def sources_digest(kernel="tc_sym"):
     import hashlib
     h = hashlib.sha256()
-    for rel in TRAFFIC_SOURCES:
+    for rel in TRAFFIC_SOURCES.get(kernel, TRAFFIC_SOURCES["tc_sym"]):
         with open(os.path.join(ROOT, rel), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -84,7 +88,7 @@ def recorded_traffic(kernel, workload, ns_steps):
     d = os.path.join(ROOT, "profiles")
     if not os.path.isdir(d):
         return None, None
-    digest = sources_digest()
+    digest = sources_digest(kernel)
     for name in sorted(os.listdir(d)):
         if not name.endswith(".md"):
             continue

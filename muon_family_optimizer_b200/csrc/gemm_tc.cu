@@ -375,9 +375,9 @@ __device__ __forceinline__ void epi_combine(const Epilogue& E, int gi, int gj0, 
 #pragma unroll
         for (int q = 0; q < 32; ++q) v[q] *= s;
     }
-    if (E.diag != 0.f) {   // static indices only: keeps v in registers
+    if (E.diag != 0.f && (unsigned)(gi - gj0) < 32u) {   // only a chunk crossing the diagonal
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
+        for (int q = 0; q < 32; ++q)   // static indices only: keeps v in registers
             if (gi == gj0 + q) v[q] += E.diag;
     }
 }
