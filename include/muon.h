@@ -309,6 +309,15 @@ typedef struct {
 MUON_API muon_status muon_trace_enable(int enable);
 MUON_API int muon_trace_read(muon_trace_record* out, int max);
 
+/*
+ * Self-test of the failure path: one block runs the library's bounded wait
+ * on a barrier that nothing completes, with a limit of wait_ms milliseconds
+ * (1..4000); the wait gives up, ORs MUON_FLAG_TIMEOUT into *d_status (device,
+ * required) and the kernel returns normally.  No pages' counterpart: it lets a
+ * caller check that a stuck wait ends in a status word, not a hung GPU.
+ */
+MUON_API muon_status muon_wait_selftest(int wait_ms, int* d_status, muon_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 MUON_API const char* muon_status_string(muon_status status);
 

@@ -107,6 +107,8 @@ def lib():
         L.muon_lite_step_batched.argtypes = [ctypes.POINTER(LiteParam), ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.POINTER(HParams), ctypes.POINTER(Schedule), vp,
                                              ctypes.c_size_t, vp, vp]
+        L.muon_wait_selftest.restype = st
+        L.muon_wait_selftest.argtypes = [ctypes.c_int, vp, vp]
         L.adamw_step_batched.restype = st
         L.adamw_step_batched.argtypes = [ctypes.POINTER(VecParam), ctypes.c_int, ctypes.c_int,
                                          ctypes.POINTER(AdamWHParams), ctypes.c_int, vp, vp]
@@ -269,6 +271,11 @@ def adamw_step_batched(params, w_dtype, hp, step, d_status=None, stream=None):
     h = AdamWHParams(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
     _check(lib().adamw_step_batched(arr, len(arr), int(w_dtype), ctypes.byref(h), int(step), _ptr(d_status),
                                     _stream_ptr(stream)), "adamw_step_batched")
+
+
+def muon_wait_selftest(wait_ms, d_status, stream=None):
+    """Run the bounded-wait self-test (see include/muon.h): sets FLAG_TIMEOUT in d_status."""
+    _check(lib().muon_wait_selftest(int(wait_ms), _ptr(d_status), _stream_ptr(stream)), "muon_wait_selftest")
 
 
 def ns_polar_workspace_size(batch, rows, cols, dtype):

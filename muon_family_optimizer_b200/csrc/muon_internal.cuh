@@ -34,12 +34,15 @@ template <> __device__ __forceinline__ float from_float<float>(float x) { return
 // Two 16-bit values packed in a 32-bit word (low half first), without taking
 // addresses of register variables.
 template <typename T> __device__ __forceinline__ uint32_t pack2(float a, float b);
+// a in the low half, b in the high half; both rounded to nearest even (one
+// paired conversion)
 template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
-    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a)) |
-           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 template <> __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
-    return (uint32_t)__half_as_ushort(__float2half_rn(a)) | ((uint32_t)__half_as_ushort(__float2half_rn(b)) << 16);
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 template <typename T> __device__ __forceinline__ float unpack_lo(uint32_t w);
 template <typename T> __device__ __forceinline__ float unpack_hi(uint32_t w);
@@ -174,14 +177,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // the CTA-wide abort flag is raised or the time limit is reached (which
 // raises the flag and reports MUON_FLAG_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* d_status) {
+                                          int* d_status, unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     unsigned long long t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (*abort_flag) return false;
-            if (global_ns() - t0 > kWaitLimitNs) {
+            if (global_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 if (d_status) atomicOr(d_status, MUON_FLAG_TIMEOUT);
                 return false;
