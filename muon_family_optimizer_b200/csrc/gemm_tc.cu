@@ -372,8 +372,10 @@ __device__ __forceinline__ void epi_combine(const Epilogue& E, int gi, int gj0, 
         }
     } else {
         const float s = sc * E.alpha;
+        if (s != 1.f) {   // uniform: most products have no scale after the first step
 #pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] *= s;
+            for (int q = 0; q < 32; ++q) v[q] *= s;
+        }
     }
     if (E.diag != 0.f && (unsigned)(gi - gj0) < 32u) {   // only a chunk crossing the diagonal
 #pragma unroll
