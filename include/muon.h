@@ -69,7 +69,7 @@ typedef struct CUstream_st* muon_stream_t;
 typedef enum {
     MUON_OK = 0,
     MUON_ERR_INVALID_ARG = 1,   /* NULL pointer, bad size, bad enum, bad schedule */
-    MUON_ERR_UNSUPPORTED = 2,   /* valid request this build cannot run (no sm_100 device, shape limits) */
+    MUON_ERR_UNSUPPORTED = 2,   /* valid request the library cannot run (no sm_100 device, shape limits) */
     MUON_ERR_WORKSPACE = 3,     /* workspace NULL, misaligned or smaller than the size query */
     MUON_ERR_NONFINITE = 4,     /* host-side name for MUON_FLAG_NONFINITE */
     MUON_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed (see cudaGetLastError) */
