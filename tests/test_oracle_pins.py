@@ -305,3 +305,18 @@ def test_muon_step_is_the_composition_of_its_parts():
     Xr = oracle.round_bf16(M2.T) / (np.linalg.norm(M2) + 1e-7)
     Ob = oracle.ns_poly(Xr, [QUINTIC] * 5).T
     np.testing.assert_allclose(outb["O"], Ob, atol=1e-12)
+
+
+def test_ns_poly_scalar_table():
+    """Singular values 1 and 0.1 follow the composed scalar quintic step by step
+    (tests/golden/quintic_scalar_table.txt); a 1 x 1 input x gives sign(x) phi_5(1)."""
+    g = load_golden("quintic_scalar_table.txt")
+    X = np.diag([1.0, 0.1])
+    for k in range(1, 6):
+        Y = oracle.ns_poly(X, [QUINTIC] * k)
+        assert abs(Y[0, 0] - g["sigma1"][k - 1]) <= 1e-9, k
+        assert abs(Y[1, 1] - g["sigma01"][k - 1]) <= 1e-9, k
+        assert abs(Y[0, 1]) == 0.0 and abs(Y[1, 0]) == 0.0
+    for x in (2.5, -0.3):
+        O = oracle.orthogonalise(np.array([[x]]), [QUINTIC] * 5, eps=0.0)
+        assert abs(O[0, 0] - np.sign(x) * g["sigma1"][4]) <= 1e-9
