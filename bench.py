@@ -225,6 +225,51 @@ def cpu_baseline(w, ns_steps):
             "ms_per_step_extrapolated": secs * full / fl * 1e3}
 
 
+def group_parity(w, ns_steps, dev):
+    """Maximum relative errors per shape group: one matrix of each (s, l) group,
+    one step on the GPU through muon_step_batched (with O stored) and the same
+    step in the fp64 oracle from the same 16-bit inputs (the iteration started
+    from the same rounded momentum).  Returns {"s x l": {"O": e, "W": e, "M": e}}."""
+    import numpy as np
+    import torch
+    import muon_family_optimizer_b200 as mo
+    import oracle
+    from muon_family_optimizer_b200 import synthetic as syn
+    w_dt, ns_dt = w["w_dtype"], w["ns_dtype"]
+    seen, pick = set(), []
+    for j, (r, c) in enumerate(w["shapes"]):
+        key = (min(r, c), max(r, c))
+        if key not in seen:
+            seen.add(key)
+            pick.append((j, r, c))
+    host, params = [], []
+    for j, r, c in pick:
+        st = dict(W=syn.initial_weight(w["name"], j, r, c).to(w_dt), G=syn.gradient(w["name"], j, 0, r, c).to(w_dt),
+                  G_prev=syn.gradient(w["name"], j, 8, r, c).to(w_dt), A=torch.zeros(r, c), M=torch.zeros(r, c))
+        host.append(st)
+        p = {k: v.to(dev).contiguous() for k, v in st.items()}
+        p["O_out"] = torch.empty(r, c, device=dev)
+        params.append(p)
+    ws = torch.empty(mo.muon_workspace_size(params, mo._dtype_code(ns_dt)), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    mo.muon_step_batched(params, mo._dtype_code(w_dt), mo._dtype_code(ns_dt), w["hp"],
+                         mo.quintic_schedule(ns_steps), ws, d_status=status)
+    torch.cuda.synchronize(dev)
+    rnd = {torch.bfloat16: oracle.ROUND_BF16, torch.float16: oracle.ROUND_FP16}.get(ns_dt, oracle.ROUND_NONE)
+    hp = w["hp"]
+    rel = lambda a, b: float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+    out = {}
+    for (j, r, c), st, p in zip(pick, host, params):
+        f = {k: v.double().numpy() for k, v in st.items()}
+        ref = oracle.muon_step(f["W"], f["G"], f["G_prev"], f["A"], f["M"], mu=hp["mu"], eta=hp["eta"],
+                               lam=hp["lambda"], gamma=hp["gamma"], beta_a=hp["beta_a"], alpha=hp["alpha"],
+                               coeffs=[tuple(syn.QUINTIC)] * ns_steps, round_to=rnd)
+        g = {k: p[k].double().cpu().numpy() for k in ("W", "M", "O_out")}
+        out[f"{min(r, c)}x{max(r, c)}"] = {"O": rel(g["O_out"], ref["O"]), "W": rel(g["W"], ref["W"]),
+                                          "M": rel(g["M"], ref["M"]), "status": int(status.item())}
+    return out
+
+
 def run_reference(args, w, ns_steps):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -609,8 +654,11 @@ def main():
                "timing": "wall clock over the loop, H2D of step i+1 overlapped with step i"}
 
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, ns_steps)
+        if not lite:
+            parity = group_parity(w, ns_steps, dev)
 
     if rank == 0:
         groups, _ = describe(args.workload, w)
@@ -630,6 +678,8 @@ def main():
                 "dense_equivalent": {"value": world * ns_flops_dense(shapes, ns_steps) * args.steps / (ms_total / 1e3) / 1e12,
                                      "unit": "TFLOP/s", "note": "symmetric products counted in full (not the headline)"},
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "parity": parity and {"vs": "fp64 oracle from the same 16-bit inputs, one matrix per shape group, "
+                                            "relative Frobenius", "groups": parity},
                 "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clk,
                 "launch": args.launch + (" (one CUDA graph per step)" if graphs is not None else ""),
                 "kernel_timing": f"per-kernel device time from {ktrace} eagerly launched steps, each launch "
