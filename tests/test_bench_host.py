@@ -1,0 +1,56 @@
+"""Host logic of bench.py (CPU).
+
+The headline metric counts algorithmic Newton-Schulz flops: per quintic step
+and matrix (s x l wide view) s^2 l for X X^T (half of the dense product), s^3
+for A A (half) and 2 s^2 l for B X.  Checked against values worked out from
+that definition: 5 steps of a 768 x 2048 matrix = 5 (3 * 768^2 * 2048 + 768^3).
+The roofline's DRAM-traffic figure is read from an ncu record only while the
+kernel sources still hash to the recorded digest.
+"""
+import json
+import os
+import shutil
+
+import pytest
+
+import bench
+from muon_family_optimizer_b200 import synthetic as syn
+
+
+@pytest.mark.parametrize("shape,expect", [((768, 2048), 20.38e9), ((2048, 768), 20.38e9),
+                                          ((1024, 4096), 69.79e9), ((4096, 14336), 3.952e12),
+                                          ((2048, 16384), 1.0737e12), ((1024, 1024), 21.47e9)])
+def test_ns_flops_per_matrix(shape, expect):
+    assert abs(bench.ns_flops([shape], 5) - expect) / expect < 1e-3
+
+
+@pytest.mark.parametrize("workload,expect", [("gpt2_small", 1.1415e12), ("llama_430m", 7.086e12),
+                                             ("llama3_8b", 471.8e12)])
+def test_ns_flops_per_workload(workload, expect):
+    assert abs(bench.ns_flops(syn.WORKLOADS[workload]["shapes"], 5) - expect) / expect < 1e-3
+
+
+def test_dense_equivalent_counts_symmetric_products_in_full():
+    s, l = 768, 3072
+    assert bench.ns_flops_dense([(s, l)], 1) == 4.0 * s * s * l + 2.0 * s ** 3
+    assert abs(bench.ns_flops_dense(syn.WORKLOADS["llama3_8b"]["shapes"], 5) - 665.9e12) / 665.9e12 < 1e-3
+
+
+def test_recorded_traffic_requires_matching_sources(tmp_path, monkeypatch):
+    root = tmp_path / "repo"
+    for rel in set(sum((list(v) for v in bench.TRAFFIC_SOURCES.values()), [])):
+        dst = root / rel
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        shutil.copy(os.path.join(bench.ROOT, rel), dst)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    (root / "profiles").mkdir()
+    rec = {"kernel": "tc_sym", "workload": "gpt2_small", "ns_steps": 5, "bytes_per_launch": 123456,
+           "sources": bench.sources_digest("tc_sym")}
+    (root / "profiles" / "k.md").write_text("# summary\n\ntraffic-record: " + json.dumps(rec) + "\n")
+    assert bench.recorded_traffic("tc_sym", "gpt2_small", 5) == (123456.0, "profiles/k.md")
+    assert bench.recorded_traffic("tc_sym", "llama_430m", 5) == (None, None)      # other workload
+    assert bench.recorded_traffic("tc_sym", "gpt2_small", 14) == (None, None)     # other schedule
+    # a change to one of the kernel's sources retires the record
+    with open(root / "muon_family_optimizer_b200" / "csrc" / "gemm_tc.cu", "a") as fh:
+        fh.write("\n// changed\n")
+    assert bench.recorded_traffic("tc_sym", "gpt2_small", 5) == (None, None)
