@@ -45,10 +45,11 @@ def parse():
                     help="replay each step as a captured CUDA graph (default) or launch it eagerly")
     ap.add_argument("--variant", default="mona", choices=["mona", "lite"],
                     help="mona: G_prev and A state (default); lite: MONA-Lite, one bfloat16 buffer B")
-    ap.add_argument("--route", default="step", choices=["step", "gram", "direct", "adamw"],
+    ap.add_argument("--route", default="step", choices=["step", "gram", "direct", "adamw", "limuon"],
                     help="step: the optimizer step (default); gram / direct: the orthogonalisation alone "
                          "(gram_polar / ns_polar, converged schedule) of the workload's matrices, one batch per shape; "
-                         "adamw: the AdamW step of the model's vector-valued parameters")
+                         "adamw: the AdamW step of the model's vector-valued parameters; "
+                         "limuon: the LiMuon step (randomized SVD, r = 16, p = 16) of the workload's matrices")
     return ap.parse_args()
 
 
@@ -370,6 +371,154 @@ def run_adamw_route(args, w):
     del graph
 
 
+# LiMuon: rank r, oversampling p (k = r + p columns of the test matrix)
+LIMUON_HP = dict(mu=0.95, eta=0.02, gamma=1.0, rank=16, oversample=16, **{"lambda": 0.0})
+# fp32 FMA peak: 148 SMs x 128 lanes x 2 flops at the 1965 MHz maximum SM clock
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+LIMUON_KERNELS = ["lim_sketch", "lim_qr", "lim_project", "lim_factor", "lim_update"]
+
+
+def limuon_kernel_work(shapes, k, w_bytes=2):
+    """Algorithmic bytes and fp32 flops per launch of the five LiMuon kernels
+    for matrices `shapes` (one launch each): per element, the sketch reads G
+    and M and writes M (w_bytes + 8), the projection reads M (4), the update
+    reads and writes W (2 w_bytes); each of the three products is k FMAs per
+    element; the k-column factors add 4 k bytes per row / column."""
+    el = sum(r * c for r, c in shapes)
+    rk = sum(r for r, _ in shapes) * k
+    ck = sum(c for _, c in shapes) * k
+    by = [el * (w_bytes + 8) + 4 * rk, 8 * rk, el * 4 + 4 * (rk + ck), 4 * (ck + 2 * rk),
+          el * 2 * w_bytes + 4 * (rk + ck)]
+    fl = [2.0 * el * k, 0.0, 2.0 * el * k, 0.0, 2.0 * el * k]
+    return by, fl
+
+
+def run_limuon_route(args, w):
+    """Time limuon_step_batched on the workload's matrices (bf16 W and G, fp32
+    M, one Gaussian test matrix per distinct column count), with the first
+    step of one matrix per shape group checked against the fp64 oracle."""
+    import numpy as np
+    import torch
+    import muon_family_optimizer_b200 as mo
+    from muon_family_optimizer_b200 import synthetic as syn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    hp = LIMUON_HP
+    k = hp["rank"] + hp["oversample"]
+    shapes = [tuple(sh) for sh in w["shapes"]]
+    omegas, params = {}, []
+    for j, (r, c) in enumerate(shapes):
+        if c not in omegas:
+            omegas[c] = torch.randn(c, k, generator=torch.Generator(device=dev).manual_seed(c), device=dev)
+        params.append(dict(W=syn.initial_weight(w["name"], j, r, c).to(torch.bfloat16).to(dev),
+                           G=syn.gradient(w["name"], j, 0, r, c, device=dev).to(torch.bfloat16),
+                           M=torch.zeros(r, c, device=dev), Omega=omegas[c]))
+    # parity: the first step of one matrix per shape group, O stored
+    pick = {}
+    for j, sh in enumerate(shapes):
+        pick.setdefault(sh, j)
+    probe = [dict(W=params[j]["W"].clone(), G=params[j]["G"], M=torch.zeros_like(params[j]["M"]),
+                  Omega=params[j]["Omega"], O_out=torch.empty_like(params[j]["M"])) for j in pick.values()]
+    ws = torch.empty(mo.limuon_workspace_size(params, hp), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    mo.limuon_step_batched(probe, mo.BF16, hp, ws, d_status=status)
+    torch.cuda.synchronize(dev)
+    parity, cpu = {}, None
+    if not args.no_cpu_baseline:
+        # CPU-baseline leg: the fp64 oracle's LiMuon step on one matrix per shape group,
+        # timed, and its O compared with the GPU's
+        from oracle import limuon as lim
+        secs, el_sample = 0.0, 0
+        for ((r, c), j), p in zip(pick.items(), probe):
+            W0 = params[j]["W"].double().cpu().numpy()       # not yet stepped
+            G = p["G"].double().cpu().numpy()
+            Om = p["Omega"].double().cpu().numpy()
+            t0 = time.perf_counter()
+            ref = lim.limuon_step(W0, G, np.zeros_like(G), Om, mu=hp["mu"],
+                                  eta=hp["eta"], lam=hp["lambda"], gamma=hp["gamma"], rank=hp["rank"])
+            secs += time.perf_counter() - t0
+            el_sample += r * c
+            O = lim.rsvd_orthogonal(p["M"].double().cpu().numpy(), Om, hp["rank"])
+            Og = p["O_out"].double().cpu().numpy()
+            parity[f"{r}x{c}"] = {"O": float(np.linalg.norm(Og - O) / max(np.linalg.norm(O), 1e-300)),
+                                  "W": float(np.linalg.norm(p["W"].double().cpu().numpy() - ref["W"])
+                                             / np.linalg.norm(ref["W"])),
+                                  "status": int(status.item())}
+        el_all = sum(r * c for r, c in shapes)
+        cpu = {"value": secs * el_all / el_sample * 1e3, "unit": "ms", "cores": len(os.sched_getaffinity(0)),
+               "kind": "oracle", "sample": f"one matrix per shape group ({', '.join(f'{r}x{c}' for r, c in pick)}): "
+                                           f"fp64 LiMuon step (numpy QR and SVD), {secs:.2f} s, scaled to all "
+                                           f"{len(shapes)} matrices by element count"}
+    arr = mo.make_rsvd_params(params)
+    for _ in range(args.warmup):
+        mo.limuon_step_batched(arr, mo.BF16, hp, ws, d_status=status)
+    torch.cuda.synchronize(dev)
+    # per-kernel device times: one traced eager pass
+    mo.muon_trace_enable(True)
+    mo.muon_trace_read()
+    n_tr = 5
+    for _ in range(n_tr):
+        mo.limuon_step_batched(arr, mo.BF16, hp, ws, d_status=status)
+    torch.cuda.synchronize(dev)
+    recs = mo.muon_trace_read()
+    mo.muon_trace_enable(False)
+    per = len(recs) // n_tr
+    kms = [0.0] * per
+    for i, (_, _, ms_) in enumerate(recs):
+        kms[i % per] += ms_ / n_tr
+    stream = torch.cuda.current_stream(dev)
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    with torch.cuda.graph(graph, stream=cap):
+        mo.limuon_step_batched(arr, mo.BF16, hp, ws, d_status=status, stream=torch.cuda.current_stream(dev))
+    for _ in range(3):
+        graph.replay()
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    by, fl = limuon_kernel_work(shapes, k)
+    pk, src = peaks()
+    kernels = {}
+    for i, name in enumerate(LIMUON_KERNELS[:per]):
+        t = kms[i] / 1e3
+        kernels[name] = {"us": kms[i] * 1e3, "GB/s": by[i] / t / 1e9, "TFLOP/s": fl[i] / t / 1e12,
+                         "hbm_frac": by[i] / t / 1e9 / pk["hbm_gbs"], "alu_frac": fl[i] / t / 1e12 / FP32_ALU_TFLOPS}
+    top = max(range(per), key=lambda i: kms[i])
+    t_top = kms[top] / 1e3
+    # the binding roof of the dominant kernel: the larger of its memory and arithmetic times
+    if fl[top] / (FP32_ALU_TFLOPS * 1e12) > by[top] / (pk["hbm_gbs"] * 1e9):
+        roof = {"bound": "alu", "achieved": fl[top] / t_top / 1e12, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": fl[top] / t_top / 1e12 / FP32_ALU_TFLOPS, "traffic": None,
+                "peak_source": "fp32 FMA units x 1965 MHz maximum SM clock (derived)"}
+    else:
+        roof = {"bound": "hbm", "achieved": by[top] / t_top / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": by[top] / t_top / 1e9 / pk["hbm_gbs"], "traffic": None, "peak_source": f"{src} (copy)"}
+    roof["kernel"] = LIMUON_KERNELS[top]
+    el = sum(r * c for r, c in shapes)
+    line = {"metric": "LiMuon optimizer step time, ms", "value": ms, "unit": "ms", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 W/G, fp32 M and products, fp64 k x k factors",
+            "data": "synthetic",
+            "config": {"workload": f"{w['name']}: {len(shapes)} matrices, {el} elements, rank {hp['rank']}, "
+                                   f"oversampling {hp['oversample']}",
+                       "l2": f"inputs larger than L2: {el * 14 / 1e9:.2f} GB of W, G and M per step",
+                       "kernels": kernels, "launches_per_step": per},
+            "roofline": roof, "cpu_baseline": cpu,
+            "parity": {"vs": "fp64 oracle from the GPU's own fp32 momentum, relative Frobenius", "groups": parity},
+            "gpu_launches": per * args.steps, "clocks": clk, "launch": "graph (one CUDA graph per step)"}
+    print(json.dumps(line), flush=True)
+    del graph
+
+
 def run_polar_route(args, w):
     """Time gram_polar (Gram route with restarts and the 1.05 divisor) or ns_polar
     with the same converged schedule on the workload's matrices (log-spaced
@@ -456,6 +605,8 @@ def main():
         return run_reference(args, w, ns_steps)
     if args.route == "adamw":
         return run_adamw_route(args, w)
+    if args.route == "limuon":
+        return run_limuon_route(args, w)
     if args.route != "step":
         return run_polar_route(args, w)
 

@@ -221,6 +221,57 @@ MUON_API muon_status adamw_step_batched(const muon_vec_param* params, int n, muo
                                muon_stream_t stream);
 
 /*
+ * LiMuon ([LiMuon] section "Метод": Muon's momentum, with the update taken
+ * from a randomized SVD of the momentum).  The page gives no formulas; read
+ * as the basic randomized SVD of Halko, Martinsson and Tropp ("Finding
+ * structure with randomness", 2011) in place of the Newton-Schulz iteration:
+ *     M <- mu M + G
+ *     Y = M Omega,  Q = orth(Y),  B = Q^T M = U~ S V^T,  U = Q U~
+ *     O = U_r V_r^T over the r = rank largest singular values
+ *     W <- W - eta (gamma O + lambda W)
+ * Omega (cols x k, k = rank + oversample <= 64) is the caller's test matrix:
+ * the method draws it (Gaussian, fresh or fixed) and passes it in.  Singular
+ * values at or below 1e-5 of the largest count as zero and are left out, so a
+ * rank-deficient M gives a partial isometry and M = 0 gives O = 0.  Y, Q and
+ * the products run in fp32; the k x k Gram, Cholesky and eigen steps in fp64.
+ */
+typedef struct {
+    int rows, cols;       /* >= 1 */
+    void* W;              /* rows x cols, w_dtype, updated in place */
+    const void* G;        /* rows x cols, w_dtype, this step's gradient (read only) */
+    float* M;             /* rows x cols, fp32 momentum, updated in place (zero initially) */
+    const float* Omega;   /* cols x k fp32 test matrix, row-major, read only; parameters with the
+                             same cols may share one */
+    float gamma;          /* per-matrix gamma; NaN means "use hparams.gamma" */
+    float* O_out;         /* optional rows x cols fp32: receives O; NULL to skip */
+} muon_rsvd_param;
+
+typedef struct {
+    float mu, eta, lambda, gamma;
+    int rank;             /* r >= 1 */
+    int oversample;       /* p >= 0; k = r + p <= 64 (else MUON_ERR_UNSUPPORTED) */
+} muon_rsvd_hparams;
+
+/* Bytes of workspace limuon_step_batched needs (only rows/cols are read). */
+MUON_API muon_status limuon_workspace_size(const muon_rsvd_param* params, int n, const muon_rsvd_hparams* hp,
+                                           size_t* bytes);
+
+/*
+ * One LiMuon step for n matrix parameters, asynchronous on `stream`: five
+ * launches per 128 parameters (fused momentum pass and sketch; per-matrix
+ * QR; projection; per-matrix eigen-decomposition; O fused with the weight
+ * update, O never stored unless O_out is given).  workspace: device,
+ * 256-byte aligned, at least limuon_workspace_size bytes; no state is kept
+ * in it between calls.  Argument errors return before any launch.  A matrix
+ * whose new momentum holds a non-finite value keeps its W, and
+ * MUON_FLAG_NONFINITE is OR-ed into *d_status (when given).  Parameters may
+ * not overlap one another (Omega excepted, which is only read).
+ */
+MUON_API muon_status limuon_step_batched(const muon_rsvd_param* params, int n, muon_dtype w_dtype,
+                                         const muon_rsvd_hparams* hp, void* workspace, size_t ws_bytes,
+                                         int* d_status, muon_stream_t stream);
+
+/*
  * Bytes of workspace ns_polar / gram_polar need for a batch of rows x cols
  * matrices in `dtype`.
  */
@@ -297,7 +348,9 @@ typedef enum {
     MUON_KERNEL_UPD = 2,       /* tcgen05 update product X <- aX + BX, Q Xb (work = flops) */
     MUON_KERNEL_SIMT = 3,      /* fp32 CUDA-core product (work = flops) */
     MUON_KERNEL_OTHER = 4,     /* identity fill (work = bytes) */
-    MUON_KERNEL_ADAMW = 5      /* AdamW streaming pass over vector parameters (work = bytes) */
+    MUON_KERNEL_ADAMW = 5,     /* AdamW streaming pass over vector parameters (work = bytes) */
+    MUON_KERNEL_RSVD = 6,      /* LiMuon streaming passes: momentum + sketch, projection, update (work = bytes) */
+    MUON_KERNEL_RSVD_SMALL = 7 /* LiMuon per-matrix factorisations: QR, eigen-decomposition (work = bytes) */
 } muon_kernel_kind;
 
 typedef struct {

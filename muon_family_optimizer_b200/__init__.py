@@ -64,14 +64,26 @@ class VecParam(ctypes.Structure):
                 ("m", ctypes.c_void_p), ("v", ctypes.c_void_p)]
 
 
+class RsvdParam(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("cols", ctypes.c_int), ("W", ctypes.c_void_p),
+                ("G", ctypes.c_void_p), ("M", ctypes.c_void_p), ("Omega", ctypes.c_void_p),
+                ("gamma", ctypes.c_float), ("O_out", ctypes.c_void_p)]
+
+
+class RsvdHParams(ctypes.Structure):
+    _fields_ = [("mu", ctypes.c_float), ("eta", ctypes.c_float), ("lambda_", ctypes.c_float),
+                ("gamma", ctypes.c_float), ("rank", ctypes.c_int), ("oversample", ctypes.c_int)]
+
+
 class AdamWHParams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float)]
 
 
-KERNEL_PREPASS, KERNEL_SYM, KERNEL_UPD, KERNEL_SIMT, KERNEL_OTHER, KERNEL_ADAMW = range(6)
+(KERNEL_PREPASS, KERNEL_SYM, KERNEL_UPD, KERNEL_SIMT, KERNEL_OTHER, KERNEL_ADAMW, KERNEL_RSVD,
+ KERNEL_RSVD_SMALL) = range(8)
 KERNEL_NAMES = {KERNEL_PREPASS: "prepass", KERNEL_SYM: "tc_sym", KERNEL_UPD: "tc_upd", KERNEL_ADAMW: "adamw",
-                KERNEL_SIMT: "simt", KERNEL_OTHER: "other"}
+                KERNEL_SIMT: "simt", KERNEL_OTHER: "other", KERNEL_RSVD: "rsvd", KERNEL_RSVD_SMALL: "rsvd_small"}
 TRACE_CAPACITY = 8192
 
 
@@ -107,6 +119,11 @@ def lib():
         L.muon_lite_step_batched.argtypes = [ctypes.POINTER(LiteParam), ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.POINTER(HParams), ctypes.POINTER(Schedule), vp,
                                              ctypes.c_size_t, vp, vp]
+        L.limuon_workspace_size.restype = st
+        L.limuon_workspace_size.argtypes = [ctypes.POINTER(RsvdParam), ctypes.c_int, ctypes.POINTER(RsvdHParams), sz]
+        L.limuon_step_batched.restype = st
+        L.limuon_step_batched.argtypes = [ctypes.POINTER(RsvdParam), ctypes.c_int, ctypes.c_int,
+                                          ctypes.POINTER(RsvdHParams), vp, ctypes.c_size_t, vp, vp]
         L.muon_wait_selftest.restype = st
         L.muon_wait_selftest.argtypes = [ctypes.c_int, vp, vp]
         L.adamw_step_batched.restype = st
@@ -271,6 +288,54 @@ def adamw_step_batched(params, w_dtype, hp, step, d_status=None, stream=None):
     h = AdamWHParams(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
     _check(lib().adamw_step_batched(arr, len(arr), int(w_dtype), ctypes.byref(h), int(step), _ptr(d_status),
                                     _stream_ptr(stream)), "adamw_step_batched")
+
+
+def make_rsvd_params(params):
+    """params: list of dicts with torch tensors W, G (same dtype), M (float32), Omega (float32,
+    cols x k), optional O_out (float32) and gamma (float); rows x cols, contiguous."""
+    import torch
+    arr = (RsvdParam * len(params))()
+    for i, p in enumerate(params):
+        W = p["W"]
+        if W.dim() != 2:
+            raise ValueError(f"param {i}: W must be 2-D")
+        rows, cols = W.shape
+        for k in ("W", "G", "M", "Omega") + (("O_out",) if p.get("O_out") is not None else ()):
+            if not p[k].is_contiguous():
+                raise ValueError(f"param {i}: {k} must be contiguous")
+        if p["G"].shape != W.shape or p["M"].shape != W.shape or p["G"].dtype != W.dtype:
+            raise ValueError(f"param {i}: G must match W; M must be rows x cols")
+        if p["M"].dtype != torch.float32 or p["Omega"].dtype != torch.float32 or p["Omega"].dim() != 2 \
+                or p["Omega"].shape[0] != cols:
+            raise ValueError(f"param {i}: M must be float32 and Omega float32 cols x k")
+        O = p.get("O_out")
+        if O is not None and (O.shape != W.shape or O.dtype != torch.float32):
+            raise ValueError(f"param {i}: O_out must be float32 rows x cols")
+        arr[i] = RsvdParam(rows, cols, W.data_ptr(), p["G"].data_ptr(), p["M"].data_ptr(), p["Omega"].data_ptr(),
+                           float(p.get("gamma", float("nan"))), O.data_ptr() if O is not None else None)
+    return arr
+
+
+def _rsvd_hp(hp):
+    return RsvdHParams(hp["mu"], hp["eta"], hp["lambda"], hp["gamma"], int(hp["rank"]), int(hp["oversample"]))
+
+
+def limuon_workspace_size(params, hp):
+    arr = params if isinstance(params, ctypes.Array) else make_rsvd_params(params)
+    out = ctypes.c_size_t(0)
+    h = _rsvd_hp(hp)
+    _check(lib().limuon_workspace_size(arr, len(arr), ctypes.byref(h), ctypes.byref(out)), "limuon_workspace_size")
+    return out.value
+
+
+def limuon_step_batched(params, w_dtype, hp, workspace, d_status=None, stream=None):
+    """One LiMuon step (see include/muon.h).  hp: dict with mu, eta, lambda, gamma, rank,
+    oversample; every Omega has rank + oversample columns."""
+    arr = params if isinstance(params, ctypes.Array) else make_rsvd_params(params)
+    h = _rsvd_hp(hp)
+    _check(lib().limuon_step_batched(arr, len(arr), int(w_dtype), ctypes.byref(h), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _ptr(d_status),
+                                     _stream_ptr(stream)), "limuon_step_batched")
 
 
 def muon_wait_selftest(wait_ms, d_status, stream=None):

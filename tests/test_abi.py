@@ -58,6 +58,12 @@ int main(void) {
   printf("muon_lite_param %zu\n", sizeof(muon_lite_param));
   printf("muon_vec_param %zu\n", sizeof(muon_vec_param));
   printf("muon_adamw_hparams %zu\n", sizeof(muon_adamw_hparams));
+  printf("muon_rsvd_param %zu\n", sizeof(muon_rsvd_param));
+  printf("muon_rsvd_hparams %zu\n", sizeof(muon_rsvd_hparams));
+  P(muon_rsvd_param, rows) P(muon_rsvd_param, cols) P(muon_rsvd_param, W) P(muon_rsvd_param, G)
+  P(muon_rsvd_param, M) P(muon_rsvd_param, Omega) P(muon_rsvd_param, gamma) P(muon_rsvd_param, O_out)
+  P(muon_rsvd_hparams, mu) P(muon_rsvd_hparams, eta) P(muon_rsvd_hparams, lambda) P(muon_rsvd_hparams, gamma)
+  P(muon_rsvd_hparams, rank) P(muon_rsvd_hparams, oversample)
   P(muon_vec_param, n) P(muon_vec_param, W) P(muon_vec_param, G) P(muon_vec_param, m) P(muon_vec_param, v)
   P(muon_adamw_hparams, lr) P(muon_adamw_hparams, beta1) P(muon_adamw_hparams, beta2) P(muon_adamw_hparams, eps)
   P(muon_adamw_hparams, weight_decay)
@@ -87,9 +93,12 @@ def test_binding_struct_layout_matches_header(tmp_path):
     assert int(got["muon_lite_param"]) == ctypes.sizeof(mo.LiteParam)
     assert int(got["muon_vec_param"]) == ctypes.sizeof(mo.VecParam)
     assert int(got["muon_adamw_hparams"]) == ctypes.sizeof(mo.AdamWHParams)
+    assert int(got["muon_rsvd_param"]) == ctypes.sizeof(mo.RsvdParam)
+    assert int(got["muon_rsvd_hparams"]) == ctypes.sizeof(mo.RsvdHParams)
     py = {"muon_param": mo.Param, "muon_schedule": mo.Schedule, "muon_hparams": mo.HParams,
           "muon_lite_param": mo.LiteParam, "muon_vec_param": mo.VecParam,
-          "muon_adamw_hparams": mo.AdamWHParams}
+          "muon_adamw_hparams": mo.AdamWHParams, "muon_rsvd_param": mo.RsvdParam,
+          "muon_rsvd_hparams": mo.RsvdHParams}
     for key, val in got.items():
         if "." not in key:
             continue
@@ -187,3 +196,34 @@ def test_adamw_argument_checks(lib):
     assert L.adamw_step_batched(nul, 1, mo.BF16, ctypes.byref(good), 1, None, None) == mo.ERR_INVALID_ARG
     empty = (mo.VecParam * 1)(mo.VecParam(0, p, p, p, p))
     assert L.adamw_step_batched(empty, 1, mo.BF16, ctypes.byref(good), 1, None, None) == mo.ERR_INVALID_ARG
+
+
+def test_limuon_argument_checks(lib):
+    L = lib
+    buf = ctypes.create_string_buffer(4096)
+    p = ctypes.cast(buf, ctypes.c_void_p).value
+    ws = (p + 255) & ~255
+    good = mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 16, 16)
+    one = (mo.RsvdParam * 1)(mo.RsvdParam(4, 8, p, p, p, p, float("nan"), None))
+    size = ctypes.c_size_t(0)
+    assert L.limuon_workspace_size(one, 1, ctypes.byref(good), ctypes.byref(size)) == mo.OK
+    # 4 per-matrix flags, then Y (4 x 32 floats) and B^T (8 x 32 floats), each 256-byte aligned
+    assert size.value == 256 + 512 + 1024
+    big = mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 40, 8)
+    assert L.limuon_workspace_size(one, 1, ctypes.byref(big), ctypes.byref(size)) == mo.OK
+    assert size.value == 256 + 1024 + 2048                 # k = 48 runs on 64 columns
+    too_big = mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 60, 5)
+    assert L.limuon_workspace_size(one, 1, ctypes.byref(too_big), ctypes.byref(size)) == mo.ERR_UNSUPPORTED
+    for bad in (mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 0, 4), mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 4, -1),
+                mo.RsvdHParams(float("nan"), 0.02, 0.0, 1.0, 4, 4), mo.RsvdHParams(0.95, float("inf"), 0.0, 1.0, 4, 4)):
+        assert L.limuon_workspace_size(one, 1, ctypes.byref(bad), ctypes.byref(size)) == mo.ERR_INVALID_ARG
+        assert L.limuon_step_batched(one, 1, mo.BF16, ctypes.byref(bad), ws, 2048, None, None) == mo.ERR_INVALID_ARG
+    assert L.limuon_step_batched(one, 0, mo.BF16, ctypes.byref(good), ws, 2048, None, None) == mo.ERR_INVALID_ARG
+    assert L.limuon_step_batched(one, 1, 7, ctypes.byref(good), ws, 2048, None, None) == mo.ERR_INVALID_ARG
+    assert L.limuon_step_batched(one, 1, mo.BF16, ctypes.byref(good), ws, 1000, None, None) == mo.ERR_WORKSPACE
+    assert L.limuon_step_batched(one, 1, mo.BF16, ctypes.byref(good), None, 4096, None, None) == mo.ERR_WORKSPACE
+    assert L.limuon_step_batched(one, 1, mo.BF16, ctypes.byref(good), ws + 16, 2048, None, None) == mo.ERR_INVALID_ARG
+    nul = (mo.RsvdParam * 1)(mo.RsvdParam(4, 8, p, p, p, None, float("nan"), None))
+    assert L.limuon_step_batched(nul, 1, mo.BF16, ctypes.byref(good), ws, 2048, None, None) == mo.ERR_INVALID_ARG
+    empty = (mo.RsvdParam * 1)(mo.RsvdParam(0, 8, p, p, p, p, float("nan"), None))
+    assert L.limuon_workspace_size(empty, 1, ctypes.byref(good), ctypes.byref(size)) == mo.ERR_INVALID_ARG
