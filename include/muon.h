@@ -17,6 +17,10 @@
  *           by Newton-Schulz on the small Gram matrix, half of every symmetric
  *           product computed and mirrored, restarts, and a division by
  *           1.02-1.05 so that the eigenvalues stay inside [0, 1].
+ *   [LiMuon] "LiMuon: Light and Fast Muon Optimizer for Large Models"
+ *           (arxiv.sitesynth.xyz digest 2509.14562v1), section "Метод":
+ *           Muon's momentum with the update taken from a randomized SVD
+ *           (limuon_step_batched below).
  *
  * Iteration used by every entry point (readings of the pages, which name
  * Newton-Schulz but print no coefficients): on the wide view X (s x l,

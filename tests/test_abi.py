@@ -227,3 +227,18 @@ def test_limuon_argument_checks(lib):
     assert L.limuon_step_batched(nul, 1, mo.BF16, ctypes.byref(good), ws, 2048, None, None) == mo.ERR_INVALID_ARG
     empty = (mo.RsvdParam * 1)(mo.RsvdParam(0, 8, p, p, p, p, float("nan"), None))
     assert L.limuon_workspace_size(empty, 1, ctypes.byref(good), ctypes.byref(size)) == mo.ERR_INVALID_ARG
+
+
+def test_limuon_binding_validates_tensors():
+    import torch
+    W = torch.zeros(4, 8, dtype=torch.bfloat16)
+    ok = dict(W=W, G=torch.zeros(4, 8, dtype=torch.bfloat16), M=torch.zeros(4, 8), Omega=torch.zeros(8, 5))
+    arr = mo.make_rsvd_params([ok])
+    assert arr[0].rows == 4 and arr[0].cols == 8 and arr[0].Omega == ok["Omega"].data_ptr()
+    import math
+    assert math.isnan(arr[0].gamma) and arr[0].O_out is None
+    for bad in (dict(ok, M=torch.zeros(4, 8, dtype=torch.float64)), dict(ok, Omega=torch.zeros(7, 5)),
+                dict(ok, G=torch.zeros(4, 8)), dict(ok, O_out=torch.zeros(4, 8, dtype=torch.bfloat16)),
+                dict(ok, W=torch.zeros(32, dtype=torch.bfloat16)), dict(ok, M=torch.zeros(8, 4).t())):
+        with pytest.raises(ValueError):
+            mo.make_rsvd_params([bad])

@@ -54,3 +54,18 @@ def test_recorded_traffic_requires_matching_sources(tmp_path, monkeypatch):
     with open(root / "muon_family_optimizer_b200" / "csrc" / "gemm_tc.cu", "a") as fh:
         fh.write("\n// changed\n")
     assert bench.recorded_traffic("tc_sym", "gpt2_small", 5) == (None, None)
+
+
+def test_limuon_kernel_work_counts():
+    # one 4 x 6 matrix, k = 3, 16-bit W/G: per element the sketch moves 2 + 4 + 4 bytes, the
+    # projection 4, the update 2 + 2; each of the three products is 3 FMAs per element
+    by, fl = bench.limuon_kernel_work([(4, 6)], 3)
+    assert by == [24 * 10 + 4 * 12, 8 * 12, 24 * 4 + 4 * (12 + 18), 4 * (18 + 24), 24 * 4 + 4 * (12 + 18)]
+    assert fl == [2.0 * 24 * 3, 0.0, 2.0 * 24 * 3, 0.0, 2.0 * 24 * 3]
+    by32, _ = bench.limuon_kernel_work([(4, 6)], 3, w_bytes=4)
+    assert by32[0] - by[0] == 24 * 2 and by32[4] - by[4] == 24 * 4
+
+
+def test_fp32_alu_peak_from_unit_counts():
+    assert abs(bench.FP32_ALU_TFLOPS - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
+    assert 74.0 < bench.FP32_ALU_TFLOPS < 75.0
