@@ -7,7 +7,10 @@ or cannot be loaded, every call raises.
 
 Names follow the C ABI: :func:`muon_step_batched`, :func:`ns_polar`,
 :func:`gram_polar`, :func:`muon_workspace_size`, :func:`ns_polar_workspace_size`,
-:func:`gram_polar_workspace_size`, :func:`muon_status_string`.
+:func:`gram_polar_workspace_size`, :func:`muon_lite_step_batched` (MONA-Lite),
+:func:`adamw_step_batched` (vector parameters), :func:`limuon_step_batched` and
+:func:`limuon_workspace_size` (LiMuon), :func:`ns_polar_noalloc`,
+:func:`muon_status_string`.
 """
 import ctypes
 import math
