@@ -52,6 +52,9 @@ def test_hand_examples(mod=lim):
         assert np.allclose(mod.rsvd_orthogonal(Ms, I2, r), g[f"O_signs_r{r}"].reshape(3, 2), rtol=0, atol=1e-14)
     assert np.allclose(mod.rsvd_orthogonal(g["M_rank1"].reshape(2, 2), I2, 2), g["O_rank1_r2"].reshape(2, 2),
                        rtol=0, atol=1e-14)
+    # one test column: the sketch keeps only range(M Omega), so O is not M's own top factor
+    assert np.allclose(mod.rsvd_orthogonal(g["M_k1"].reshape(2, 3), g["Omega_k1"].reshape(3, 1), 1),
+                       g["O_k1_r1"].reshape(2, 3), rtol=0, atol=1e-14)
 
 
 def test_step_hand_example(mod=lim):
