@@ -5,13 +5,17 @@ A step is one call of muon_step_batched over every matrix of the workload:
 the fused MONA pre-pass with the Frobenius norms, 5 quintic Newton-Schulz
 steps on tensor cores (grouped by shape), and the weight update fused into
 the last step.  Inputs are synthetic (seeded; shapes of the named model).
+The default workload is the largest configuration that fits one GPU: the
+Llama-3-8B layer set (224 matrices, 6.98 G elements).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 value = Newton-Schulz TFLOP/s over all ranks (algorithmic flops: symmetric
 products count the half they need), timed with CUDA events on the step's
-stream between barriers, max over ranks.  Under torchrun each rank steps its
-own copy of the workload (weak scaling, no collective on the data path).
+stream between barriers, max over ranks.  Under torchrun the matrices are
+partitioned across the ranks (flop-balanced, whole matrices) and every step
+ends with one all-gather of the updated weights (strong scaling: the model's
+step is shared); --replicas makes each rank step its own copy instead.
 --impl reference times the fp64 CPU oracle on a bounded sample instead.
 """
 import argparse
@@ -34,9 +38,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="gpt2_small")
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama3_8b")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="take only the first N layers of a layered workload (smaller cases for profiling)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="under torchrun: every rank steps its own copy of the workload (weak scaling) "
+                         "instead of its share of one model (strong scaling, the default)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ns-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -81,10 +90,13 @@ def sources_digest(kernel="tc_sym"):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel, workload, ns_steps):
+def recorded_traffic(kernel, workload, ns_steps, elements=None):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
     ``kernel`` from the ncu summaries under profiles/: a line
-    ``traffic-record: {json}`` written when the counters were taken.  None when
+    ``traffic-record: {json}`` written when the counters were taken.  A record
+    taken on a leading slice of the workload's layers (its "elements" below the
+    launch's) is scaled to the launch by elements: every matrix of a shape
+    group is processed alike, so the traffic grows in proportion.  None when
     no record matches the workload or the kernel sources changed since."""
     d = os.path.join(ROOT, "profiles")
     if not os.path.isdir(d):
@@ -103,7 +115,11 @@ def recorded_traffic(kernel, workload, ns_steps):
                     continue
                 if (rec.get("kernel") == kernel and rec.get("workload") == workload
                         and rec.get("ns_steps") == ns_steps and rec.get("sources") == digest):
-                    return float(rec["bytes_per_launch"]), f"profiles/{name}"
+                    b = float(rec["bytes_per_launch"])
+                    rec_el = rec.get("elements")
+                    if rec_el and elements and rec_el != elements:
+                        return b * elements / rec_el, f"profiles/{name} (scaled by elements from {rec_el})"
+                    return b, f"profiles/{name}"
     return None, None
 
 
@@ -190,13 +206,14 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle (baseline and reference arm)
 
-def oracle_sample_run(w, shapes, seed_base=0):
-    """One full MONA/Muon step in fp64 on the given shapes; returns seconds."""
+def oracle_sample_run(w, picks, seed_base=0):
+    """One full MONA/Muon step in fp64 on the matrices `picks` ((j, rows, cols),
+    j = the matrix's index in the workload); returns seconds."""
     import numpy as np
     import oracle
     from muon_family_optimizer_b200 import synthetic as syn
     arrays = []
-    for j, (r, c) in enumerate(shapes):
+    for j, r, c in picks:
         W = syn.initial_weight(w["name"], j, r, c).double().numpy()
         G = syn.gradient(w["name"], j, seed_base, r, c).double().numpy()
         Gp = syn.gradient(w["name"], j, seed_base + 8, r, c).double().numpy()
@@ -209,20 +226,47 @@ def oracle_sample_run(w, shapes, seed_base=0):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, ns_steps):
+def shape_groups(shapes):
+    """Matrices of each (short side, long side) group: [(cost, [(j, rows, cols), ...])],
+    cheapest group first (cost = one matrix's algorithmic NS flops)."""
+    groups = {}
+    for j, (r, c) in enumerate(shapes):
+        groups.setdefault((min(r, c), max(r, c)), []).append((j, r, c))
+    out = [(ns_flops([(m[0][1], m[0][2])], 5), m) for m in groups.values()]
+    return sorted(out, key=lambda x: x[0])
+
+
+# fp64 oracle work per matrix beyond which it is left out of the bench's CPU legs
+# (a 4096 x 4096 matrix is 1.4 TFLOP: about half a minute on 16 host cores)
+ORACLE_MATRIX_FLOPS = 2.5e11
+
+
+def cpu_baseline(w, ns_steps, budget_s=25.0, floor_s=10.0):
+    """The fp64 oracle's rate on a bounded sample of the workload: one matrix of
+    each shape group, cheapest first, while the predicted time stays within
+    budget_s, then further matrices of the cheapest group until floor_s."""
     import oracle
-    seen, sample = set(), []
-    for r, c in w["shapes"]:
-        key = (min(r, c), max(r, c))
-        if key not in seen:
-            seen.add(key)
-            sample.append((r, c))
-    secs = oracle_sample_run(w, sample)
-    fl = ns_flops(sample, ns_steps)
+    groups = shape_groups(w["shapes"])
+    picks, secs, fl = [], 0.0, 0.0
+    for cost, members in groups:
+        if picks and (cost > ORACLE_MATRIX_FLOPS or secs + cost * secs / fl > budget_s):
+            break
+        secs += oracle_sample_run(w, [members[0]])
+        fl += ns_flops([members[0][1:]], ns_steps)
+        picks.append(members[0])
+    more = iter(groups[0][1][1:])
+    for m in more:
+        if secs >= floor_s:
+            break
+        secs += oracle_sample_run(w, [m])
+        fl += ns_flops([m[1:]], ns_steps)
+        picks.append(m)
     full = ns_flops(w["shapes"], ns_steps)
+    from collections import Counter
+    desc = ", ".join(f"{n} x {r}x{c}" for (r, c), n in Counter((r, c) for _, r, c in picks).items())
     return {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"one matrix per shape group ({', '.join(f'{r}x{c}' for r, c in sample)}): full "
-                      f"fp64 MONA step with {ns_steps} quintic steps, {secs:.2f} s",
+            "sample": f"{len(picks)} matrices of the workload ({desc}): full fp64 MONA step with {ns_steps} "
+                      f"quintic steps each, {secs:.2f} s; rate = their algorithmic NS flops / time",
             "ms_per_step_extrapolated": secs * full / fl * 1e3}
 
 
@@ -230,18 +274,22 @@ def group_parity(w, ns_steps, dev):
     """Maximum relative errors per shape group: one matrix of each (s, l) group,
     one step on the GPU through muon_step_batched (with O stored) and the same
     step in the fp64 oracle from the same 16-bit inputs (the iteration started
-    from the same rounded momentum).  Returns {"s x l": {"O": e, "W": e, "M": e}}."""
+    from the same rounded momentum).  Groups whose oracle step would take more
+    than a few seconds are listed as skipped (the full-size GPU tests check
+    them).  Returns {"s x l": {"O": e, "W": e, "M": e}}."""
     import numpy as np
     import torch
     import muon_family_optimizer_b200 as mo
     import oracle
     from muon_family_optimizer_b200 import synthetic as syn
     w_dt, ns_dt = w["w_dtype"], w["ns_dtype"]
-    seen, pick = set(), []
-    for j, (r, c) in enumerate(w["shapes"]):
-        key = (min(r, c), max(r, c))
-        if key not in seen:
-            seen.add(key)
+    pick, out = [], {}
+    for cost, members in shape_groups(w["shapes"]):
+        j, r, c = members[0]
+        if cost > ORACLE_MATRIX_FLOPS:
+            out[f"{min(r, c)}x{max(r, c)}"] = {"skipped": f"{cost / 1e12:.2f} TFLOP per matrix in fp64; "
+                                                           "checked by the full-size GPU tests"}
+        else:
             pick.append((j, r, c))
     host, params = [], []
     for j, r, c in pick:
@@ -251,6 +299,8 @@ def group_parity(w, ns_steps, dev):
         p = {k: v.to(dev).contiguous() for k, v in st.items()}
         p["O_out"] = torch.empty(r, c, device=dev)
         params.append(p)
+    if not params:
+        return out
     ws = torch.empty(mo.muon_workspace_size(params, mo._dtype_code(ns_dt)), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     mo.muon_step_batched(params, mo._dtype_code(w_dt), mo._dtype_code(ns_dt), w["hp"],
@@ -259,7 +309,6 @@ def group_parity(w, ns_steps, dev):
     rnd = {torch.bfloat16: oracle.ROUND_BF16, torch.float16: oracle.ROUND_FP16}.get(ns_dt, oracle.ROUND_NONE)
     hp = w["hp"]
     rel = lambda a, b: float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
-    out = {}
     for (j, r, c), st, p in zip(pick, host, params):
         f = {k: v.double().numpy() for k, v in st.items()}
         ref = oracle.muon_step(f["W"], f["G"], f["G_prev"], f["A"], f["M"], mu=hp["mu"], eta=hp["eta"],
@@ -272,43 +321,44 @@ def group_parity(w, ns_steps, dev):
 
 
 def run_reference(args, w, ns_steps):
+    """The reference arm: the fp64 oracle on the host cores.  Each timed step is
+    one full MONA step of one matrix of the workload (the shape groups whose
+    oracle step takes at most a few seconds, in turn), so K steps finish within
+    minutes; value = algorithmic NS flops / time, ms_per_step = the timed
+    sample step, the whole-workload time extrapolated by flops."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle
-    shapes_by_group = []
-    seen = set()
-    for r, c in w["shapes"]:
-        key = (min(r, c), max(r, c))
-        if key not in seen:
-            seen.add(key)
-            shapes_by_group.append((r, c))
-    # one matrix per step, cycling through the shape groups, smallest first
-    shapes_by_group.sort(key=lambda rc: rc[0] * rc[1])
+    groups = [members for cost, members in shape_groups(w["shapes"]) if cost <= ORACLE_MATRIX_FLOPS]
+    if not groups:
+        groups = [shape_groups(w["shapes"])[0][1]]
+    # step i takes group i % len(groups), cycling through that group's matrices
+    order = [groups[i % len(groups)][(i // len(groups)) % len(groups[i % len(groups)])]
+             for i in range(args.warmup + args.steps)]
     for i in range(args.warmup):
-        oracle_sample_run(w, [shapes_by_group[i % len(shapes_by_group)]], seed_base=i)
+        oracle_sample_run(w, [order[i]], seed_base=i)
     fl = secs = 0.0
     steps = 0
-    budget = 150.0
-    t_start = time.perf_counter()
     for i in range(args.steps):
-        sh = shapes_by_group[i % len(shapes_by_group)]
-        secs += oracle_sample_run(w, [sh], seed_base=i)
-        fl += ns_flops([sh], ns_steps)
+        m = order[args.warmup + i]
+        secs += oracle_sample_run(w, [m], seed_base=i)
+        fl += ns_flops([m[1:]], ns_steps)
         steps += 1
-        if time.perf_counter() - t_start > budget:
-            break
     value = fl / secs / 1e12
     full = ns_flops(w["shapes"], ns_steps)
-    ms_step = secs / fl * full * 1e3
-    groups, nel = describe(args.workload, w)
+    groups_desc, nel = describe(args.workload, w)
+    from collections import Counter
+    used = ", ".join(f"{r}x{c}" for (r, c) in Counter((m[1], m[2]) for m in order[args.warmup:]))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-            "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": secs / steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{args.workload}: {groups}", "elements": nel, "ns_steps": ns_steps},
+            "config": {"workload": f"{w['name']}: {groups_desc}", "elements": nel, "ns_steps": ns_steps},
+            "ms_per_step_extrapolated": secs / fl * full * 1e3,
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-                             "sample": f"{steps} timed steps, each one full fp64 MONA step of one matrix "
-                                       "(cycling through the shape groups); ms_per_step extrapolated"},
+                             "sample": f"{steps} timed steps, each one full fp64 MONA step of one matrix of the "
+                                       f"workload ({used}); ms_per_step is that sample step, "
+                                       "ms_per_step_extrapolated the whole workload by flops"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -595,11 +645,28 @@ def run_polar_route(args, w):
     del g
 
 
-def main():
-    args = parse()
+def select_workload(args):
     from muon_family_optimizer_b200 import synthetic as syn
     w = dict(syn.WORKLOADS[args.workload])
     w["name"] = args.workload
+    if args.layers:
+        if not w.get("layer_size"):
+            raise SystemExit(f"--layers: {args.workload} has no layer structure")
+        n = args.layers * w["layer_size"]
+        if n > len(w["shapes"]):
+            raise SystemExit(f"--layers: {args.workload} has {len(w['shapes']) // w['layer_size']} layers")
+        w["shapes"] = w["shapes"][:n]
+    return w
+
+
+def workload_label(args, w):
+    name = args.workload + (f"[{args.layers} layers]" if args.layers else "")
+    return name
+
+
+def main():
+    args = parse()
+    w = select_workload(args)
     ns_steps = args.ns_steps
     if args.impl == "reference":
         return run_reference(args, w, ns_steps)
@@ -609,10 +676,15 @@ def main():
         return run_limuon_route(args, w)
     if args.route != "step":
         return run_polar_route(args, w)
+    return run_step_route(args, w, ns_steps)
 
+
+def run_step_route(args, w, ns_steps):
     import torch
     import torch.distributed as dist
     import muon_family_optimizer_b200 as mo
+    from muon_family_optimizer_b200 import sharding
+    from muon_family_optimizer_b200 import synthetic as syn
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -622,24 +694,34 @@ def main():
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    sharded = world > 1 and not args.replicas
+    lite = args.variant == "lite"
 
     w_dt, ns_dt = w["w_dtype"], w["ns_dtype"]
     shapes = w["shapes"]
-    # ---- state (each rank its own copy); gradients live in one buffer per set
+    assignment = sharding.partition(shapes, world) if sharded else None
+    owned = assignment[rank] if sharded else list(range(len(shapes)))
+    # ---- state: weights of every matrix (replicas); gradients and optimizer
+    # state of the matrices this rank steps; two gradient sets in one buffer each
+    nel_owned = sum(shapes[j][0] * shapes[j][1] for j in owned)
     nel = sum(r * c for r, c in shapes)
     esz = torch.empty((), dtype=w_dt).element_size()
-    gbuf = [torch.empty(nel, dtype=w_dt, device=dev) for _ in range(2)]
-    params = [[], []]
-    off = 0
+    gbuf = [torch.empty(max(1, nel_owned), dtype=w_dt, device=dev) for _ in range(2)]
+    full = [[None] * len(shapes), [None] * len(shapes)]   # per gradient set: every matrix's dict
     torch.manual_seed(1234 + rank)
     cache = {}
+    off = 0
+    mine = set(owned)
     for j, (r, c) in enumerate(shapes):
+        W = syn.initial_weight(args.workload, j, r, c, device=dev).to(w_dt)
+        if j not in mine:
+            full[0][j] = full[1][j] = dict(W=W)
+            continue
         key = (r, c)
         if key not in cache:
             cache[key] = [syn.gradient(args.workload, j, t, r, c, device=dev) for t in range(2)]
-        W = syn.initial_weight(args.workload, j, r, c, device=dev).to(w_dt)
         M = torch.zeros(r, c, dtype=torch.float32, device=dev)
-        if args.variant == "lite":
+        if lite:
             B = (cache[key][1] * -0.01).to(torch.bfloat16).contiguous()
         else:
             Gp = cache[key][1].to(w_dt).contiguous()
@@ -648,23 +730,33 @@ def main():
             g = gbuf[t][off:off + r * c].view(r, c)
             sign = torch.randint(0, 2, (1, c), device=dev, dtype=torch.int8).float() * 2 - 1
             g.copy_(cache[key][t] * sign)
-            params[t].append(dict(W=W, G=g, B=B, M=M) if args.variant == "lite" else
-                             dict(W=W, G=g, G_prev=Gp, A=A, M=M))
+            full[t][j] = dict(W=W, G=g, B=B, M=M) if lite else dict(W=W, G=g, G_prev=Gp, A=A, M=M)
         off += r * c
     del cache
-    lite = args.variant == "lite"
-    arrs = [(mo.make_lite_params if lite else mo.make_params)(p) for p in params]
+    params = [[full[t][j] for j in owned] for t in range(2)]
+    arrs = [(mo.make_lite_params if lite else mo.make_params)(p) for p in params] if owned else None
     sched = mo.quintic_schedule(ns_steps)
-    ws = torch.empty((mo.muon_lite_workspace_size if lite else mo.muon_workspace_size)(arrs[0], mo._dtype_code(ns_dt)),
-                     dtype=torch.uint8, device=dev)
+    ws_size = ((mo.muon_lite_workspace_size if lite else mo.muon_workspace_size)(arrs[0], mo._dtype_code(ns_dt))
+               if owned else 256)
+    ws = torch.empty(ws_size, dtype=torch.uint8, device=dev)
     step_fn = mo.muon_lite_step_batched if lite else mo.muon_step_batched
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     wcode, ncode = mo._dtype_code(w_dt), mo._dtype_code(ns_dt)
+    if sharded and lite:
+        raise SystemExit("the sharded step runs the MONA variant; use --replicas with --variant lite")
+    xbuf = None
+    if sharded:
+        per = sharding.exchange_numel([full[0][j]["W"] for j in range(len(shapes))], assignment)
+        xbuf = (torch.empty(per, dtype=w_dt, device=dev), torch.empty(world * per, dtype=w_dt, device=dev))
 
     def step(i, st=None):
-        step_fn(arrs[i % 2], wcode, ncode, w["hp"], sched, ws, d_status=status,
-                stream=st if st is not None else stream)
+        st = st if st is not None else stream
+        if sharded:
+            sharding.sharded_step(full[i % 2], wcode, ncode, w["hp"], sched, ws, rank, world, d_status=status,
+                                  stream=st, buffers=xbuf)
+        elif owned:
+            step_fn(arrs[i % 2], wcode, ncode, w["hp"], sched, ws, d_status=status, stream=st)
 
     for i in range(args.warmup):
         step(i)
@@ -674,8 +766,9 @@ def main():
 
     # One step per gradient set captured as a CUDA graph (the library's launches
     # are plain stream work: capturable once its one-time set-up ran above).
+    # The sharded step (with its collective) is launched eagerly.
     graphs = None
-    if args.launch == "graph":
+    if args.launch == "graph" and not sharded:
         graphs = []
         cap = torch.cuda.Stream(dev)
         for i in range(2):
@@ -715,16 +808,18 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_total = float(t.item())
     ms_step = ms_total / args.steps
-    fl_step = ns_flops(shapes, ns_steps)
-    value = world * fl_step * args.steps / (ms_total / 1e3) / 1e12
+    fl_step = ns_flops(shapes, ns_steps)          # the whole model's step
+    copies = 1 if sharded else world               # model steps per timed step, all ranks
+    value = copies * fl_step * args.steps / (ms_total / 1e3) / 1e12
 
-    # ---- per-kernel device times: the same steps launched eagerly with every
-    # launch of the library bracketed by CUDA events on its stream
-    ktrace = min(args.steps, 50)
+    # ---- per-kernel device times: steps launched eagerly with every launch of
+    # the library bracketed by CUDA events on its stream (about 5 s of steps)
+    ktrace = max(2, min(args.steps, 50, int(5000.0 / max(ms_step, 1e-3))))
     mo.muon_trace_enable(True)
     mo.muon_trace_read()
     for i in range(ktrace):
-        step(i)
+        if owned:
+            step_fn(arrs[i % 2], wcode, ncode, w["hp"], sched, ws, d_status=status, stream=stream)
     torch.cuda.synchronize(dev)
     mo.muon_trace_enable(False)
     recs = mo.muon_trace_read()
@@ -745,7 +840,8 @@ def main():
             sustained = ms_total > 1000.0
             peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
             ach, unit, bound = d["work"] / (d["ms"] / 1e3) / 1e12, "TFLOP/s", "tensor"
-        traffic, traffic_src = recorded_traffic(dom, args.workload, ns_steps)
+        nel_launch = nel_owned
+        traffic, traffic_src = recorded_traffic(dom, args.workload, ns_steps, elements=nel_launch)
         roofline = {"bound": bound, "kernel": dom, "achieved": ach, "peak": peak, "unit": unit,
                     "frac": ach / peak, "traffic": traffic,
                     "traffic_source": traffic_src or "no ncu record for the current kernel sources",
@@ -760,11 +856,13 @@ def main():
     launches_per_step = len(recs) / max(1, ktrace)
 
     # ---- end to end through the public API: each step's gradients copied from
-    # pinned host memory (on a copy stream, overlapping the previous step),
-    # the step, then a device->host read of the step's status word
+    # pinned host memory (one host set, into the two device buffers in turn, on
+    # a copy stream overlapping the previous step), the step, then a
+    # device->host read of the step's status word
     e2e = None
     if not args.no_e2e:
-        host_g = [gbuf[t].cpu().pin_memory() for t in range(2)]
+        host_g = torch.empty(gbuf[0].numel(), dtype=w_dt, pin_memory=True)
+        host_g.copy_(gbuf[0])
         host_status = torch.zeros(1, dtype=torch.int32).pin_memory()
         s_copy = torch.cuda.Stream(dev)
         copied = [torch.cuda.Event() for _ in range(2)]
@@ -772,12 +870,12 @@ def main():
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-        k = max(3, min(args.steps, 50))
+        k = max(3, min(args.steps, 50, int(10000.0 / max(ms_step, 1e-3))))
 
         def issue_copy(i):
             with torch.cuda.stream(s_copy):
                 s_copy.wait_event(used[i % 2])          # buffer no longer read by step i-2
-                gbuf[i % 2].copy_(host_g[i % 2], non_blocking=True)
+                gbuf[i % 2].copy_(host_g, non_blocking=True)
                 copied[i % 2].record(s_copy)
 
         for e in used:
@@ -796,17 +894,24 @@ def main():
                 raise RuntimeError(f"device status {int(host_status.item())}")
         e_s = time.perf_counter() - t0
         e_ms = e_s * 1e3
+        h2d = float(nel_owned * esz)
         if world > 1:
             t = torch.tensor([e_ms], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
-        e2e = {"value": world * fl_step * k / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": nel * esz, "d2h_bytes_per_step": 4, "ms_per_step": e_ms / k,
-               "timing": "wall clock over the loop, H2D of step i+1 overlapped with step i"}
+            t = torch.tensor([h2d], device=dev, dtype=torch.float64)
+            dist.all_reduce(t)
+            h2d = float(t.item())
+        e2e = {"value": copies * fl_step * k / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4 * world, "ms_per_step": e_ms / k,
+               "steps": k, "timing": "wall clock over the loop, H2D of step i+1 overlapped with step i"}
+        del host_g
 
     cpu = None
     parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        del gbuf, params, arrs, full, ws, graphs
+        torch.cuda.empty_cache()
         cpu = cpu_baseline(w, ns_steps)
         if not lite:
             parity = group_parity(w, ns_steps, dev)
@@ -816,25 +921,31 @@ def main():
         # W, G, G_prev (w dtype), A, M (fp32); MONA-Lite: W, G, B (bf16), M
         state_bytes = nel * (2 * esz + 2 + 4) if lite else nel * (3 * esz + 8)
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "strong" if sharded else "weak",
                 "vs_baseline": None, "dtype": {torch.bfloat16: "bf16", torch.float16: "fp16",
                                                torch.float32: "fp32"}[ns_dt],
                 "data": "synthetic (seeded; shapes of the named model, random values)",
-                "config": {"workload": f"{args.workload}{' (MONA-Lite)' if lite else ''}: {groups} (wide view s x l)",
+                "config": {"workload": f"{workload_label(args, w)}{' (MONA-Lite)' if lite else ''}: {groups} "
+                                       "(wide view s x l)",
                            "variant": args.variant, "elements": nel,
                            "ns_steps": ns_steps, "w_dtype": str(w_dt).replace("torch.", ""),
                            "state_bytes": state_bytes,
                            "l2": f"inputs larger than L2: {state_bytes / 1e9:.2f} GB of state per step",
-                           "parallelism": f"{world} replica(s), each rank steps its own copy"},
-                "dense_equivalent": {"value": world * ns_flops_dense(shapes, ns_steps) * args.steps / (ms_total / 1e3) / 1e12,
+                           "parallelism": (f"sharded over {world} ranks: whole matrices, flop-balanced, one "
+                                           "all-gather of the updated weights per step" if sharded else
+                                           f"{world} replica(s), each rank steps its own copy")},
+                "dense_equivalent": {"value": copies * ns_flops_dense(shapes, ns_steps) * args.steps
+                                     / (ms_total / 1e3) / 1e12,
                                      "unit": "TFLOP/s", "note": "symmetric products counted in full (not the headline)"},
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
                 "parity": parity and {"vs": "fp64 oracle from the same 16-bit inputs, one matrix per shape group, "
                                             "relative Frobenius", "groups": parity},
                 "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clk,
-                "launch": args.launch + (" (one CUDA graph per step)" if graphs is not None else ""),
-                "kernel_timing": f"per-kernel device time from {ktrace} eagerly launched steps, each launch "
-                                 "bracketed by CUDA events on its stream"}
+                "launch": args.launch + (" (one CUDA graph per step)" if graphs is not None else
+                                         " (eager: the sharded step's collective)" if sharded else ""),
+                "kernel_timing": f"per-kernel device time from {ktrace} eagerly launched steps of this rank's "
+                                 "matrices, each launch bracketed by CUDA events on its stream"}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

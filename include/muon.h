@@ -321,7 +321,10 @@ MUON_API muon_status gram_polar(const void* X_in, void* X_out, int batch, int ro
  * cudaMalloc, cudaFree or allocating library routine is called.
  *   - The first call on each device looks up the scratch array's device
  *     address (cudaGetSymbolAddress, with that device current); make that
- *     first call before any stream capture.
+ *     first call before any stream capture.  The address is remembered with
+ *     the id of the CUDA context it was taken in and looked up again when a
+ *     call finds a different context current (after cudaDeviceReset, say);
+ *     such a call, too, should come before any capture.
  *   - All calls on a device share the scratch, which keeps the previous
  *     call's contents (each call clears what must start at zero).  Calls that
  *     overlap on the GPU (unordered streams) race: order them.

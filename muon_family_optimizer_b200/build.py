@@ -43,16 +43,21 @@ def up_to_date():
 def build(force=False, verbose=False, extra=()):
     if not force and up_to_date():
         return LIB
-    objs = []
+    from concurrent.futures import ThreadPoolExecutor
     builddir = os.path.join(HERE, "_build")
     os.makedirs(builddir, exist_ok=True)
+    jobs = []
     for src in sources():
         obj = os.path.join(builddir, os.path.basename(src) + ".o")
         cmd = [NVCC, "-c", src, "-o", obj] + [f for f in FLAGS if f != "-shared"] + list(extra)
         if verbose:
             print(" ".join(cmd))
-        subprocess.check_call(cmd)
-        objs.append(obj)
+        jobs.append((cmd, obj))
+    # one nvcc per translation unit, in parallel
+    with ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1))) as pool:
+        for f in [pool.submit(subprocess.check_call, cmd) for cmd, _ in jobs]:
+            f.result()
+    objs = [obj for _, obj in jobs]
     cmd = [NVCC, "-shared", "-o", LIB + ".tmp"] + objs + ["-gencode", "arch=compute_100a,code=sm_100a",
                                                            "-cudart", "static", "-Xcompiler", "-fPIC"]
     subprocess.check_call(cmd)

@@ -48,6 +48,7 @@ constexpr int kGramRows = 64;     // rows of Y / B^T staged per Gram chunk
 constexpr double kDrop = 1e-10;   // Cholesky pivot / squared column norm below which a column is dropped
 constexpr double kTau2 = 1e-10;   // (singular value / largest)^2 at or below which it counts as zero
 constexpr int kMaxSweeps = 30;
+constexpr int kMaxDevices = 64;    // devices whose kernel attributes are tracked
 
 struct LimEntry {
     void* W; const void* G; float* M; const float* Omega; float* O_out;
@@ -588,16 +589,25 @@ cudaError_t allow_smem(K kernel, size_t bytes) {
 template <int KT, int W_DT>
 muon_status launch_all(LimParams& prm, cudaStream_t s, int sketch_blocks, int proj_blocks, int upd_blocks,
                        double elems, double rows_k, double cols_k) {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        cudaError_t e[5] = {allow_smem(lim_sketch<KT, W_DT>, sketch_smem(KT)), allow_smem(lim_qr<KT>, qr_smem(KT)),
-                            allow_smem(lim_project<KT>, project_smem(KT)), allow_smem(lim_factor<KT>, factor_smem(KT)),
-                            allow_smem(lim_update<KT, W_DT>, update_smem(KT))};
-        for (cudaError_t x : e)
-            if (x != cudaSuccess) attr_err = x;
-    });
-    if (attr_err != cudaSuccess) return MUON_ERR_CUDA;
+    // The shared-memory limit is a per-device attribute of each kernel: set it
+    // once on every device this instantiation is launched on.
+    static std::mutex mu;
+    static bool configured[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MUON_ERR_UNSUPPORTED;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!configured[dev]) {
+            cudaError_t e[5] = {allow_smem(lim_sketch<KT, W_DT>, sketch_smem(KT)), allow_smem(lim_qr<KT>, qr_smem(KT)),
+                                allow_smem(lim_project<KT>, project_smem(KT)),
+                                allow_smem(lim_factor<KT>, factor_smem(KT)),
+                                allow_smem(lim_update<KT, W_DT>, update_smem(KT))};
+            for (cudaError_t x : e)
+                if (x != cudaSuccess) return MUON_ERR_CUDA;
+            configured[dev] = true;
+        }
+    }
     const double wsz = dt_size(W_DT), k = prm.k;
     // algorithmic bytes: per element G, M read + M written; the sketch Y written (rows x k)
     trace_begin(MUON_KERNEL_RSVD, elems * (wsz + 8.0) + 4.0 * rows_k, s);

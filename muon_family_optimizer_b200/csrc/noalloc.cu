@@ -14,6 +14,8 @@
 // iteration needs to start at zero (the per-matrix sums of squares) is
 // cleared by each call, and two calls that overlap on the GPU (different
 // streams without ordering between them) race on the same memory.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "gemm.h"
@@ -25,22 +27,61 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-// Device address of g_scratch per device (in host code the array's name is
-// only a stand-in, not an address the GPU can use).
-void* g_scratch_ptr[kMaxDevices] = {};
+// Device address of g_scratch per device, valid for one CUDA context: in host
+// code the array's name is only a stand-in, not an address the GPU can use,
+// and a context that is destroyed and created again (cudaDeviceReset, or the
+// primary context released and retained) reloads this module, so the array
+// may move.  The address is therefore cached together with the unique id of
+// the context it was taken in and looked up again when the current context's
+// id differs.
+struct ScratchSlot {
+    unsigned long long ctx_id;
+    void* ptr;
+};
+ScratchSlot g_slot[kMaxDevices] = {};
 std::mutex g_scratch_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Driver entry points (the library links no driver library directly).
+template <typename Fn>
+Fn driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(p);
+}
+
+muon_status current_context_id(unsigned long long* id) {
+    static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (!get_current || !get_id) return MUON_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return MUON_ERR_CUDA;
+    return get_id(ctx, id) == CUDA_SUCCESS ? MUON_OK : MUON_ERR_CUDA;
+}
 
 muon_status scratch_for_current_device(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return MUON_ERR_UNSUPPORTED;
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id) == MUON_OK;   // false before the context exists
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    ScratchSlot& slot = g_slot[dev];
+    if (!have_id || !slot.ptr || slot.ctx_id != id) {
+        // the lookup also creates the device's context if there is none yet
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return MUON_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
+        muon_status st = current_context_id(&id);
+        if (st != MUON_OK) return st;
+        slot.ptr = p;
+        slot.ctx_id = id;
     }
-    *out = g_scratch_ptr[dev];
+    *out = slot.ptr;
     return MUON_OK;
 }
 

@@ -14,6 +14,8 @@ values are synthetic, no dataset or trained weights are involved):
   llama3_8b   32 layers x {2 x 4096x4096, 2 x 1024x4096, 2 x 14336x4096,
               4096x14336}, bf16 W/G/G_prev, fp32 A/M
 Seeds: matrix j of workload c at step t uses 1000 c + 16 j + t.
+Layered workloads give `layer_size`, the matrices per layer, so that a
+leading slice of whole layers can be taken (smaller cases of the same shapes).
 """
 import math
 
@@ -90,17 +92,18 @@ WORKLOADS = {
     "tiny": dict(index=1, shapes=[(64, 128)], w_dtype=torch.float32, ns_dtype=torch.float32,
                  grad="gaussian", muon_steps=3,
                  hp=dict(mu=0.95, eta=0.02, **{"lambda": 0.0}, gamma=1.0, beta_a=0.9, alpha=0.0)),
-    "gpt2_small": dict(index=2, shapes=_layers(12, [(768, 768)] * 4 + [(768, 3072), (3072, 768)]),
+    "gpt2_small": dict(index=2, shapes=_layers(12, [(768, 768)] * 4 + [(768, 3072), (3072, 768)]), layer_size=6,
                        w_dtype=torch.bfloat16, ns_dtype=torch.bfloat16, grad="rank16", muon_steps=3,
                        hp=dict(mu=0.95, eta=0.02, **{"lambda": 0.0}, gamma=1.0, beta_a=0.9, alpha=0.5)),
     "llama_430m": dict(index=3, shapes=_layers(24, [(1024, 1024)] * 4 + [(4096, 1024)] * 2 + [(1024, 4096)]),
+                       layer_size=7,
                        w_dtype=torch.bfloat16, ns_dtype=torch.bfloat16, grad="power", muon_steps=3,
                        hp=dict(mu=0.95, eta=0.02, **{"lambda": 0.1}, gamma=1.0, beta_a=0.9, alpha=0.5)),
     "moe_gram": dict(index=4, shapes=[(2048, 768)] * 64 + [(768, 2048)] * 64 + [(16384, 2048)],
                      w_dtype=torch.float16, ns_dtype=torch.float16, grad="logspec", muon_steps=1,
                      hp=dict(mu=0.95, eta=0.02, **{"lambda": 0.0}, gamma=1.0, beta_a=0.9, alpha=0.5)),
     "llama3_8b": dict(index=5, shapes=_layers(32, [(4096, 4096)] * 2 + [(1024, 4096)] * 2 +
-                                              [(14336, 4096)] * 2 + [(4096, 14336)]),
+                                              [(14336, 4096)] * 2 + [(4096, 14336)]), layer_size=7,
                       w_dtype=torch.bfloat16, ns_dtype=torch.bfloat16, grad="power", muon_steps=3,
                       hp=dict(mu=0.95, eta=0.02, **{"lambda": 0.1}, gamma=1.0, beta_a=0.9, alpha=0.5)),
 }

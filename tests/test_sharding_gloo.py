@@ -1,9 +1,11 @@
-"""Multi-rank host logic of the sharded step, on CPU with gloo (world size 2 and 3).
+"""Multi-rank host logic of the sharded step, on CPU with gloo (world size 2 and
+3, and two 2-rank subgroups of a 4-rank world).
 
 Each rank updates the matrices partition() gives it (the per-matrix step is the
 fp64 oracle here: the CUDA library is not needed to test the exchange), then
-gather_weights() brings every replica's W up to date.  Every rank's W, and the
-owned optimizer state, must equal a single-process oracle step of all matrices.
+gather_weights() brings every replica's W up to date with one all-gather.
+Every rank's W, and the owned optimizer state, must equal a single-process
+oracle step of all matrices.
 """
 import os
 import socket
@@ -45,25 +47,32 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, queue):
+def _worker(rank, world, port, queue, subgroups=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         oracle.set_num_threads(1)
         params = _state()
-        assignment = sharding.sharded_step(params, None, None, HP, None, None, rank, world,
+        group = None
+        grank, gworld = rank, world
+        if subgroups:
+            # two subgroups {0, 2} and {1, 3}: every rank creates both, then steps in its own
+            groups = [dist.new_group([0, 2]), dist.new_group([1, 3])]
+            group = groups[rank % 2]
+            grank, gworld = dist.get_rank(group), dist.get_world_size(group)
+        assignment = sharding.sharded_step(params, None, None, HP, None, None, grank, gworld, group=group,
                                            step_fn=lambda mine: [_oracle_step(p) for p in mine])
-        queue.put((rank, assignment, {j: {k: v.numpy().copy() for k, v in p.items()} for j, p in enumerate(params)}))
+        queue.put((grank, assignment, {j: {k: v.numpy().copy() for k, v in p.items()} for j, p in enumerate(params)}))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_sharded_step_matches_single_process(world):
+@pytest.mark.parametrize("world,subgroups", [(2, False), (3, False), (4, True)])
+def test_sharded_step_matches_single_process(world, subgroups):
     ctx = mp.get_context("spawn")
     queue = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, queue)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, queue, subgroups)) for r in range(world)]
     for p in procs:
         p.start()
     results = [queue.get(timeout=300) for _ in range(world)]
@@ -98,6 +107,13 @@ def test_partition_balanced_and_deterministic():
         assert max(loads) - sum(loads) / world <= biggest
     with pytest.raises(ValueError):
         sharding.partition(shapes, 0)
+
+
+def test_exchange_numel_is_the_largest_share():
+    ws = [torch.zeros(r, c) for r, c in SHAPES]
+    a = sharding.partition(SHAPES, 3)
+    assert sharding.exchange_numel(ws, a) == max(sum(r * c for r, c in (SHAPES[j] for j in idx)) for idx in a)
+    assert sharding.exchange_numel(ws, [[], []] + [list(range(len(SHAPES)))]) == sum(r * c for r, c in SHAPES)
 
 
 def test_partition_edge_cases():
