@@ -43,6 +43,12 @@ def parse():
     ap.add_argument("--workload", default="llama3_8b")
     ap.add_argument("--layers", type=int, default=0,
                     help="take only the first N layers of a layered workload (smaller cases for profiling)")
+    ap.add_argument("--step-route", default="direct", choices=["direct", "gram"],
+                    help="route of the headline step: the direct quintic iteration (default) or the Gram route on "
+                         "shape groups with long side >= --gram-aspect x short side (one restart before step 3)")
+    ap.add_argument("--gram-aspect", type=float, default=2.0)
+    ap.add_argument("--no-route-compare", action="store_true",
+                    help="skip timing the other route of the step (single GPU only)")
     ap.add_argument("--replicas", action="store_true",
                     help="under torchrun: every rank steps its own copy of the workload (weak scaling) "
                          "instead of its share of one model (strong scaling, the default)")
@@ -301,7 +307,7 @@ def group_parity(w, ns_steps, dev):
         params.append(p)
     if not params:
         return out
-    ws = torch.empty(mo.muon_workspace_size(params, mo._dtype_code(ns_dt)), dtype=torch.uint8, device=dev)
+    ws = torch.empty(mo.muon_workspace_size(params, mo._dtype_code(ns_dt), None), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     mo.muon_step_batched(params, mo._dtype_code(w_dt), mo._dtype_code(ns_dt), w["hp"],
                          mo.quintic_schedule(ns_steps), ws, d_status=status)
@@ -735,9 +741,14 @@ def run_step_route(args, w, ns_steps):
     del cache
     params = [[full[t][j] for j in owned] for t in range(2)]
     arrs = [(mo.make_lite_params if lite else mo.make_params)(p) for p in params] if owned else None
-    sched = mo.quintic_schedule(ns_steps)
-    ws_size = ((mo.muon_lite_workspace_size if lite else mo.muon_workspace_size)(arrs[0], mo._dtype_code(ns_dt))
-               if owned else 256)
+    scheds = {"direct": mo.quintic_schedule(ns_steps),
+              "gram": mo.quintic_gram_schedule(ns_steps, gram_aspect=args.gram_aspect)}
+    sched = scheds[args.step_route]
+    other = "gram" if args.step_route == "direct" else "direct"
+    compare = world == 1 and not args.no_route_compare
+    size_fn = mo.muon_lite_workspace_size if lite else mo.muon_workspace_size
+    ws_size = max([size_fn(arrs[0], mo._dtype_code(ns_dt), scheds[r]) for r in
+                   ((args.step_route, other) if compare else (args.step_route,))]) if owned else 256
     ws = torch.empty(ws_size, dtype=torch.uint8, device=dev)
     step_fn = mo.muon_lite_step_batched if lite else mo.muon_step_batched
     status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -750,13 +761,14 @@ def run_step_route(args, w, ns_steps):
         per = sharding.exchange_numel([full[0][j]["W"] for j in range(len(shapes))], assignment)
         xbuf = (torch.empty(per, dtype=w_dt, device=dev), torch.empty(world * per, dtype=w_dt, device=dev))
 
-    def step(i, st=None):
+    def step(i, st=None, sc=None):
         st = st if st is not None else stream
+        sc = sc if sc is not None else sched
         if sharded:
-            sharding.sharded_step(full[i % 2], wcode, ncode, w["hp"], sched, ws, rank, world, d_status=status,
+            sharding.sharded_step(full[i % 2], wcode, ncode, w["hp"], sc, ws, rank, world, d_status=status,
                                   stream=st, buffers=xbuf)
         elif owned:
-            step_fn(arrs[i % 2], wcode, ncode, w["hp"], sched, ws, d_status=status, stream=st)
+            step_fn(arrs[i % 2], wcode, ncode, w["hp"], sc, ws, d_status=status, stream=st)
 
     for i in range(args.warmup):
         step(i)
@@ -808,9 +820,7 @@ def run_step_route(args, w, ns_steps):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_total = float(t.item())
     ms_step = ms_total / args.steps
-    fl_step = ns_flops(shapes, ns_steps)          # the whole model's step
     copies = 1 if sharded else world               # model steps per timed step, all ranks
-    value = copies * fl_step * args.steps / (ms_total / 1e3) / 1e12
 
     # ---- per-kernel device times: steps launched eagerly with every launch of
     # the library bracketed by CUDA events on its stream (about 5 s of steps)
@@ -823,12 +833,24 @@ def run_step_route(args, w, ns_steps):
     torch.cuda.synchronize(dev)
     mo.muon_trace_enable(False)
     recs = mo.muon_trace_read()
+    # the work the kernels of one step do (the Gram route's own algorithmic flops)
+    fl_exec = sum(wk for kind, wk, _ in recs if kind in (mo.KERNEL_SYM, mo.KERNEL_UPD, mo.KERNEL_SIMT)) / ktrace
     per = {}
     for kind, work, ms in recs:
         d = per.setdefault(mo.KERNEL_NAMES[kind], {"launches": 0, "work": 0.0, "ms": 0.0})
         d["launches"] += 1
         d["work"] += work
         d["ms"] += ms
+    # headline work: the direct iteration's algorithmic flops, or the Gram
+    # route's own count (what its kernels execute) when it is the headline
+    fl_step = ns_flops(shapes, ns_steps)
+    if args.step_route == "gram":
+        fl_step = fl_exec
+        if sharded:     # every rank traced its own share
+            t = torch.tensor([fl_exec], device=dev, dtype=torch.float64)
+            dist.all_reduce(t)
+            fl_step = float(t.item())
+    value = copies * fl_step * args.steps / (ms_total / 1e3) / 1e12
     pk, pk_src = peaks()
     dom = max(per.items(), key=lambda kv: kv[1]["ms"])[0] if per else None
     roofline = None
@@ -854,6 +876,49 @@ def run_step_route(args, w, ns_steps):
                          ("GB/s" if name in ("prepass", "other") else "TFLOP/s"):
                              round(rate / 1e9, 1) if name in ("prepass", "other") else round(rate / 1e12, 1)}
     launches_per_step = len(recs) / max(1, ktrace)
+
+    # ---- the other route of the same step, timed the same way (one GPU)
+    route_cmp = None
+    if compare and owned and not sharded:
+        sc2 = scheds[other]
+        for i in range(2):
+            step(i, sc=sc2)
+        torch.cuda.synchronize(dev)
+        mo.muon_trace_enable(True)
+        mo.muon_trace_read()
+        step(0, sc=sc2)
+        torch.cuda.synchronize(dev)
+        mo.muon_trace_enable(False)
+        recs2 = mo.muon_trace_read()
+        fl2 = sum(wk for kind, wk, _ in recs2 if kind in (mo.KERNEL_SYM, mo.KERNEL_UPD, mo.KERNEL_SIMT))
+        g2 = []
+        cap = torch.cuda.Stream(dev)
+        for i in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                step(i, torch.cuda.current_stream(dev), sc=sc2)
+            g2.append(g)
+        for i in range(2):
+            g2[i % 2].replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            g2[i % 2].replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms2 = e0.elapsed_time(e1) / args.steps
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item())} after the {other} route")
+        gram_ms, direct_ms = (ms2, ms_step) if other == "gram" else (ms_step, ms2)
+        gram_fl, direct_fl = (fl2, fl_exec) if other == "gram" else (fl_exec, fl2)
+        route_cmp = {"other_route": other, "ms_per_step": ms2, "launches_per_step": len(recs2),
+                     "TFLOP/s": fl2 / (ms2 / 1e3) / 1e12, "flops_per_step": fl2,
+                     "gram_aspect": args.gram_aspect, "gram_restarts": list(mo.GRAM_STEP_RESTARTS),
+                     "gram_vs_direct": {"flops": gram_fl / direct_fl, "ms": gram_ms / direct_ms},
+                     "note": "same inputs and launch mode; Gram route on shape groups with long side >= "
+                             f"{args.gram_aspect:g} x short side, direct iteration elsewhere"}
+        del g2
 
     # ---- end to end through the public API: each step's gradients copied from
     # pinned host memory (one host set, into the two device buffers in turn, on
@@ -907,6 +972,8 @@ def run_step_route(args, w, ns_steps):
                "steps": k, "timing": "wall clock over the loop, H2D of step i+1 overlapped with step i"}
         del host_g
 
+    launch_desc = args.launch + (" (one CUDA graph per step)" if graphs is not None else
+                                 " (eager: the sharded step's collective)" if sharded else "")
     cpu = None
     parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -937,13 +1004,16 @@ def run_step_route(args, w, ns_steps):
                                            f"{world} replica(s), each rank steps its own copy")},
                 "dense_equivalent": {"value": copies * ns_flops_dense(shapes, ns_steps) * args.steps
                                      / (ms_total / 1e3) / 1e12,
-                                     "unit": "TFLOP/s", "note": "symmetric products counted in full (not the headline)"},
+                                     "unit": "TFLOP/s", "note": "symmetric products counted in full (not the headline)"}
+                                    if args.step_route == "direct" else None,
+                "step_route": args.step_route + (f" (Gram route where long side >= {args.gram_aspect:g} x short "
+                                                 "side)" if args.step_route == "gram" else ""),
+                "route_compare": route_cmp,
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
                 "parity": parity and {"vs": "fp64 oracle from the same 16-bit inputs, one matrix per shape group, "
                                             "relative Frobenius", "groups": parity},
                 "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clk,
-                "launch": args.launch + (" (one CUDA graph per step)" if graphs is not None else
-                                         " (eager: the sharded step's collective)" if sharded else ""),
+                "launch": launch_desc,
                 "kernel_timing": f"per-kernel device time from {ktrace} eagerly launched steps of this rank's "
                                  "matrices, each launch bracketed by CUDA events on its stream"}
         print(json.dumps(line), flush=True)

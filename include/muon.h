@@ -102,6 +102,10 @@ typedef struct {
     const int* restarts;         /* host array of step indices (0 allowed, ignored); may be NULL if n_restarts == 0 */
     int n_restarts;              /* >= 0, <= 64 */
     float scale_f;               /* >= 1: extra divisor at the start and at every restart (1.02-1.05 on the Gram route) */
+    float gram_aspect;           /* optimizer steps only: a shape group whose long side is at least gram_aspect
+                                    times its short side runs the Gram route (with restarts and scale_f);
+                                    0 keeps every group on the direct iteration.  >= 0.  ns_polar and
+                                    gram_polar ignore it. */
 } muon_schedule;
 
 /* Hyper-parameters of [MONA] section 2. */
@@ -127,20 +131,30 @@ typedef struct {
 } muon_param;
 
 /*
- * Bytes of workspace muon_step_batched needs for these parameters.
- * params: host array of n descriptors (only rows/cols are read).
- * Returns MUON_ERR_INVALID_ARG for n < 1, NULL pointers or non-positive sizes.
+ * Bytes of workspace muon_step_batched needs for these parameters under this
+ * schedule.  params: host array of n descriptors (only rows/cols are read).
+ * sched: the schedule the step will use (its gram_aspect decides which shape
+ * groups need the Gram route's larger workspace); NULL sizes every group for
+ * the direct iteration.
+ * Returns MUON_ERR_INVALID_ARG for n < 1, NULL pointers, non-positive sizes or
+ * an invalid schedule.
  */
 MUON_API muon_status muon_workspace_size(const muon_param* params, int n, muon_dtype ns_dtype,
-                                size_t* bytes);
+                                const muon_schedule* sched, size_t* bytes);
 
 /*
  * One optimizer step ([MONA] section 2, steps 1-4) for n matrix parameters.
  *   1. One fused pass over every element: A, M, G_prev updated in place as in
  *      steps 1-4, the Frobenius norm of the new M accumulated per matrix, and
  *      M written in ns_dtype (wide view) to the workspace.
- *   2. The quintic iteration above on every matrix (matrices with the same
- *      (short side, long side) are batched together).
+ *   2. The iteration above on every matrix (matrices with the same
+ *      (short side, long side) are batched together): the direct iteration,
+ *      or the Gram route for the shape groups sched->gram_aspect selects
+ *      ([POLAR]: elongated matrices iterate on their small s x s Gram
+ *      matrix; in exact arithmetic both routes give the same O).  A matrix
+ *      whose short side is below 16 is iterated in fp32 on CUDA cores
+ *      whatever ns_dtype says (its 16-bit intermediates would cost accuracy
+ *      for no measurable time).
  *   3. W <- W - eta (gamma O + lambda W), fused into the last iteration step;
  *      O never reaches memory unless O_out is given.
  * w_dtype: element type of W, G and G_prev (MUON_BF16, MUON_FP16 or MUON_FP32).
@@ -176,9 +190,10 @@ typedef struct {
     float* O_out;      /* optional rows x cols fp32: receives O; NULL to skip */
 } muon_lite_param;
 
-/* Bytes of workspace muon_lite_step_batched needs (only rows/cols are read). */
+/* Bytes of workspace muon_lite_step_batched needs (only rows/cols are read;
+ * sched as for muon_workspace_size). */
 MUON_API muon_status muon_lite_workspace_size(const muon_lite_param* params, int n, muon_dtype ns_dtype,
-                                     size_t* bytes);
+                                     const muon_schedule* sched, size_t* bytes);
 
 /*
  * One MONA-Lite optimizer step for n matrix parameters: the fused pass above
@@ -290,6 +305,11 @@ MUON_API muon_status gram_polar_workspace_size(int batch, int rows, int cols, mu
  * matrix i at X_in + i * batch_stride elements (batch_stride >= rows*cols).
  * X_out: device, same layout and dtype; may equal X_in.
  * dtype MUON_BF16 / MUON_FP16 run on tensor cores, MUON_FP32 on CUDA cores.
+ * A MUON_BF16 batch is iterated in fp16 ([POLAR]: fp16 is the recommended
+ * type; bfloat16's 8 significant bits lose the small singular directions at
+ * condition numbers near 1e3): one extra read of the input sums its squares,
+ * and the copy the iteration starts from is X / (||X||_F + eps), which fp16
+ * holds without overflow.  Input and output stay bfloat16.
  */
 MUON_API muon_status ns_polar(const void* X_in, void* X_out, int batch, int rows, int cols,
                      long long batch_stride, muon_dtype dtype, const muon_schedule* sched,

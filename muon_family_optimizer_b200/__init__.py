@@ -42,7 +42,7 @@ class NsCoeff(ctypes.Structure):
 class Schedule(ctypes.Structure):
     _fields_ = [("n_steps", ctypes.c_int), ("coeffs", ctypes.POINTER(NsCoeff)),
                 ("eps", ctypes.c_float), ("restarts", ctypes.POINTER(ctypes.c_int)),
-                ("n_restarts", ctypes.c_int), ("scale_f", ctypes.c_float)]
+                ("n_restarts", ctypes.c_int), ("scale_f", ctypes.c_float), ("gram_aspect", ctypes.c_float)]
 
 
 class HParams(ctypes.Structure):
@@ -111,13 +111,15 @@ def lib():
         L.muon_status_string.restype = ctypes.c_char_p
         L.muon_status_string.argtypes = [st]
         L.muon_workspace_size.restype = st
-        L.muon_workspace_size.argtypes = [ctypes.POINTER(Param), ctypes.c_int, ctypes.c_int, sz]
+        L.muon_workspace_size.argtypes = [ctypes.POINTER(Param), ctypes.c_int, ctypes.c_int,
+                                          ctypes.POINTER(Schedule), sz]
         L.muon_step_batched.restype = st
         L.muon_step_batched.argtypes = [ctypes.POINTER(Param), ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.POINTER(HParams), ctypes.POINTER(Schedule), vp,
                                         ctypes.c_size_t, vp, vp]
         L.muon_lite_workspace_size.restype = st
-        L.muon_lite_workspace_size.argtypes = [ctypes.POINTER(LiteParam), ctypes.c_int, ctypes.c_int, sz]
+        L.muon_lite_workspace_size.argtypes = [ctypes.POINTER(LiteParam), ctypes.c_int, ctypes.c_int,
+                                               ctypes.POINTER(Schedule), sz]
         L.muon_lite_step_batched.restype = st
         L.muon_lite_step_batched.argtypes = [ctypes.POINTER(LiteParam), ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                              ctypes.POINTER(HParams), ctypes.POINTER(Schedule), vp,
@@ -163,19 +165,35 @@ def _check(status, where):
         raise MuonError(status, where)
 
 
-def make_schedule(coeffs, eps=1e-7, restarts=(), scale_f=1.0):
-    """Build a C schedule; the returned object keeps its arrays alive."""
+def make_schedule(coeffs, eps=1e-7, restarts=(), scale_f=1.0, gram_aspect=0.0):
+    """Build a C schedule; the returned object keeps its arrays alive.
+    gram_aspect > 0: in an optimizer step, shape groups with long side >=
+    gram_aspect * short side run the Gram route (restarts, scale_f)."""
     coeffs = [tuple(c) for c in coeffs]
     arr = (NsCoeff * len(coeffs))(*[NsCoeff(*c) for c in coeffs])
     rs = list(restarts)
     rarr = (ctypes.c_int * max(1, len(rs)))(*rs) if rs else None
-    s = Schedule(len(coeffs), arr, eps, rarr, len(rs), scale_f)
+    s = Schedule(len(coeffs), arr, eps, rarr, len(rs), scale_f, gram_aspect)
     s._keep = (arr, rarr)
     return s
 
 
 def quintic_schedule(n_steps=5, eps=1e-7, scale_f=1.0):
     return make_schedule([QUINTIC] * n_steps, eps=eps, scale_f=scale_f)
+
+
+# Restart of the Gram route inside the 5-step quintic optimizer step: before
+# step 3.  Without a restart, 16-bit rounding leaves small negative eigenvalues
+# in R that the quintic h(R) R h(R) multiplies by about 12 each step until they
+# dominate; one restart recomputes R from Xb and keeps the result as close to
+# the exact iteration as the direct route's (emulated and measured).
+GRAM_STEP_RESTARTS = (3,)
+
+
+def quintic_gram_schedule(n_steps=5, gram_aspect=2.0, eps=1e-7, restarts=GRAM_STEP_RESTARTS):
+    """The quintic step schedule with the Gram route on shape groups whose long
+    side is at least gram_aspect times the short side."""
+    return make_schedule([QUINTIC] * n_steps, eps=eps, restarts=restarts, scale_f=1.0, gram_aspect=gram_aspect)
 
 
 def _dtype_code(t):
@@ -210,11 +228,12 @@ def make_params(params):
     return arr
 
 
-def muon_workspace_size(params, ns_dtype):
+def muon_workspace_size(params, ns_dtype, schedule=None):
+    """Workspace bytes of muon_step_batched; schedule None sizes the direct route."""
     arr = params if isinstance(params, ctypes.Array) else make_params(params)
     out = ctypes.c_size_t(0)
-    _check(lib().muon_workspace_size(arr, len(arr), int(ns_dtype), ctypes.byref(out)),
-           "muon_workspace_size")
+    _check(lib().muon_workspace_size(arr, len(arr), int(ns_dtype), ctypes.byref(schedule) if schedule else None,
+                                     ctypes.byref(out)), "muon_workspace_size")
     return out.value
 
 
@@ -251,10 +270,11 @@ def make_lite_params(params):
     return arr
 
 
-def muon_lite_workspace_size(params, ns_dtype):
+def muon_lite_workspace_size(params, ns_dtype, schedule=None):
     arr = params if isinstance(params, ctypes.Array) else make_lite_params(params)
     out = ctypes.c_size_t(0)
-    _check(lib().muon_lite_workspace_size(arr, len(arr), int(ns_dtype), ctypes.byref(out)),
+    _check(lib().muon_lite_workspace_size(arr, len(arr), int(ns_dtype),
+                                          ctypes.byref(schedule) if schedule else None, ctypes.byref(out)),
            "muon_lite_workspace_size")
     return out.value
 

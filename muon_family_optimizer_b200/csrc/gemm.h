@@ -55,7 +55,10 @@ struct PrepParams {
     int n;
     long long total_tiles;
     int in_dt, x0_dt, mode;   // mode 0 = MONA pre-pass, 1 = copy (normalisation input of ns/gram_polar),
-                              // 2 = MONA-Lite (Gp holds the bfloat16 buffer B, A unused)
+                              // 2 = MONA-Lite (Gp holds the bfloat16 buffer B, A unused),
+                              // 3 = norm only (sums of squares of the batch input, nothing stored)
+    int prescale;             // copy mode after a norm pass: store X / (||X|| + eps), sums left as they are
+    float eps;
     float beta_a, alpha, mu;
     double* sumsq;
 };

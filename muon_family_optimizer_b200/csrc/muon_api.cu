@@ -32,6 +32,7 @@ muon_status check_schedule(const muon_schedule* s) {
     if (!(s->scale_f >= 1.f) || !isfinite(s->scale_f)) return MUON_ERR_INVALID_ARG;
     if (s->n_restarts < 0 || s->n_restarts > kMaxRestarts) return MUON_ERR_INVALID_ARG;
     if (s->n_restarts > 0 && !s->restarts) return MUON_ERR_INVALID_ARG;
+    if (!(s->gram_aspect >= 0.f) || !isfinite(s->gram_aspect)) return MUON_ERR_INVALID_ARG;
     for (int i = 0; i < s->n_restarts; ++i)
         if (s->restarts[i] < 0 || s->restarts[i] >= s->n_steps) return MUON_ERR_INVALID_ARG;
     for (int k = 0; k < s->n_steps; ++k) {
@@ -58,10 +59,18 @@ muon_status check_device() {
 
 // ---------------------------------------------------------------- layouts
 
+// Smallest short side the tensor-core path takes inside an optimizer step:
+// narrower matrices (at most 15 rows in the wide view) are iterated in fp32 on
+// CUDA cores, where their 16-bit intermediates would cost more accuracy than
+// their negligible work saves.
+constexpr int kMinTcSide = 16;
+
 // A batch of same-shape matrices in the wide view (s <= l).
 struct Group {
     int s = 0, l = 0;
     std::vector<int> members;        // indices into the caller's parameter array
+    int dt = DT_BF16;                // element type of this group's iteration
+    int gram = 0;                    // 1: the Gram route, 0: the direct iteration
     long long ldl = 0, lds = 0;      // padded row strides of s x l and s x s buffers
     size_t x[2] = {0, 0};            // s x l ping-pong
     size_t sq[6] = {0, 0, 0, 0, 0, 0};   // s x s buffers (direct route uses 2, Gram route 6)
@@ -73,22 +82,29 @@ struct Layout {
     std::vector<Group> groups;
 };
 
-void place_group(Group& g, size_t& off, int esz, int nsq) {
+void place_group(Group& g, size_t& off) {
     const long long cnt = (long long)g.members.size();
+    const int esz = dt_size(g.dt);
     g.ldl = pad8(g.l);
     g.lds = pad8(g.s);
     for (int i = 0; i < 2; ++i) {
         g.x[i] = off;
         off = align_up(off + (size_t)cnt * g.s * g.ldl * esz, kAlign);
     }
-    for (int i = 0; i < nsq; ++i) {
+    for (int i = 0; i < (g.gram ? 6 : 2); ++i) {
         g.sq[i] = off;
         off = align_up(off + (size_t)cnt * g.s * g.lds * esz, kAlign);
     }
 }
 
-// Parameters grouped by (s, l); a group holds at most kMaxGroupMembers.
-Layout step_layout(const muon_param* params, int n, int ns_dt) {
+// Whether a shape group of an optimizer step runs the Gram route.
+bool gram_group(const muon_schedule* sch, int s, int l, int dt) {
+    return sch && dt != DT_FP32 && sch->gram_aspect > 0.f && (double)l >= (double)sch->gram_aspect * s;
+}
+
+// Parameters grouped by (s, l); a group holds at most kMaxGroupMembers.  The
+// schedule (may be NULL: every group direct) selects the Gram route per group.
+Layout step_layout(const muon_param* params, int n, int ns_dt, const muon_schedule* sch) {
     Layout L;
     std::map<std::pair<int, int>, std::vector<int>> by_shape;
     for (int i = 0; i < n; ++i) {
@@ -103,6 +119,8 @@ Layout step_layout(const muon_param* params, int n, int ns_dt) {
             Group g;
             g.s = kv.first.first;
             g.l = kv.first.second;
+            g.dt = (ns_dt != DT_FP32 && g.s < kMinTcSide) ? DT_FP32 : ns_dt;
+            g.gram = gram_group(sch, g.s, g.l, g.dt) ? 1 : 0;
             g.members.assign(all.begin() + b, all.begin() + std::min(all.size(), b + kMaxGroupMembers));
             groups.push_back(g);
         }
@@ -116,30 +134,31 @@ Layout step_layout(const muon_param* params, int n, int ns_dt) {
     off = align_up(off + 256, kAlign);
     L.sumsq = off;
     off = align_up(off + sizeof(double) * (size_t)n, kAlign);
-    const int esz = dt_size(ns_dt);
     int slot = 0;
     for (Group& g : groups) {
         g.sumsq0 = slot;
         slot += (int)g.members.size();
-        place_group(g, off, esz, 2);
+        place_group(g, off);
     }
     L.groups = groups;
     L.total = off;
     return L;
 }
 
-Layout batch_layout(int batch, int rows, int cols, int dt, int nsq) {
+Layout batch_layout(int batch, int rows, int cols, int dt, int gram) {
     Layout L;
     Group g;
     g.s = std::min(rows, cols);
     g.l = std::max(rows, cols);
+    g.dt = dt;
+    g.gram = gram;
     g.members.resize(batch);
     size_t off = 0;
     L.status = off;
     off = align_up(off + 256, kAlign);
     L.sumsq = off;
     off = align_up(off + sizeof(double) * (size_t)batch, kAlign);
-    place_group(g, off, dt_size(dt), nsq);
+    place_group(g, off);
     L.groups.push_back(g);
     L.total = off;
     return L;
@@ -151,6 +170,7 @@ inline void* at(void* ws, size_t off) { return static_cast<char*>(ws) + off; }
 
 struct Runner {
     int dt;                 // element type of the iteration
+    bool prenorm = false;   // the wide views already hold X / (||X|| + eps): no norm scale in the products
     FinalCtx fc;
     cudaStream_t stream;
 
@@ -199,13 +219,41 @@ GemmOp upd_op(int count, int s, int l, const void* A, long long lda, long long s
     return o;
 }
 
-// The direct quintic iteration on every group of `L`, starting from the
-// unnormalised wide views in x[0] (norms in sumsq).  The last step's
-// epilogue is `final_epi` (FIN_OUT or FIN_WUPD) with the given table.
-muon_status run_direct(Runner& R, const Layout& L, void* ws, const muon_schedule* sch,
-                       const std::vector<std::vector<FinalEntry>>& fin_per_group, int final_kind) {
-    const int esz = dt_size(R.dt);
-    const double* sumsq = static_cast<const double*>(at(ws, L.sumsq));
+using GroupList = std::vector<const Group*>;
+using FinalTables = std::vector<std::vector<FinalEntry>>;   // per group of a GroupList: its W-update rows
+
+// The last product of the iteration, one op per group (ops[i] belongs to
+// group i): FIN_OUT writes the caller's output; FIN_WUPD updates W through
+// each group's rows of the final table.  A launch carries at most
+// kMaxProblems ops and kMaxFinal table rows.
+muon_status run_final(Runner& R, const std::vector<GemmOp>& ops, const FinalTables& fins, int final_kind) {
+    std::vector<GemmOp> batch;
+    std::vector<FinalEntry> fin;
+    for (size_t i = 0; i < ops.size(); ++i) {
+        GemmOp o = ops[i];
+        const int rows_needed = final_kind == FIN_WUPD ? o.count : 0;
+        if (!batch.empty() && (batch.size() == (size_t)kMaxProblems || (int)fin.size() + rows_needed > kMaxFinal)) {
+            muon_status st = R.run(batch, fin);
+            if (st != MUON_OK) return st;
+            batch.clear();
+            fin.clear();
+        }
+        o.epi.fin = final_kind;
+        if (rows_needed) {
+            o.epi.fin_base = (int)fin.size();
+            fin.insert(fin.end(), fins[i].begin(), fins[i].end());
+        }
+        batch.push_back(o);
+    }
+    return R.run(batch, fin);
+}
+
+// The direct quintic iteration on the groups `gs` (all of R.dt), starting
+// from the unnormalised wide views in x[0] (norms in sumsq).  The last step's
+// epilogue is `final_kind` (FIN_OUT or FIN_WUPD with the groups' tables).
+muon_status run_direct(Runner& R, const GroupList& gs, void* ws, const double* sumsq, const muon_schedule* sch,
+                       const FinalTables& fins, int final_kind) {
+    if (gs.empty()) return MUON_OK;
     const float f = sch->scale_f;
     int cur = 0;
     for (int k = 0; k < sch->n_steps; ++k) {
@@ -215,19 +263,21 @@ muon_status run_direct(Runner& R, const Layout& L, void* ws, const muon_schedule
         const bool last = k == sch->n_steps - 1;
         // A = X X^T (scaled by pre^2, and by 1/(|M|+eps)^2 at the first step)
         std::vector<GemmOp> ops;
-        for (const Group& g : L.groups) {
+        for (const Group* gp : gs) {
+            const Group& g = *gp;
             const int cnt = (int)g.members.size();
             const long long sx = (long long)g.s * g.ldl, ss = (long long)g.s * g.lds;
             Epilogue e = epi_store(at(ws, g.sq[0]), g.lds, ss);
             e.sc_mul = pre * pre;
-            if (first) { e.sumsq = sumsq + g.sumsq0; e.eps = sch->eps; e.sc_pow = 2; }
+            if (first && !R.prenorm) { e.sumsq = sumsq + g.sumsq0; e.eps = sch->eps; e.sc_pow = 2; }
             ops.push_back(sym_op(cnt, g.s, g.l, at(ws, g.x[cur]), g.ldl, sx, at(ws, g.x[cur]), g.ldl, sx, e));
         }
         muon_status st = R.run(ops, {});
         if (st != MUON_OK) return st;
         // B' = a I + b A + c A A   (the a X term of the step rides on the diagonal)
         ops.clear();
-        for (const Group& g : L.groups) {
+        for (const Group* gp : gs) {
+            const Group& g = *gp;
             const int cnt = (int)g.members.size();
             const long long ss = (long long)g.s * g.lds;
             Epilogue e = epi_store(at(ws, g.sq[1]), g.lds, ss);
@@ -239,104 +289,131 @@ muon_status run_direct(Runner& R, const Layout& L, void* ws, const muon_schedule
         if (st != MUON_OK) return st;
         // X' = pre B' X   (and 1/(|M|+eps) at the first step); on the last
         // step the result goes to the caller (FIN_OUT) or into W (FIN_WUPD).
-        // A launch carries at most kMaxProblems groups and kMaxFinal table rows.
         ops.clear();
-        std::vector<FinalEntry> fin;
-        for (size_t gi = 0; gi < L.groups.size(); ++gi) {
-            const Group& g = L.groups[gi];
+        for (const Group* gp : gs) {
+            const Group& g = *gp;
             const int cnt = (int)g.members.size();
             const long long sx = (long long)g.s * g.ldl, ss = (long long)g.s * g.lds;
             Epilogue e = epi_store(at(ws, g.x[cur ^ 1]), g.ldl, sx);
             e.sc_mul = pre;
-            if (first) { e.sumsq = sumsq + g.sumsq0; e.eps = sch->eps; e.sc_pow = 1; }
-            const int rows_needed = (last && final_kind == FIN_WUPD) ? cnt : 0;
-            if (!ops.empty() && (ops.size() == (size_t)kMaxProblems || (int)fin.size() + rows_needed > kMaxFinal)) {
-                st = R.run(ops, fin);
-                if (st != MUON_OK) return st;
-                ops.clear();
-                fin.clear();
-            }
-            if (last) {
-                e.fin = final_kind;
-                e.check = sumsq + g.sumsq0;
-                if (rows_needed) {
-                    e.fin_base = (int)fin.size();
-                    fin.insert(fin.end(), fin_per_group[gi].begin(), fin_per_group[gi].end());
-                }
-            }
+            if (first && !R.prenorm) { e.sumsq = sumsq + g.sumsq0; e.eps = sch->eps; e.sc_pow = 1; }
+            if (last) e.check = sumsq + g.sumsq0;
             ops.push_back(upd_op(cnt, g.s, g.l, at(ws, g.sq[1]), g.lds, ss, at(ws, g.x[cur]), g.ldl, sx, e));
         }
-        st = R.run(ops, fin);
+        st = last ? run_final(R, ops, fins, final_kind) : R.run(ops, {});
         if (st != MUON_OK) return st;
         cur ^= 1;
     }
     return MUON_OK;
 }
 
-// The Gram route for one batch group (see include/muon.h).
-muon_status run_gram(Runner& R, const Layout& L, void* ws, const muon_schedule* sch) {
-    const Group& g = L.groups[0];
-    const int cnt = (int)g.members.size();
-    const long long sx = (long long)g.s * g.ldl, ss = (long long)g.s * g.lds;
-    const double* sumsq = static_cast<const double*>(at(ws, L.sumsq)) + g.sumsq0;
+// The Gram route (see include/muon.h) on the groups `gs` (all of R.dt, each
+// with six s x s buffers), starting from the unnormalised wide views in x[0];
+// the last product's epilogue is `final_kind` as for run_direct.  Every launch
+// carries the same product for all groups.
+muon_status run_gram(Runner& R, const GroupList& gs, void* ws, const double* sumsq, const muon_schedule* sch,
+                     const FinalTables& fins, int final_kind) {
+    if (gs.empty()) return MUON_OK;
     const float f = sch->scale_f;
-    // buffer roles: indices into g.sq
+    // buffer roles: indices into each group's sq[]
     int iR = 0, iRn = 1, iH = 2, iQ = 3, iQn = 4, iT = 5;
     int xb = 0;                 // current Xb buffer
     bool xb_raw = true;         // Xb still holds the unnormalised input (scale pending)
     bool q_identity = true;
-    auto sq = [&](int i) { return at(ws, g.sq[i]); };
-    auto xbuf = [&](int i) { return at(ws, g.x[i]); };
+    auto sq = [&](const Group& g, int i) { return at(ws, g.sq[i]); };
+    auto xbuf = [&](const Group& g, int i) { return at(ws, g.x[i]); };
+    auto strides = [](const Group& g, long long& sx, long long& ss) {
+        sx = (long long)g.s * g.ldl;
+        ss = (long long)g.s * g.lds;
+    };
+    // one symmetric s x s product per group: D = A B^T (A, B, D given as buffer roles)
+    auto sym_all = [&](int ia, int ib, int id, bool with_band, const muon_ns_coeff* poly) -> muon_status {
+        std::vector<GemmOp> ops;
+        for (const Group* gp : gs) {
+            const Group& g = *gp;
+            long long sx, ss;
+            strides(g, sx, ss);
+            Epilogue e = epi_store(sq(g, id), g.lds, ss);
+            if (poly) {   // h = a I + b R + c R R
+                e.alpha = poly->c; e.beta = poly->b; e.diag = poly->a;
+                e.Cin = sq(g, ia); e.ldc = g.lds; e.strideC = ss;
+            }
+            ops.push_back(sym_op((int)g.members.size(), g.s, g.s, sq(g, ia), g.lds, ss, sq(g, ib), g.lds, ss, e, 1, 1,
+                                 with_band ? 1 : 0));
+        }
+        return R.run(ops, {});
+    };
+    // R = Xb Xb^T (normalised when Xb is still the raw input)
+    auto gram_all = [&](float sc_mul, bool normalise) -> muon_status {
+        std::vector<GemmOp> ops;
+        for (const Group* gp : gs) {
+            const Group& g = *gp;
+            long long sx, ss;
+            strides(g, sx, ss);
+            Epilogue e = epi_store(sq(g, iR), g.lds, ss);
+            e.sc_mul = sc_mul;
+            if (normalise && !R.prenorm) { e.sumsq = sumsq + g.sumsq0; e.eps = sch->eps; e.sc_pow = 2; }
+            ops.push_back(sym_op((int)g.members.size(), g.s, g.l, xbuf(g, xb), g.ldl, sx, xbuf(g, xb), g.ldl, sx, e));
+        }
+        return R.run(ops, {});
+    };
+    // Xb' = scale Q Xb (the pending normalisation folded in): into the other
+    // Xb buffer, or (final) to the caller / W
+    auto apply_q = [&](bool final) -> muon_status {
+        std::vector<GemmOp> ops;
+        for (const Group* gp : gs) {
+            const Group& g = *gp;
+            long long sx, ss;
+            strides(g, sx, ss);
+            if (q_identity) {
+                muon_status st = fill_identity(sq(g, iQ), R.dt, (int)g.members.size(), g.s, g.lds, ss, R.stream);
+                if (st != MUON_OK) return st;
+            }
+            Epilogue e = final ? epi_store(nullptr, 0, 0) : epi_store(xbuf(g, xb ^ 1), g.ldl, sx);
+            e.sc_mul = final ? 1.f : 1.f / f;
+            if (xb_raw) {
+                e.sc_mul *= 1.f / f;
+                if (!R.prenorm) { e.sumsq = sumsq + g.sumsq0; e.eps = sch->eps; e.sc_pow = 1; }
+            }
+            if (final) e.check = sumsq + g.sumsq0;
+            ops.push_back(upd_op((int)g.members.size(), g.s, g.l, sq(g, iQ), g.lds, ss, xbuf(g, xb), g.ldl, sx, e));
+        }
+        return final ? run_final(R, ops, fins, final_kind) : R.run(ops, {});
+    };
 
     // R = Xb Xb^T / ((|X|+eps) f)^2
-    {
-        Epilogue e = epi_store(sq(iR), g.lds, ss);
-        e.sc_mul = 1.f / (f * f); e.sumsq = sumsq; e.eps = sch->eps; e.sc_pow = 2;
-        muon_status st = R.run({sym_op(cnt, g.s, g.l, xbuf(xb), g.ldl, sx, xbuf(xb), g.ldl, sx, e)}, {});
-        if (st != MUON_OK) return st;
-    }
-    auto apply_q = [&](Epilogue e) -> muon_status {
-        // Xb' = scale * Q Xb  (the pending normalisation folded in)
-        if (xb_raw) { e.sc_mul *= 1.f / f; e.sumsq = sumsq; e.eps = sch->eps; e.sc_pow = 1; }
-        if (q_identity) {
-            muon_status st = fill_identity(sq(iQ), R.dt, cnt, g.s, g.lds, ss, R.stream);
-            if (st != MUON_OK) return st;
-        }
-        return R.run({upd_op(cnt, g.s, g.l, sq(iQ), g.lds, ss, xbuf(xb), g.ldl, sx, e)}, {});
-    };
+    muon_status st = gram_all(1.f / (f * f), true);
+    if (st != MUON_OK) return st;
     for (int k = 0; k < sch->n_steps; ++k) {
         const muon_ns_coeff c = sch->coeffs[k];
-        muon_status st;
         if (is_restart(sch, k)) {
             // Xb <- Q Xb / f;  R <- Xb Xb^T;  Q <- I
-            Epilogue e = epi_store(xbuf(xb ^ 1), g.ldl, sx);
-            e.sc_mul = 1.f / f;
-            st = apply_q(e);
+            st = apply_q(false);
             if (st != MUON_OK) return st;
             xb ^= 1;
             xb_raw = false;
             q_identity = true;
-            Epilogue e2 = epi_store(sq(iR), g.lds, ss);
-            st = R.run({sym_op(cnt, g.s, g.l, xbuf(xb), g.ldl, sx, xbuf(xb), g.ldl, sx, e2)}, {});
+            st = gram_all(1.f, false);
             if (st != MUON_OK) return st;
         }
         // h = a I + b R + c R R
-        {
-            Epilogue e = epi_store(sq(iH), g.lds, ss);
-            e.alpha = c.c; e.beta = c.b; e.diag = c.a;
-            e.Cin = sq(iR); e.ldc = g.lds; e.strideC = ss;
-            st = R.run({sym_op(cnt, g.s, g.s, sq(iR), g.lds, ss, sq(iR), g.lds, ss, e, 1, 1, 1)}, {});
-            if (st != MUON_OK) return st;
-        }
+        st = sym_all(iR, iR, iH, true, &c);
+        if (st != MUON_OK) return st;
         const bool need_r = k + 1 < sch->n_steps && !is_restart(sch, k + 1);
         // Q <- h Q  and  T = h R  (one launch)
         std::vector<GemmOp> ops;
-        if (!q_identity)
-            ops.push_back(sym_op(cnt, g.s, g.s, sq(iH), g.lds, ss, sq(iQ), g.lds, ss, epi_store(sq(iQn), g.lds, ss),
-                                 1, 1, 1));
-        if (need_r)
-            ops.push_back(sym_op(cnt, g.s, g.s, sq(iH), g.lds, ss, sq(iR), g.lds, ss, epi_store(sq(iT), g.lds, ss),
-                                 1, 1));
+        for (const Group* gp : gs) {
+            const Group& g = *gp;
+            long long sx, ss;
+            strides(g, sx, ss);
+            const int cnt = (int)g.members.size();
+            if (!q_identity)
+                ops.push_back(sym_op(cnt, g.s, g.s, sq(g, iH), g.lds, ss, sq(g, iQ), g.lds, ss,
+                                     epi_store(sq(g, iQn), g.lds, ss), 1, 1, 1));
+            if (need_r)
+                ops.push_back(sym_op(cnt, g.s, g.s, sq(g, iH), g.lds, ss, sq(g, iR), g.lds, ss,
+                                     epi_store(sq(g, iT), g.lds, ss), 1, 1));
+        }
         st = R.run(ops, {});
         if (st != MUON_OK) return st;
         const int h_buf = iH;     // h stays in this buffer until the end of the step
@@ -348,17 +425,13 @@ muon_status run_gram(Runner& R, const Layout& L, void* ws, const muon_schedule* 
         }
         // R <- (h R) h
         if (need_r) {
-            st = R.run({sym_op(cnt, g.s, g.s, sq(iT), g.lds, ss, sq(h_buf), g.lds, ss,
-                               epi_store(sq(iRn), g.lds, ss), 1, 1)}, {});
+            st = sym_all(iT, h_buf, iRn, false, nullptr);
             if (st != MUON_OK) return st;
             std::swap(iR, iRn);
         }
     }
-    // X = Q Xb  -> caller's output
-    Epilogue e = epi_store(nullptr, 0, 0);
-    e.fin = FIN_OUT;
-    e.check = sumsq;
-    return apply_q(e);
+    // X = Q Xb  -> the caller's output or W
+    return apply_q(true);
 }
 
 }  // namespace
@@ -391,11 +464,16 @@ static muon_status check_params(const muon_param* params, int n) {
     return MUON_OK;
 }
 
-muon_status muon_workspace_size(const muon_param* params, int n, muon_dtype ns_dtype, size_t* bytes) {
+muon_status muon_workspace_size(const muon_param* params, int n, muon_dtype ns_dtype, const muon_schedule* sched,
+                                size_t* bytes) {
     if (!bytes || !valid_dtype(ns_dtype)) return MUON_ERR_INVALID_ARG;
     muon_status st = check_params(params, n);
     if (st != MUON_OK) return st;
-    *bytes = step_layout(params, n, ns_dtype).total;
+    if (sched) {
+        st = check_schedule(sched);
+        if (st != MUON_OK) return st;
+    }
+    *bytes = step_layout(params, n, ns_dtype, sched).total;
     return MUON_OK;
 }
 
@@ -414,7 +492,7 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
     const float hv[6] = {hp->mu, hp->eta, hp->lambda, hp->gamma, hp->beta_a, hp->alpha};
     for (float v : hv)
         if (!isfinite(v)) return MUON_ERR_INVALID_ARG;
-    Layout L = step_layout(params, n, ns_dtype);
+    Layout L = step_layout(params, n, ns_dtype, sched);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) || ws_bytes < L.total)
         return MUON_ERR_WORKSPACE;
     st = check_device();
@@ -424,48 +502,55 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
     double* sumsq = static_cast<double*>(at(workspace, L.sumsq));
     if (cudaMemsetAsync(sumsq, 0, sizeof(double) * n, stream_) != cudaSuccess) return MUON_ERR_CUDA;
 
-    // 1. fused MONA pre-pass + norms + wide-view copies
-    PrepParams pp;
-    memset(&pp, 0, sizeof(pp));
-    pp.in_dt = w_dtype; pp.x0_dt = ns_dtype; pp.mode = lite ? 2 : 0;
-    pp.beta_a = hp->beta_a; pp.alpha = hp->alpha; pp.mu = hp->mu;
-    pp.sumsq = sumsq;
+    // 1. fused MONA pre-pass + norms + wide-view copies: one launch per
+    //    element type of the copies (the iteration's, and fp32 for narrow groups)
     const size_t in_sz = dt_size(w_dtype);
-    for (const Group& g : L.groups) {
-        for (size_t j = 0; j < g.members.size(); ++j) {
-            const muon_param& p = params[g.members[j]];
-            PrepEntry& E = pp.e[pp.n++];
-            E.G = p.G; E.Gp = p.G_prev; E.A = p.A; E.M = p.M;
-            E.rows = p.rows; E.cols = p.cols; E.count = 1;
-            E.transposed = p.rows > p.cols;
-            E.X0 = static_cast<char*>(at(workspace, g.x[0])) + j * (size_t)g.s * g.ldl * dt_size(ns_dtype);
-            E.ld = g.ldl;
-            E.sumsq_index = g.sumsq0 + (int)j;
-            const uintptr_t al = reinterpret_cast<uintptr_t>(p.G) | reinterpret_cast<uintptr_t>(p.G_prev) |
-                                 reinterpret_cast<uintptr_t>(p.A) | reinterpret_cast<uintptr_t>(p.M);
-            E.vec_ok = (p.cols % 8 == 0) && (al & 15) == 0 && in_sz >= 2;
-            if (pp.n == kMaxPrep) {
-                st = prep_run(pp, stream_);
-                if (st != MUON_OK) return st;
-                pp.n = 0;
+    for (int x0_dt : {(int)ns_dtype, (int)DT_FP32}) {
+        if (x0_dt == DT_FP32 && (int)ns_dtype == DT_FP32) break;
+        PrepParams pp;
+        memset(&pp, 0, sizeof(pp));
+        pp.in_dt = w_dtype; pp.x0_dt = x0_dt; pp.mode = lite ? 2 : 0;
+        pp.beta_a = hp->beta_a; pp.alpha = hp->alpha; pp.mu = hp->mu;
+        pp.sumsq = sumsq;
+        for (const Group& g : L.groups) {
+            if (g.dt != x0_dt) continue;
+            for (size_t j = 0; j < g.members.size(); ++j) {
+                const muon_param& p = params[g.members[j]];
+                PrepEntry& E = pp.e[pp.n++];
+                E.G = p.G; E.Gp = p.G_prev; E.A = p.A; E.M = p.M;
+                E.rows = p.rows; E.cols = p.cols; E.count = 1;
+                E.transposed = p.rows > p.cols;
+                E.X0 = static_cast<char*>(at(workspace, g.x[0])) + j * (size_t)g.s * g.ldl * dt_size(g.dt);
+                E.ld = g.ldl;
+                E.sumsq_index = g.sumsq0 + (int)j;
+                const uintptr_t al = reinterpret_cast<uintptr_t>(p.G) | reinterpret_cast<uintptr_t>(p.G_prev) |
+                                     reinterpret_cast<uintptr_t>(p.A) | reinterpret_cast<uintptr_t>(p.M);
+                E.vec_ok = (p.cols % 8 == 0) && (al & 15) == 0 && in_sz >= 2;
+                if (pp.n == kMaxPrep) {
+                    st = prep_run(pp, stream_);
+                    if (st != MUON_OK) return st;
+                    pp.n = 0;
+                }
             }
         }
-    }
-    if (pp.n > 0) {
-        st = prep_run(pp, stream_);
-        if (st != MUON_OK) return st;
+        if (pp.n > 0) {
+            st = prep_run(pp, stream_);
+            if (st != MUON_OK) return st;
+        }
     }
 
-    // 2-3. iteration with the weight update fused into its last step
+    // 2-3. iteration with the weight update fused into its last step: the
+    //      direct groups of the iteration's type, the Gram-route groups, and
+    //      the narrow groups in fp32
     Runner R;
-    R.dt = ns_dtype;
     R.stream = stream_;
     memset(&R.fc, 0, sizeof(R.fc));
     R.fc.w_dt = w_dtype;
     R.fc.eta = hp->eta;
     R.fc.lambda = hp->lambda;
     R.fc.d_status = status;
-    std::vector<std::vector<FinalEntry>> fins;
+    GroupList direct16, gram16, direct32;
+    FinalTables fin_d16, fin_g16, fin_d32;
     for (const Group& g : L.groups) {
         std::vector<FinalEntry> f;
         for (int idx : g.members) {
@@ -479,9 +564,17 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
             fe.vec_ok = (p.cols % 8 == 0) && (al & 15) == 0;
             f.push_back(fe);
         }
-        fins.push_back(f);
+        if (g.dt != (int)ns_dtype) { direct32.push_back(&g); fin_d32.push_back(f); }
+        else if (g.gram) { gram16.push_back(&g); fin_g16.push_back(f); }
+        else { direct16.push_back(&g); fin_d16.push_back(f); }
     }
-    return run_direct(R, L, workspace, sched, fins, FIN_WUPD);
+    R.dt = ns_dtype;
+    st = run_direct(R, direct16, workspace, sumsq, sched, fin_d16, FIN_WUPD);
+    if (st != MUON_OK) return st;
+    st = run_gram(R, gram16, workspace, sumsq, sched, fin_g16, FIN_WUPD);
+    if (st != MUON_OK) return st;
+    R.dt = DT_FP32;
+    return run_direct(R, direct32, workspace, sumsq, sched, fin_d32, FIN_WUPD);
 }
 
 muon_status muon_step_batched(const muon_param* params, int n, muon_dtype w_dtype, muon_dtype ns_dtype,
@@ -502,10 +595,11 @@ static std::vector<muon_param> lite_as_params(const muon_lite_param* lp, int n) 
     return out;
 }
 
-muon_status muon_lite_workspace_size(const muon_lite_param* params, int n, muon_dtype ns_dtype, size_t* bytes) {
+muon_status muon_lite_workspace_size(const muon_lite_param* params, int n, muon_dtype ns_dtype,
+                                     const muon_schedule* sched, size_t* bytes) {
     if (!params || n < 1) return MUON_ERR_INVALID_ARG;
     std::vector<muon_param> p = lite_as_params(params, n);
-    return muon_workspace_size(p.data(), n, ns_dtype, bytes);
+    return muon_workspace_size(p.data(), n, ns_dtype, sched, bytes);
 }
 
 muon_status muon_lite_step_batched(const muon_lite_param* params, int n, muon_dtype w_dtype, muon_dtype ns_dtype,
@@ -527,13 +621,13 @@ static muon_status check_batch(const void* X_in, void* X_out, int batch, int row
 
 muon_status ns_polar_workspace_size(int batch, int rows, int cols, muon_dtype dtype, size_t* bytes) {
     if (!bytes || batch < 1 || rows < 1 || cols < 1 || !valid_dtype(dtype)) return MUON_ERR_INVALID_ARG;
-    *bytes = batch_layout(batch, rows, cols, dtype, 2).total;
+    *bytes = batch_layout(batch, rows, cols, dtype, 0).total;
     return MUON_OK;
 }
 
 muon_status gram_polar_workspace_size(int batch, int rows, int cols, muon_dtype dtype, size_t* bytes) {
     if (!bytes || batch < 1 || rows < 1 || cols < 1 || !valid_dtype(dtype)) return MUON_ERR_INVALID_ARG;
-    *bytes = batch_layout(batch, rows, cols, dtype, 6).total;
+    *bytes = batch_layout(batch, rows, cols, dtype, 1).total;
     return MUON_OK;
 }
 
@@ -545,7 +639,13 @@ static muon_status polar_common(int route, const void* X_in, void* X_out, int ba
     st = check_schedule(sched);
     if (st != MUON_OK) return st;
     if (batch == 1) batch_stride = (long long)rows * cols;
-    Layout L = batch_layout(batch, rows, cols, dtype, route == 0 ? 2 : 6);
+    // A bfloat16 input is iterated in fp16 ([POLAR]: fp16 is the recommended
+    // type; its three extra significand bits carry the small singular
+    // directions at condition numbers near 1e3): the copy of the input is
+    // divided by its norm first, which puts it in fp16's range.  Storage in and
+    // out stays bfloat16; both types take the same workspace.
+    const int it_dt = (int)dtype == DT_BF16 ? (int)DT_FP16 : (int)dtype;
+    Layout L = batch_layout(batch, rows, cols, it_dt, route);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) || ws_bytes < L.total)
         return MUON_ERR_WORKSPACE;
     st = check_device();
@@ -558,18 +658,27 @@ static muon_status polar_common(int route, const void* X_in, void* X_out, int ba
 
     PrepParams pp;
     memset(&pp, 0, sizeof(pp));
-    pp.in_dt = dtype; pp.x0_dt = dtype; pp.mode = 1; pp.sumsq = sumsq; pp.n = 1;
+    pp.in_dt = dtype; pp.x0_dt = it_dt; pp.mode = 1; pp.sumsq = sumsq; pp.n = 1; pp.eps = sched->eps;
     PrepEntry& E = pp.e[0];
     E.X = X_in; E.x_stride = batch_stride;
     E.X0 = at(workspace, g.x[0]); E.x0_stride = (long long)g.s * g.ldl; E.ld = g.ldl;
     E.rows = rows; E.cols = cols; E.count = batch; E.transposed = rows > cols;
     E.sumsq_index = 0;
     E.vec_ok = (cols % 8 == 0) && (batch_stride % 8 == 0) && (reinterpret_cast<uintptr_t>(X_in) & 15) == 0;
+    const bool prenorm = it_dt != (int)dtype;
+    if (prenorm) {
+        pp.mode = 3;                  // norms first
+        st = prep_run(pp, stream_);
+        if (st != MUON_OK) return st;
+        pp.mode = 1;
+        pp.prescale = 1;              // then the normalised copy
+    }
     st = prep_run(pp, stream_);
     if (st != MUON_OK) return st;
 
     Runner R;
-    R.dt = dtype;
+    R.dt = it_dt;
+    R.prenorm = prenorm;
     R.stream = stream_;
     memset(&R.fc, 0, sizeof(R.fc));
     R.fc.out_dt = dtype;
@@ -578,8 +687,10 @@ static muon_status polar_common(int route, const void* X_in, void* X_out, int ba
     R.fc.out_transposed = rows > cols;
     R.fc.out_vec = (cols % 8 == 0) && (batch_stride % 8 == 0) && (reinterpret_cast<uintptr_t>(X_out) & 15) == 0;
     R.fc.d_status = status;
-    if (route == 0) return run_direct(R, L, workspace, sched, {}, FIN_OUT);
-    return run_gram(R, L, workspace, sched);
+    const GroupList gs = {&L.groups[0]};
+    const FinalTables none(1);
+    if (route == 0) return run_direct(R, gs, workspace, sumsq, sched, none, FIN_OUT);
+    return run_gram(R, gs, workspace, sumsq, sched, none, FIN_OUT);
 }
 
 muon_status ns_polar(const void* X_in, void* X_out, int batch, int rows, int cols, long long batch_stride,

@@ -8,7 +8,10 @@
 // new M per matrix (Frobenius norm) and M rounded to the iteration's element
 // type, written in the wide view (transposed when rows > cols) into the
 // workspace.  COPY mode does the last two for a batch of input matrices
-// (ns_polar / gram_polar).
+// (ns_polar / gram_polar); NORM mode only sums the squares, so that a
+// following COPY pass can write the copy already divided by (||X|| + eps)
+// (prescale) -- the iteration of a bfloat16 input runs in fp16, whose range
+// needs the normalised values.
 //
 // Traffic per element (bf16 G/G_prev, fp32 A/M, bf16 copy): 12 bytes read,
 // 12 bytes written; the norm costs no extra bytes.  Tiles of 32 rows x 64
@@ -85,7 +88,7 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
         const int tr = E.flat ? 0 : (int)(tt / E.tiles_c), tc = E.flat ? 0 : (int)(tt % E.tiles_c);
         const int key = E.sumsq_index + b;
         if (key != cur) {   // uniform over the block
-            if (cur >= 0) {
+            if (cur >= 0 && !p.prescale) {
                 double s = block_sum(acc, red);
                 if (threadIdx.x == 0) atomicAdd(&p.sumsq[cur], s);
             }
@@ -161,10 +164,17 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
                 store8_dt(E.M, idx[h], DT_FP32, vec[h], nvalid[h], x[h]);
                 store8_dt(E.Gp, idx[h], DT_BF16, vec[h], nvalid[h], bb[h]);
             }
-        } else {
+        } else {   // COPY or NORM
             const void* X = static_cast<const char*>(E.X) + (size_t)b * E.x_stride * dt_size(IN_DT);
 #pragma unroll
             for (int h = 0; h < H; ++h) load8_in<IN_DT>(X, idx[h], vec[h], nvalid[h], x[h]);
+            if (p.prescale) {   // the norm is complete: store X / (||X|| + eps)
+                const float sc = (float)(1.0 / (sqrt(p.sumsq[key]) + (double)p.eps));
+#pragma unroll
+                for (int h = 0; h < H; ++h)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) x[h][i] *= sc;
+            }
         }
         float part = 0.f;
 #pragma unroll
@@ -172,6 +182,7 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
 #pragma unroll
             for (int i = 0; i < 8; ++i) part += x[h][i] * x[h][i];
         acc += (double)part;
+        if (p.mode == 3) continue;   // NORM: nothing to store (uniform over the block)
 
         void* X0 = static_cast<char*>(E.X0) + (size_t)b * E.x0_stride * dt_size(X0_DT);
         if (!E.transposed) {
@@ -203,7 +214,7 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
             __syncthreads();
         }
     }
-    if (cur >= 0) {
+    if (cur >= 0 && !p.prescale) {
         double s = block_sum(acc, red);
         if (threadIdx.x == 0) atomicAdd(&p.sumsq[cur], s);
     }
@@ -253,9 +264,9 @@ muon_status prep_run(PrepParams& prm, cudaStream_t stream) {
     for (int i = 0; i < prm.n; ++i) elems += (double)prm.e[i].rows * prm.e[i].cols * prm.e[i].count;
     const int isz = dt_size(prm.in_dt), xsz = dt_size(prm.x0_dt);
     // MONA: read G, G_prev, A, M; write A, M, G_prev, X0.  COPY: read X, write X0.
-    // MONA-Lite: read G, B, M; write B, M, X0.
+    // MONA-Lite: read G, B, M; write B, M, X0.  NORM: read X.
     const double per = prm.mode == 0 ? 3.0 * isz + 16.0 + xsz
-                     : prm.mode == 2 ? isz + 12.0 + xsz : (double)(isz + xsz);
+                     : prm.mode == 2 ? isz + 12.0 + xsz : prm.mode == 3 ? (double)isz : (double)(isz + xsz);
     trace_begin(MUON_KERNEL_PREPASS, elems * per, stream);
     // element types are compile-time in the kernel: loads and stores stay in registers
 #define MUON_PREP(I, X)                                                   \

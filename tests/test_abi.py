@@ -73,6 +73,7 @@ int main(void) {
   P(muon_param, A) P(muon_param, M) P(muon_param, gamma) P(muon_param, O_out)
   P(muon_schedule, n_steps) P(muon_schedule, coeffs) P(muon_schedule, eps)
   P(muon_schedule, restarts) P(muon_schedule, n_restarts) P(muon_schedule, scale_f)
+  P(muon_schedule, gram_aspect)
   P(muon_hparams, mu) P(muon_hparams, eta) P(muon_hparams, lambda) P(muon_hparams, gamma)
   P(muon_hparams, beta_a) P(muon_hparams, alpha)
   return 0;
@@ -126,6 +127,33 @@ def test_workspace_size_queries_are_host_only(lib):
     lower = 2 * (2 * 768 * 3072 * 2) + 2 * (2 * 768 * 768 * 2) + 4 * (768 * 768 * 2)
     assert lower <= n16 <= lower + 64 * 1024
     assert mo.ns_polar_workspace_size(4, 100, 300, mo.BF16) < mo.gram_polar_workspace_size(4, 100, 300, mo.BF16)
+    # a schedule with the Gram route on elongated groups: the 768x3072 group takes
+    # four more 768x768 buffers, the square group stays direct
+    gram = mo.quintic_gram_schedule(5, gram_aspect=2.0)
+    assert mo.muon_workspace_size(arr, mo.BF16, gram) - n16 in range(4 * 2 * 768 * 768 * 2,
+                                                                     4 * 2 * 768 * 768 * 2 + 8 * 1024)
+    assert mo.muon_workspace_size(arr, mo.BF16, mo.quintic_schedule(5)) == n16
+    assert mo.muon_workspace_size(arr, mo.BF16, mo.quintic_gram_schedule(5, gram_aspect=5.0)) == n16
+
+
+def test_narrow_groups_take_fp32_buffers(lib):
+    # a short side below 16 is iterated in fp32 whatever the iteration type:
+    # its buffers are sized in 4-byte elements
+    arr = (mo.Param * 1)()
+    arr[0].rows, arr[0].cols = 15, 1000
+    n16 = mo.muon_workspace_size(arr, mo.BF16)
+    assert n16 == mo.muon_workspace_size(arr, mo.FP32)
+    arr[0].rows = 16
+    assert mo.muon_workspace_size(arr, mo.BF16) < mo.muon_workspace_size(arr, mo.FP32)
+
+
+def test_schedule_gram_aspect_is_validated(lib):
+    arr = (mo.Param * 1)()
+    arr[0].rows, arr[0].cols = 64, 256
+    sz = ctypes.c_size_t(0)
+    for bad in (-1.0, float("nan"), float("inf")):
+        sched = mo.make_schedule([mo.QUINTIC] * 5, gram_aspect=bad)
+        assert lib.muon_workspace_size(arr, 1, mo.BF16, ctypes.byref(sched), ctypes.byref(sz)) == mo.ERR_INVALID_ARG
 
 
 def test_invalid_arguments_are_rejected_before_any_launch(lib):
@@ -164,8 +192,8 @@ def test_lite_entry_points_host_checks(lib):
     # same iteration workspace as the full step
     assert mo.muon_lite_workspace_size(lite, mo.BF16) == mo.muon_workspace_size(arr, mo.BF16)
     sz = ctypes.c_size_t(0)
-    assert L.muon_lite_workspace_size(None, 1, mo.BF16, ctypes.byref(sz)) == mo.ERR_INVALID_ARG
-    assert L.muon_lite_workspace_size(lite, 0, mo.BF16, ctypes.byref(sz)) == mo.ERR_INVALID_ARG
+    assert L.muon_lite_workspace_size(None, 1, mo.BF16, None, ctypes.byref(sz)) == mo.ERR_INVALID_ARG
+    assert L.muon_lite_workspace_size(lite, 0, mo.BF16, None, ctypes.byref(sz)) == mo.ERR_INVALID_ARG
     sched = mo.quintic_schedule(5)
     hp = mo.HParams(0.9, 0.02, 0.0, 1.0, 0.9, 0.5)
     buf = ctypes.create_string_buffer(64)

@@ -70,10 +70,11 @@ def sampled_mona_check(before, after, hp, n=4096, seed=0):
     assert np.array_equal(take(after["G_prev"]), Gp)
 
 
-def run_step(params, w):
-    sched = mo.quintic_schedule(5)
+def run_step(params, w, sched=None):
+    sched = sched if sched is not None else mo.quintic_schedule(5)
     arr = mo.make_params(params)
-    ws = torch.empty(mo.muon_workspace_size(arr, mo._dtype_code(w["ns_dtype"])), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(mo.muon_workspace_size(arr, mo._dtype_code(w["ns_dtype"]), sched), dtype=torch.uint8,
+                     device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     mo.muon_step_batched(arr, mo._dtype_code(w["w_dtype"]), mo._dtype_code(w["ns_dtype"]), w["hp"], sched, ws,
                          d_status=status)
@@ -146,18 +147,45 @@ def test_llama3_8b_full_step():
     for j, sh in enumerate(shapes):
         firsts.setdefault(sh, j)
     w, params = build_state("llama3_8b", dev, o_out_for=set(firsts.values()))
-    small = firsts[(1024, 4096)]
+    small, square = firsts[(1024, 4096)], firsts[(4096, 4096)]
     keep = set(firsts.values()) | set(range(0, len(params), 23))
     before = {j: {k: v.clone() for k, v in params[j].items() if k != "O_out"} for j in keep}
     assert run_step(params, w) == 0
+    # whole-matrix parity where the fp64 oracle takes at most a minute or two:
+    # the 1024 x 4096 and one 4096 x 4096 matrix, element by element
     oracle_full_check(before[small], params[small], w["hp"])
+    oracle_full_check(before[square], params[square], w["hp"])
     for sh, j in firsts.items():
         weight_consistency(before[j], params[j], w["hp"])
-        if sh != (1024, 4096):
+        if sh not in ((1024, 4096), (4096, 4096)):
             spectrum_check(params[j]["M"], params[j]["O_out"])
     for j in keep:
         sampled_mona_check(before[j], params[j], w["hp"], seed=j)
         assert torch.equal(params[j]["G_prev"], before[j]["G"])
+    del params, before
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("workload", ["gpt2_small", "llama_430m"])
+def test_full_step_gram_route(workload):
+    """The whole layer set in one call with the Gram route on the elongated
+    groups (768 x 3072, 1024 x 4096 and their transposes: long side >= 2 x short
+    side; one restart before step 3), the square groups direct.  One matrix per
+    shape against the oracle's step (in exact arithmetic both routes give the
+    same O), sampled elementwise state everywhere."""
+    dev = torch.device("cuda")
+    shapes = syn.WORKLOADS[workload]["shapes"]
+    firsts = {}
+    for j, sh in enumerate(shapes):
+        firsts.setdefault(sh, j)
+    w, params = build_state(workload, dev, o_out_for=set(firsts.values()))
+    before = [{k: v.clone() for k, v in p.items() if k != "O_out"} for p in params]
+    assert run_step(params, w, mo.quintic_gram_schedule(5, gram_aspect=2.0)) == 0
+    for j in firsts.values():
+        oracle_full_check(before[j], params[j], w["hp"])
+        weight_consistency(before[j], params[j], w["hp"])
+    for j in range(0, len(params), 5):
+        sampled_mona_check(before[j], params[j], w["hp"], seed=j)
     del params, before
     torch.cuda.empty_cache()
 
