@@ -431,21 +431,27 @@ def run_adamw_route(args, w):
 LIMUON_HP = dict(mu=0.95, eta=0.02, gamma=1.0, rank=16, oversample=16, **{"lambda": 0.0})
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 flops at the 1965 MHz maximum SM clock
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-LIMUON_KERNELS = ["lim_sketch", "lim_qr", "lim_project", "lim_factor", "lim_update"]
+LIMUON_KERNELS = ["lim_sketch", "lim_chol", "lim_rowmul_q", "lim_project", "lim_eig", "lim_rowmul_z", "lim_update"]
 
 
 def limuon_kernel_work(shapes, k, w_bytes=2):
-    """Algorithmic bytes and fp32 flops per launch of the five LiMuon kernels
-    for matrices `shapes` (one launch each): per element, the sketch reads G
-    and M and writes M (w_bytes + 8), the projection reads M (4), the update
-    reads and writes W (2 w_bytes); each of the three products is k FMAs per
-    element; the k-column factors add 4 k bytes per row / column."""
+    """Algorithmic bytes and fp32/fp64 flops per launch of the seven LiMuon
+    kernels for matrices `shapes` (one launch each): per element, the sketch
+    reads G and M and writes M (w_bytes + 8), the projection reads M (4), the
+    update reads and writes W (2 w_bytes); each of these three products is k
+    FMAs per element and moves its k-column factor (4 k bytes per row / column).
+    The row transforms read and write the rows x KT factor (8 KT bytes per row,
+    2 k^2 flops); the Cholesky and eigen steps move two KT x KT fp64 matrices
+    per matrix."""
+    kt = 32 if k <= 32 else 64
     el = sum(r * c for r, c in shapes)
-    rk = sum(r for r, _ in shapes) * k
+    rows = sum(r for r, _ in shapes)
+    rk = rows * k
     ck = sum(c for _, c in shapes) * k
-    by = [el * (w_bytes + 8) + 4 * rk, 8 * rk, el * 4 + 4 * (rk + ck), 4 * (ck + 2 * rk),
-          el * 2 * w_bytes + 4 * (rk + ck)]
-    fl = [2.0 * el * k, 0.0, 2.0 * el * k, 0.0, 2.0 * el * k]
+    small = 2 * 8 * kt * kt * len(shapes)
+    by = [el * (w_bytes + 8) + 4 * rk, small, 8 * rows * kt + small // 2, el * 4 + 4 * (rk + ck), small,
+          8 * rows * kt + small // 2, el * 2 * w_bytes + 4 * (rk + ck)]
+    fl = [2.0 * el * k, 0.0, 2.0 * rows * k * k, 2.0 * el * k, 0.0, 2.0 * rows * k * k, 2.0 * el * k]
     return by, fl
 
 

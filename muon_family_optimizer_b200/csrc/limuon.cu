@@ -10,21 +10,32 @@
 //     W <- W - eta (gamma O + lambda W)
 // Singular values at or below 1e-5 of the largest count as zero.
 //
-// Five launches per batch of up to 128 matrices (k = r + p <= 64, templated
-// on KT = 32 or 64 columns):
-//   1 lim_sketch   fused momentum pass and Y = M Omega: reads G and M, writes
-//                  M (10 bytes per element for 16-bit G), k FMAs per element.
-//   2 lim_qr       per matrix, one block: Q = Y R^-1 by Cholesky QR in fp64
-//                  (Gram Y^T Y, Cholesky; a column whose pivot falls to 1e-10
-//                  of its squared norm lies in the span of the previous ones
-//                  and is dropped: its Q column is zero).
-//   3 lim_project  B^T = M^T Q: reads M once more (4 bytes per element).
-//   4 lim_factor   per matrix, one block, fp64: C = B B^T = E L E^T by cyclic
-//                  Jacobi in parallel (round-robin) order; with the r largest
-//                  eigenvalues, O = Q E_r L_r^{-1/2} E_r^T B, so the kernel
-//                  forms Z = Q P, P = E_r L_r^{-1/2} E_r^T, in Q's place.
-//   5 lim_update   O = Z B row tile by row tile, fused with the weight update
-//                  (reads and writes W: 4 bytes per element for 16-bit W).
+// With C = B B^T = E L E^T (so U~ = E, S^2 = L) and V_r^T = L_r^{-1/2} E_r^T B:
+//     O = Q P B,   P = E_r L_r^{-1/2} E_r^T      (k x k)
+// and Q = Y R^-1 with Y^T Y = R^T R (Cholesky QR).  Every pass over an l x s
+// array streams; everything per matrix touches only k x k data:
+//   1 lim_sketch   M <- mu M + G and Y = M Omega, 128-row blocks over 64-column
+//                  chunks double-buffered in shared memory (cp.async); each
+//                  block adds its rows' share of the Gram Y^T Y (fp64) to the
+//                  matrix's k x k sum.  Reads G and M, writes M.
+//   2 lim_chol     per matrix (k x k): Cholesky of Y^T Y in fp64 (a column whose
+//                  pivot falls to 1e-10 of its squared norm lies in the span of
+//                  the previous ones and is dropped: its Q column is zero), R^-1.
+//   3 lim_rowmul   Q = Y R^-1, row by row in place (fp64 sums), all matrices'
+//                  rows in one grid.
+//   4 lim_project  B^T = M^T Q, 128-column blocks over 32-row chunks (three
+//                  cp.async stages); each block adds its columns' share of
+//                  B B^T (fp64) to the matrix's k x k sum.  Reads M.
+//   5 lim_eig      per matrix (k x k): cyclic Jacobi on B B^T in fp64,
+//                  round-robin order (k/2 disjoint rotations per round), a
+//                  rotation only while |C_pq| > 1e-15 sqrt(C_pp C_qq) (and
+//                  above 1e-16 of the trace: fp64 noise), stop after a sweep
+//                  without one; P from the r largest eigenpairs.
+//   6 lim_rowmul   Z = Q P in place.
+//   7 lim_update   O = Z B on 128 x 128 tiles, fused with the weight update
+//                  (reads and writes W; O never stored unless O_out is given).
+// A non-finite momentum element or k x k factor marks its matrix: its W is
+// kept and MUON_FLAG_NONFINITE raised.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -39,26 +50,33 @@ namespace {
 
 constexpr int kLimMax = 128;      // matrices per launch
 constexpr int kThreads = 256;
-constexpr int kSketchRows = 64;   // lim_sketch: rows per block
-constexpr int kChunk = 128;       // columns per smem chunk (sketch, project, update)
-constexpr int kMsLd = kChunk + 4; // padded row of a staged M tile
-constexpr int kProjRows = 32;     // lim_project: rows per chunk
-constexpr int kUpdRows = 32;      // lim_update: rows per tile
-constexpr int kGramRows = 64;     // rows of Y / B^T staged per Gram chunk
+constexpr int kSmallThreads = 64; // per-matrix k x k kernels
+constexpr int kSkRows = 128;      // lim_sketch: rows per block
+constexpr int kSkCols = 64;       // lim_sketch: columns per chunk (two stages)
+constexpr int kPjCols = 128;      // lim_project: columns per block
+constexpr int kPjRows = 32;       // lim_project: rows per chunk
+constexpr int kPjStages = 3;
+constexpr int kUpRows = 128;      // lim_update: tile rows
+constexpr int kUpCols = 128;      // lim_update: tile columns
+constexpr int kBsLd = kUpCols + 4;   // padded row of the staged B tile
 constexpr double kDrop = 1e-10;   // Cholesky pivot / squared column norm below which a column is dropped
 constexpr double kTau2 = 1e-10;   // (singular value / largest)^2 at or below which it counts as zero
+constexpr double kRotTol = 1e-15; // Jacobi: rotate while |C_pq| > kRotTol sqrt(C_pp C_qq)
 constexpr int kMaxSweeps = 30;
 constexpr int kMaxDevices = 64;    // devices whose kernel attributes are tracked
 
 struct LimEntry {
     void* W; const void* G; float* M; const float* Omega; float* O_out;
-    float* Y;        // rows x KT workspace: Y, then Q, then Z
+    float* Y;        // rows x KT workspace: Y, then Q, then Z (in place)
     float* Bt;       // cols x KT workspace: B^T
-    int* bad;        // this matrix's non-finite flag (workspace)
+    double* Gy;      // KT x KT: Y^T Y, upper triangle summed by lim_sketch (zeroed per call)
+    double* Cg;      // KT x KT: B B^T, upper triangle summed by lim_project (zeroed per call)
+    double* K;       // KT x KT: R^-1 (lim_chol), then P (lim_eig)
+    int* bad;        // this matrix's non-finite flag (workspace, zeroed per call)
     int rows, cols;
     float gamma;
-    int vec_ok;      // W, G, M 16-byte aligned and cols % 8 == 0
-    int t_sketch, t_proj, t_upd;   // first block of this matrix in each launch's grid
+    int vec_ok;      // W, G, M, O_out 16-byte aligned and cols % 8 == 0
+    int t_sketch, t_rows, t_proj, t_upd;   // first block of this matrix in each launch's grid
 };
 
 struct LimParams {
@@ -68,77 +86,161 @@ struct LimParams {
     int* d_status;
 };
 
+// The matrix that block b of a launch works on: the last entry whose first
+// block is <= b (which: 0 sketch, 1 row transforms, 2 projection, 3 update).
 __device__ __forceinline__ int find_entry(const LimParams& p, int b, int which) {
-    int lo = 0, hi = p.n - 1;        // last entry whose first block is <= b
+    int lo = 0, hi = p.n - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        const int t = which == 0 ? p.e[mid].t_sketch : which == 1 ? p.e[mid].t_proj : p.e[mid].t_upd;
+        const LimEntry& e = p.e[mid];
+        const int t = which == 0 ? e.t_sketch : which == 1 ? e.t_rows : which == 2 ? e.t_proj : e.t_upd;
         if (t <= b) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
 
+__device__ __forceinline__ void mark_bad(const LimParams& p, const LimEntry& E) {
+    atomicOr(E.bad, 1);
+    if (p.d_status) atomicOr(p.d_status, MUON_FLAG_NONFINITE);
+}
+
+// Entry e of the upper triangle (row-major, a <= b) of a KT x KT matrix.
+template <int KT>
+__device__ __forceinline__ void upper_entry(int e, int& a, int& b) {
+    a = 0;
+    while (e >= KT - a) { e -= KT - a; ++a; }
+    b = a + e;
+}
+
+// Add this block's share S = X^T X of a k x k Gram matrix (X: `n` rows of KT
+// floats in shared memory, columns >= k ignored) to the upper triangle of the
+// fp64 sum `dst`.
+template <int KT>
+__device__ __forceinline__ void add_gram(const float* X, int n, int k, double* dst) {
+    constexpr int NE = KT * (KT + 1) / 2;
+    for (int e = threadIdx.x; e < NE; e += blockDim.x) {
+        int a, b;
+        upper_entry<KT>(e, a, b);
+        if (b >= k) continue;
+        double s = 0.0;
+        for (int rr = 0; rr < n; ++rr) s = fma((double)X[rr * KT + a], (double)X[rr * KT + b], s);
+        if (s != 0.0) atomicAdd(&dst[a * KT + b], s);
+    }
+}
+
 // ---------------------------------------------------------------------------
-// 1. momentum + sketch
+// 1. momentum + sketch (+ share of Y^T Y)
 // ---------------------------------------------------------------------------
+template <int G_DT>
+__host__ __device__ constexpr int g_size() { return G_DT == DT_FP32 ? 4 : 2; }
+
+template <int G_DT>
+__host__ __device__ constexpr int sketch_stage_bytes() { return kSkRows * kSkCols * (g_size<G_DT>() + 4); }
+
 template <int KT, int G_DT>
-__global__ void __launch_bounds__(kThreads) lim_sketch(const __grid_constant__ LimParams p) {
+__global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant__ LimParams p) {
     constexpr int H = KT / 32;
-    extern __shared__ __align__(16) float smem[];
-    float* Ms = smem;                              // [kSketchRows][kMsLd]
-    float* Os = smem + kSketchRows * kMsLd;        // [kChunk][KT]
+    constexpr int GSZ = g_size<G_DT>();
+    constexpr int kGBytes = kSkRows * kSkCols * GSZ;
+    constexpr int kStage = sketch_stage_bytes<G_DT>();
+    extern __shared__ __align__(16) unsigned char sm[];
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 0)];
-    const int row0 = (blockIdx.x - E.t_sketch) * kSketchRows;
+    const int row0 = (blockIdx.x - E.t_sketch) * kSkRows;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float acc[8][H];
+    const int nchunks = (E.cols + kSkCols - 1) / kSkCols;
+    float acc[16][H];
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
+    for (int r = 0; r < 16; ++r)
 #pragma unroll
         for (int h = 0; h < H; ++h) acc[r][h] = 0.f;
     bool bad = false;
-    for (int c0 = 0; c0 < E.cols; c0 += kChunk) {
-#pragma unroll 1
-        for (int pass = 0; pass < kSketchRows * kChunk / (8 * kThreads); ++pass) {
-            const int g = threadIdx.x + kThreads * pass;
-            const int rr = g >> 4, cc = (g & 15) * 8;
-            const int i = row0 + rr, j = c0 + cc;
-            float m[8];
-            if (i < E.rows && j < E.cols) {
-                const long long idx = (long long)i * E.cols + j;
-                const int nvalid = min(8, E.cols - j);
-                const bool vec = E.vec_ok && nvalid == 8;
-                float g8[8];
-                load8_dt(E.G, idx, G_DT, vec, nvalid, g8);
-                load8_dt(E.M, idx, DT_FP32, vec, nvalid, m);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    m[q] = q < nvalid ? fmaf(p.mu, m[q], g8[q]) : 0.f;
-                    bad |= !isfinite(m[q]);
-                }
-                store8_dt(E.M, idx, DT_FP32, vec, nvalid, m);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) m[q] = 0.f;
+
+    // Chunk c (columns c*kSkCols..) of G and M into stage s: raw G in its own
+    // type, then M in fp32, row-major [kSkRows][kSkCols]; zeros outside the matrix.
+    auto issue = [&](int c, int s) {
+        const int c0 = c * kSkCols;
+        unsigned char* gs = sm + s * kStage;
+        float* ms = reinterpret_cast<float*>(gs + kGBytes);
+        if (E.vec_ok) {
+            constexpr int GP = kSkCols * GSZ / 16, GE = 16 / GSZ;    // 16-byte pieces per row, elements per piece
+            for (int q = threadIdx.x; q < kSkRows * GP; q += kThreads) {
+                const int rr = q / GP, pc = q % GP, i = row0 + rr, j = c0 + pc * GE;
+                const bool in = i < E.rows && j < E.cols;
+                const char* src = static_cast<const char*>(E.G) + (in ? ((long long)i * E.cols + j) * GSZ : 0);
+                cp_async16(gs + (rr * kSkCols + pc * GE) * GSZ, src, in ? 16u : 0u);
             }
-            float4* dst = reinterpret_cast<float4*>(Ms + rr * kMsLd + cc);
-            dst[0] = make_float4(m[0], m[1], m[2], m[3]);
-            dst[1] = make_float4(m[4], m[5], m[6], m[7]);
+            constexpr int MP = kSkCols / 4;
+            for (int q = threadIdx.x; q < kSkRows * MP; q += kThreads) {
+                const int rr = q / MP, pc = q % MP, i = row0 + rr, j = c0 + pc * 4;
+                const bool in = i < E.rows && j < E.cols;
+                cp_async16(ms + rr * kSkCols + pc * 4, E.M + (in ? (long long)i * E.cols + j : 0), in ? 16u : 0u);
+            }
+        } else {
+            for (int q = threadIdx.x; q < kSkRows * kSkCols; q += kThreads) {
+                const int rr = q / kSkCols, cc = q % kSkCols, i = row0 + rr, j = c0 + cc;
+                const bool in = i < E.rows && j < E.cols;
+                const long long idx = (long long)i * E.cols + j;
+                st_elem(gs, rr * kSkCols + cc, G_DT, in ? ld_elem(E.G, idx, G_DT) : 0.f);
+                ms[rr * kSkCols + cc] = in ? E.M[idx] : 0.f;
+            }
         }
-        for (int idx = threadIdx.x; idx < kChunk * KT; idx += kThreads) {
-            const int jj = idx / KT, t = idx % KT;
-            Os[idx] = (t < p.k && c0 + jj < E.cols) ? E.Omega[(long long)(c0 + jj) * p.k + t] : 0.f;
+        cp_async_commit();
+    };
+
+    issue(0, 0);
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1;
+        if (c + 1 < nchunks) {
+            issue(c + 1, s ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();                       // chunk c complete for every thread
+        const int c0 = c * kSkCols;
+        unsigned char* gs = sm + s * kStage;
+        float* ms = reinterpret_cast<float*>(gs + kGBytes);
+        // momentum: M <- mu M + G, back to global memory and kept for the product
+#pragma unroll
+        for (int it = 0; it < kSkRows * kSkCols / (8 * kThreads); ++it) {
+            const int q = threadIdx.x + kThreads * it;
+            const int rr = q / (kSkCols / 8), cc = (q % (kSkCols / 8)) * 8;
+            const int i = row0 + rr, j = c0 + cc;
+            float g[8], m[8];
+            load8_dt(gs, rr * kSkCols + cc, G_DT, true, 8, g);
+            float4* mp = reinterpret_cast<float4*>(ms + rr * kSkCols + cc);
+            const float4 m0 = mp[0], m1 = mp[1];
+            m[0] = m0.x; m[1] = m0.y; m[2] = m0.z; m[3] = m0.w;
+            m[4] = m1.x; m[5] = m1.y; m[6] = m1.z; m[7] = m1.w;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                m[e] = fmaf(p.mu, m[e], g[e]);   // zero outside the matrix
+                bad |= !isfinite(m[e]);
+            }
+            mp[0] = make_float4(m[0], m[1], m[2], m[3]);
+            mp[1] = make_float4(m[4], m[5], m[6], m[7]);
+            if (i < E.rows && j < E.cols) {
+                const int nvalid = min(8, E.cols - j);
+                store8_dt(E.M, (long long)i * E.cols + j, DT_FP32, E.vec_ok != 0, nvalid, m);
+            }
         }
         __syncthreads();
+        // Y rows 16 warp + r, column lane + 32 h: += M chunk x Omega chunk
 #pragma unroll 2
-        for (int jj = 0; jj < kChunk; jj += 4) {
+        for (int jj = 0; jj < kSkCols; jj += 4) {
             float om[4][H];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < 4; ++q) {
+                const int j = c0 + jj + q;
 #pragma unroll
-                for (int h = 0; h < H; ++h) om[q][h] = Os[(jj + q) * KT + lane + 32 * h];
+                for (int h = 0; h < H; ++h) {
+                    const int t = lane + 32 * h;
+                    om[q][h] = (j < E.cols && t < p.k) ? __ldg(E.Omega + (long long)j * p.k + t) : 0.f;
+                }
+            }
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const float4 mv = *reinterpret_cast<const float4*>(Ms + (8 * warp + r) * kMsLd + jj);
+            for (int r = 0; r < 16; ++r) {
+                const float4 mv = *reinterpret_cast<const float4*>(ms + (16 * warp + r) * kSkCols + jj);
 #pragma unroll
                 for (int h = 0; h < H; ++h) {
                     acc[r][h] = fmaf(mv.x, om[0][h], acc[r][h]);
@@ -148,84 +250,52 @@ __global__ void __launch_bounds__(kThreads) lim_sketch(const __grid_constant__ L
                 }
             }
         }
-        __syncthreads();
+        __syncthreads();                       // stage s free for chunk c + 2
     }
+    // Y to the workspace, and this block's rows' share of Y^T Y
+    float* ys = reinterpret_cast<float*>(sm);  // [kSkRows][KT]
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int i = row0 + 8 * warp + r;
-        if (i >= E.rows) continue;
+    for (int r = 0; r < 16; ++r) {
+        const int rr = 16 * warp + r, i = row0 + rr;
 #pragma unroll
-        for (int h = 0; h < H; ++h) E.Y[(long long)i * KT + lane + 32 * h] = acc[r][h];
-    }
-    if (__syncthreads_or(bad) && threadIdx.x == 0) {
-        atomicOr(E.bad, 1);
-        if (p.d_status) atomicOr(p.d_status, MUON_FLAG_NONFINITE);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Gram matrix G = X^T X (k x k, fp64) of an n x KT fp32 array (columns >= k
-// ignored), into Gm[KT * KT] (shared); stage: kGramRows x KT floats (shared).
-// ---------------------------------------------------------------------------
-template <int KT>
-__device__ void gram_fp64(const float* X, int n, int k, double* Gm, float* stage) {
-    constexpr int NE = KT * (KT + 1) / 2;
-    constexpr int PER = (NE + kThreads - 1) / kThreads;
-    int ea[PER], eb[PER];
-    double acc[PER];
-#pragma unroll
-    for (int q = 0; q < PER; ++q) {
-        // entry e -> (a, b), a <= b, row-major over the upper triangle
-        int e = threadIdx.x + kThreads * q, a = 0;
-        if (e < NE) {
-            while (e >= KT - a) { e -= KT - a; ++a; }
-            ea[q] = a; eb[q] = a + e;
-        } else {
-            ea[q] = eb[q] = -1;
-        }
-        acc[q] = 0.0;
-    }
-    for (int r0 = 0; r0 < n; r0 += kGramRows) {
-        __syncthreads();
-        for (int idx = threadIdx.x; idx < kGramRows * KT; idx += kThreads) {
-            const int rr = idx / KT, t = idx % KT;
-            stage[idx] = (r0 + rr < n && t < k) ? X[(long long)(r0 + rr) * KT + t] : 0.f;
-        }
-        __syncthreads();
-        const int nr = min(kGramRows, n - r0);
-#pragma unroll
-        for (int q = 0; q < PER; ++q) {
-            if (ea[q] < 0) continue;
-            double s = 0.0;
-            for (int rr = 0; rr < nr; ++rr)
-                s = fma((double)stage[rr * KT + ea[q]], (double)stage[rr * KT + eb[q]], s);
-            acc[q] += s;
+        for (int h = 0; h < H; ++h) {
+            ys[rr * KT + lane + 32 * h] = acc[r][h];   // zero for rows past the matrix
+            if (i < E.rows) E.Y[(long long)i * KT + lane + 32 * h] = acc[r][h];
         }
     }
-#pragma unroll
-    for (int q = 0; q < PER; ++q)
-        if (ea[q] >= 0) {
-            Gm[ea[q] * KT + eb[q]] = acc[q];
-            Gm[eb[q] * KT + ea[q]] = acc[q];
-        }
     __syncthreads();
+    add_gram<KT>(ys, min(kSkRows, E.rows - row0), p.k, E.Gy);
+    if (__syncthreads_or(bad) && threadIdx.x == 0) mark_bad(p, E);
 }
 
 // ---------------------------------------------------------------------------
-// 2. Cholesky QR (one block per matrix)
+// 2. Cholesky of Y^T Y and R^-1 (one small block per matrix, k x k only)
 // ---------------------------------------------------------------------------
 template <int KT>
-__global__ void __launch_bounds__(kThreads) lim_qr(const __grid_constant__ LimParams p) {
+__global__ void __launch_bounds__(kSmallThreads) lim_chol(const __grid_constant__ LimParams p) {
     extern __shared__ __align__(16) double dsm[];
-    double* Gm = dsm;                   // [KT][KT]: Gram, then R^-1
-    double* R = dsm + KT * KT;          // [KT][KT]: R (upper)
+    double* Gm = dsm;                   // [KT][KT]: the Gram matrix, updated in place
+    double* R = dsm + KT * KT;          // [KT][KT]: R (upper), then R^-1
     double* d0 = R + KT * KT;           // [KT]: squared column norms
-    int* ok = reinterpret_cast<int*>(d0 + KT);                  // [KT]
-    float* stage = reinterpret_cast<float*>(ok + KT);          // [kGramRows][KT]
+    int* ok = reinterpret_cast<int*>(d0 + KT);   // [KT]
+    __shared__ int nonfinite;
     const LimEntry& E = p.e[blockIdx.x];
     const int k = p.k;
-    gram_fp64<KT>(E.Y, E.rows, k, Gm, stage);
-    for (int idx = threadIdx.x; idx < KT * KT; idx += kThreads) R[idx] = 0.0;
+    if (threadIdx.x == 0) nonfinite = 0;
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < KT * KT; idx += blockDim.x) {
+        const int a = idx / KT, b = idx % KT;
+        const double v = (a < k && b < k) ? (a <= b ? E.Gy[a * KT + b] : E.Gy[b * KT + a]) : 0.0;
+        if (!isfinite(v)) nonfinite = 1;
+        Gm[idx] = v;
+        R[idx] = 0.0;
+    }
+    __syncthreads();
+    if (nonfinite) {                    // an overflow in the sketch: keep W, no factor
+        for (int idx = threadIdx.x; idx < KT * KT; idx += blockDim.x) E.K[idx] = 0.0;
+        if (threadIdx.x == 0) mark_bad(p, E);
+        return;
+    }
     if (threadIdx.x < KT) d0[threadIdx.x] = Gm[threadIdx.x * KT + threadIdx.x];
     __syncthreads();
     // right-looking Cholesky of the upper triangle: G = R^T R
@@ -233,21 +303,20 @@ __global__ void __launch_bounds__(kThreads) lim_qr(const __grid_constant__ LimPa
         const double d = Gm[j * KT + j];
         const bool keep = d > kDrop * d0[j] && d > 0.0;
         const double rj = keep ? sqrt(d) : 0.0;
-        for (int b = j + threadIdx.x; b < k; b += kThreads) R[j * KT + b] = keep ? (b == j ? rj : Gm[j * KT + b] / rj) : 0.0;
+        for (int b = j + threadIdx.x; b < k; b += blockDim.x) R[j * KT + b] = keep ? (b == j ? rj : Gm[j * KT + b] / rj) : 0.0;
         if (threadIdx.x == 0) ok[j] = keep;
         __syncthreads();
         const int m = k - j - 1;
-        for (int idx = threadIdx.x; idx < m * m; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) {
             const int a = j + 1 + idx / m, b = j + 1 + idx % m;
             if (b >= a) Gm[a * KT + b] -= R[j * KT + a] * R[j * KT + b];
         }
         __syncthreads();
     }
     // R^-1 (upper) column by column into Gm; dropped rows stay zero
-    for (int idx = threadIdx.x; idx < KT * KT; idx += kThreads) Gm[idx] = 0.0;
+    for (int idx = threadIdx.x; idx < KT * KT; idx += blockDim.x) Gm[idx] = 0.0;
     __syncthreads();
-    if (threadIdx.x < k) {
-        const int b = threadIdx.x;
+    for (int b = threadIdx.x; b < k; b += blockDim.x) {
         for (int a = b; a >= 0; --a) {
             if (!ok[a]) continue;
             double s = a == b ? 1.0 : 0.0;
@@ -256,73 +325,103 @@ __global__ void __launch_bounds__(kThreads) lim_qr(const __grid_constant__ LimPa
         }
     }
     __syncthreads();
-    // Q = Y R^-1, row by row in place
-    for (int i = threadIdx.x; i < E.rows; i += kThreads) {
-        float y[KT];
-        float* row = E.Y + (long long)i * KT;
-#pragma unroll
-        for (int t = 0; t < KT; ++t) y[t] = t < k ? row[t] : 0.f;
-#pragma unroll 4
-        for (int j = 0; j < KT; ++j) {
-            if (j >= k) break;
-            double s = 0.0;
-#pragma unroll
-            for (int a = 0; a < KT; ++a)
-                if (a <= j) s = fma((double)y[a], Gm[a * KT + j], s);
-            row[j] = (float)s;
-        }
-    }
+    for (int idx = threadIdx.x; idx < KT * KT; idx += blockDim.x) E.K[idx] = Gm[idx];
 }
 
 // ---------------------------------------------------------------------------
-// 3. B^T = M^T Q
+// 3 / 6. rows of Y times the matrix's k x k factor K, in place (fp64 sums)
 // ---------------------------------------------------------------------------
 template <int KT>
-__global__ void __launch_bounds__(kThreads) lim_project(const __grid_constant__ LimParams p) {
-    constexpr int H = KT / 32;
-    extern __shared__ __align__(16) float smem[];
-    float* Ms = smem;                          // [kProjRows][kMsLd]
-    float* Qs = smem + kProjRows * kMsLd;      // [kProjRows][KT]
+__global__ void __launch_bounds__(kThreads) lim_rowmul(const __grid_constant__ LimParams p) {
+    __shared__ double Ks[KT * KT];
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 1)];
-    const int c0 = (blockIdx.x - E.t_proj) * kChunk;
+    for (int idx = threadIdx.x; idx < KT * KT; idx += kThreads) Ks[idx] = E.K[idx];
+    __syncthreads();
+    const int i = (blockIdx.x - E.t_rows) * kThreads + threadIdx.x;
+    if (i >= E.rows) return;
+    float* row = E.Y + (long long)i * KT;
+    float y[KT];
+#pragma unroll
+    for (int t = 0; t < KT; t += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(row + t);
+        y[t] = v.x; y[t + 1] = v.y; y[t + 2] = v.z; y[t + 3] = v.w;
+    }
+    float out[KT];
+#pragma unroll 4
+    for (int j = 0; j < KT; ++j) {
+        double s = 0.0;
+#pragma unroll
+        for (int a = 0; a < KT; ++a) s = fma((double)y[a], Ks[a * KT + j], s);
+        out[j] = (float)s;
+    }
+#pragma unroll
+    for (int t = 0; t < KT; t += 4)
+        *reinterpret_cast<float4*>(row + t) = make_float4(out[t], out[t + 1], out[t + 2], out[t + 3]);
+}
+
+// ---------------------------------------------------------------------------
+// 4. B^T = M^T Q (+ share of B B^T)
+// ---------------------------------------------------------------------------
+template <int KT>
+__host__ __device__ constexpr int project_stage_floats() { return kPjRows * kPjCols + kPjRows * KT; }
+
+template <int KT>
+__global__ void __launch_bounds__(kThreads, 3) lim_project(const __grid_constant__ LimParams p) {
+    constexpr int H = KT / 32;
+    constexpr int kStage = project_stage_floats<KT>();
+    extern __shared__ __align__(16) float fsm[];
+    const LimEntry& E = p.e[find_entry(p, blockIdx.x, 2)];
+    const int c0 = (blockIdx.x - E.t_proj) * kPjCols;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nchunks = (E.rows + kPjRows - 1) / kPjRows;
     float acc[16][H];
 #pragma unroll
     for (int c = 0; c < 16; ++c)
 #pragma unroll
         for (int h = 0; h < H; ++h) acc[c][h] = 0.f;
-    for (int i0 = 0; i0 < E.rows; i0 += kProjRows) {
-#pragma unroll
-        for (int pass = 0; pass < kProjRows * kChunk / (8 * kThreads); ++pass) {
-            const int g = threadIdx.x + kThreads * pass;
-            const int rr = g >> 4, cc = (g & 15) * 8;
-            const int i = i0 + rr, j = c0 + cc;
-            float m[8];
-            if (i < E.rows && j < E.cols) {
-                const long long idx = (long long)i * E.cols + j;
-                const int nvalid = min(8, E.cols - j);
-                load8_dt(E.M, idx, DT_FP32, E.vec_ok && nvalid == 8, nvalid, m);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) m[q] = q < nvalid ? m[q] : 0.f;
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) m[q] = 0.f;
+
+    // rows i0.. of M (this block's columns) and of Q into stage s
+    auto issue = [&](int ch, int s) {
+        const int i0 = ch * kPjRows;
+        float* ms = fsm + s * kStage;
+        float* qs = ms + kPjRows * kPjCols;
+        if (E.vec_ok) {
+            constexpr int MP = kPjCols / 4;
+            for (int q = threadIdx.x; q < kPjRows * MP; q += kThreads) {
+                const int rr = q / MP, pc = q % MP, i = i0 + rr, j = c0 + pc * 4;
+                const bool in = i < E.rows && j < E.cols;
+                cp_async16(ms + rr * kPjCols + pc * 4, E.M + (in ? (long long)i * E.cols + j : 0), in ? 16u : 0u);
             }
-            float4* dst = reinterpret_cast<float4*>(Ms + rr * kMsLd + cc);
-            dst[0] = make_float4(m[0], m[1], m[2], m[3]);
-            dst[1] = make_float4(m[4], m[5], m[6], m[7]);
+        } else {
+            for (int q = threadIdx.x; q < kPjRows * kPjCols; q += kThreads) {
+                const int rr = q / kPjCols, cc = q % kPjCols, i = i0 + rr, j = c0 + cc;
+                ms[q] = (i < E.rows && j < E.cols) ? E.M[(long long)i * E.cols + j] : 0.f;
+            }
         }
-        for (int idx = threadIdx.x; idx < kProjRows * KT; idx += kThreads) {
-            const int rr = idx / KT, t = idx % KT;
-            Qs[idx] = (i0 + rr < E.rows && t < p.k) ? E.Y[(long long)(i0 + rr) * KT + t] : 0.f;
+        constexpr int QP = KT / 4;
+        for (int q = threadIdx.x; q < kPjRows * QP; q += kThreads) {
+            const int rr = q / QP, pc = q % QP, i = i0 + rr;
+            const bool in = i < E.rows;
+            cp_async16(qs + rr * KT + pc * 4, E.Y + (in ? (long long)i * KT + pc * 4 : 0), in ? 16u : 0u);
         }
+        cp_async_commit();
+    };
+
+    for (int ch = 0; ch < kPjStages - 1; ++ch)
+        if (ch < nchunks) issue(ch, ch); else cp_async_commit();   // empty groups keep the count uniform
+    for (int ch = 0; ch < nchunks; ++ch) {
+        if (ch + kPjStages - 1 < nchunks) issue(ch + kPjStages - 1, (ch + kPjStages - 1) % kPjStages);
+        else cp_async_commit();
+        cp_async_wait<kPjStages - 1>();
         __syncthreads();
-#pragma unroll 2
-        for (int rr = 0; rr < kProjRows; ++rr) {
+        const float* ms = fsm + (ch % kPjStages) * kStage;
+        const float* qs = ms + kPjRows * kPjCols;
+#pragma unroll 4
+        for (int rr = 0; rr < kPjRows; ++rr) {
             float qv[H];
 #pragma unroll
-            for (int h = 0; h < H; ++h) qv[h] = Qs[rr * KT + lane + 32 * h];
-            const float4* mrow = reinterpret_cast<const float4*>(Ms + rr * kMsLd + 16 * warp);
+            for (int h = 0; h < H; ++h) qv[h] = qs[rr * KT + lane + 32 * h];
+            const float4* mrow = reinterpret_cast<const float4*>(ms + rr * kPjCols + 16 * warp);
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
                 const float4 mv = mrow[c4];
@@ -335,83 +434,95 @@ __global__ void __launch_bounds__(kThreads) lim_project(const __grid_constant__ 
                 }
             }
         }
-        __syncthreads();
+        __syncthreads();                       // this stage is refilled next
     }
+    cp_async_wait<0>();
+    // B^T to the workspace, and this block's columns' share of B B^T
+    float* bs = fsm;                           // [kPjCols][KT]
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
-        const int j = c0 + 16 * warp + c;
-        if (j >= E.cols) continue;
+        const int cc = 16 * warp + c, j = c0 + cc;
 #pragma unroll
-        for (int h = 0; h < H; ++h) E.Bt[(long long)j * KT + lane + 32 * h] = acc[c][h];
+        for (int h = 0; h < H; ++h) {
+            bs[cc * KT + lane + 32 * h] = acc[c][h];
+            if (j < E.cols) E.Bt[(long long)j * KT + lane + 32 * h] = acc[c][h];
+        }
     }
+    __syncthreads();
+    add_gram<KT>(bs, min(kPjCols, E.cols - c0), p.k, E.Cg);
 }
 
 // ---------------------------------------------------------------------------
-// 4. eigen-decomposition of B B^T and Z = Q P (one block per matrix)
+// 5. eigen-decomposition of B B^T and P = E_r L_r^{-1/2} E_r^T (one small
+//    block per matrix, k x k only)
 // ---------------------------------------------------------------------------
 template <int KT>
-__global__ void __launch_bounds__(kThreads) lim_factor(const __grid_constant__ LimParams p) {
+__global__ void __launch_bounds__(kSmallThreads) lim_eig(const __grid_constant__ LimParams p) {
     extern __shared__ __align__(16) double dsm[];
     double* C = dsm;                    // [KT][KT]
     double* Ev = dsm + KT * KT;         // [KT][KT] eigenvectors (columns)
     double* cs = Ev + KT * KT;          // [KT/2] cosines
     double* sn = cs + KT / 2;           // [KT/2] sines
     double* lam = sn + KT / 2;          // [KT] eigenvalues
-    double* red = lam + KT;             // [2 * 8] reduction scratch
-    int* pp = reinterpret_cast<int*>(red + 16);   // [KT/2]
+    int* pp = reinterpret_cast<int*>(lam + KT);   // [KT/2]
     int* pq = pp + KT / 2;                         // [KT/2]
-    float* stage = reinterpret_cast<float*>(pq + KT / 2);   // [kGramRows][KT]
+    __shared__ int rotated, nonfinite;
     const LimEntry& E = p.e[blockIdx.x];
     const int k = p.k, ke = k + (k & 1), n = ke - 1;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    gram_fp64<KT>(E.Bt, E.cols, k, C, stage);
-    for (int idx = threadIdx.x; idx < KT * KT; idx += kThreads) Ev[idx] = (idx / KT == idx % KT) ? 1.0 : 0.0;
+    if (threadIdx.x == 0) nonfinite = 0;
     __syncthreads();
-    for (int sweep = 0; sweep < kMaxSweeps; ++sweep) {
-        double off = 0.0, tot = 0.0;
-        for (int idx = threadIdx.x; idx < ke * ke; idx += kThreads) {
-            const int a = idx / ke, b = idx % ke;
-            const double v = C[a * KT + b] * C[a * KT + b];
-            tot += v;
-            if (a != b) off += v;
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-            off += __shfl_xor_sync(0xffffffffu, off, o);
-            tot += __shfl_xor_sync(0xffffffffu, tot, o);
-        }
-        if (lane == 0) { red[warp] = off; red[8 + warp] = tot; }
+    for (int idx = threadIdx.x; idx < KT * KT; idx += blockDim.x) {
+        const int a = idx / KT, b = idx % KT;
+        const double v = (a < k && b < k) ? (a <= b ? E.Cg[a * KT + b] : E.Cg[b * KT + a]) : 0.0;
+        if (!isfinite(v)) nonfinite = 1;
+        C[idx] = v;
+        Ev[idx] = a == b ? 1.0 : 0.0;
+    }
+    __syncthreads();
+    if (nonfinite || *E.bad) {          // no factor for a marked matrix: its W is kept
+        for (int idx = threadIdx.x; idx < KT * KT; idx += blockDim.x) E.K[idx] = 0.0;
+        if (nonfinite && threadIdx.x == 0) mark_bad(p, E);
+        return;
+    }
+    // Off-diagonal entries at the fp64 rounding level of the whole matrix are
+    // noise, not coupling: below kRotTol * trace no rotation is made, so a
+    // pair of negligible eigenvalues cannot keep the sweeps going.
+    double tr = 0.0;
+    for (int a = 0; a < k; ++a) tr += fabs(C[a * KT + a]);
+    const double floor_abs = kRotTol * 0.1 * tr;
+    for (int sweep = 0; sweep < kMaxSweeps && n > 0; ++sweep) {
+        if (threadIdx.x == 0) rotated = 0;
         __syncthreads();
-        off = 0.0; tot = 0.0;
-        for (int w = 0; w < kThreads / 32; ++w) { off += red[w]; tot += red[8 + w]; }
-        __syncthreads();
-        if (!(off > 1e-30 * tot)) break;          // also leaves on tot == 0
         for (int rd = 0; rd < n; ++rd) {
             if (threadIdx.x < ke / 2) {
                 const int i = threadIdx.x;
                 int a = i == 0 ? n : (rd + i) % n, b = i == 0 ? rd : (rd - i + n) % n;
                 if (a > b) { const int t = a; a = b; b = t; }
-                const double apq = C[a * KT + b];
+                const double apq = C[a * KT + b], app = C[a * KT + a], aqq = C[b * KT + b];
                 double c = 1.0, s = 0.0;
-                if (apq != 0.0) {
-                    const double tau = (C[b * KT + b] - C[a * KT + a]) / (2.0 * apq);
+                if (fabs(apq) > kRotTol * sqrt(fabs(app * aqq)) && fabs(apq) > floor_abs) {
+                    const double tau = (aqq - app) / (2.0 * apq);
                     const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
                     c = 1.0 / sqrt(1.0 + t * t);
                     s = t * c;
+                    rotated = 1;
                 }
                 pp[i] = a; pq[i] = b; cs[i] = c; sn[i] = s;
             }
             __syncthreads();
-            for (int idx = threadIdx.x; idx < (ke / 2) * ke; idx += kThreads) {   // rows p, q <- J^T C
+            for (int idx = threadIdx.x; idx < (ke / 2) * ke; idx += blockDim.x) {   // rows p, q <- J^T C
                 const int i = idx / ke, col = idx % ke;
                 const double c = cs[i], s = sn[i];
+                if (s == 0.0) continue;
                 const double x = C[pp[i] * KT + col], y = C[pq[i] * KT + col];
                 C[pp[i] * KT + col] = c * x - s * y;
                 C[pq[i] * KT + col] = s * x + c * y;
             }
             __syncthreads();
-            for (int idx = threadIdx.x; idx < (ke / 2) * ke; idx += kThreads) {   // columns p, q <- C J, E J
+            for (int idx = threadIdx.x; idx < (ke / 2) * ke; idx += blockDim.x) {   // columns p, q <- C J, E J
                 const int i = idx / ke, row = idx % ke;
                 const double c = cs[i], s = sn[i];
+                if (s == 0.0) continue;
                 const double x = C[row * KT + pp[i]], y = C[row * KT + pq[i]];
                 C[row * KT + pp[i]] = c * x - s * y;
                 C[row * KT + pq[i]] = s * x + c * y;
@@ -421,6 +532,9 @@ __global__ void __launch_bounds__(kThreads) lim_factor(const __grid_constant__ L
             }
             __syncthreads();
         }
+        const bool again = rotated != 0;       // read by every thread before the next reset
+        __syncthreads();
+        if (!again) break;                     // a sweep without a rotation: converged
     }
     // the r largest eigenvalues above kTau2 * largest: weights 1 / sqrt(lambda)
     if (threadIdx.x < k) lam[threadIdx.x] = C[threadIdx.x * KT + threadIdx.x];
@@ -429,40 +543,25 @@ __global__ void __launch_bounds__(kThreads) lim_factor(const __grid_constant__ L
     for (int a = 0; a < k; ++a) lmax = fmax(lmax, lam[a]);
     double* wgt = cs;                   // reuse: [KT] weights (cs and sn are contiguous)
     __syncthreads();
-    if (threadIdx.x < k) {
-        const int a = threadIdx.x;
+    for (int a = threadIdx.x; a < k; a += blockDim.x) {
         int rank = 0;
         for (int b = 0; b < k; ++b) rank += (lam[b] > lam[a]) || (lam[b] == lam[a] && b < a);
         const bool sel = lmax > 0.0 && rank < p.r && lam[a] > kTau2 * lmax;
         wgt[a] = sel ? 1.0 / sqrt(lam[a]) : 0.0;
     }
     __syncthreads();
-    // P = E diag(w) E^T into C
-    for (int idx = threadIdx.x; idx < KT * KT; idx += kThreads) {
+    // P = E diag(w) E^T
+    for (int idx = threadIdx.x; idx < KT * KT; idx += blockDim.x) {
         const int a = idx / KT, b = idx % KT;
         double s = 0.0;
         if (a < k && b < k)
             for (int e = 0; e < k; ++e) s += Ev[a * KT + e] * wgt[e] * Ev[b * KT + e];
-        C[idx] = s;
-    }
-    __syncthreads();
-    // Z = Q P, row by row in place
-    for (int i = threadIdx.x; i < E.rows; i += kThreads) {
-        float q[KT];
-        float* row = E.Y + (long long)i * KT;
-#pragma unroll
-        for (int t = 0; t < KT; ++t) q[t] = t < k ? row[t] : 0.f;
-        for (int j = 0; j < KT; ++j) {
-            double s = 0.0;
-#pragma unroll
-            for (int a = 0; a < KT; ++a) s = fma((double)q[a], C[a * KT + j], s);
-            row[j] = (float)s;
-        }
+        E.K[idx] = s;
     }
 }
 
 // ---------------------------------------------------------------------------
-// 5. O = Z B and the weight update
+// 7. O = Z B and the weight update
 // ---------------------------------------------------------------------------
 template <int W_DT>
 __device__ __forceinline__ void load4_w(const void* base, long long idx, bool vec, int nvalid, float* v) {
@@ -499,40 +598,52 @@ __device__ __forceinline__ void store4_w(void* base, long long idx, bool vec, in
         if (c < nvalid) st_elem(base, idx + c, W_DT, v[c]);
 }
 
+template <int KT>
+__host__ __device__ constexpr int update_smem_floats() { return kUpRows * KT + KT * kBsLd; }
+
 template <int KT, int W_DT>
-__global__ void __launch_bounds__(kThreads) lim_update(const __grid_constant__ LimParams p) {
-    extern __shared__ __align__(16) float smem[];
-    float* Zs = smem;                          // [kUpdRows][KT]
-    float* Bs = smem + kUpdRows * KT;          // [KT][kMsLd]: B = (B^T)^T, this tile's columns
-    const LimEntry& E = p.e[find_entry(p, blockIdx.x, 2)];
+__global__ void __launch_bounds__(kThreads, 2) lim_update(const __grid_constant__ LimParams p) {
+    extern __shared__ __align__(16) float fsm[];
+    float* Zs = fsm;                           // [kUpRows][KT]
+    float* Bs = fsm + kUpRows * KT;            // [KT][kBsLd]: B = (B^T)^T, this tile's columns
+    const LimEntry& E = p.e[find_entry(p, blockIdx.x, 3)];
     const int tile = blockIdx.x - E.t_upd;
-    const int tiles_c = (E.cols + kChunk - 1) / kChunk;
-    const int row0 = (tile / tiles_c) * kUpdRows, c0 = (tile % tiles_c) * kChunk;
+    const int tiles_c = (E.cols + kUpCols - 1) / kUpCols;
+    const int row0 = (tile / tiles_c) * kUpRows, c0 = (tile % tiles_c) * kUpCols;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int idx = threadIdx.x; idx < kUpdRows * KT; idx += kThreads) {
-        const int rr = idx / KT;
-        Zs[idx] = row0 + rr < E.rows ? E.Y[(long long)(row0 + rr) * KT + idx % KT] : 0.f;
+    constexpr int ZP = KT / 4;
+    for (int q = threadIdx.x; q < kUpRows * ZP; q += kThreads) {
+        const int rr = q / ZP, pc = q % ZP, i = row0 + rr;
+        const bool in = i < E.rows;
+        cp_async16(Zs + rr * KT + pc * 4, E.Y + (in ? (long long)i * KT + pc * 4 : 0), in ? 16u : 0u);
     }
-    for (int idx = threadIdx.x; idx < kChunk * KT; idx += kThreads) {
-        const int jj = idx / KT, t = idx % KT;
-        Bs[t * kMsLd + jj] = c0 + jj < E.cols ? E.Bt[(long long)(c0 + jj) * KT + t] : 0.f;
+    cp_async_commit();
+    for (int q = threadIdx.x; q < kUpCols * ZP; q += kThreads) {
+        const int jj = q % kUpCols, t4 = q / kUpCols, j = c0 + jj;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j < E.cols) v = *reinterpret_cast<const float4*>(E.Bt + (long long)j * KT + 4 * t4);
+        Bs[(4 * t4 + 0) * kBsLd + jj] = v.x;
+        Bs[(4 * t4 + 1) * kBsLd + jj] = v.y;
+        Bs[(4 * t4 + 2) * kBsLd + jj] = v.z;
+        Bs[(4 * t4 + 3) * kBsLd + jj] = v.w;
     }
+    cp_async_wait<0>();
     __syncthreads();
-    float o[4][4];
+    float o[16][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < 16; ++r)
 #pragma unroll
         for (int c = 0; c < 4; ++c) o[r][c] = 0.f;
-#pragma unroll 2
-    for (int t = 0; t < KT; t += 4) {
-        float4 z[4], b[4];
+    const int kk = (p.k + 3) & ~3;             // columns of Z past k are zero
+#pragma unroll 1
+    for (int t = 0; t < kk; t += 4) {
+        float4 b[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) z[r] = *reinterpret_cast<const float4*>(Zs + (4 * warp + r) * KT + t);
+        for (int q = 0; q < 4; ++q) b[q] = *reinterpret_cast<const float4*>(Bs + (t + q) * kBsLd + 4 * lane);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) b[q] = *reinterpret_cast<const float4*>(Bs + (t + q) * kMsLd + 4 * lane);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const float zz[4] = {z[r].x, z[r].y, z[r].z, z[r].w};
+        for (int r = 0; r < 16; ++r) {
+            const float4 z = *reinterpret_cast<const float4*>(Zs + (16 * warp + r) * KT + t);
+            const float zz[4] = {z.x, z.y, z.z, z.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 o[r][0] = fmaf(zz[q], b[q].x, o[r][0]);
@@ -548,8 +659,8 @@ __global__ void __launch_bounds__(kThreads) lim_update(const __grid_constant__ L
     const int nvalid = min(4, E.cols - j);
     const bool vec = E.vec_ok && nvalid == 4;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int i = row0 + 4 * warp + r;
+    for (int r = 0; r < 16; ++r) {
+        const int i = row0 + 16 * warp + r;
         if (i >= E.rows) break;
         const long long idx = (long long)i * E.cols + j;
         if (E.O_out) {
@@ -571,24 +682,32 @@ __global__ void __launch_bounds__(kThreads) lim_update(const __grid_constant__ L
 // ---------------------------------------------------------------------------
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-constexpr size_t sketch_smem(int KT) { return sizeof(float) * (kSketchRows * kMsLd + kChunk * KT); }
-constexpr size_t project_smem(int KT) { return sizeof(float) * (kProjRows * kMsLd + kProjRows * KT); }
-constexpr size_t update_smem(int KT) { return sizeof(float) * (kUpdRows * KT + KT * kMsLd); }
-constexpr size_t qr_smem(int KT) {
-    return sizeof(double) * (2 * KT * KT + KT) + sizeof(int) * KT + sizeof(float) * kGramRows * KT;
-}
-constexpr size_t factor_smem(int KT) {
-    return sizeof(double) * (2 * KT * KT + KT / 2 * 2 + KT + 16) + sizeof(int) * KT + sizeof(float) * kGramRows * KT;
-}
+template <int KT, int G_DT>
+constexpr size_t sketch_smem() { return 2 * (size_t)sketch_stage_bytes<G_DT>(); }
+template <int KT>
+constexpr size_t project_smem() { return sizeof(float) * kPjStages * project_stage_floats<KT>(); }
+template <int KT>
+constexpr size_t update_smem() { return sizeof(float) * update_smem_floats<KT>(); }
+template <int KT>
+constexpr size_t chol_smem() { return sizeof(double) * (2 * KT * KT + KT) + sizeof(int) * KT; }
+template <int KT>
+constexpr size_t eig_smem() { return sizeof(double) * (2 * KT * KT + KT / 2 * 2 + KT) + sizeof(int) * KT; }
+
+static_assert(sketch_smem<64, DT_FP32>() >= sizeof(float) * kSkRows * 64, "sketch Y staging fits a stage");
+static_assert(project_smem<64>() >= sizeof(float) * kPjCols * 64, "projection B^T staging fits the stages");
 
 template <typename K>
 cudaError_t allow_smem(K kernel, size_t bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+struct LaunchShape {
+    int sketch, rows, proj, upd;       // blocks of the grid-wide launches
+    double elems, rows_k, cols_k, rows_total;
+};
+
 template <int KT, int W_DT>
-muon_status launch_all(LimParams& prm, cudaStream_t s, int sketch_blocks, int proj_blocks, int upd_blocks,
-                       double elems, double rows_k, double cols_k) {
+muon_status launch_all(LimParams& prm, cudaStream_t s, const LaunchShape& L) {
     // The shared-memory limit is a per-device attribute of each kernel: set it
     // once on every device this instantiation is launched on.
     static std::mutex mu;
@@ -599,32 +718,40 @@ muon_status launch_all(LimParams& prm, cudaStream_t s, int sketch_blocks, int pr
     {
         std::lock_guard<std::mutex> lock(mu);
         if (!configured[dev]) {
-            cudaError_t e[5] = {allow_smem(lim_sketch<KT, W_DT>, sketch_smem(KT)), allow_smem(lim_qr<KT>, qr_smem(KT)),
-                                allow_smem(lim_project<KT>, project_smem(KT)),
-                                allow_smem(lim_factor<KT>, factor_smem(KT)),
-                                allow_smem(lim_update<KT, W_DT>, update_smem(KT))};
+            cudaError_t e[5] = {allow_smem(lim_sketch<KT, W_DT>, sketch_smem<KT, W_DT>()),
+                                allow_smem(lim_chol<KT>, chol_smem<KT>()),
+                                allow_smem(lim_project<KT>, project_smem<KT>()),
+                                allow_smem(lim_eig<KT>, eig_smem<KT>()),
+                                allow_smem(lim_update<KT, W_DT>, update_smem<KT>())};
             for (cudaError_t x : e)
                 if (x != cudaSuccess) return MUON_ERR_CUDA;
             configured[dev] = true;
         }
     }
-    const double wsz = dt_size(W_DT), k = prm.k;
-    // algorithmic bytes: per element G, M read + M written; the sketch Y written (rows x k)
-    trace_begin(MUON_KERNEL_RSVD, elems * (wsz + 8.0) + 4.0 * rows_k, s);
-    lim_sketch<KT, W_DT><<<sketch_blocks, kThreads, sketch_smem(KT), s>>>(prm);
+    const double wsz = dt_size(W_DT), k = prm.k, kk = (double)KT * KT * 8.0 * prm.n;
+    // algorithmic bytes (MUON_KERNEL_RSVD: the passes over the matrices; _SMALL: the k x k work)
+    trace_begin(MUON_KERNEL_RSVD, L.elems * (wsz + 8.0) + 4.0 * L.rows_k, s);       // G, M read; M, Y written
+    lim_sketch<KT, W_DT><<<L.sketch, kThreads, sketch_smem<KT, W_DT>(), s>>>(prm);
     trace_end(s);
-    trace_begin(MUON_KERNEL_RSVD_SMALL, 2.0 * rows_k * k, s);     // Y read, Q written
-    lim_qr<KT><<<prm.n, kThreads, qr_smem(KT), s>>>(prm);
+    trace_begin(MUON_KERNEL_RSVD_SMALL, 2.0 * kk, s);                                // Gram read, R^-1 written
+    lim_chol<KT><<<prm.n, kSmallThreads, chol_smem<KT>(), s>>>(prm);
     trace_end(s);
-    trace_begin(MUON_KERNEL_RSVD, elems * 4.0 + 4.0 * (rows_k + cols_k), s);   // M, Q read; B^T written
-    lim_project<KT><<<proj_blocks, kThreads, project_smem(KT), s>>>(prm);
+    trace_begin(MUON_KERNEL_RSVD_SMALL, 8.0 * L.rows_total * KT + kk, s);           // Y read and written
+    lim_rowmul<KT><<<L.rows, kThreads, 0, s>>>(prm);
     trace_end(s);
-    trace_begin(MUON_KERNEL_RSVD_SMALL, 4.0 * (cols_k + 2.0 * rows_k), s);     // B^T, Q read; Z written
-    lim_factor<KT><<<prm.n, kThreads, factor_smem(KT), s>>>(prm);
+    trace_begin(MUON_KERNEL_RSVD, L.elems * 4.0 + 4.0 * (L.rows_k + L.cols_k), s);  // M, Q read; B^T written
+    lim_project<KT><<<L.proj, kThreads, project_smem<KT>(), s>>>(prm);
     trace_end(s);
-    trace_begin(MUON_KERNEL_RSVD, elems * 2.0 * wsz + 4.0 * (rows_k + cols_k), s);   // W read and written
-    lim_update<KT, W_DT><<<upd_blocks, kThreads, update_smem(KT), s>>>(prm);
+    trace_begin(MUON_KERNEL_RSVD_SMALL, 2.0 * kk, s);                                // Gram read, P written
+    lim_eig<KT><<<prm.n, kSmallThreads, eig_smem<KT>(), s>>>(prm);
     trace_end(s);
+    trace_begin(MUON_KERNEL_RSVD_SMALL, 8.0 * L.rows_total * KT + kk, s);           // Q read, Z written
+    lim_rowmul<KT><<<L.rows, kThreads, 0, s>>>(prm);
+    trace_end(s);
+    trace_begin(MUON_KERNEL_RSVD, L.elems * 2.0 * wsz + 4.0 * (L.rows_k + L.cols_k), s);   // W read and written
+    lim_update<KT, W_DT><<<L.upd, kThreads, update_smem<KT>(), s>>>(prm);
+    trace_end(s);
+    (void)k;
     return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
@@ -653,6 +780,26 @@ muon_status check_shapes(const muon_rsvd_param* params, int n) {
     return MUON_OK;
 }
 
+// Workspace: the per-matrix flags, then the k x k sums that start at zero
+// (Y^T Y, B B^T), then the k x k factors, then per matrix Y and B^T.
+struct WsLayout {
+    size_t flags, zero_bytes, gy, cg, kf, mats, total;
+};
+
+WsLayout ws_layout(const muon_rsvd_param* params, int n, int KT) {
+    WsLayout L;
+    const size_t kk = sizeof(double) * (size_t)KT * KT * n;
+    L.flags = 0;
+    L.gy = align256(sizeof(int) * (size_t)n);
+    L.cg = L.gy + align256(kk);
+    L.zero_bytes = L.cg + align256(kk);
+    L.kf = L.zero_bytes;
+    L.mats = L.kf + align256(kk);
+    L.total = L.mats;
+    for (int i = 0; i < n; ++i) L.total += matrix_ws(params[i].rows, params[i].cols, KT);
+    return L;
+}
+
 }  // namespace
 }  // namespace muon
 
@@ -666,10 +813,7 @@ muon_status limuon_workspace_size(const muon_rsvd_param* params, int n, const mu
     if (st != MUON_OK) return st;
     if ((st = check_hp(hp)) != MUON_OK) return st;
     if (!bytes) return MUON_ERR_INVALID_ARG;
-    const int KT = kt_for(hp->rank + hp->oversample);
-    size_t total = align256(sizeof(int) * (size_t)n);
-    for (int i = 0; i < n; ++i) total += matrix_ws(params[i].rows, params[i].cols, KT);
-    *bytes = total;
+    *bytes = ws_layout(params, n, kt_for(hp->rank + hp->oversample)).total;
     return MUON_OK;
 }
 
@@ -688,10 +832,15 @@ muon_status limuon_step_batched(const muon_rsvd_param* params, int n, muon_dtype
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return MUON_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int k = hp->rank + hp->oversample, KT = kt_for(k);
+    const WsLayout W = ws_layout(params, n, KT);
     char* ws = static_cast<char*>(workspace);
-    int* bad = reinterpret_cast<int*>(ws);
-    if (cudaMemsetAsync(bad, 0, sizeof(int) * (size_t)n, s) != cudaSuccess) return MUON_ERR_CUDA;
-    char* cur = ws + align256(sizeof(int) * (size_t)n);
+    // flags and the two Gram sums start at zero
+    if (cudaMemsetAsync(ws, 0, W.zero_bytes, s) != cudaSuccess) return MUON_ERR_CUDA;
+    int* bad = reinterpret_cast<int*>(ws + W.flags);
+    double* gy = reinterpret_cast<double*>(ws + W.gy);
+    double* cg = reinterpret_cast<double*>(ws + W.cg);
+    double* kf = reinterpret_cast<double*>(ws + W.kf);
+    char* cur = ws + W.mats;
     static LimParams prm;              // large: kept off the stack, filled and consumed per launch
     static std::mutex mu;
     std::lock_guard<std::mutex> lock(mu);
@@ -701,8 +850,8 @@ muon_status limuon_step_batched(const muon_rsvd_param* params, int n, muon_dtype
         prm.k = k; prm.r = hp->rank;
         prm.mu = hp->mu; prm.eta = hp->eta; prm.lambda = hp->lambda;
         prm.d_status = d_status;
-        long long ts = 0, tp = 0, tu = 0;
-        double elems = 0.0, rows_k = 0.0, cols_k = 0.0;
+        long long ts = 0, tr = 0, tp = 0, tu = 0;
+        LaunchShape L = {};
         for (int i = 0; i < prm.n; ++i) {
             const muon_rsvd_param& q = params[b + i];
             LimEntry& E = prm.e[i];
@@ -710,30 +859,34 @@ muon_status limuon_step_batched(const muon_rsvd_param* params, int n, muon_dtype
             E.rows = q.rows; E.cols = q.cols;
             E.gamma = std::isnan(q.gamma) ? hp->gamma : q.gamma;
             E.bad = bad + b + i;
+            const size_t kk = (size_t)KT * KT * (b + i);
+            E.Gy = gy + kk; E.Cg = cg + kk; E.K = kf + kk;
             E.Y = reinterpret_cast<float*>(cur);
             E.Bt = reinterpret_cast<float*>(cur + align256(sizeof(float) * (size_t)q.rows * KT));
             cur += matrix_ws(q.rows, q.cols, KT);
             const uintptr_t al = reinterpret_cast<uintptr_t>(q.W) | reinterpret_cast<uintptr_t>(q.G) |
                                  reinterpret_cast<uintptr_t>(q.M) | reinterpret_cast<uintptr_t>(q.O_out);
             E.vec_ok = (al & 15) == 0 && q.cols % 8 == 0;
-            E.t_sketch = (int)ts; E.t_proj = (int)tp; E.t_upd = (int)tu;
-            ts += (q.rows + kSketchRows - 1) / kSketchRows;
-            tp += (q.cols + kChunk - 1) / kChunk;
-            tu += (long long)((q.rows + kUpdRows - 1) / kUpdRows) * ((q.cols + kChunk - 1) / kChunk);
-            elems += (double)q.rows * q.cols;
-            rows_k += (double)q.rows * k;
-            cols_k += (double)q.cols * k;
+            E.t_sketch = (int)ts; E.t_rows = (int)tr; E.t_proj = (int)tp; E.t_upd = (int)tu;
+            ts += (q.rows + kSkRows - 1) / kSkRows;
+            tr += (q.rows + kThreads - 1) / kThreads;
+            tp += (q.cols + kPjCols - 1) / kPjCols;
+            tu += (long long)((q.rows + kUpRows - 1) / kUpRows) * ((q.cols + kUpCols - 1) / kUpCols);
+            L.elems += (double)q.rows * q.cols;
+            L.rows_k += (double)q.rows * k;
+            L.cols_k += (double)q.cols * k;
+            L.rows_total += q.rows;
         }
-        if (ts > INT32_MAX || tp > INT32_MAX || tu > INT32_MAX) return MUON_ERR_UNSUPPORTED;
-        const int a = (int)ts, pj = (int)tp, u = (int)tu;
+        if (ts > INT32_MAX || tr > INT32_MAX || tp > INT32_MAX || tu > INT32_MAX) return MUON_ERR_UNSUPPORTED;
+        L.sketch = (int)ts; L.rows = (int)tr; L.proj = (int)tp; L.upd = (int)tu;
         if (KT == 32) {
-            if (w_dtype == MUON_BF16) st = launch_all<32, DT_BF16>(prm, s, a, pj, u, elems, rows_k, cols_k);
-            else if (w_dtype == MUON_FP16) st = launch_all<32, DT_FP16>(prm, s, a, pj, u, elems, rows_k, cols_k);
-            else st = launch_all<32, DT_FP32>(prm, s, a, pj, u, elems, rows_k, cols_k);
+            if (w_dtype == MUON_BF16) st = launch_all<32, DT_BF16>(prm, s, L);
+            else if (w_dtype == MUON_FP16) st = launch_all<32, DT_FP16>(prm, s, L);
+            else st = launch_all<32, DT_FP32>(prm, s, L);
         } else {
-            if (w_dtype == MUON_BF16) st = launch_all<64, DT_BF16>(prm, s, a, pj, u, elems, rows_k, cols_k);
-            else if (w_dtype == MUON_FP16) st = launch_all<64, DT_FP16>(prm, s, a, pj, u, elems, rows_k, cols_k);
-            else st = launch_all<64, DT_FP32>(prm, s, a, pj, u, elems, rows_k, cols_k);
+            if (w_dtype == MUON_BF16) st = launch_all<64, DT_BF16>(prm, s, L);
+            else if (w_dtype == MUON_FP16) st = launch_all<64, DT_FP16>(prm, s, L);
+            else st = launch_all<64, DT_FP32>(prm, s, L);
         }
         if (st != MUON_OK) return st;
     }

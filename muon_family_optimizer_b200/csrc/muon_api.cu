@@ -505,8 +505,10 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
     // 1. fused MONA pre-pass + norms + wide-view copies: one launch per
     //    element type of the copies (the iteration's, and fp32 for narrow groups)
     const size_t in_sz = dt_size(w_dtype);
-    for (int x0_dt : {(int)ns_dtype, (int)DT_FP32}) {
-        if (x0_dt == DT_FP32 && (int)ns_dtype == DT_FP32) break;
+    const int n_x0 = (int)ns_dtype == DT_FP32 ? 1 : 2;
+    const int x0_types[2] = {(int)ns_dtype, DT_FP32};
+    for (int t = 0; t < n_x0; ++t) {
+        const int x0_dt = x0_types[t];
         PrepParams pp;
         memset(&pp, 0, sizeof(pp));
         pp.in_dt = w_dtype; pp.x0_dt = x0_dt; pp.mode = lite ? 2 : 0;

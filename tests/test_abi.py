@@ -235,11 +235,12 @@ def test_limuon_argument_checks(lib):
     one = (mo.RsvdParam * 1)(mo.RsvdParam(4, 8, p, p, p, p, float("nan"), None))
     size = ctypes.c_size_t(0)
     assert L.limuon_workspace_size(one, 1, ctypes.byref(good), ctypes.byref(size)) == mo.OK
-    # 4 per-matrix flags, then Y (4 x 32 floats) and B^T (8 x 32 floats), each 256-byte aligned
-    assert size.value == 256 + 512 + 1024
+    # the per-matrix flag, three k x k fp64 matrices (Y^T Y, B B^T, the factor) on 32 columns,
+    # then Y (4 x 32 floats) and B^T (8 x 32 floats), each region 256-byte aligned
+    assert size.value == 256 + 3 * 32 * 32 * 8 + 512 + 1024
     big = mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 40, 8)
     assert L.limuon_workspace_size(one, 1, ctypes.byref(big), ctypes.byref(size)) == mo.OK
-    assert size.value == 256 + 1024 + 2048                 # k = 48 runs on 64 columns
+    assert size.value == 256 + 3 * 64 * 64 * 8 + 1024 + 2048   # k = 48 runs on 64 columns
     too_big = mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 60, 5)
     assert L.limuon_workspace_size(one, 1, ctypes.byref(too_big), ctypes.byref(size)) == mo.ERR_UNSUPPORTED
     for bad in (mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 0, 4), mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 4, -1),
@@ -250,7 +251,8 @@ def test_limuon_argument_checks(lib):
     assert L.limuon_step_batched(one, 1, 7, ctypes.byref(good), ws, 2048, None, None) == mo.ERR_INVALID_ARG
     assert L.limuon_step_batched(one, 1, mo.BF16, ctypes.byref(good), ws, 1000, None, None) == mo.ERR_WORKSPACE
     assert L.limuon_step_batched(one, 1, mo.BF16, ctypes.byref(good), None, 4096, None, None) == mo.ERR_WORKSPACE
-    assert L.limuon_step_batched(one, 1, mo.BF16, ctypes.byref(good), ws + 16, 2048, None, None) == mo.ERR_INVALID_ARG
+    assert L.limuon_step_batched(one, 1, mo.BF16, ctypes.byref(good), ws + 16, 1 << 20, None, None) == \
+        mo.ERR_INVALID_ARG
     nul = (mo.RsvdParam * 1)(mo.RsvdParam(4, 8, p, p, p, None, float("nan"), None))
     assert L.limuon_step_batched(nul, 1, mo.BF16, ctypes.byref(good), ws, 2048, None, None) == mo.ERR_INVALID_ARG
     empty = (mo.RsvdParam * 1)(mo.RsvdParam(0, 8, p, p, p, p, float("nan"), None))

@@ -57,13 +57,18 @@ def test_recorded_traffic_requires_matching_sources(tmp_path, monkeypatch):
 
 
 def test_limuon_kernel_work_counts():
-    # one 4 x 6 matrix, k = 3, 16-bit W/G: per element the sketch moves 2 + 4 + 4 bytes, the
-    # projection 4, the update 2 + 2; each of the three products is 3 FMAs per element
+    # one 4 x 6 matrix, k = 3 (32-column factors), 16-bit W/G: per element the sketch moves
+    # 2 + 4 + 4 bytes, the projection 4, the update 2 + 2; each of these three products is
+    # 3 FMAs per element; the row transforms move 4 rows of 32 floats each way and do
+    # 2 k^2 flops per row; the two k x k steps move two 32 x 32 fp64 matrices
     by, fl = bench.limuon_kernel_work([(4, 6)], 3)
-    assert by == [24 * 10 + 4 * 12, 8 * 12, 24 * 4 + 4 * (12 + 18), 4 * (18 + 24), 24 * 4 + 4 * (12 + 18)]
-    assert fl == [2.0 * 24 * 3, 0.0, 2.0 * 24 * 3, 0.0, 2.0 * 24 * 3]
+    small = 2 * 8 * 32 * 32
+    assert by == [24 * 10 + 4 * 12, small, 8 * 4 * 32 + small // 2, 24 * 4 + 4 * (12 + 18), small,
+                  8 * 4 * 32 + small // 2, 24 * 4 + 4 * (12 + 18)]
+    assert fl == [2.0 * 24 * 3, 0.0, 2.0 * 4 * 9, 2.0 * 24 * 3, 0.0, 2.0 * 4 * 9, 2.0 * 24 * 3]
     by32, _ = bench.limuon_kernel_work([(4, 6)], 3, w_bytes=4)
-    assert by32[0] - by[0] == 24 * 2 and by32[4] - by[4] == 24 * 4
+    assert by32[0] - by[0] == 24 * 2 and by32[6] - by[6] == 24 * 4
+    assert len(bench.LIMUON_KERNELS) == len(by)
 
 
 def test_fp32_alu_peak_from_unit_counts():

@@ -163,6 +163,26 @@ def test_limuon_nonfinite_keeps_weights():
     assert not torch.equal(params[0]["W"], W0)
 
 
+def test_limuon_overflow_in_the_sketch_keeps_weights():
+    # a finite momentum whose sketch Y = M Omega overflows fp32 (entries of
+    # 2.85e38 times Gaussian weights, summed over 200 columns): the k x k Gram
+    # of Y is not finite, the matrix is marked, its W kept and the flag raised;
+    # the other matrix steps
+    hp = _hp(8, 8)
+    params = _params([(64, 96), (48, 200)], torch.float32, 16, 8)
+    for p in params:
+        rows, cols = p["W"].shape
+        p["G"] = _planted(rows, cols, 8, p["seed"]).to(torch.float32).cuda()
+    params[1]["G"].zero_()
+    params[1]["M"].fill_(3e38)          # mu M + 0 stays finite; the sums over 200 columns do not
+    W0, W1 = params[0]["W"].clone(), params[1]["W"].clone()
+    st = _run(params, torch.float32, hp)
+    assert st & mo.FLAG_NONFINITE
+    assert torch.isfinite(params[1]["M"]).all()
+    assert torch.equal(params[1]["W"], W1)
+    assert not torch.equal(params[0]["W"], W0)
+
+
 def test_limuon_many_parameters_two_launches():
     shapes = [(24 + (i % 5) * 8, 40 + (i % 7) * 4) for i in range(130)]
     hp = _hp(4, 4)
