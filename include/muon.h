@@ -240,6 +240,24 @@ MUON_API muon_status adamw_step_batched(const muon_vec_param* params, int n, muo
                                muon_stream_t stream);
 
 /*
+ * One optimizer step for a whole model: the n matrix parameters exactly as
+ * muon_step_batched, and the nvec vector-valued parameters (embeddings,
+ * biases, norm weights: [MONA] section 2, "Ontwerprichtlijnen") with AdamW
+ * exactly as adamw_step_batched -- their elements are further work items of
+ * the step's fused pre-pass launch, so the model needs no separate AdamW pass.
+ * vecs: host array of nvec descriptors (NULL when nvec == 0); every W and G
+ * of them in w_dtype, m and v fp32.  adamw, step: as adamw_step_batched
+ * (ignored when nvec == 0).  workspace: muon_workspace_size of the matrix
+ * parameters under `sched` (the vectors need none).  Errors, ownership and
+ * asynchrony as muon_step_batched and adamw_step_batched; a vector element
+ * with a non-finite gradient keeps its state and sets MUON_FLAG_NONFINITE.
+ */
+MUON_API muon_status muon_model_step(const muon_param* params, int n, const muon_vec_param* vecs, int nvec,
+                                     muon_dtype w_dtype, muon_dtype ns_dtype, const muon_hparams* hp,
+                                     const muon_adamw_hparams* adamw, int step, const muon_schedule* sched,
+                                     void* workspace, size_t ws_bytes, int* d_status, muon_stream_t stream);
+
+/*
  * LiMuon ([LiMuon] section "Метод": Muon's momentum, with the update taken
  * from a randomized SVD of the momentum).  The page gives no formulas; read
  * as the basic randomized SVD of Halko, Martinsson and Tropp ("Finding

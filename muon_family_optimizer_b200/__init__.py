@@ -8,7 +8,8 @@ or cannot be loaded, every call raises.
 Names follow the C ABI: :func:`muon_step_batched`, :func:`ns_polar`,
 :func:`gram_polar`, :func:`muon_workspace_size`, :func:`ns_polar_workspace_size`,
 :func:`gram_polar_workspace_size`, :func:`muon_lite_step_batched` (MONA-Lite),
-:func:`adamw_step_batched` (vector parameters), :func:`limuon_step_batched` and
+:func:`adamw_step_batched` (vector parameters), :func:`muon_model_step` (matrices and
+vector parameters in one step), :func:`limuon_step_batched` and
 :func:`limuon_workspace_size` (LiMuon), :func:`ns_polar_noalloc`,
 :func:`muon_status_string`.
 """
@@ -131,6 +132,11 @@ def lib():
                                           ctypes.POINTER(RsvdHParams), vp, ctypes.c_size_t, vp, vp]
         L.muon_wait_selftest.restype = st
         L.muon_wait_selftest.argtypes = [ctypes.c_int, vp, vp]
+        L.muon_model_step.restype = st
+        L.muon_model_step.argtypes = [ctypes.POINTER(Param), ctypes.c_int, ctypes.POINTER(VecParam), ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, ctypes.POINTER(HParams),
+                                      ctypes.POINTER(AdamWHParams), ctypes.c_int, ctypes.POINTER(Schedule), vp,
+                                      ctypes.c_size_t, vp, vp]
         L.adamw_step_batched.restype = st
         L.adamw_step_batched.argtypes = [ctypes.POINTER(VecParam), ctypes.c_int, ctypes.c_int,
                                          ctypes.POINTER(AdamWHParams), ctypes.c_int, vp, vp]
@@ -249,6 +255,26 @@ def muon_step_batched(params, w_dtype, ns_dtype, hp, schedule, workspace, d_stat
     _check(lib().muon_step_batched(arr, len(arr), int(w_dtype), int(ns_dtype), ctypes.byref(h),
                                    ctypes.byref(schedule), _ptr(workspace), workspace.numel(),
                                    _ptr(d_status), _stream_ptr(stream)), "muon_step_batched")
+
+
+def muon_model_step(params, vecs, w_dtype, ns_dtype, hp, adamw_hp, step, schedule, workspace, d_status=None,
+                    stream=None):
+    """One step of a whole model (see include/muon.h): the matrices as
+    muon_step_batched, the vector-valued parameters with AdamW as items of the
+    same pre-pass launch.  vecs: list of dicts (see make_vec_params), a ctypes
+    VecParam array, or None; adamw_hp: dict with lr, beta1, beta2, eps,
+    weight_decay; step: t >= 1."""
+    arr = params if isinstance(params, ctypes.Array) else make_params(params)
+    varr = None
+    if vecs is not None and len(vecs):
+        varr = vecs if isinstance(vecs, ctypes.Array) else make_vec_params(vecs)
+    h = HParams(hp["mu"], hp["eta"], hp["lambda"], hp["gamma"], hp["beta_a"], hp["alpha"])
+    a = AdamWHParams(adamw_hp["lr"], adamw_hp["beta1"], adamw_hp["beta2"], adamw_hp["eps"],
+                     adamw_hp["weight_decay"]) if adamw_hp else None
+    _check(lib().muon_model_step(arr, len(arr), varr, len(varr) if varr is not None else 0, int(w_dtype),
+                                 int(ns_dtype), ctypes.byref(h), ctypes.byref(a) if a else None, int(step),
+                                 ctypes.byref(schedule), _ptr(workspace), workspace.numel(), _ptr(d_status),
+                                 _stream_ptr(stream)), "muon_model_step")
 
 
 def make_lite_params(params):

@@ -17,6 +17,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "adamw_elem.cuh"
 #include "gemm.h"
 
 namespace muon {
@@ -39,8 +40,7 @@ struct AdamWParams {
     VecEntry e[kMaxVec];
     int n;
     long long total_runs;
-    float lr, b1, b2, eps, wd;
-    float ic1, ic2;   // 1 / (1 - b1^t), 1 / (1 - b2^t)
+    AdamWCoeffs c;
     int* d_status;
 };
 
@@ -63,19 +63,7 @@ __global__ void __launch_bounds__(256, 4) adamw_kernel(const __grid_constant__ A
         load8_dt(E.G, idx, W_DT, vec, nvalid, g);
         load8_dt(E.m, idx, DT_FP32, vec, nvalid, m);
         load8_dt(E.v, idx, DT_FP32, vec, nvalid, v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (!isfinite(g[i])) {       // keep this element's state
-                bad |= i < nvalid;
-                continue;
-            }
-            const float mn = p.b1 * m[i] + (1.f - p.b1) * g[i];
-            const float vn = p.b2 * v[i] + (1.f - p.b2) * g[i] * g[i];
-            const float upd = (mn * p.ic1) / (sqrtf(vn * p.ic2) + p.eps);
-            w[i] = w[i] - p.lr * (upd + p.wd * w[i]);
-            m[i] = mn;
-            v[i] = vn;
-        }
+        bad |= adamw8(p.c, w, g, m, v, nvalid);
         store8_dt(E.W, idx, W_DT, vec, nvalid, w);
         store8_dt(E.m, idx, DT_FP32, vec, nvalid, m);
         store8_dt(E.v, idx, DT_FP32, vec, nvalid, v);
@@ -116,12 +104,10 @@ muon_status launch_adamw(AdamWParams& prm, int w_dtype, cudaStream_t stream) {
 
 using namespace muon;
 
-extern "C" {
+namespace muon {
 
-muon_status adamw_step_batched(const muon_vec_param* params, int n, muon_dtype w_dtype, const muon_adamw_hparams* hp,
-                               int step, int* d_status, muon_stream_t stream) {
+muon_status adamw_check(const muon_vec_param* params, int n, const muon_adamw_hparams* hp, int step) {
     if (!params || n < 1 || !hp || step < 1) return MUON_ERR_INVALID_ARG;
-    if (w_dtype != MUON_BF16 && w_dtype != MUON_FP16 && w_dtype != MUON_FP32) return MUON_ERR_INVALID_ARG;
     const float hv[5] = {hp->lr, hp->beta1, hp->beta2, hp->eps, hp->weight_decay};
     for (float x : hv)
         if (!std::isfinite(x)) return MUON_ERR_INVALID_ARG;
@@ -132,6 +118,26 @@ muon_status adamw_step_batched(const muon_vec_param* params, int n, muon_dtype w
         if (q.n < 1 || !q.W || !q.G || !q.m || !q.v) return MUON_ERR_INVALID_ARG;
         if (q.n > (1LL << 40)) return MUON_ERR_UNSUPPORTED;
     }
+    return MUON_OK;
+}
+
+AdamWCoeffs adamw_coeffs(const muon_adamw_hparams* hp, int step) {
+    AdamWCoeffs c;
+    c.lr = hp->lr; c.b1 = hp->beta1; c.b2 = hp->beta2; c.eps = hp->eps; c.wd = hp->weight_decay;
+    c.ic1 = (float)(1.0 / (1.0 - std::pow((double)hp->beta1, (double)step)));
+    c.ic2 = (float)(1.0 / (1.0 - std::pow((double)hp->beta2, (double)step)));
+    return c;
+}
+
+}  // namespace muon
+
+extern "C" {
+
+muon_status adamw_step_batched(const muon_vec_param* params, int n, muon_dtype w_dtype, const muon_adamw_hparams* hp,
+                               int step, int* d_status, muon_stream_t stream) {
+    if (w_dtype != MUON_BF16 && w_dtype != MUON_FP16 && w_dtype != MUON_FP32) return MUON_ERR_INVALID_ARG;
+    muon_status chk = adamw_check(params, n, hp, step);
+    if (chk != MUON_OK) return chk;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     static AdamWParams prm;            // large: kept off the stack, filled and consumed per launch
     static std::mutex mu;
@@ -139,9 +145,7 @@ muon_status adamw_step_batched(const muon_vec_param* params, int n, muon_dtype w
     for (int b = 0; b < n; b += kMaxVec) {
         memset(&prm, 0, sizeof(prm));
         prm.n = std::min(kMaxVec, n - b);
-        prm.lr = hp->lr; prm.b1 = hp->beta1; prm.b2 = hp->beta2; prm.eps = hp->eps; prm.wd = hp->weight_decay;
-        prm.ic1 = (float)(1.0 / (1.0 - std::pow((double)hp->beta1, (double)step)));
-        prm.ic2 = (float)(1.0 / (1.0 - std::pow((double)hp->beta2, (double)step)));
+        prm.c = adamw_coeffs(hp, step);
         prm.d_status = d_status;
         for (int i = 0; i < prm.n; ++i) {
             const muon_vec_param& q = params[b + i];

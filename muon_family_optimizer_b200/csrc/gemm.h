@@ -2,6 +2,7 @@
 // Newton-Schulz iteration and the two back ends that run it.
 #pragma once
 
+#include "adamw_elem.cuh"
 #include "epilogue.cuh"
 
 namespace muon {
@@ -37,16 +38,20 @@ muon_status simt_run(const GemmOp* ops, int nops, const FinalCtx& fc, const Fina
 }
 
 // Fused elementwise passes ahead of the iteration (prepass.cu).
-constexpr int kMaxPrep = 128;
+constexpr int kMaxPrep = 192;
 
 struct PrepEntry {
     const void* G; void* Gp; float* A; float* M;   // MONA mode: this parameter's state
+                                                   // (AdamW item: G the gradient, Gp the weights W,
+                                                   //  A the first moment m, M the second moment v)
     const void* X; long long x_stride;             // COPY mode: batch input
     void* X0; long long x0_stride, ld;             // wide-view destination
     int rows, cols, count, transposed, vec_ok;
     int sumsq_index;
     int tiles_c;
     int flat;          // set by prep_run: processed as one contiguous array
+    int kind;          // 0: a matrix of the launch's mode; 1: an AdamW vector item of nel elements
+    long long nel;
     long long tiles_per_mat, tile_begin;
 };
 
@@ -61,9 +66,16 @@ struct PrepParams {
     float eps;
     float beta_a, alpha, mu;
     double* sumsq;
+    // AdamW items (kind 1), after every matrix entry of the launch
+    AdamWCoeffs adam;
+    int* d_status;
 };
 
 muon_status prep_run(PrepParams& prm, cudaStream_t stream);
+
+// AdamW host helpers (adamw.cu): argument checks and the launch's coefficients.
+muon_status adamw_check(const muon_vec_param* params, int n, const muon_adamw_hparams* hp, int step);
+AdamWCoeffs adamw_coeffs(const muon_adamw_hparams* hp, int step);
 
 // Launch tracing (trace.cu): no-ops unless muon_trace_enable(1) was called.
 void trace_begin(int kind, double work, cudaStream_t stream);

@@ -477,10 +477,19 @@ muon_status muon_workspace_size(const muon_param* params, int n, muon_dtype ns_d
     return MUON_OK;
 }
 
+// Optional vector-valued parameters of a whole-model step (AdamW items of the
+// pre-pass launch).
+struct VecItems {
+    const muon_vec_param* vecs = nullptr;
+    int n = 0;
+    AdamWCoeffs c = {};
+};
+
 // lite: MONA-Lite state (G_prev holds the bfloat16 buffer B, A is unused).
 static muon_status step_common(const muon_param* params, int n, muon_dtype w_dtype, muon_dtype ns_dtype,
                                const muon_hparams* hp, const muon_schedule* sched, void* workspace,
-                               size_t ws_bytes, int* d_status, muon_stream_t stream, bool lite) {
+                               size_t ws_bytes, int* d_status, muon_stream_t stream, bool lite,
+                               const VecItems& vec = VecItems()) {
     if (!valid_dtype(w_dtype) || !valid_dtype(ns_dtype) || !hp) return MUON_ERR_INVALID_ARG;
     muon_status st = check_params(params, n);
     if (st != MUON_OK) return st;
@@ -528,6 +537,27 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
                 const uintptr_t al = reinterpret_cast<uintptr_t>(p.G) | reinterpret_cast<uintptr_t>(p.G_prev) |
                                      reinterpret_cast<uintptr_t>(p.A) | reinterpret_cast<uintptr_t>(p.M);
                 E.vec_ok = (p.cols % 8 == 0) && (al & 15) == 0 && in_sz >= 2;
+                if (pp.n == kMaxPrep) {
+                    st = prep_run(pp, stream_);
+                    if (st != MUON_OK) return st;
+                    pp.n = 0;
+                }
+            }
+        }
+        if (t == 0) {
+            // the vector-valued parameters' AdamW as further items of the same launch
+            pp.adam = vec.c;
+            pp.d_status = status;
+            for (int i = 0; i < vec.n; ++i) {
+                const muon_vec_param& q = vec.vecs[i];
+                PrepEntry& E = pp.e[pp.n++];
+                E.kind = 1;
+                E.nel = q.n;
+                E.G = q.G; E.Gp = q.W; E.A = q.m; E.M = q.v;
+                E.rows = E.cols = 1; E.ld = 1; E.count = 1;
+                const uintptr_t al = reinterpret_cast<uintptr_t>(q.W) | reinterpret_cast<uintptr_t>(q.G) |
+                                     reinterpret_cast<uintptr_t>(q.m) | reinterpret_cast<uintptr_t>(q.v);
+                E.vec_ok = (al & 15) == 0 && in_sz >= 2;
                 if (pp.n == kMaxPrep) {
                     st = prep_run(pp, stream_);
                     if (st != MUON_OK) return st;
@@ -583,6 +613,22 @@ muon_status muon_step_batched(const muon_param* params, int n, muon_dtype w_dtyp
                               const muon_hparams* hp, const muon_schedule* sched, void* workspace,
                               size_t ws_bytes, int* d_status, muon_stream_t stream) {
     return step_common(params, n, w_dtype, ns_dtype, hp, sched, workspace, ws_bytes, d_status, stream, false);
+}
+
+muon_status muon_model_step(const muon_param* params, int n, const muon_vec_param* vecs, int nvec,
+                            muon_dtype w_dtype, muon_dtype ns_dtype, const muon_hparams* hp,
+                            const muon_adamw_hparams* adamw, int step, const muon_schedule* sched,
+                            void* workspace, size_t ws_bytes, int* d_status, muon_stream_t stream) {
+    if (nvec < 0) return MUON_ERR_INVALID_ARG;
+    VecItems v;
+    if (nvec > 0) {
+        muon_status st = adamw_check(vecs, nvec, adamw, step);
+        if (st != MUON_OK) return st;
+        v.vecs = vecs;
+        v.n = nvec;
+        v.c = adamw_coeffs(adamw, step);
+    }
+    return step_common(params, n, w_dtype, ns_dtype, hp, sched, workspace, ws_bytes, d_status, stream, false, v);
 }
 
 // MONA-Lite descriptors as the common path's (B in the G_prev slot, no A).

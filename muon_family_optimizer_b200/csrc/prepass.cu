@@ -79,10 +79,30 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
     int cur = -1;
     double acc = 0.0;
     int ei = 0;
+    bool bad = false;                        // an AdamW item saw a non-finite gradient
     for (long long t = t_begin; t < t_end; ++t) {
         while (ei + 1 < p.n && t >= p.e[ei + 1].tile_begin) ++ei;
         const PrepEntry& E = p.e[ei];
         const long long local = t - E.tile_begin;
+        if (E.kind == 1) {
+            // AdamW item (uniform over the block): TR*TC consecutive elements,
+            // 8 per thread; nothing of the iteration follows
+            const long long e0 = local * (TR * TC) + (long long)threadIdx.x * 8;
+            const int nv = (int)max(0LL, min(8LL, E.nel - e0));
+            if (nv > 0) {
+                const bool vec = E.vec_ok && nv == 8;
+                float w[8], g[8], m[8], v[8];
+                load8_in<IN_DT>(E.G, e0, vec, nv, g);
+                load8_dt(E.Gp, e0, IN_DT, vec, nv, w);
+                load8_dt(E.A, e0, DT_FP32, vec, nv, m);
+                load8_dt(E.M, e0, DT_FP32, vec, nv, v);
+                bad |= adamw8(p.adam, w, g, m, v, nv);
+                store8_dt(E.Gp, e0, IN_DT, vec, nv, w);
+                store8_dt(E.A, e0, DT_FP32, vec, nv, m);
+                store8_dt(E.M, e0, DT_FP32, vec, nv, v);
+            }
+            continue;
+        }
         const int b = (int)(local / E.tiles_per_mat);
         const long long tt = local - (long long)b * E.tiles_per_mat;
         const int tr = E.flat ? 0 : (int)(tt / E.tiles_c), tc = E.flat ? 0 : (int)(tt % E.tiles_c);
@@ -218,6 +238,7 @@ __global__ void __launch_bounds__(256, 4) prep_kernel(const __grid_constant__ Pr
         double s = block_sum(acc, red);
         if (threadIdx.x == 0) atomicAdd(&p.sumsq[cur], s);
     }
+    if (__syncthreads_or(bad) && threadIdx.x == 0 && p.d_status) atomicOr(p.d_status, MUON_FLAG_NONFINITE);
 }
 
 __global__ void identity_kernel(void* D, int dt, int count, int s, long long ld, long long stride) {
@@ -245,6 +266,7 @@ muon_status prep_run(PrepParams& prm, cudaStream_t stream) {
         // streams per array instead of TR separate row segments)
         E.flat = !E.transposed && E.ld == E.cols;
         if (E.flat) E.tiles_per_mat = ((long long)E.rows * E.cols + TR * TC - 1) / (TR * TC);
+        if (E.kind == 1) E.tiles_per_mat = (E.nel + TR * TC - 1) / (TR * TC);
         E.tile_begin = tiles;
         tiles += E.tiles_per_mat * E.count;
     }
@@ -260,14 +282,18 @@ muon_status prep_run(PrepParams& prm, cudaStream_t stream) {
         occ = 1;
     const long long want = (long long)nsm * (occ > 0 ? occ : 1);
     const int grid = (int)(tiles < want ? tiles : want);
-    double elems = 0.0;
-    for (int i = 0; i < prm.n; ++i) elems += (double)prm.e[i].rows * prm.e[i].cols * prm.e[i].count;
+    double elems = 0.0, vec_elems = 0.0;
+    for (int i = 0; i < prm.n; ++i) {
+        if (prm.e[i].kind == 1) vec_elems += (double)prm.e[i].nel;
+        else elems += (double)prm.e[i].rows * prm.e[i].cols * prm.e[i].count;
+    }
     const int isz = dt_size(prm.in_dt), xsz = dt_size(prm.x0_dt);
     // MONA: read G, G_prev, A, M; write A, M, G_prev, X0.  COPY: read X, write X0.
     // MONA-Lite: read G, B, M; write B, M, X0.  NORM: read X.
+    // AdamW item: read G, W, m, v; write W, m, v.
     const double per = prm.mode == 0 ? 3.0 * isz + 16.0 + xsz
                      : prm.mode == 2 ? isz + 12.0 + xsz : prm.mode == 3 ? (double)isz : (double)(isz + xsz);
-    trace_begin(MUON_KERNEL_PREPASS, elems * per, stream);
+    trace_begin(MUON_KERNEL_PREPASS, elems * per + vec_elems * (3.0 * isz + 16.0), stream);
     // element types are compile-time in the kernel: loads and stores stay in registers
 #define MUON_PREP(I, X)                                                   \
     if (prm.in_dt == I && prm.x0_dt == X) prep_kernel<I, X><<<grid, 256, 0, stream>>>(prm);

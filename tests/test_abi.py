@@ -272,3 +272,27 @@ def test_limuon_binding_validates_tensors():
                 dict(ok, W=torch.zeros(32, dtype=torch.bfloat16)), dict(ok, M=torch.zeros(8, 4).t())):
         with pytest.raises(ValueError):
             mo.make_rsvd_params([bad])
+
+
+def test_model_step_argument_checks(lib):
+    L = lib
+    buf = ctypes.create_string_buffer(4096)
+    p = ctypes.cast(buf, ctypes.c_void_p).value
+    arr = (mo.Param * 1)()
+    arr[0].rows, arr[0].cols = 4, 4
+    arr[0].W = arr[0].G = arr[0].G_prev = arr[0].A = arr[0].M = p
+    hp = mo.HParams(0.9, 0.02, 0.0, 1.0, 0.9, 0.5)
+    sched = mo.quintic_schedule(5)
+    good = mo.AdamWHParams(1e-3, 0.9, 0.999, 1e-8, 0.1)
+    vec = (mo.VecParam * 1)(mo.VecParam(8, p, p, p, p))
+    args = lambda v, nv, a, t, ws=p, size=16: (arr, 1, v, nv, mo.BF16, mo.BF16, ctypes.byref(hp), a, t,
+                                               ctypes.byref(sched), ws, size, None, None)
+    assert L.muon_model_step(*args(vec, -1, ctypes.byref(good), 1)) == mo.ERR_INVALID_ARG
+    assert L.muon_model_step(*args(vec, 1, None, 1)) == mo.ERR_INVALID_ARG                 # no AdamW hparams
+    assert L.muon_model_step(*args(vec, 1, ctypes.byref(good), 0)) == mo.ERR_INVALID_ARG   # step t < 1
+    bad = mo.AdamWHParams(1e-3, 1.0, 0.999, 1e-8, 0.1)                                        # beta1 = 1
+    assert L.muon_model_step(*args(vec, 1, ctypes.byref(bad), 1)) == mo.ERR_INVALID_ARG
+    nul = (mo.VecParam * 1)(mo.VecParam(8, p, None, p, p))
+    assert L.muon_model_step(*args(nul, 1, ctypes.byref(good), 1)) == mo.ERR_INVALID_ARG
+    # without vectors the AdamW arguments are not read; a too small workspace is then the error
+    assert L.muon_model_step(*args(None, 0, None, 0)) == mo.ERR_WORKSPACE

@@ -135,3 +135,69 @@ def test_adamw_nonfinite_gradient_element_keeps_state():
         assert p["W"][i].item() == W0[i].item() and p["m"][i].item() == 0.5 and p["v"][i].item() == 0.25
     changed = (p["W"] != W0).sum().item()
     assert changed > 900
+
+
+def test_model_step_fuses_adamw_into_the_step_launch():
+    # muon_model_step: the matrices exactly as muon_step_batched and the vectors
+    # exactly as adamw_step_batched (the same per-element arithmetic, as items of
+    # the step's pre-pass launch): both compared bit for bit with the separate
+    # calls, and the vectors against the oracle within this file's bounds
+    from muon_family_optimizer_b200 import synthetic as syn
+    hp = dict(mu=0.95, eta=0.02, gamma=1.0, beta_a=0.9, alpha=0.5, **{"lambda": 0.1})
+    shapes = [(256, 384), (384, 256), (64, 96)]
+
+    def mats():
+        out = []
+        for j, (r, c) in enumerate(shapes):
+            out.append(dict(W=syn.initial_weight("gpt2_small", j, r, c).to(torch.bfloat16).cuda(),
+                            G=syn.gradient("gpt2_small", j, 0, r, c).to(torch.bfloat16).cuda(),
+                            G_prev=syn.gradient("gpt2_small", j, 8, r, c).to(torch.bfloat16).cuda(),
+                            A=torch.zeros(r, c, device="cuda"), M=torch.zeros(r, c, device="cuda")))
+        return out
+
+    def vecs(state, t):
+        out = []
+        for j, st in enumerate(state):
+            shape = st["W"].shape
+            out.append(dict(W=torch.from_numpy(st["W"]).to(torch.bfloat16).cuda(),
+                            G=_grad(shape, t, j, torch.bfloat16).cuda(),
+                            m=torch.from_numpy(st["m"]).float().cuda(), v=torch.from_numpy(st["v"]).float().cuda()))
+        return out
+
+    sizes = [768, 2304, 65541, (3, 5)]
+    state = _state(torch.bfloat16, sizes)
+    sched = mo.quintic_schedule(5)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for t in (1, 2):
+        A, B = mats(), mats()
+        VA, VB = vecs(state, t), vecs(state, t)
+        ws = torch.empty(mo.muon_workspace_size(A, mo.BF16, sched), dtype=torch.uint8, device="cuda")
+        mo.muon_model_step(A, VA, mo.BF16, mo.BF16, hp, HP, t, sched, ws, d_status=status)
+        mo.muon_step_batched(B, mo.BF16, mo.BF16, hp, sched, ws)
+        mo.adamw_step_batched(VB, mo.BF16, HP, t)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        for a, b in zip(A, B):
+            for k in ("W", "G_prev", "A", "M"):
+                assert torch.equal(a[k], b[k]), k
+        for j, (a, b) in enumerate(zip(VA, VB)):
+            for k in ("W", "m", "v"):
+                assert torch.equal(a[k], b[k]), (j, k)
+            st = state[j]
+            g = a["G"].double().cpu().numpy()
+            W_ref, m_ref, v_ref = oracle.adamw(st["W"], g, st["m"], st["v"], lr=HP32["lr"], beta1=HP32["beta1"],
+                                               beta2=HP32["beta2"], eps=HP32["eps"],
+                                               weight_decay=HP32["weight_decay"], step=t)
+            # (the per-element bounds of this file hold for adamw_step_batched, equal bit for bit)
+            assert np.allclose(a["m"].double().cpu().numpy(), m_ref, rtol=1e-5, atol=0.0)
+            assert np.allclose(a["W"].double().cpu().numpy(), W_ref, rtol=2.0 ** -7, atol=1e-7)
+            state[j] = dict(W=_round(W_ref, torch.bfloat16), m=oracle.round_fp32(m_ref), v=oracle.round_fp32(v_ref))
+    # a non-finite vector gradient: that element keeps its state, the flag is raised
+    A, V = mats(), vecs(state, 3)
+    V[1]["G"][7] = float("nan")
+    w7 = V[1]["W"][7].clone()
+    status.zero_()
+    mo.muon_model_step(A, V, mo.BF16, mo.BF16, hp, HP, 3, sched, ws, d_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & mo.FLAG_NONFINITE
+    assert torch.equal(V[1]["W"][7], w7)
