@@ -60,11 +60,13 @@ def parse():
                     help="replay each step as a captured CUDA graph (default) or launch it eagerly")
     ap.add_argument("--variant", default="mona", choices=["mona", "lite"],
                     help="mona: G_prev and A state (default); lite: MONA-Lite, one bfloat16 buffer B")
-    ap.add_argument("--route", default="step", choices=["step", "gram", "direct", "adamw", "limuon"],
+    ap.add_argument("--route", default="step", choices=["step", "gram", "direct", "adamw", "limuon", "model"],
                     help="step: the optimizer step (default); gram / direct: the orthogonalisation alone "
                          "(gram_polar / ns_polar, converged schedule) of the workload's matrices, one batch per shape; "
                          "adamw: the AdamW step of the model's vector-valued parameters; "
-                         "limuon: the LiMuon step (randomized SVD, r = 16, p = 16) of the workload's matrices")
+                         "limuon: the LiMuon step (randomized SVD, r = 16, p = 16) of the workload's matrices; "
+                         "model: muon_model_step (matrices plus the vector-valued parameters' AdamW in one pre-pass "
+                         "launch) against the two separate calls")
     return ap.parse_args()
 
 
@@ -427,6 +429,76 @@ def run_adamw_route(args, w):
     del graph
 
 
+def run_model_route(args, w):
+    """Time muon_model_step (the matrices' MONA step with the vector-valued
+    parameters' AdamW as items of its pre-pass launch) against
+    muon_step_batched followed by adamw_step_batched on the same state."""
+    import torch
+    import muon_family_optimizer_b200 as mo
+    from muon_family_optimizer_b200 import synthetic as syn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    if w["name"] not in syn.VECTOR_SHAPES:
+        raise SystemExit(f"--route model: no vector-valued parameters for {w['name']}")
+    shapes = w["shapes"]
+    mats = []
+    for j, (r, c) in enumerate(shapes):
+        G = syn.gradient(w["name"], j, 0, r, c, device=dev)
+        mats.append(dict(W=syn.initial_weight(w["name"], j, r, c, device=dev).to(torch.bfloat16),
+                         G=G.to(torch.bfloat16), G_prev=(G * 0.5).to(torch.bfloat16),
+                         A=torch.zeros(r, c, device=dev), M=torch.zeros(r, c, device=dev)))
+    g = torch.Generator(device=dev).manual_seed(77)
+    vecs = []
+    for sh in syn.VECTOR_SHAPES[w["name"]]:
+        vecs.append(dict(W=(torch.randn(sh, generator=g, device=dev) * 0.02).to(torch.bfloat16),
+                         G=torch.randn(sh, generator=g, device=dev).to(torch.bfloat16),
+                         m=torch.zeros(sh, device=dev), v=torch.zeros(sh, device=dev)))
+    arr, varr = mo.make_params(mats), mo.make_vec_params(vecs)
+    sched = mo.quintic_schedule(args.ns_steps)
+    ws = torch.empty(mo.muon_workspace_size(arr, mo.BF16, sched), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ahp = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1)
+    fused = lambda st: mo.muon_model_step(arr, varr, mo.BF16, mo.BF16, w["hp"], ahp, 5, sched, ws,
+                                          d_status=status, stream=st)
+
+    def separate(st):
+        mo.muon_step_batched(arr, mo.BF16, mo.BF16, w["hp"], sched, ws, d_status=status, stream=st)
+        mo.adamw_step_batched(varr, mo.BF16, ahp, 5, d_status=status, stream=st)
+
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for name, fn in (("fused", fused), ("separate", separate)):
+        for _ in range(args.warmup):
+            fn(stream)
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        with torch.cuda.graph(graph, stream=cap):
+            fn(torch.cuda.current_stream(dev))
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        out[name] = e0.elapsed_time(e1) / args.steps
+        del graph
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+    nvec = sum(v["W"].numel() for v in vecs)
+    fl = ns_flops(shapes, args.ns_steps)
+    line = {"metric": "Muon + AdamW model step time, ms", "value": out["fused"], "unit": "ms", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": out["fused"], "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w['name']}: {len(shapes)} matrices + {len(vecs)} vector-valued parameters "
+                                   f"({nvec} elements)", "ns_steps": args.ns_steps},
+            "separate_calls_ms": out["separate"], "NS_TFLOP/s": fl / (out["fused"] / 1e3) / 1e12,
+            "launch": "graph (one CUDA graph per step)"}
+    print(json.dumps(line), flush=True)
+
+
 # LiMuon: rank r, oversampling p (k = r + p columns of the test matrix)
 LIMUON_HP = dict(mu=0.95, eta=0.02, gamma=1.0, rank=16, oversample=16, **{"lambda": 0.0})
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 flops at the 1965 MHz maximum SM clock
@@ -686,6 +758,8 @@ def main():
         return run_adamw_route(args, w)
     if args.route == "limuon":
         return run_limuon_route(args, w)
+    if args.route == "model":
+        return run_model_route(args, w)
     if args.route != "step":
         return run_polar_route(args, w)
     return run_step_route(args, w, ns_steps)

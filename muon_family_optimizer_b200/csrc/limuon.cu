@@ -14,7 +14,7 @@
 //     O = Q P B,   P = E_r L_r^{-1/2} E_r^T      (k x k)
 // and Q = Y R^-1 with Y^T Y = R^T R (Cholesky QR).  Every pass over an l x s
 // array streams; everything per matrix touches only k x k data:
-//   1 lim_sketch   M <- mu M + G and Y = M Omega, 128-row blocks over 64-column
+//   1 lim_sketch   M <- mu M + G and Y = M Omega, 64-row blocks over 64-column
 //                  chunks double-buffered in shared memory (cp.async); each
 //                  block adds its rows' share of the Gram Y^T Y (fp64) to the
 //                  matrix's k x k sum.  Reads G and M, writes M.
@@ -51,8 +51,9 @@ namespace {
 constexpr int kLimMax = 128;      // matrices per launch
 constexpr int kThreads = 256;
 constexpr int kSmallThreads = 64; // per-matrix k x k kernels
-constexpr int kSkRows = 128;      // lim_sketch: rows per block
+constexpr int kSkRows = 64;       // lim_sketch: rows per block
 constexpr int kSkCols = 64;       // lim_sketch: columns per chunk (two stages)
+constexpr int kSkLd = kSkCols + 4;   // padded row of a staged M chunk
 constexpr int kPjCols = 128;      // lim_project: columns per block
 constexpr int kPjRows = 32;       // lim_project: rows per chunk
 constexpr int kPjStages = 3;
@@ -134,33 +135,41 @@ __device__ __forceinline__ void add_gram(const float* X, int n, int k, double* d
 template <int G_DT>
 __host__ __device__ constexpr int g_size() { return G_DT == DT_FP32 ? 4 : 2; }
 
-template <int G_DT>
-__host__ __device__ constexpr int sketch_stage_bytes() { return kSkRows * kSkCols * (g_size<G_DT>() + 4); }
+// One stage of the sketch: raw G [kSkRows][kSkCols] in its own type, M
+// [kSkRows][kSkLd] fp32 (updated in place), Omega [kSkCols][KT] fp32.
+template <int KT, int G_DT>
+__host__ __device__ constexpr int sketch_stage_bytes() {
+    return kSkRows * kSkCols * g_size<G_DT>() + kSkRows * kSkLd * 4 + kSkCols * KT * 4;
+}
 
 template <int KT, int G_DT>
 __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant__ LimParams p) {
-    constexpr int H = KT / 32;
     constexpr int GSZ = g_size<G_DT>();
     constexpr int kGBytes = kSkRows * kSkCols * GSZ;
-    constexpr int kStage = sketch_stage_bytes<G_DT>();
+    constexpr int kMBytes = kSkRows * kSkLd * 4;
+    constexpr int kStage = sketch_stage_bytes<KT, G_DT>();
+    // register tile of the product: RPT rows x 4 columns of Y per thread
+    constexpr int CG = KT / 4, RG = kThreads / CG, RPT = kSkRows / RG;
+    static_assert(RPT * RG == kSkRows && RPT >= 1, "row tiling");
     extern __shared__ __align__(16) unsigned char sm[];
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 0)];
     const int row0 = (blockIdx.x - E.t_sketch) * kSkRows;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tx = threadIdx.x % CG, ty = threadIdx.x / CG;
     const int nchunks = (E.cols + kSkCols - 1) / kSkCols;
-    float acc[16][H];
+    const bool om_vec = (p.k & 3) == 0;       // Omega rows 16-byte aligned
+    float acc[RPT][4];
 #pragma unroll
-    for (int r = 0; r < 16; ++r)
+    for (int r = 0; r < RPT; ++r)
 #pragma unroll
-        for (int h = 0; h < H; ++h) acc[r][h] = 0.f;
+        for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
     bool bad = false;
 
-    // Chunk c (columns c*kSkCols..) of G and M into stage s: raw G in its own
-    // type, then M in fp32, row-major [kSkRows][kSkCols]; zeros outside the matrix.
+    // Chunk c (columns c*kSkCols..) of G, M and Omega into stage s; zeros outside.
     auto issue = [&](int c, int s) {
         const int c0 = c * kSkCols;
         unsigned char* gs = sm + s * kStage;
         float* ms = reinterpret_cast<float*>(gs + kGBytes);
+        float* os = reinterpret_cast<float*>(gs + kGBytes + kMBytes);
         if (E.vec_ok) {
             constexpr int GP = kSkCols * GSZ / 16, GE = 16 / GSZ;    // 16-byte pieces per row, elements per piece
             for (int q = threadIdx.x; q < kSkRows * GP; q += kThreads) {
@@ -173,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
             for (int q = threadIdx.x; q < kSkRows * MP; q += kThreads) {
                 const int rr = q / MP, pc = q % MP, i = row0 + rr, j = c0 + pc * 4;
                 const bool in = i < E.rows && j < E.cols;
-                cp_async16(ms + rr * kSkCols + pc * 4, E.M + (in ? (long long)i * E.cols + j : 0), in ? 16u : 0u);
+                cp_async16(ms + rr * kSkLd + pc * 4, E.M + (in ? (long long)i * E.cols + j : 0), in ? 16u : 0u);
             }
         } else {
             for (int q = threadIdx.x; q < kSkRows * kSkCols; q += kThreads) {
@@ -181,7 +190,20 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
                 const bool in = i < E.rows && j < E.cols;
                 const long long idx = (long long)i * E.cols + j;
                 st_elem(gs, rr * kSkCols + cc, G_DT, in ? ld_elem(E.G, idx, G_DT) : 0.f);
-                ms[rr * kSkCols + cc] = in ? E.M[idx] : 0.f;
+                ms[rr * kSkLd + cc] = in ? E.M[idx] : 0.f;
+            }
+        }
+        if (om_vec) {
+            constexpr int OP = KT / 4;
+            for (int q = threadIdx.x; q < kSkCols * OP; q += kThreads) {
+                const int jj = q / OP, pc = q % OP, j = c0 + jj;
+                const bool in = j < E.cols && pc * 4 < p.k;
+                cp_async16(os + jj * KT + pc * 4, E.Omega + (in ? (long long)j * p.k + pc * 4 : 0), in ? 16u : 0u);
+            }
+        } else {
+            for (int q = threadIdx.x; q < kSkCols * KT; q += kThreads) {
+                const int jj = q / KT, t = q % KT, j = c0 + jj;
+                os[q] = (j < E.cols && t < p.k) ? E.Omega[(long long)j * p.k + t] : 0.f;
             }
         }
         cp_async_commit();
@@ -200,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
         const int c0 = c * kSkCols;
         unsigned char* gs = sm + s * kStage;
         float* ms = reinterpret_cast<float*>(gs + kGBytes);
+        const float* os = reinterpret_cast<const float*>(gs + kGBytes + kMBytes);
         // momentum: M <- mu M + G, back to global memory and kept for the product
 #pragma unroll
         for (int it = 0; it < kSkRows * kSkCols / (8 * kThreads); ++it) {
@@ -208,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
             const int i = row0 + rr, j = c0 + cc;
             float g[8], m[8];
             load8_dt(gs, rr * kSkCols + cc, G_DT, true, 8, g);
-            float4* mp = reinterpret_cast<float4*>(ms + rr * kSkCols + cc);
+            float4* mp = reinterpret_cast<float4*>(ms + rr * kSkLd + cc);
             const float4 m0 = mp[0], m1 = mp[1];
             m[0] = m0.x; m[1] = m0.y; m[2] = m0.z; m[3] = m0.w;
             m[4] = m1.x; m[5] = m1.y; m[6] = m1.z; m[7] = m1.w;
@@ -225,28 +248,22 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
             }
         }
         __syncthreads();
-        // Y rows 16 warp + r, column lane + 32 h: += M chunk x Omega chunk
+        // Y[ty*RPT + r][4 tx + c] += sum_jj M[ty*RPT + r][jj] Omega[jj][4 tx + c]
 #pragma unroll 2
         for (int jj = 0; jj < kSkCols; jj += 4) {
-            float om[4][H];
+            float4 o[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int j = c0 + jj + q;
+            for (int q = 0; q < 4; ++q) o[q] = *reinterpret_cast<const float4*>(os + (jj + q) * KT + 4 * tx);
 #pragma unroll
-                for (int h = 0; h < H; ++h) {
-                    const int t = lane + 32 * h;
-                    om[q][h] = (j < E.cols && t < p.k) ? __ldg(E.Omega + (long long)j * p.k + t) : 0.f;
-                }
-            }
+            for (int r = 0; r < RPT; ++r) {
+                const float4 mv = *reinterpret_cast<const float4*>(ms + (ty * RPT + r) * kSkLd + jj);
+                const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const float4 mv = *reinterpret_cast<const float4*>(ms + (16 * warp + r) * kSkCols + jj);
-#pragma unroll
-                for (int h = 0; h < H; ++h) {
-                    acc[r][h] = fmaf(mv.x, om[0][h], acc[r][h]);
-                    acc[r][h] = fmaf(mv.y, om[1][h], acc[r][h]);
-                    acc[r][h] = fmaf(mv.z, om[2][h], acc[r][h]);
-                    acc[r][h] = fmaf(mv.w, om[3][h], acc[r][h]);
+                for (int q = 0; q < 4; ++q) {
+                    acc[r][0] = fmaf(mm[q], o[q].x, acc[r][0]);
+                    acc[r][1] = fmaf(mm[q], o[q].y, acc[r][1]);
+                    acc[r][2] = fmaf(mm[q], o[q].z, acc[r][2]);
+                    acc[r][3] = fmaf(mm[q], o[q].w, acc[r][3]);
                 }
             }
         }
@@ -255,13 +272,11 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
     // Y to the workspace, and this block's rows' share of Y^T Y
     float* ys = reinterpret_cast<float*>(sm);  // [kSkRows][KT]
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        const int rr = 16 * warp + r, i = row0 + rr;
-#pragma unroll
-        for (int h = 0; h < H; ++h) {
-            ys[rr * KT + lane + 32 * h] = acc[r][h];   // zero for rows past the matrix
-            if (i < E.rows) E.Y[(long long)i * KT + lane + 32 * h] = acc[r][h];
-        }
+    for (int r = 0; r < RPT; ++r) {
+        const int rr = ty * RPT + r, i = row0 + rr;
+        const float4 v = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+        *reinterpret_cast<float4*>(ys + rr * KT + 4 * tx) = v;      // zero for rows past the matrix
+        if (i < E.rows) *reinterpret_cast<float4*>(E.Y + (long long)i * KT + 4 * tx) = v;
     }
     __syncthreads();
     add_gram<KT>(ys, min(kSkRows, E.rows - row0), p.k, E.Gy);
@@ -346,17 +361,20 @@ __global__ void __launch_bounds__(kThreads) lim_rowmul(const __grid_constant__ L
         const float4 v = *reinterpret_cast<const float4*>(row + t);
         y[t] = v.x; y[t + 1] = v.y; y[t + 2] = v.z; y[t + 3] = v.w;
     }
-    float out[KT];
-#pragma unroll 4
-    for (int j = 0; j < KT; ++j) {
-        double s = 0.0;
+    // four output columns at a time, stored as they are formed (the row was read whole)
+#pragma unroll 1
+    for (int j = 0; j < KT; j += 4) {
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
 #pragma unroll
-        for (int a = 0; a < KT; ++a) s = fma((double)y[a], Ks[a * KT + j], s);
-        out[j] = (float)s;
+        for (int a = 0; a < KT; ++a) {
+            const double ya = (double)y[a];
+            s0 = fma(ya, Ks[a * KT + j], s0);
+            s1 = fma(ya, Ks[a * KT + j + 1], s1);
+            s2 = fma(ya, Ks[a * KT + j + 2], s2);
+            s3 = fma(ya, Ks[a * KT + j + 3], s3);
+        }
+        *reinterpret_cast<float4*>(row + j) = make_float4((float)s0, (float)s1, (float)s2, (float)s3);
     }
-#pragma unroll
-    for (int t = 0; t < KT; t += 4)
-        *reinterpret_cast<float4*>(row + t) = make_float4(out[t], out[t + 1], out[t + 2], out[t + 3]);
 }
 
 // ---------------------------------------------------------------------------
@@ -367,18 +385,20 @@ __host__ __device__ constexpr int project_stage_floats() { return kPjRows * kPjC
 
 template <int KT>
 __global__ void __launch_bounds__(kThreads, 3) lim_project(const __grid_constant__ LimParams p) {
-    constexpr int H = KT / 32;
     constexpr int kStage = project_stage_floats<KT>();
+    // register tile: JPT columns of M (rows of B^T) x 4 columns of Q per thread
+    constexpr int CG = KT / 4, JG = kThreads / CG, JPT = kPjCols / JG;
+    static_assert(JPT * JG == kPjCols && JPT % 4 == 0, "column tiling");
     extern __shared__ __align__(16) float fsm[];
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 2)];
     const int c0 = (blockIdx.x - E.t_proj) * kPjCols;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tt = threadIdx.x % CG, tj = threadIdx.x / CG;
     const int nchunks = (E.rows + kPjRows - 1) / kPjRows;
-    float acc[16][H];
+    float acc[JPT][4];
 #pragma unroll
-    for (int c = 0; c < 16; ++c)
+    for (int c = 0; c < JPT; ++c)
 #pragma unroll
-        for (int h = 0; h < H; ++h) acc[c][h] = 0.f;
+        for (int h = 0; h < 4; ++h) acc[c][h] = 0.f;
 
     // rows i0.. of M (this block's columns) and of Q into stage s
     auto issue = [&](int ch, int s) {
@@ -418,20 +438,16 @@ __global__ void __launch_bounds__(kThreads, 3) lim_project(const __grid_constant
         const float* qs = ms + kPjRows * kPjCols;
 #pragma unroll 4
         for (int rr = 0; rr < kPjRows; ++rr) {
-            float qv[H];
+            const float4 q4 = *reinterpret_cast<const float4*>(qs + rr * KT + 4 * tt);
+            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-            for (int h = 0; h < H; ++h) qv[h] = qs[rr * KT + lane + 32 * h];
-            const float4* mrow = reinterpret_cast<const float4*>(ms + rr * kPjCols + 16 * warp);
+            for (int c4 = 0; c4 < JPT / 4; ++c4) {
+                const float4 mv = *reinterpret_cast<const float4*>(ms + rr * kPjCols + tj * JPT + 4 * c4);
+                const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const float4 mv = mrow[c4];
+                for (int e = 0; e < 4; ++e)
 #pragma unroll
-                for (int h = 0; h < H; ++h) {
-                    acc[4 * c4 + 0][h] = fmaf(mv.x, qv[h], acc[4 * c4 + 0][h]);
-                    acc[4 * c4 + 1][h] = fmaf(mv.y, qv[h], acc[4 * c4 + 1][h]);
-                    acc[4 * c4 + 2][h] = fmaf(mv.z, qv[h], acc[4 * c4 + 2][h]);
-                    acc[4 * c4 + 3][h] = fmaf(mv.w, qv[h], acc[4 * c4 + 3][h]);
-                }
+                    for (int h = 0; h < 4; ++h) acc[4 * c4 + e][h] = fmaf(mm[e], qv[h], acc[4 * c4 + e][h]);
             }
         }
         __syncthreads();                       // this stage is refilled next
@@ -440,24 +456,25 @@ __global__ void __launch_bounds__(kThreads, 3) lim_project(const __grid_constant
     // B^T to the workspace, and this block's columns' share of B B^T
     float* bs = fsm;                           // [kPjCols][KT]
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        const int cc = 16 * warp + c, j = c0 + cc;
-#pragma unroll
-        for (int h = 0; h < H; ++h) {
-            bs[cc * KT + lane + 32 * h] = acc[c][h];
-            if (j < E.cols) E.Bt[(long long)j * KT + lane + 32 * h] = acc[c][h];
-        }
+    for (int c = 0; c < JPT; ++c) {
+        const int cc = tj * JPT + c, j = c0 + cc;
+        const float4 v = make_float4(acc[c][0], acc[c][1], acc[c][2], acc[c][3]);
+        *reinterpret_cast<float4*>(bs + cc * KT + 4 * tt) = v;
+        if (j < E.cols) *reinterpret_cast<float4*>(E.Bt + (long long)j * KT + 4 * tt) = v;
     }
     __syncthreads();
     add_gram<KT>(bs, min(kPjCols, E.cols - c0), p.k, E.Cg);
 }
 
 // ---------------------------------------------------------------------------
-// 5. eigen-decomposition of B B^T and P = E_r L_r^{-1/2} E_r^T (one small
-//    block per matrix, k x k only)
+// 5. eigen-decomposition of B B^T and P = E_r L_r^{-1/2} E_r^T (one block per
+//    matrix, k x k only).  A round applies k/2 disjoint rotations J at once:
+//    C <- J^T C J touches the 2 x 2 blocks (rows of pair i, columns of pair j),
+//    each updated by one thread from its own four entries, so a round is one
+//    pass over C (and E <- E J) after the rotations are chosen.
 // ---------------------------------------------------------------------------
 template <int KT>
-__global__ void __launch_bounds__(kSmallThreads) lim_eig(const __grid_constant__ LimParams p) {
+__global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimParams p) {
     extern __shared__ __align__(16) double dsm[];
     double* C = dsm;                    // [KT][KT]
     double* Ev = dsm + KT * KT;         // [KT][KT] eigenvectors (columns)
@@ -468,7 +485,7 @@ __global__ void __launch_bounds__(kSmallThreads) lim_eig(const __grid_constant__
     int* pq = pp + KT / 2;                         // [KT/2]
     __shared__ int rotated, nonfinite;
     const LimEntry& E = p.e[blockIdx.x];
-    const int k = p.k, ke = k + (k & 1), n = ke - 1;
+    const int k = p.k, ke = k + (k & 1), n = ke - 1, np = ke / 2;
     if (threadIdx.x == 0) nonfinite = 0;
     __syncthreads();
     for (int idx = threadIdx.x; idx < KT * KT; idx += blockDim.x) {
@@ -485,7 +502,7 @@ __global__ void __launch_bounds__(kSmallThreads) lim_eig(const __grid_constant__
         return;
     }
     // Off-diagonal entries at the fp64 rounding level of the whole matrix are
-    // noise, not coupling: below kRotTol * trace no rotation is made, so a
+    // noise, not coupling: below 0.1 kRotTol * trace no rotation is made, so a
     // pair of negligible eigenvalues cannot keep the sweeps going.
     double tr = 0.0;
     for (int a = 0; a < k; ++a) tr += fabs(C[a * KT + a]);
@@ -494,7 +511,7 @@ __global__ void __launch_bounds__(kSmallThreads) lim_eig(const __grid_constant__
         if (threadIdx.x == 0) rotated = 0;
         __syncthreads();
         for (int rd = 0; rd < n; ++rd) {
-            if (threadIdx.x < ke / 2) {
+            if (threadIdx.x < np) {
                 const int i = threadIdx.x;
                 int a = i == 0 ? n : (rd + i) % n, b = i == 0 ? rd : (rd - i + n) % n;
                 if (a > b) { const int t = a; a = b; b = t; }
@@ -510,22 +527,23 @@ __global__ void __launch_bounds__(kSmallThreads) lim_eig(const __grid_constant__
                 pp[i] = a; pq[i] = b; cs[i] = c; sn[i] = s;
             }
             __syncthreads();
-            for (int idx = threadIdx.x; idx < (ke / 2) * ke; idx += blockDim.x) {   // rows p, q <- J^T C
-                const int i = idx / ke, col = idx % ke;
-                const double c = cs[i], s = sn[i];
-                if (s == 0.0) continue;
-                const double x = C[pp[i] * KT + col], y = C[pq[i] * KT + col];
-                C[pp[i] * KT + col] = c * x - s * y;
-                C[pq[i] * KT + col] = s * x + c * y;
+            for (int idx = threadIdx.x; idx < np * np; idx += blockDim.x) {   // C <- J^T C J, block by block
+                const int i = idx / np, j = idx % np;
+                const double c1 = cs[i], s1 = sn[i], c2 = cs[j], s2 = sn[j];
+                if (s1 == 0.0 && s2 == 0.0) continue;
+                const int a1 = pp[i], b1 = pq[i], a2 = pp[j], b2 = pq[j];
+                const double x = C[a1 * KT + a2], y = C[a1 * KT + b2], z = C[b1 * KT + a2], w = C[b1 * KT + b2];
+                const double r0 = c1 * x - s1 * z, r1 = c1 * y - s1 * w;   // rows a1, b1 rotated
+                const double r2 = s1 * x + c1 * z, r3 = s1 * y + c1 * w;
+                C[a1 * KT + a2] = c2 * r0 - s2 * r1;                      // then columns a2, b2
+                C[a1 * KT + b2] = s2 * r0 + c2 * r1;
+                C[b1 * KT + a2] = c2 * r2 - s2 * r3;
+                C[b1 * KT + b2] = s2 * r2 + c2 * r3;
             }
-            __syncthreads();
-            for (int idx = threadIdx.x; idx < (ke / 2) * ke; idx += blockDim.x) {   // columns p, q <- C J, E J
-                const int i = idx / ke, row = idx % ke;
+            for (int idx = threadIdx.x; idx < ke * np; idx += blockDim.x) {   // E <- E J
+                const int row = idx / np, i = idx % np;
                 const double c = cs[i], s = sn[i];
                 if (s == 0.0) continue;
-                const double x = C[row * KT + pp[i]], y = C[row * KT + pq[i]];
-                C[row * KT + pp[i]] = c * x - s * y;
-                C[row * KT + pq[i]] = s * x + c * y;
                 const double u = Ev[row * KT + pp[i]], v = Ev[row * KT + pq[i]];
                 Ev[row * KT + pp[i]] = c * u - s * v;
                 Ev[row * KT + pq[i]] = s * u + c * v;
@@ -683,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 2) lim_update(const __grid_constant_
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 template <int KT, int G_DT>
-constexpr size_t sketch_smem() { return 2 * (size_t)sketch_stage_bytes<G_DT>(); }
+constexpr size_t sketch_smem() { return 2 * (size_t)sketch_stage_bytes<KT, G_DT>(); }
 template <int KT>
 constexpr size_t project_smem() { return sizeof(float) * kPjStages * project_stage_floats<KT>(); }
 template <int KT>
@@ -743,7 +761,7 @@ muon_status launch_all(LimParams& prm, cudaStream_t s, const LaunchShape& L) {
     lim_project<KT><<<L.proj, kThreads, project_smem<KT>(), s>>>(prm);
     trace_end(s);
     trace_begin(MUON_KERNEL_RSVD_SMALL, 2.0 * kk, s);                                // Gram read, P written
-    lim_eig<KT><<<prm.n, kSmallThreads, eig_smem<KT>(), s>>>(prm);
+    lim_eig<KT><<<prm.n, kThreads, eig_smem<KT>(), s>>>(prm);
     trace_end(s);
     trace_begin(MUON_KERNEL_RSVD_SMALL, 8.0 * L.rows_total * KT + kk, s);           // Q read, Z written
     lim_rowmul<KT><<<L.rows, kThreads, 0, s>>>(prm);

@@ -70,6 +70,7 @@ struct Group {
     int s = 0, l = 0;
     std::vector<int> members;        // indices into the caller's parameter array
     int dt = DT_BF16;                // element type of this group's iteration
+    int x0_dt = DT_BF16;             // element type of the pre-pass copy of M (x[0])
     int gram = 0;                    // 1: the Gram route, 0: the direct iteration
     long long ldl = 0, lds = 0;      // padded row strides of s x l and s x s buffers
     size_t x[2] = {0, 0};            // s x l ping-pong
@@ -121,6 +122,16 @@ Layout step_layout(const muon_param* params, int n, int ns_dt, const muon_schedu
             g.l = kv.first.second;
             g.dt = (ns_dt != DT_FP32 && g.s < kMinTcSide) ? DT_FP32 : ns_dt;
             g.gram = gram_group(sch, g.s, g.l, g.dt) ? 1 : 0;
+            g.x0_dt = g.dt;
+            if (g.gram) {
+                // The Gram route iterates in fp16 whatever the 16-bit type ([POLAR]:
+                // fp16 is recommended; with bfloat16's 8 bits rounding turns small
+                // eigenvalues of R negative and the polynomial h R h multiplies them
+                // about 12 times a step): the pre-pass copy of M is bfloat16 (any
+                // range), then divided by its norm into fp16 (x[1]).
+                g.x0_dt = DT_BF16;
+                g.dt = DT_FP16;
+            }
             g.members.assign(all.begin() + b, all.begin() + std::min(all.size(), b + kMaxGroupMembers));
             groups.push_back(g);
         }
@@ -308,16 +319,17 @@ muon_status run_direct(Runner& R, const GroupList& gs, void* ws, const double* s
 }
 
 // The Gram route (see include/muon.h) on the groups `gs` (all of R.dt, each
-// with six s x s buffers), starting from the unnormalised wide views in x[0];
+// with six s x s buffers), starting from the wide views in x[xb0] (normalised
+// already when R.prenorm);
 // the last product's epilogue is `final_kind` as for run_direct.  Every launch
 // carries the same product for all groups.
 muon_status run_gram(Runner& R, const GroupList& gs, void* ws, const double* sumsq, const muon_schedule* sch,
-                     const FinalTables& fins, int final_kind) {
+                     const FinalTables& fins, int final_kind, int xb0 = 0) {
     if (gs.empty()) return MUON_OK;
     const float f = sch->scale_f;
     // buffer roles: indices into each group's sq[]
     int iR = 0, iRn = 1, iH = 2, iQ = 3, iQn = 4, iT = 5;
-    int xb = 0;                 // current Xb buffer
+    int xb = xb0;               // current Xb buffer
     bool xb_raw = true;         // Xb still holds the unnormalised input (scale pending)
     bool q_identity = true;
     auto sq = [&](const Group& g, int i) { return at(ws, g.sq[i]); };
@@ -514,8 +526,13 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
     // 1. fused MONA pre-pass + norms + wide-view copies: one launch per
     //    element type of the copies (the iteration's, and fp32 for narrow groups)
     const size_t in_sz = dt_size(w_dtype);
-    const int n_x0 = (int)ns_dtype == DT_FP32 ? 1 : 2;
-    const int x0_types[2] = {(int)ns_dtype, DT_FP32};
+    int x0_types[3], n_x0 = 0;
+    x0_types[n_x0++] = (int)ns_dtype;
+    for (const Group& g : L.groups) {
+        bool seen = false;
+        for (int t = 0; t < n_x0; ++t) seen |= x0_types[t] == g.x0_dt;
+        if (!seen) x0_types[n_x0++] = g.x0_dt;
+    }
     for (int t = 0; t < n_x0; ++t) {
         const int x0_dt = x0_types[t];
         PrepParams pp;
@@ -524,14 +541,14 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
         pp.beta_a = hp->beta_a; pp.alpha = hp->alpha; pp.mu = hp->mu;
         pp.sumsq = sumsq;
         for (const Group& g : L.groups) {
-            if (g.dt != x0_dt) continue;
+            if (g.x0_dt != x0_dt) continue;
             for (size_t j = 0; j < g.members.size(); ++j) {
                 const muon_param& p = params[g.members[j]];
                 PrepEntry& E = pp.e[pp.n++];
                 E.G = p.G; E.Gp = p.G_prev; E.A = p.A; E.M = p.M;
                 E.rows = p.rows; E.cols = p.cols; E.count = 1;
                 E.transposed = p.rows > p.cols;
-                E.X0 = static_cast<char*>(at(workspace, g.x[0])) + j * (size_t)g.s * g.ldl * dt_size(g.dt);
+                E.X0 = static_cast<char*>(at(workspace, g.x[0])) + j * (size_t)g.s * g.ldl * dt_size(g.x0_dt);
                 E.ld = g.ldl;
                 E.sumsq_index = g.sumsq0 + (int)j;
                 const uintptr_t al = reinterpret_cast<uintptr_t>(p.G) | reinterpret_cast<uintptr_t>(p.G_prev) |
@@ -571,6 +588,32 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
         }
     }
 
+    // 1b. Gram-route groups: x[1] = x[0] / (||M|| + eps) in fp16 (norms complete)
+    {
+        PrepParams pp;
+        memset(&pp, 0, sizeof(pp));
+        pp.in_dt = DT_BF16; pp.x0_dt = DT_FP16; pp.mode = 1; pp.prescale = 1; pp.eps = sched->eps;
+        pp.sumsq = sumsq;
+        for (const Group& g : L.groups) {
+            if (!g.gram) continue;
+            PrepEntry& E = pp.e[pp.n++];
+            E.X = at(workspace, g.x[0]); E.x_stride = (long long)g.s * g.ldl;
+            E.X0 = at(workspace, g.x[1]); E.x0_stride = (long long)g.s * g.ldl; E.ld = g.ldl;
+            E.rows = g.s; E.cols = (int)g.ldl; E.count = (int)g.members.size(); E.transposed = 0;
+            E.sumsq_index = g.sumsq0;
+            E.vec_ok = 1;             // rows of ldl elements (a multiple of 8), 1024-byte aligned buffers
+            if (pp.n == kMaxPrep) {
+                st = prep_run(pp, stream_);
+                if (st != MUON_OK) return st;
+                pp.n = 0;
+            }
+        }
+        if (pp.n > 0) {
+            st = prep_run(pp, stream_);
+            if (st != MUON_OK) return st;
+        }
+    }
+
     // 2-3. iteration with the weight update fused into its last step: the
     //      direct groups of the iteration's type, the Gram-route groups, and
     //      the narrow groups in fp32
@@ -596,15 +639,18 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
             fe.vec_ok = (p.cols % 8 == 0) && (al & 15) == 0;
             f.push_back(fe);
         }
-        if (g.dt != (int)ns_dtype) { direct32.push_back(&g); fin_d32.push_back(f); }
-        else if (g.gram) { gram16.push_back(&g); fin_g16.push_back(f); }
+        if (g.gram) { gram16.push_back(&g); fin_g16.push_back(f); }
+        else if (g.dt != (int)ns_dtype) { direct32.push_back(&g); fin_d32.push_back(f); }
         else { direct16.push_back(&g); fin_d16.push_back(f); }
     }
     R.dt = ns_dtype;
     st = run_direct(R, direct16, workspace, sumsq, sched, fin_d16, FIN_WUPD);
     if (st != MUON_OK) return st;
-    st = run_gram(R, gram16, workspace, sumsq, sched, fin_g16, FIN_WUPD);
+    R.dt = DT_FP16;
+    R.prenorm = true;          // the Gram groups start from their normalised fp16 copies in x[1]
+    st = run_gram(R, gram16, workspace, sumsq, sched, fin_g16, FIN_WUPD, 1);
     if (st != MUON_OK) return st;
+    R.prenorm = false;
     R.dt = DT_FP32;
     return run_direct(R, direct32, workspace, sumsq, sched, fin_d32, FIN_WUPD);
 }

@@ -44,7 +44,9 @@ def _state():
 
 def test_sharded_step_world_one_is_the_library_step():
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
-    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    from datetime import timedelta
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0),
+                            timeout=timedelta(seconds=60))
     try:
         params = _state()
         host = [{k: v.double().cpu().numpy() for k, v in p.items()} for p in params]
