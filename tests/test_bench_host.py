@@ -74,3 +74,43 @@ def test_limuon_kernel_work_counts():
 def test_fp32_alu_peak_from_unit_counts():
     assert abs(bench.FP32_ALU_TFLOPS - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
     assert 74.0 < bench.FP32_ALU_TFLOPS < 75.0
+
+
+def test_layers_slice_keeps_whole_layers():
+    class A:
+        workload, layers = "llama3_8b", 1
+    w = bench.select_workload(A)
+    assert w["shapes"] == syn.WORKLOADS["llama3_8b"]["shapes"][:7]
+    A.layers = 32
+    assert len(bench.select_workload(A)["shapes"]) == 224
+    A.layers = 33
+    with pytest.raises(SystemExit):
+        bench.select_workload(A)
+    A.workload, A.layers = "moe_gram", 1          # no layer structure
+    with pytest.raises(SystemExit):
+        bench.select_workload(A)
+
+
+def test_shape_groups_cheapest_first():
+    g = bench.shape_groups(syn.WORKLOADS["llama3_8b"]["shapes"])
+    assert [len(m) for _, m in g] == [64, 64, 96]
+    costs = [c for c, _ in g]
+    assert costs == sorted(costs)
+    # both orientations of a shape share a group
+    assert {(r, c) for _, r, c in g[2][1]} == {(14336, 4096), (4096, 14336)}
+
+
+def test_recorded_traffic_scales_a_layer_slice_by_elements(tmp_path, monkeypatch):
+    root = tmp_path / "repo"
+    for rel in set(sum((list(v) for v in bench.TRAFFIC_SOURCES.values()), [])):
+        dst = root / rel
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        shutil.copy(os.path.join(bench.ROOT, rel), dst)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    (root / "profiles").mkdir()
+    rec = {"kernel": "tc_upd", "workload": "llama3_8b", "ns_steps": 5, "bytes_per_launch": 1000.0,
+           "elements": 218103808, "sources": bench.sources_digest("tc_upd")}
+    (root / "profiles" / "k.md").write_text("traffic-record: " + json.dumps(rec) + "\n")
+    b, src = bench.recorded_traffic("tc_upd", "llama3_8b", 5, elements=32 * 218103808)
+    assert b == 32000.0 and "scaled" in src
+    assert bench.recorded_traffic("tc_upd", "llama3_8b", 5, elements=218103808)[0] == 1000.0
