@@ -19,6 +19,11 @@ struct GemmOp {
     // Symmetric result that an update product will read on CTA pairs: also
     // store the first tile below the diagonal (exact mirror of the one above).
     int band;
+    // Operand stored transposed in full (tensor-core path; a matrix copied in
+    // its parameter's orientation, K x M instead of M x K): SYM A (a_tr) / B
+    // (b_tr) are read as MN-major tiles; UPD B (b_tr: N x K, K contiguous) as
+    // K-major tiles.
+    int a_tr, b_tr;
     int count, M, N, K;
     const void* A; long long lda, strideA;
     const void* B; long long ldb, strideB;

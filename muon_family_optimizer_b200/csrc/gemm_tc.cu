@@ -74,12 +74,14 @@ struct Cfg {
 struct TcProblem {
     CUtensorMap mapA;    // A rows, K-major boxes 64 (K) x 128 (M)
     CUtensorMap mapAt;   // A symmetric: transposed reads, boxes 64 (M) x 64 (K)
-    CUtensorMap mapB;    // SYM: B rows, boxes 64 (K) x 128 (N); UPD: X panel, boxes 64 (N) x 64 (K)
+    CUtensorMap mapB;    // SYM: B rows, boxes 64 (K) x 128 (N); UPD: X panel, boxes 64 (N) x 64 (K),
+                         // or (b_tr) X stored N x K, boxes 64 (K) x BN/2 (N)
     CUtensorMap mapBt;   // B symmetric: transposed reads, boxes 64 (N) x 64 (K)
     CUtensorMap mapD;    // output stores, boxes 64 (N) x 32 (M)
     CUtensorMap mapDt;   // band: transposed stores, boxes 32 (M) x 64 (N), no swizzle
     int count, M, N, K;
     int tiles_m, tiles_n, tiles_per_mat, sym, a_sym, b_sym, band;
+    int a_tr, b_tr;      // operands stored transposed in full (see GemmOp)
     int same_ab;         // A and B are one operand: a diagonal tile loads one panel for both
     long long tile_begin;
     Epilogue epi;
@@ -529,8 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     }
     if (warp == 0 && lane == 0) {
         for (int i = 0; i < p.nprob; ++i) {
-            prefetch_tensormap(&p.prob[i].mapA);
-            prefetch_tensormap(&p.prob[i].mapB);
+            prefetch_tensormap(p.prob[i].a_tr ? &p.prob[i].mapAt : &p.prob[i].mapA);
+            prefetch_tensormap(p.prob[i].sym && p.prob[i].b_tr ? &p.prob[i].mapBt : &p.prob[i].mapB);
         }
     }
     if (warp == 1) {
@@ -571,9 +573,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 // A diagonal tile of a product whose operands are one matrix (X X^T,
                 // S S) needs the same rows as A and as B: one panel serves both.
                 const bool one_panel = !B_MN && P.same_ab && ti == tj;
-                uint32_t bytes = C::kABytes + (B_MN ? nchunk * 64 * BK * 2 : (one_panel ? 0 : C::kBBytes));
+                // an update product whose X is stored transposed loads whole K-major boxes
+                const bool b_kmaj = B_MN && P.b_tr;
+                uint32_t bytes = C::kABytes + (B_MN ? (b_kmaj ? C::kBBytes : nchunk * 64 * BK * 2)
+                                                    : (one_panel ? 0 : C::kBBytes));
                 if (PAIR) {   // the leader's barrier counts both CTAs' boxes
-                    bytes = B_MN ? 2 * C::kABytes + (chunks(tj * BN) + chunks(tj * BN + kBCols)) * 64 * BK * 2
+                    bytes = B_MN ? (b_kmaj ? 2 * (C::kABytes + C::kBBytes)
+                                           : 2 * C::kABytes + (chunks(tj * BN) + chunks(tj * BN + kBCols)) * 64 * BK * 2)
                                  : 2 * (C::kABytes + (one_panel ? 0 : C::kBBytes));
                 }
                 for (int kb = 0; kb < nkb; ++kb) {
@@ -585,8 +591,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     // decision is taken on the pair's first 128-row (128-column) block,
                     // so both halves agree (such operands also store the first tile
                     // below the diagonal).
-                    const bool at = P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti);
-                    const bool bt = !B_MN && P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj);
+                    const bool at = P.a_tr || (P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti));
+                    const bool bt = !B_MN && (P.b_tr || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj)));
                     const uint32_t fb = PAIR ? mapa_shared(smem_u32(&full_bar[stage]), 0) : 0u;
                     auto load = [&](const CUtensorMap* map, void* dst, int x, int y) {
                         if (PAIR) tma_load_3d_pair(map, fb, dst, x, y, m);
@@ -599,7 +605,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     } else {
                         load(&P.mapA, sa, kb * BK, rows0);
                     }
-                    if (B_MN) {
+                    if (b_kmaj) {
+                        load(&P.mapB, sb, kb * BK, bcol0);
+                    } else if (B_MN) {
                         for (int c = 0; c < nchunk; ++c) load(&P.mapB, sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK);
                     } else if (one_panel) {
                         // B is the A panel just loaded
@@ -654,8 +662,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, abort_flag, d_status)) { ok = false; break; }
                     tc_fence_after();
-                    const bool at = P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti);   // A block read transposed
-                    const bool bm = B_MN || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj));   // B block MN-major
+                    const bool at = P.a_tr || (P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti));   // A block read transposed
+                    const bool bm = B_MN ? !P.b_tr : (P.b_tr || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj)));   // B block MN-major
                     const uint32_t idesc = idesc0 | (at ? 1u << 15 : 0u) | (bm ? 1u << 16 : 0u);
                     const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t sb = one_panel ? sa : sa + C::kABytes;
@@ -1041,16 +1049,27 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         P.a_sym = o.a_sym;
         P.b_sym = sym ? o.b_sym : 0;
         P.band = sym ? (pair ? 1 : o.band) : 0;
-        P.same_ab = sym && o.A == o.B && o.lda == o.ldb && o.strideA == o.strideB && o.a_sym == o.b_sym;
-        // A operand: M rows x K (K contiguous); a symmetric A is also read transposed
-        if (!encode_map(&P.mapA, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, BK, BM)) return MUON_ERR_CUDA;
-        if (o.a_sym && !encode_map(&P.mapAt, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, 64, BK))
+        P.a_tr = o.a_tr;
+        P.b_tr = o.b_tr;
+        P.same_ab = sym && o.A == o.B && o.lda == o.ldb && o.strideA == o.strideB && o.a_sym == o.b_sym &&
+                    o.a_tr == o.b_tr;
+        // A operand: M rows x K (K contiguous); a symmetric A is also read transposed;
+        // a transposed A (K rows x M) only transposed
+        if (!o.a_tr && !encode_map(&P.mapA, dt, o.A, o.K, o.M, o.count, o.lda, o.strideA, BK, BM))
+            return MUON_ERR_CUDA;
+        if ((o.a_sym || o.a_tr) && !encode_map(&P.mapAt, dt, o.A, o.a_tr ? o.M : o.K, o.a_tr ? o.K : o.M, o.count,
+                                               o.lda, o.strideA, 64, BK))
             return MUON_ERR_CUDA;
         if (sym) {
             // each CTA of a pair loads half of the tile's B rows
-            if (!encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK, pair ? BN / 2 : BN))
+            if (!o.b_tr && !encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK, pair ? BN / 2 : BN))
                 return MUON_ERR_CUDA;
-            if (o.b_sym && !encode_map(&P.mapBt, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, 64, BK))
+            if ((o.b_sym || o.b_tr) && !encode_map(&P.mapBt, dt, o.B, o.b_tr ? o.N : o.K, o.b_tr ? o.K : o.N,
+                                                   o.count, o.ldb, o.strideB, 64, BK))
+                return MUON_ERR_CUDA;
+        } else if (o.b_tr) {
+            // X stored N x K (K contiguous); boxes of BK (K) x the CTA's N columns
+            if (!encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK, pair ? BN / 2 : BN))
                 return MUON_ERR_CUDA;
         } else {
             // X panel: K rows x N (N contiguous); boxes of 64 (N) x BK (K)

@@ -72,7 +72,12 @@ struct Group {
     int dt = DT_BF16;                // element type of this group's iteration
     int x0_dt = DT_BF16;             // element type of the pre-pass copy of M (x[0])
     int gram = 0;                    // 1: the Gram route, 0: the direct iteration
+    // Members with rows <= cols come first (n_wide of them).  When param_tr is
+    // set, the pre-pass copies a taller member in its own orientation (l x s,
+    // row stride lds) and the first step's products read it transposed.
+    int n_wide = 0, param_tr = 0;
     long long ldl = 0, lds = 0;      // padded row strides of s x l and s x s buffers
+    long long xs = 0;                // elements per member in the s x l buffers
     size_t x[2] = {0, 0};            // s x l ping-pong
     size_t sq[6] = {0, 0, 0, 0, 0, 0};   // s x s buffers (direct route uses 2, Gram route 6)
     int sumsq0 = 0;                  // first sumsq slot of this group
@@ -88,9 +93,11 @@ void place_group(Group& g, size_t& off) {
     const int esz = dt_size(g.dt);
     g.ldl = pad8(g.l);
     g.lds = pad8(g.s);
+    g.xs = (long long)g.s * g.ldl;
+    if (g.param_tr && g.n_wide < cnt) g.xs = std::max(g.xs, (long long)g.l * g.lds);
     for (int i = 0; i < 2; ++i) {
         g.x[i] = off;
-        off = align_up(off + (size_t)cnt * g.s * g.ldl * esz, kAlign);
+        off = align_up(off + (size_t)cnt * g.xs * esz, kAlign);
     }
     for (int i = 0; i < (g.gram ? 6 : 2); ++i) {
         g.sq[i] = off;
@@ -133,6 +140,12 @@ Layout step_layout(const muon_param* params, int n, int ns_dt, const muon_schedu
                 g.dt = DT_FP16;
             }
             g.members.assign(all.begin() + b, all.begin() + std::min(all.size(), b + kMaxGroupMembers));
+            std::stable_partition(g.members.begin(), g.members.end(),
+                                  [&](int i) { return params[i].rows <= params[i].cols; });
+            g.n_wide = 0;
+            for (int i : g.members) g.n_wide += params[i].rows <= params[i].cols;
+            // the tensor-core direct groups read a taller member in its own orientation
+            g.param_tr = (!g.gram && g.dt != DT_FP32) ? 1 : 0;
             groups.push_back(g);
         }
     }
@@ -213,6 +226,7 @@ GemmOp sym_op(int count, int n, int k, const void* A, long long lda, long long s
               long long ldb, long long sB, const Epilogue& e, int a_sym = 0, int b_sym = 0, int band = 0) {
     GemmOp o;
     o.sym = 1; o.a_sym = a_sym; o.b_sym = b_sym; o.band = band; o.count = count; o.M = n; o.N = n; o.K = k;
+    o.a_tr = 0; o.b_tr = 0;
     o.A = A; o.lda = lda; o.strideA = sA;
     o.B = B; o.ldb = ldb; o.strideB = sB;
     o.epi = e;
@@ -224,6 +238,7 @@ GemmOp upd_op(int count, int s, int l, const void* A, long long lda, long long s
               long long ldx, long long sX, const Epilogue& e) {
     GemmOp o;
     o.sym = 0; o.a_sym = 1; o.b_sym = 0; o.band = 0; o.count = count; o.M = s; o.N = l; o.K = s;
+    o.a_tr = 0; o.b_tr = 0;
     o.A = A; o.lda = lda; o.strideA = sA;
     o.B = X; o.ldb = ldx; o.strideB = sX;
     o.epi = e;
@@ -259,29 +274,54 @@ muon_status run_final(Runner& R, const std::vector<GemmOp>& ops, const FinalTabl
     return R.run(batch, fin);
 }
 
+// The members of a group as the first products see them: the wide members
+// (rows <= cols), then -- read transposed when the group copies them in their
+// own orientation -- the taller ones.  {first member, count, transposed}.
+struct Part {
+    int first, count, tr;
+};
+
+std::vector<Part> first_parts(const Group& g) {
+    const int cnt = (int)g.members.size();
+    if (!g.param_tr || g.n_wide == cnt) return {{0, cnt, 0}};
+    if (g.n_wide == 0) return {{0, cnt, 1}};
+    return {{0, g.n_wide, 0}, {g.n_wide, cnt - g.n_wide, 1}};
+}
+
 // The direct quintic iteration on the groups `gs` (all of R.dt), starting
-// from the unnormalised wide views in x[0] (norms in sumsq).  The last step's
+// from the unnormalised copies in x[0] (norms in sumsq).  The last step's
 // epilogue is `final_kind` (FIN_OUT or FIN_WUPD with the groups' tables).
 muon_status run_direct(Runner& R, const GroupList& gs, void* ws, const double* sumsq, const muon_schedule* sch,
                        const FinalTables& fins, int final_kind) {
     if (gs.empty()) return MUON_OK;
     const float f = sch->scale_f;
+    const int esz = dt_size(R.dt);
     int cur = 0;
     for (int k = 0; k < sch->n_steps; ++k) {
         const muon_ns_coeff c = sch->coeffs[k];
         const bool first = k == 0;
         const float pre = first ? 1.f / f : (is_restart(sch, k) ? 1.f / f : 1.f);
         const bool last = k == sch->n_steps - 1;
+        // member ranges of each product: the first step reads transposed copies
+        // of the taller members separately, later steps the wide views only
+        auto parts = [&](const Group& g) {
+            return first ? first_parts(g) : std::vector<Part>{{0, (int)g.members.size(), 0}};
+        };
         // A = X X^T (scaled by pre^2, and by 1/(|M|+eps)^2 at the first step)
         std::vector<GemmOp> ops;
         for (const Group* gp : gs) {
             const Group& g = *gp;
-            const int cnt = (int)g.members.size();
-            const long long sx = (long long)g.s * g.ldl, ss = (long long)g.s * g.lds;
-            Epilogue e = epi_store(at(ws, g.sq[0]), g.lds, ss);
-            e.sc_mul = pre * pre;
-            if (first && !R.prenorm) { e.sumsq = sumsq + g.sumsq0; e.eps = sch->eps; e.sc_pow = 2; }
-            ops.push_back(sym_op(cnt, g.s, g.l, at(ws, g.x[cur]), g.ldl, sx, at(ws, g.x[cur]), g.ldl, sx, e));
+            const long long ss = (long long)g.s * g.lds;
+            for (const Part& q : parts(g)) {
+                Epilogue e = epi_store(static_cast<char*>(at(ws, g.sq[0])) + (size_t)q.first * ss * esz, g.lds, ss);
+                e.sc_mul = pre * pre;
+                if (first && !R.prenorm) { e.sumsq = sumsq + g.sumsq0 + q.first; e.eps = sch->eps; e.sc_pow = 2; }
+                const void* X = static_cast<char*>(at(ws, g.x[cur])) + (size_t)q.first * g.xs * esz;
+                const long long ldx = q.tr ? g.lds : g.ldl;
+                GemmOp o = sym_op(q.count, g.s, g.l, X, ldx, g.xs, X, ldx, g.xs, e);
+                o.a_tr = o.b_tr = q.tr;
+                ops.push_back(o);
+            }
         }
         muon_status st = R.run(ops, {});
         if (st != MUON_OK) return st;
@@ -301,17 +341,28 @@ muon_status run_direct(Runner& R, const GroupList& gs, void* ws, const double* s
         // X' = pre B' X   (and 1/(|M|+eps) at the first step); on the last
         // step the result goes to the caller (FIN_OUT) or into W (FIN_WUPD).
         ops.clear();
-        for (const Group* gp : gs) {
-            const Group& g = *gp;
-            const int cnt = (int)g.members.size();
-            const long long sx = (long long)g.s * g.ldl, ss = (long long)g.s * g.lds;
-            Epilogue e = epi_store(at(ws, g.x[cur ^ 1]), g.ldl, sx);
-            e.sc_mul = pre;
-            if (first && !R.prenorm) { e.sumsq = sumsq + g.sumsq0; e.eps = sch->eps; e.sc_pow = 1; }
-            if (last) e.check = sumsq + g.sumsq0;
-            ops.push_back(upd_op(cnt, g.s, g.l, at(ws, g.sq[1]), g.lds, ss, at(ws, g.x[cur]), g.ldl, sx, e));
+        FinalTables op_fins;
+        for (size_t gi = 0; gi < gs.size(); ++gi) {
+            const Group& g = *gs[gi];
+            const long long ss = (long long)g.s * g.lds;
+            for (const Part& q : parts(g)) {
+                Epilogue e = epi_store(static_cast<char*>(at(ws, g.x[cur ^ 1])) + (size_t)q.first * g.xs * esz,
+                                       g.ldl, g.xs);
+                e.sc_mul = pre;
+                if (first && !R.prenorm) { e.sumsq = sumsq + g.sumsq0 + q.first; e.eps = sch->eps; e.sc_pow = 1; }
+                if (last) e.check = sumsq + g.sumsq0 + q.first;
+                const void* B = static_cast<char*>(at(ws, g.sq[1])) + (size_t)q.first * ss * esz;
+                const void* X = static_cast<char*>(at(ws, g.x[cur])) + (size_t)q.first * g.xs * esz;
+                GemmOp o = upd_op(q.count, g.s, g.l, B, g.lds, ss, X, q.tr ? g.lds : g.ldl, g.xs, e);
+                o.b_tr = q.tr;
+                ops.push_back(o);
+                if (last && final_kind == FIN_WUPD)
+                    op_fins.emplace_back(fins[gi].begin() + q.first, fins[gi].begin() + q.first + q.count);
+                else
+                    op_fins.emplace_back();
+            }
         }
-        st = last ? run_final(R, ops, fins, final_kind) : R.run(ops, {});
+        st = last ? run_final(R, ops, op_fins, final_kind) : R.run(ops, {});
         if (st != MUON_OK) return st;
         cur ^= 1;
     }
@@ -335,7 +386,7 @@ muon_status run_gram(Runner& R, const GroupList& gs, void* ws, const double* sum
     auto sq = [&](const Group& g, int i) { return at(ws, g.sq[i]); };
     auto xbuf = [&](const Group& g, int i) { return at(ws, g.x[i]); };
     auto strides = [](const Group& g, long long& sx, long long& ss) {
-        sx = (long long)g.s * g.ldl;
+        sx = g.xs;
         ss = (long long)g.s * g.lds;
     };
     // one symmetric s x s product per group: D = A B^T (A, B, D given as buffer roles)
@@ -547,9 +598,11 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
                 PrepEntry& E = pp.e[pp.n++];
                 E.G = p.G; E.Gp = p.G_prev; E.A = p.A; E.M = p.M;
                 E.rows = p.rows; E.cols = p.cols; E.count = 1;
-                E.transposed = p.rows > p.cols;
-                E.X0 = static_cast<char*>(at(workspace, g.x[0])) + j * (size_t)g.s * g.ldl * dt_size(g.x0_dt);
-                E.ld = g.ldl;
+                // wide copy (a taller member transposed), or the member's own orientation
+                const bool own = g.param_tr && p.rows > p.cols;
+                E.transposed = p.rows > p.cols && !own;
+                E.X0 = static_cast<char*>(at(workspace, g.x[0])) + j * (size_t)g.xs * dt_size(g.x0_dt);
+                E.ld = own ? g.lds : g.ldl;
                 E.sumsq_index = g.sumsq0 + (int)j;
                 const uintptr_t al = reinterpret_cast<uintptr_t>(p.G) | reinterpret_cast<uintptr_t>(p.G_prev) |
                                      reinterpret_cast<uintptr_t>(p.A) | reinterpret_cast<uintptr_t>(p.M);
@@ -597,8 +650,8 @@ static muon_status step_common(const muon_param* params, int n, muon_dtype w_dty
         for (const Group& g : L.groups) {
             if (!g.gram) continue;
             PrepEntry& E = pp.e[pp.n++];
-            E.X = at(workspace, g.x[0]); E.x_stride = (long long)g.s * g.ldl;
-            E.X0 = at(workspace, g.x[1]); E.x0_stride = (long long)g.s * g.ldl; E.ld = g.ldl;
+            E.X = at(workspace, g.x[0]); E.x_stride = g.xs;
+            E.X0 = at(workspace, g.x[1]); E.x0_stride = g.xs; E.ld = g.ldl;
             E.rows = g.s; E.cols = (int)g.ldl; E.count = (int)g.members.size(); E.transposed = 0;
             E.sumsq_index = g.sumsq0;
             E.vec_ok = 1;             // rows of ldl elements (a multiple of 8), 1024-byte aligned buffers
@@ -755,7 +808,7 @@ static muon_status polar_common(int route, const void* X_in, void* X_out, int ba
     pp.in_dt = dtype; pp.x0_dt = it_dt; pp.mode = 1; pp.sumsq = sumsq; pp.n = 1; pp.eps = sched->eps;
     PrepEntry& E = pp.e[0];
     E.X = X_in; E.x_stride = batch_stride;
-    E.X0 = at(workspace, g.x[0]); E.x0_stride = (long long)g.s * g.ldl; E.ld = g.ldl;
+    E.X0 = at(workspace, g.x[0]); E.x0_stride = g.xs; E.ld = g.ldl;
     E.rows = rows; E.cols = cols; E.count = batch; E.transposed = rows > cols;
     E.sumsq_index = 0;
     E.vec_ok = (cols % 8 == 0) && (batch_stride % 8 == 0) && (reinterpret_cast<uintptr_t>(X_in) & 15) == 0;
