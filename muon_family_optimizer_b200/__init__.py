@@ -18,7 +18,8 @@ import math
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmuon_b200.so")
+# the library next to this file; MUON_B200_LIB names another build of it (A/B comparisons)
+LIB_PATH = os.environ.get("MUON_B200_LIB") or os.path.join(_HERE, "libmuon_b200.so")
 
 BF16, FP16, FP32 = 0, 1, 2
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_NONFINITE, ERR_CUDA, ERR_TIMEOUT = range(7)

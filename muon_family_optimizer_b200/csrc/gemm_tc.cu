@@ -659,23 +659,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
                 const bool one_panel = !B_MN && P.same_ab && ti == tj;   // B read from the A panel
+                // Operand layouts of the tile, decided once: A (and a symmetric B) blocks left
+                // of the diagonal block kb_a (kb_b) are read transposed; a transposed operand
+                // is read transposed throughout.  The per-k-block work of this single issuing
+                // thread stays a few integer operations per MMA.
+                const int kb_a = P.a_tr ? nkb : (P.a_sym ? (PAIR ? 2 * ti : ti) * 2 : 0);
+                const int kb_b = B_MN ? (P.b_tr ? 0 : nkb) : (P.b_tr ? nkb : (P.b_sym ? (PAIR ? 2 * tj : tj) * 2 : 0));
+                // shared-memory descriptors of a stage's first slice (address field added per stage),
+                // and the step from one 16-deep slice to the next, in 16-byte units:
+                // K-major 32 bytes further in each swizzled 128-byte row; MN-major 16 rows
+                // of 128 bytes further, 64-element MN chunks 64 x BK x 2 bytes apart
+                const uint64_t desc_k = smem_desc_sw128(0, 16, 1024), desc_mn = smem_desc_sw128(0, 64 * BK * 2, 1024);
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, abort_flag, d_status)) { ok = false; break; }
                     tc_fence_after();
-                    const bool at = P.a_tr || (P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti));   // A block read transposed
-                    const bool bm = B_MN ? !P.b_tr : (P.b_tr || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj)));   // B block MN-major
+                    const bool at = kb < kb_a;     // A block read transposed
+                    const bool bm = kb < kb_b;     // B block MN-major
                     const uint32_t idesc = idesc0 | (at ? 1u << 15 : 0u) | (bm ? 1u << 16 : 0u);
                     const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t sb = one_panel ? sa : sa + C::kABytes;
+                    const uint64_t ad0 = (at ? desc_mn : desc_k) | (uint64_t)((sa >> 4) & 0x3FFFu);
+                    const uint64_t bd0 = (bm ? desc_mn : desc_k) | (uint64_t)((sb >> 4) & 0x3FFFu);
+                    const uint64_t a_step = at ? 2048 >> 4 : 32 >> 4, b_step = bm ? 2048 >> 4 : 32 >> 4;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        // K-major: the k-th 16-element slice sits 32 bytes further in each
-                        // swizzled 128-byte row; MN-major: 16 rows of 128 bytes further,
-                        // 64-element MN chunks 64 x BK x 2 bytes apart.
-                        const uint64_t ad = at ? smem_desc_sw128(sa + k * 2048, 64 * BK * 2, 1024)
-                                               : smem_desc_sw128(sa + k * 32, 16, 1024);
-                        const uint64_t bd = bm ? smem_desc_sw128(sb + k * 2048, 64 * BK * 2, 1024)
-                                               : smem_desc_sw128(sb + k * 32, 16, 1024);
+                        const uint64_t ad = ad0 + (uint64_t)k * a_step, bd = bd0 + (uint64_t)k * b_step;
                         if (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
                         else tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
                     }

@@ -223,28 +223,39 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
         unsigned char* gs = sm + s * kStage;
         float* ms = reinterpret_cast<float*>(gs + kGBytes);
         const float* os = reinterpret_cast<const float*>(gs + kGBytes + kMBytes);
-        // momentum: M <- mu M + G, back to global memory and kept for the product
+        // momentum: M <- mu M + G, back to global memory and kept for the product;
+        // 4 consecutive elements per thread, so a warp's 16-byte accesses are
+        // consecutive in shared memory
 #pragma unroll
-        for (int it = 0; it < kSkRows * kSkCols / (8 * kThreads); ++it) {
+        for (int it = 0; it < kSkRows * kSkCols / (4 * kThreads); ++it) {
             const int q = threadIdx.x + kThreads * it;
-            const int rr = q / (kSkCols / 8), cc = (q % (kSkCols / 8)) * 8;
+            const int rr = q / (kSkCols / 4), cc = (q % (kSkCols / 4)) * 4;
             const int i = row0 + rr, j = c0 + cc;
-            float g[8], m[8];
-            load8_dt(gs, rr * kSkCols + cc, G_DT, true, 8, g);
-            float4* mp = reinterpret_cast<float4*>(ms + rr * kSkLd + cc);
-            const float4 m0 = mp[0], m1 = mp[1];
-            m[0] = m0.x; m[1] = m0.y; m[2] = m0.z; m[3] = m0.w;
-            m[4] = m1.x; m[5] = m1.y; m[6] = m1.z; m[7] = m1.w;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                m[e] = fmaf(p.mu, m[e], g[e]);   // zero outside the matrix
-                bad |= !isfinite(m[e]);
+            float g[4];
+            if (GSZ == 2) {
+                const uint2 u = *reinterpret_cast<const uint2*>(gs + (rr * kSkCols + cc) * 2);
+                using T = typename std::conditional<G_DT == DT_BF16, __nv_bfloat16, __half>::type;
+                g[0] = unpack_lo<T>(u.x); g[1] = unpack_hi<T>(u.x); g[2] = unpack_lo<T>(u.y); g[3] = unpack_hi<T>(u.y);
+            } else {
+                const float4 u = *reinterpret_cast<const float4*>(gs + (rr * kSkCols + cc) * 4);
+                g[0] = u.x; g[1] = u.y; g[2] = u.z; g[3] = u.w;
             }
-            mp[0] = make_float4(m[0], m[1], m[2], m[3]);
-            mp[1] = make_float4(m[4], m[5], m[6], m[7]);
+            float4* mp = reinterpret_cast<float4*>(ms + rr * kSkLd + cc);
+            float4 m = *mp;
+            m.x = fmaf(p.mu, m.x, g[0]);      // zero outside the matrix
+            m.y = fmaf(p.mu, m.y, g[1]);
+            m.z = fmaf(p.mu, m.z, g[2]);
+            m.w = fmaf(p.mu, m.w, g[3]);
+            bad |= !isfinite(m.x) || !isfinite(m.y) || !isfinite(m.z) || !isfinite(m.w);
+            *mp = m;
             if (i < E.rows && j < E.cols) {
-                const int nvalid = min(8, E.cols - j);
-                store8_dt(E.M, (long long)i * E.cols + j, DT_FP32, E.vec_ok != 0, nvalid, m);
+                float* dst = E.M + (long long)i * E.cols + j;
+                if (E.vec_ok) {
+                    *reinterpret_cast<float4*>(dst) = m;
+                } else {
+                    const float mv[4] = {m.x, m.y, m.z, m.w};
+                    for (int e = 0; e < 4 && j + e < E.cols; ++e) dst[e] = mv[e];
+                }
             }
         }
         __syncthreads();
@@ -475,10 +486,11 @@ __global__ void __launch_bounds__(kThreads, 3) lim_project(const __grid_constant
 // ---------------------------------------------------------------------------
 template <int KT>
 __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimParams p) {
+    constexpr int LD = KT + 1;          // padded rows: a column of C spreads over the banks
     extern __shared__ __align__(16) double dsm[];
-    double* C = dsm;                    // [KT][KT]
-    double* Ev = dsm + KT * KT;         // [KT][KT] eigenvectors (columns)
-    double* cs = Ev + KT * KT;          // [KT/2] cosines
+    double* C = dsm;                    // [KT][LD]
+    double* Ev = dsm + KT * LD;         // [KT][LD] eigenvectors (columns)
+    double* cs = Ev + KT * LD;          // [KT/2] cosines
     double* sn = cs + KT / 2;           // [KT/2] sines
     double* lam = sn + KT / 2;          // [KT] eigenvalues
     int* pp = reinterpret_cast<int*>(lam + KT);   // [KT/2]
@@ -492,8 +504,8 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
         const int a = idx / KT, b = idx % KT;
         const double v = (a < k && b < k) ? (a <= b ? E.Cg[a * KT + b] : E.Cg[b * KT + a]) : 0.0;
         if (!isfinite(v)) nonfinite = 1;
-        C[idx] = v;
-        Ev[idx] = a == b ? 1.0 : 0.0;
+        C[a * LD + b] = v;
+        Ev[a * LD + b] = a == b ? 1.0 : 0.0;
     }
     __syncthreads();
     if (nonfinite || *E.bad) {          // no factor for a marked matrix: its W is kept
@@ -505,7 +517,7 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
     // noise, not coupling: below 0.1 kRotTol * trace no rotation is made, so a
     // pair of negligible eigenvalues cannot keep the sweeps going.
     double tr = 0.0;
-    for (int a = 0; a < k; ++a) tr += fabs(C[a * KT + a]);
+    for (int a = 0; a < k; ++a) tr += fabs(C[a * LD + a]);
     const double floor_abs = kRotTol * 0.1 * tr;
     for (int sweep = 0; sweep < kMaxSweeps && n > 0; ++sweep) {
         if (threadIdx.x == 0) rotated = 0;
@@ -515,7 +527,7 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
                 const int i = threadIdx.x;
                 int a = i == 0 ? n : (rd + i) % n, b = i == 0 ? rd : (rd - i + n) % n;
                 if (a > b) { const int t = a; a = b; b = t; }
-                const double apq = C[a * KT + b], app = C[a * KT + a], aqq = C[b * KT + b];
+                const double apq = C[a * LD + b], app = C[a * LD + a], aqq = C[b * LD + b];
                 double c = 1.0, s = 0.0;
                 if (fabs(apq) > kRotTol * sqrt(fabs(app * aqq)) && fabs(apq) > floor_abs) {
                     const double tau = (aqq - app) / (2.0 * apq);
@@ -532,21 +544,21 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
                 const double c1 = cs[i], s1 = sn[i], c2 = cs[j], s2 = sn[j];
                 if (s1 == 0.0 && s2 == 0.0) continue;
                 const int a1 = pp[i], b1 = pq[i], a2 = pp[j], b2 = pq[j];
-                const double x = C[a1 * KT + a2], y = C[a1 * KT + b2], z = C[b1 * KT + a2], w = C[b1 * KT + b2];
+                const double x = C[a1 * LD + a2], y = C[a1 * LD + b2], z = C[b1 * LD + a2], w = C[b1 * LD + b2];
                 const double r0 = c1 * x - s1 * z, r1 = c1 * y - s1 * w;   // rows a1, b1 rotated
                 const double r2 = s1 * x + c1 * z, r3 = s1 * y + c1 * w;
-                C[a1 * KT + a2] = c2 * r0 - s2 * r1;                      // then columns a2, b2
-                C[a1 * KT + b2] = s2 * r0 + c2 * r1;
-                C[b1 * KT + a2] = c2 * r2 - s2 * r3;
-                C[b1 * KT + b2] = s2 * r2 + c2 * r3;
+                C[a1 * LD + a2] = c2 * r0 - s2 * r1;                      // then columns a2, b2
+                C[a1 * LD + b2] = s2 * r0 + c2 * r1;
+                C[b1 * LD + a2] = c2 * r2 - s2 * r3;
+                C[b1 * LD + b2] = s2 * r2 + c2 * r3;
             }
             for (int idx = threadIdx.x; idx < ke * np; idx += blockDim.x) {   // E <- E J
                 const int row = idx / np, i = idx % np;
                 const double c = cs[i], s = sn[i];
                 if (s == 0.0) continue;
-                const double u = Ev[row * KT + pp[i]], v = Ev[row * KT + pq[i]];
-                Ev[row * KT + pp[i]] = c * u - s * v;
-                Ev[row * KT + pq[i]] = s * u + c * v;
+                const double u = Ev[row * LD + pp[i]], v = Ev[row * LD + pq[i]];
+                Ev[row * LD + pp[i]] = c * u - s * v;
+                Ev[row * LD + pq[i]] = s * u + c * v;
             }
             __syncthreads();
         }
@@ -555,7 +567,7 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
         if (!again) break;                     // a sweep without a rotation: converged
     }
     // the r largest eigenvalues above kTau2 * largest: weights 1 / sqrt(lambda)
-    if (threadIdx.x < k) lam[threadIdx.x] = C[threadIdx.x * KT + threadIdx.x];
+    if (threadIdx.x < k) lam[threadIdx.x] = C[threadIdx.x * LD + threadIdx.x];
     __syncthreads();
     double lmax = 0.0;
     for (int a = 0; a < k; ++a) lmax = fmax(lmax, lam[a]);
@@ -573,7 +585,7 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
         const int a = idx / KT, b = idx % KT;
         double s = 0.0;
         if (a < k && b < k)
-            for (int e = 0; e < k; ++e) s += Ev[a * KT + e] * wgt[e] * Ev[b * KT + e];
+            for (int e = 0; e < k; ++e) s += Ev[a * LD + e] * wgt[e] * Ev[b * LD + e];
         E.K[idx] = s;
     }
 }
@@ -616,36 +628,60 @@ __device__ __forceinline__ void store4_w(void* base, long long idx, bool vec, in
         if (c < nvalid) st_elem(base, idx + c, W_DT, v[c]);
 }
 
+// Shared memory of lim_update: Z rows [kUpRows][KT], B [KT][kBsLd] (the tile's
+// columns of B = (B^T)^T), the B^T tile as loaded [kUpCols][KT], and the
+// tile of W [kUpRows][kUpCols] in W's type.
 template <int KT>
-__host__ __device__ constexpr int update_smem_floats() { return kUpRows * KT + KT * kBsLd; }
+__host__ __device__ constexpr int update_smem_floats() { return kUpRows * KT + KT * kBsLd + kUpCols * KT; }
+
+template <int KT, int W_DT>
+__host__ __device__ constexpr int update_smem_bytes() {
+    return update_smem_floats<KT>() * 4 + kUpRows * kUpCols * g_size<W_DT>();
+}
 
 template <int KT, int W_DT>
 __global__ void __launch_bounds__(kThreads, 2) lim_update(const __grid_constant__ LimParams p) {
+    constexpr int WSZ = g_size<W_DT>();
     extern __shared__ __align__(16) float fsm[];
     float* Zs = fsm;                           // [kUpRows][KT]
-    float* Bs = fsm + kUpRows * KT;            // [KT][kBsLd]: B = (B^T)^T, this tile's columns
+    float* Bs = Zs + kUpRows * KT;             // [KT][kBsLd]
+    float* Bts = Bs + KT * kBsLd;              // [kUpCols][KT]
+    unsigned char* Ws = reinterpret_cast<unsigned char*>(Bts + kUpCols * KT);   // [kUpRows][kUpCols]
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 3)];
     const int tile = blockIdx.x - E.t_upd;
     const int tiles_c = (E.cols + kUpCols - 1) / kUpCols;
     const int row0 = (tile / tiles_c) * kUpRows, c0 = (tile % tiles_c) * kUpCols;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool skip = *E.bad != 0;
+    // every global read of the tile in one asynchronous group: Z rows, the
+    // B^T rows of the tile's columns, and (aligned rows) the tile of W
     constexpr int ZP = KT / 4;
     for (int q = threadIdx.x; q < kUpRows * ZP; q += kThreads) {
         const int rr = q / ZP, pc = q % ZP, i = row0 + rr;
         const bool in = i < E.rows;
         cp_async16(Zs + rr * KT + pc * 4, E.Y + (in ? (long long)i * KT + pc * 4 : 0), in ? 16u : 0u);
     }
-    cp_async_commit();
     for (int q = threadIdx.x; q < kUpCols * ZP; q += kThreads) {
-        const int jj = q % kUpCols, t4 = q / kUpCols, j = c0 + jj;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (j < E.cols) v = *reinterpret_cast<const float4*>(E.Bt + (long long)j * KT + 4 * t4);
-        Bs[(4 * t4 + 0) * kBsLd + jj] = v.x;
-        Bs[(4 * t4 + 1) * kBsLd + jj] = v.y;
-        Bs[(4 * t4 + 2) * kBsLd + jj] = v.z;
-        Bs[(4 * t4 + 3) * kBsLd + jj] = v.w;
+        const int jj = q / ZP, pc = q % ZP, j = c0 + jj;
+        const bool in = j < E.cols;
+        cp_async16(Bts + jj * KT + pc * 4, E.Bt + (in ? (long long)j * KT + pc * 4 : 0), in ? 16u : 0u);
     }
+    if (E.vec_ok && !skip) {
+        constexpr int WP = kUpCols * WSZ / 16, WE = 16 / WSZ;   // 16-byte pieces per row, elements per piece
+        for (int q = threadIdx.x; q < kUpRows * WP; q += kThreads) {
+            const int rr = q / WP, pc = q % WP, i = row0 + rr, j = c0 + pc * WE;
+            const bool in = i < E.rows && j < E.cols;
+            const char* src = static_cast<const char*>(E.W) + (in ? ((long long)i * E.cols + j) * WSZ : 0);
+            cp_async16(Ws + (rr * kUpCols + pc * WE) * WSZ, src, in ? 16u : 0u);
+        }
+    }
+    cp_async_commit();
     cp_async_wait<0>();
+    __syncthreads();
+    for (int q = threadIdx.x; q < kUpCols * KT; q += kThreads) {   // B = (B^T)^T, shared to shared
+        const int t = q % KT, jj = q / KT;
+        Bs[t * kBsLd + jj] = Bts[jj * KT + t];
+    }
     __syncthreads();
     float o[16][4];
 #pragma unroll
@@ -671,14 +707,13 @@ __global__ void __launch_bounds__(kThreads, 2) lim_update(const __grid_constant_
             }
         }
     }
-    const bool skip = *E.bad != 0;
     const int j = c0 + 4 * lane;
     if (j >= E.cols) return;
     const int nvalid = min(4, E.cols - j);
     const bool vec = E.vec_ok && nvalid == 4;
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-        const int i = row0 + 16 * warp + r;
+        const int rr = 16 * warp + r, i = row0 + rr;
         if (i >= E.rows) break;
         const long long idx = (long long)i * E.cols + j;
         if (E.O_out) {
@@ -688,7 +723,8 @@ __global__ void __launch_bounds__(kThreads, 2) lim_update(const __grid_constant_
         }
         if (skip) continue;
         float w[4];
-        load4_w<W_DT>(E.W, idx, vec, nvalid, w);
+        if (vec) load4_w<W_DT>(Ws, (long long)rr * kUpCols + 4 * lane, true, 4, w);   // staged
+        else load4_w<W_DT>(E.W, idx, false, nvalid, w);
 #pragma unroll
         for (int c = 0; c < 4; ++c) w[c] = w[c] - p.eta * (E.gamma * o[r][c] + p.lambda * w[c]);
         store4_w<W_DT>(E.W, idx, vec, nvalid, w);
@@ -704,12 +740,12 @@ template <int KT, int G_DT>
 constexpr size_t sketch_smem() { return 2 * (size_t)sketch_stage_bytes<KT, G_DT>(); }
 template <int KT>
 constexpr size_t project_smem() { return sizeof(float) * kPjStages * project_stage_floats<KT>(); }
-template <int KT>
-constexpr size_t update_smem() { return sizeof(float) * update_smem_floats<KT>(); }
+template <int KT, int W_DT>
+constexpr size_t update_smem() { return (size_t)update_smem_bytes<KT, W_DT>(); }
 template <int KT>
 constexpr size_t chol_smem() { return sizeof(double) * (2 * KT * KT + KT) + sizeof(int) * KT; }
 template <int KT>
-constexpr size_t eig_smem() { return sizeof(double) * (2 * KT * KT + KT / 2 * 2 + KT) + sizeof(int) * KT; }
+constexpr size_t eig_smem() { return sizeof(double) * (2 * KT * (KT + 1) + KT / 2 * 2 + KT) + sizeof(int) * KT; }
 
 static_assert(sketch_smem<64, DT_FP32>() >= sizeof(float) * kSkRows * 64, "sketch Y staging fits a stage");
 static_assert(project_smem<64>() >= sizeof(float) * kPjCols * 64, "projection B^T staging fits the stages");
@@ -740,7 +776,7 @@ muon_status launch_all(LimParams& prm, cudaStream_t s, const LaunchShape& L) {
                                 allow_smem(lim_chol<KT>, chol_smem<KT>()),
                                 allow_smem(lim_project<KT>, project_smem<KT>()),
                                 allow_smem(lim_eig<KT>, eig_smem<KT>()),
-                                allow_smem(lim_update<KT, W_DT>, update_smem<KT>())};
+                                allow_smem(lim_update<KT, W_DT>, update_smem<KT, W_DT>())};
             for (cudaError_t x : e)
                 if (x != cudaSuccess) return MUON_ERR_CUDA;
             configured[dev] = true;
@@ -767,7 +803,7 @@ muon_status launch_all(LimParams& prm, cudaStream_t s, const LaunchShape& L) {
     lim_rowmul<KT><<<L.rows, kThreads, 0, s>>>(prm);
     trace_end(s);
     trace_begin(MUON_KERNEL_RSVD, L.elems * 2.0 * wsz + 4.0 * (L.rows_k + L.cols_k), s);   // W read and written
-    lim_update<KT, W_DT><<<L.upd, kThreads, update_smem<KT>(), s>>>(prm);
+    lim_update<KT, W_DT><<<L.upd, kThreads, update_smem<KT, W_DT>(), s>>>(prm);
     trace_end(s);
     (void)k;
     return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
