@@ -492,7 +492,11 @@ __device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int cb0, 
     }
 }
 
-template <int BN, bool B_MN, bool PAIR, bool FIN, typename T>
+// TRX: the launch may hold operands stored transposed in full (the first step
+// of an optimizer step); without it the operand layouts of every k-block are
+// compile-time or per-problem symmetric-storage decisions only, which keeps
+// the single MMA-issuing thread's work per instruction minimal.
+template <int BN, bool B_MN, bool PAIR, bool FIN, bool TRX, typename T>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
     static_assert(!PAIR || BN == 256, "CTA pairs compute 256 x 256 tiles");
     static_assert(!FIN || B_MN, "the final step is an update product");
@@ -531,8 +535,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     }
     if (warp == 0 && lane == 0) {
         for (int i = 0; i < p.nprob; ++i) {
-            prefetch_tensormap(p.prob[i].a_tr ? &p.prob[i].mapAt : &p.prob[i].mapA);
-            prefetch_tensormap(p.prob[i].sym && p.prob[i].b_tr ? &p.prob[i].mapBt : &p.prob[i].mapB);
+            prefetch_tensormap(TRX && p.prob[i].a_tr ? &p.prob[i].mapAt : &p.prob[i].mapA);
+            prefetch_tensormap(TRX && p.prob[i].sym && p.prob[i].b_tr ? &p.prob[i].mapBt : &p.prob[i].mapB);
         }
     }
     if (warp == 1) {
@@ -574,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 // S S) needs the same rows as A and as B: one panel serves both.
                 const bool one_panel = !B_MN && P.same_ab && ti == tj;
                 // an update product whose X is stored transposed loads whole K-major boxes
-                const bool b_kmaj = B_MN && P.b_tr;
+                const bool b_kmaj = B_MN && TRX && P.b_tr;
                 uint32_t bytes = C::kABytes + (B_MN ? (b_kmaj ? C::kBBytes : nchunk * 64 * BK * 2)
                                                     : (one_panel ? 0 : C::kBBytes));
                 if (PAIR) {   // the leader's barrier counts both CTAs' boxes
@@ -591,8 +595,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     // decision is taken on the pair's first 128-row (128-column) block,
                     // so both halves agree (such operands also store the first tile
                     // below the diagonal).
-                    const bool at = P.a_tr || (P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti));
-                    const bool bt = !B_MN && (P.b_tr || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj)));
+                    const bool at = (TRX && P.a_tr) || (P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti));
+                    const bool bt = !B_MN && ((TRX && P.b_tr) || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj)));
                     const uint32_t fb = PAIR ? mapa_shared(smem_u32(&full_bar[stage]), 0) : 0u;
                     auto load = [&](const CUtensorMap* map, void* dst, int x, int y) {
                         if (PAIR) tma_load_3d_pair(map, fb, dst, x, y, m);
@@ -659,31 +663,26 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
                 const bool one_panel = !B_MN && P.same_ab && ti == tj;   // B read from the A panel
-                // Operand layouts of the tile, decided once: A (and a symmetric B) blocks left
-                // of the diagonal block kb_a (kb_b) are read transposed; a transposed operand
-                // is read transposed throughout.  The per-k-block work of this single issuing
-                // thread stays a few integer operations per MMA.
-                const int kb_a = P.a_tr ? nkb : (P.a_sym ? (PAIR ? 2 * ti : ti) * 2 : 0);
-                const int kb_b = B_MN ? (P.b_tr ? 0 : nkb) : (P.b_tr ? nkb : (P.b_sym ? (PAIR ? 2 * tj : tj) * 2 : 0));
-                // shared-memory descriptors of a stage's first slice (address field added per stage),
-                // and the step from one 16-deep slice to the next, in 16-byte units:
-                // K-major 32 bytes further in each swizzled 128-byte row; MN-major 16 rows
-                // of 128 bytes further, 64-element MN chunks 64 x BK x 2 bytes apart
-                const uint64_t desc_k = smem_desc_sw128(0, 16, 1024), desc_mn = smem_desc_sw128(0, 64 * BK * 2, 1024);
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, abort_flag, d_status)) { ok = false; break; }
                     tc_fence_after();
-                    const bool at = kb < kb_a;     // A block read transposed
-                    const bool bm = kb < kb_b;     // B block MN-major
+                    // A block read transposed; B block MN-major (an update product's X panel
+                    // always, unless stored transposed in full)
+                    const bool at = (TRX && P.a_tr) || (P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti));
+                    const bool bm = B_MN ? !(TRX && P.b_tr)
+                                         : ((TRX && P.b_tr) || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj)));
                     const uint32_t idesc = idesc0 | (at ? 1u << 15 : 0u) | (bm ? 1u << 16 : 0u);
                     const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t sb = one_panel ? sa : sa + C::kABytes;
-                    const uint64_t ad0 = (at ? desc_mn : desc_k) | (uint64_t)((sa >> 4) & 0x3FFFu);
-                    const uint64_t bd0 = (bm ? desc_mn : desc_k) | (uint64_t)((sb >> 4) & 0x3FFFu);
-                    const uint64_t a_step = at ? 2048 >> 4 : 32 >> 4, b_step = bm ? 2048 >> 4 : 32 >> 4;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        const uint64_t ad = ad0 + (uint64_t)k * a_step, bd = bd0 + (uint64_t)k * b_step;
+                        // K-major: the k-th 16-element slice sits 32 bytes further in each
+                        // swizzled 128-byte row; MN-major: 16 rows of 128 bytes further,
+                        // 64-element MN chunks 64 x BK x 2 bytes apart.
+                        const uint64_t ad = at ? smem_desc_sw128(sa + k * 2048, 64 * BK * 2, 1024)
+                                               : smem_desc_sw128(sa + k * 32, 16, 1024);
+                        const uint64_t bd = bm ? smem_desc_sw128(sb + k * 2048, 64 * BK * 2, 1024)
+                                               : smem_desc_sw128(sb + k * 32, 16, 1024);
                         if (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
                         else tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
                     }
@@ -988,10 +987,10 @@ static bool encode_map(CUtensorMap* map, int dt, const void* base, long long inn
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool B_MN, bool PAIR, bool FIN, typename T>
+template <int BN, bool B_MN, bool PAIR, bool FIN, bool TRX, typename T>
 static cudaError_t launch_one(const TcParams& prm, int grid, cudaStream_t stream) {
     using C = Cfg<BN, PAIR, B_MN, FIN>;
-    auto kern = tc_gemm_kernel<BN, B_MN, PAIR, FIN, T>;
+    auto kern = tc_gemm_kernel<BN, B_MN, PAIR, FIN, TRX, T>;
     static thread_local int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1109,21 +1108,26 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
     trace_begin(sym ? MUON_KERNEL_SYM : MUON_KERNEL_UPD, work, stream);
     cudaError_t e;
     const bool final_step = ops[0].epi.fin != FIN_STORE;
+    bool any_tr = false;
+    for (int i = 0; i < nops; ++i) any_tr |= ops[i].a_tr || ops[i].b_tr;
+    // one instantiation per product kind, CTA-pair mode, operand layouts and element type
+#define MUON_TC_LAUNCH(TRX, T)                                                                         \
+    do {                                                                                               \
+        if (sym) e = pair ? launch_one<256, false, true, false, TRX, T>(prm, grid, stream)             \
+                          : launch_one<128, false, false, false, TRX, T>(prm, grid, stream);           \
+        else if (final_step) e = pair ? launch_one<256, true, true, true, TRX, T>(prm, grid, stream)   \
+                               : launch_one<256, true, false, true, TRX, T>(prm, grid, stream);        \
+        else e = pair ? launch_one<256, true, true, false, TRX, T>(prm, grid, stream)                  \
+                      : launch_one<256, true, false, false, TRX, T>(prm, grid, stream);                \
+    } while (0)
     if (dt == DT_BF16) {
-        if (sym) e = pair ? launch_one<256, false, true, false, __nv_bfloat16>(prm, grid, stream)
-                          : launch_one<128, false, false, false, __nv_bfloat16>(prm, grid, stream);
-        else if (final_step) e = pair ? launch_one<256, true, true, true, __nv_bfloat16>(prm, grid, stream)
-                               : launch_one<256, true, false, true, __nv_bfloat16>(prm, grid, stream);
-        else e = pair ? launch_one<256, true, true, false, __nv_bfloat16>(prm, grid, stream)
-                      : launch_one<256, true, false, false, __nv_bfloat16>(prm, grid, stream);
+        if (any_tr) MUON_TC_LAUNCH(true, __nv_bfloat16);
+        else MUON_TC_LAUNCH(false, __nv_bfloat16);
     } else {
-        if (sym) e = pair ? launch_one<256, false, true, false, __half>(prm, grid, stream)
-                          : launch_one<128, false, false, false, __half>(prm, grid, stream);
-        else if (final_step) e = pair ? launch_one<256, true, true, true, __half>(prm, grid, stream)
-                               : launch_one<256, true, false, true, __half>(prm, grid, stream);
-        else e = pair ? launch_one<256, true, true, false, __half>(prm, grid, stream)
-                      : launch_one<256, true, false, false, __half>(prm, grid, stream);
+        if (any_tr) MUON_TC_LAUNCH(true, __half);
+        else MUON_TC_LAUNCH(false, __half);
     }
+#undef MUON_TC_LAUNCH
     trace_end(stream);
     return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
