@@ -15,7 +15,8 @@
 // and Q = Y R^-1 with Y^T Y = R^T R (Cholesky QR).  Every pass over an l x s
 // array streams; everything per matrix touches only k x k data:
 //   1 lim_sketch   M <- mu M + G and Y = M Omega, 64-row blocks over 64-column
-//                  chunks double-buffered in shared memory (cp.async); each
+//                  chunks double-buffered in shared memory (cp.async), the
+//                  product on tensor cores (tf32 x 3, fp32 accuracy); each
 //                  block adds its rows' share of the Gram Y^T Y (fp64) to the
 //                  matrix's k x k sum.  Reads G and M, writes M.
 //   2 lim_chol     per matrix (k x k): Cholesky of Y^T Y in fp64 (a column whose
@@ -24,16 +25,19 @@
 //   3 lim_rowmul   Q = Y R^-1, row by row in place (fp64 sums), all matrices'
 //                  rows in one grid.
 //   4 lim_project  B^T = M^T Q, 128-column blocks over 32-row chunks (three
-//                  cp.async stages); each block adds its columns' share of
-//                  B B^T (fp64) to the matrix's k x k sum.  Reads M.
+//                  cp.async stages), tensor cores as in 1; each block adds its
+//                  columns' share of B B^T (fp64) to the matrix's k x k sum.
+//                  Reads M.
 //   5 lim_eig      per matrix (k x k): cyclic Jacobi on B B^T in fp64,
 //                  round-robin order (k/2 disjoint rotations per round), a
 //                  rotation only while |C_pq| > 1e-15 sqrt(C_pp C_qq) (and
 //                  above 1e-16 of the trace: fp64 noise), stop after a sweep
 //                  without one; P from the r largest eigenpairs.
 //   6 lim_rowmul   Z = Q P in place.
-//   7 lim_update   O = Z B on 128 x 128 tiles, fused with the weight update
-//                  (reads and writes W; O never stored unless O_out is given).
+//   7 lim_update   O = Z B on 128 x 128 tiles (tensor cores as in 1), fused
+//                  with the weight update (reads and writes W; O never stored
+//                  unless O_out is given).
+// The sketch and the projection order their blocks longest first.
 // A non-finite momentum element or k x k factor marks its matrix: its W is
 // kept and MUON_FLAG_NONFINITE raised.
 #include <algorithm>
@@ -59,7 +63,6 @@ constexpr int kPjRows = 32;       // lim_project: rows per chunk
 constexpr int kPjStages = 3;
 constexpr int kUpRows = 128;      // lim_update: tile rows
 constexpr int kUpCols = 128;      // lim_update: tile columns
-constexpr int kBsLd = kUpCols + 4;   // padded row of the staged B tile
 constexpr double kDrop = 1e-10;   // Cholesky pivot / squared column norm below which a column is dropped
 constexpr double kTau2 = 1e-10;   // (singular value / largest)^2 at or below which it counts as zero
 constexpr double kRotTol = 1e-15; // Jacobi: rotate while |C_pq| > kRotTol sqrt(C_pp C_qq)
@@ -82,22 +85,29 @@ struct LimEntry {
 
 struct LimParams {
     LimEntry e[kLimMax];
+    // order of the matrices in each launch's grid (which: 0 sketch, 1 row
+    // transforms, 2 projection, 3 update): the sketch and the projection give
+    // the matrices with the longest blocks (most columns, most rows) the first
+    // blocks, so no long block starts in the last wave
+    unsigned char ord[4][kLimMax];
     int n, k, r;
     float mu, eta, lambda;
     int* d_status;
 };
 
-// The matrix that block b of a launch works on: the last entry whose first
-// block is <= b (which: 0 sketch, 1 row transforms, 2 projection, 3 update).
+__device__ __forceinline__ int first_block(const LimEntry& e, int which) {
+    return which == 0 ? e.t_sketch : which == 1 ? e.t_rows : which == 2 ? e.t_proj : e.t_upd;
+}
+
+// The matrix that block b of a launch works on: in the launch's order, the
+// last matrix whose first block is <= b.
 __device__ __forceinline__ int find_entry(const LimParams& p, int b, int which) {
     int lo = 0, hi = p.n - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        const LimEntry& e = p.e[mid];
-        const int t = which == 0 ? e.t_sketch : which == 1 ? e.t_rows : which == 2 ? e.t_proj : e.t_upd;
-        if (t <= b) lo = mid; else hi = mid - 1;
+        if (first_block(p.e[p.ord[which][mid]], which) <= b) lo = mid; else hi = mid - 1;
     }
-    return lo;
+    return p.ord[which][lo];
 }
 
 __device__ __forceinline__ void mark_bad(const LimParams& p, const LimEntry& E) {
@@ -130,46 +140,102 @@ __device__ __forceinline__ void add_gram(const float* X, int n, int k, double* d
 }
 
 // ---------------------------------------------------------------------------
+// Tensor-core products with fp32 accuracy.  The three products with k columns
+// (Y = M Omega, B^T = M^T Q, O = Z B) run on mma.sync m16n8k8 in tf32 with
+// each operand split as x = hi + lo (hi = x rounded to tf32, lo = the
+// remainder rounded to tf32) and the product summed as hi*lo + lo*hi + hi*hi
+// into fp32 accumulators ("3xTF32"): the dropped lo*lo term and the rounding
+// of lo are below 2^-21 of |a b| per product, under the fp32 accumulation's
+// own rounding for sums of a few hundred terms or more.  At 2 k flops per
+// element these products are below the HBM ridge once on tensor cores; the
+// legacy warp-level MMA gives that rate with the fragments in registers,
+// next to the fused momentum, Gram and weight-update code.
+// Fragments of m16n8k8 (g = lane / 4, q = lane % 4): A (16 x 8) a0 = (g, q),
+// a1 = (g + 8, q), a2 = (g, q + 4), a3 = (g + 8, q + 4); B (8 x 8) b0 = (q, g),
+// b1 = (q + 4, g); C (16 x 8) c0, c1 = (g, 2q), (g, 2q + 1); c2, c3 = the same
+// columns of row g + 8.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = to_tf32(x);
+    lo = to_tf32(x - __uint_as_float(hi));
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// d += a b with a = ah + al, b = (bh0, bh1) + (bl0, bl1): small terms first.
+__device__ __forceinline__ void mma3_tf32(float (&d)[4], const uint32_t (&ah)[4], const uint32_t (&al)[4],
+                                          uint32_t bh0, uint32_t bh1, uint32_t bl0, uint32_t bl1) {
+    mma_tf32(d, ah, bl0, bl1);
+    mma_tf32(d, al, bh0, bh1);
+    mma_tf32(d, ah, bh0, bh1);
+}
+
+// ---------------------------------------------------------------------------
 // 1. momentum + sketch (+ share of Y^T Y)
 // ---------------------------------------------------------------------------
 template <int G_DT>
 __host__ __device__ constexpr int g_size() { return G_DT == DT_FP32 ? 4 : 2; }
 
-// One stage of the sketch: raw G [kSkRows][kSkCols] in its own type, M
-// [kSkRows][kSkLd] fp32 (updated in place), Omega [kSkCols][KT] fp32.
+// Shared memory of the sketch.  Two stages of raw chunks: G [kSkRows][kSkCols]
+// in its own type, M [kSkRows][kSkLd] fp32 (its tf32 high part after the
+// momentum phase, in place), Omega [kSkCols][KT] fp32.  One buffer each of the
+// chunk's M low part [kSkRows][kSkLd] and Omega's high and low parts
+// [kSkCols][KT + 8].  Row pitches 4 (M) and 8 (Omega) words past a multiple
+// of 32 make the fragment loads conflict-free.
 template <int KT, int G_DT>
-__host__ __device__ constexpr int sketch_stage_bytes() {
-    return kSkRows * kSkCols * g_size<G_DT>() + kSkRows * kSkLd * 4 + kSkCols * KT * 4;
-}
+struct SketchSmem {
+    static constexpr int kOmLd = KT + 8;
+    static constexpr int kG = kSkRows * kSkCols * g_size<G_DT>();
+    static constexpr int kM = kSkRows * kSkLd * 4;
+    static constexpr int kOm = kSkCols * KT * 4;
+    static constexpr int kStage = kG + kM + kOm;
+    static constexpr int kMlo = 2 * kStage;
+    static constexpr int kOmHi = kMlo + kSkRows * kSkLd * 4;
+    static constexpr int kOmLo = kOmHi + kSkCols * kOmLd * 4;
+    static constexpr int kBytes = kOmLo + kSkCols * kOmLd * 4;
+};
 
 template <int KT, int G_DT>
 __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant__ LimParams p) {
+    using S = SketchSmem<KT, G_DT>;
     constexpr int GSZ = g_size<G_DT>();
-    constexpr int kGBytes = kSkRows * kSkCols * GSZ;
-    constexpr int kMBytes = kSkRows * kSkLd * 4;
-    constexpr int kStage = sketch_stage_bytes<KT, G_DT>();
-    // register tile of the product: RPT rows x 4 columns of Y per thread
-    constexpr int CG = KT / 4, RG = kThreads / CG, RPT = kSkRows / RG;
-    static_assert(RPT * RG == kSkRows && RPT >= 1, "row tiling");
+    constexpr int NT = KT / 16;                // 8-column MMA tiles per warp (a warp takes half of Y's columns)
+    static_assert(kSkRows == 64 && kThreads == 256, "four 16-row MMA tiles x two column halves");
     extern __shared__ __align__(16) unsigned char sm[];
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 0)];
     const int row0 = (blockIdx.x - E.t_sketch) * kSkRows;
-    const int tx = threadIdx.x % CG, ty = threadIdx.x / CG;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q4 = lane & 3;
+    const int mt = warp & 3, n0 = (warp >> 2) * (KT / 2);   // rows 16 mt.., columns n0.. of Y
     const int nchunks = (E.cols + kSkCols - 1) / kSkCols;
     const bool om_vec = (p.k & 3) == 0;       // Omega rows 16-byte aligned
-    float acc[RPT][4];
+    uint32_t* mlo = reinterpret_cast<uint32_t*>(sm + S::kMlo);
+    uint32_t* omh = reinterpret_cast<uint32_t*>(sm + S::kOmHi);
+    uint32_t* oml = reinterpret_cast<uint32_t*>(sm + S::kOmLo);
+    float acc[NT][4];
 #pragma unroll
-    for (int r = 0; r < RPT; ++r)
+    for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+        for (int c = 0; c < 4; ++c) acc[t][c] = 0.f;
     bool bad = false;
 
     // Chunk c (columns c*kSkCols..) of G, M and Omega into stage s; zeros outside.
     auto issue = [&](int c, int s) {
         const int c0 = c * kSkCols;
-        unsigned char* gs = sm + s * kStage;
-        float* ms = reinterpret_cast<float*>(gs + kGBytes);
-        float* os = reinterpret_cast<float*>(gs + kGBytes + kMBytes);
+        unsigned char* gs = sm + s * S::kStage;
+        float* ms = reinterpret_cast<float*>(gs + S::kG);
+        float* os = reinterpret_cast<float*>(gs + S::kG + S::kM);
         if (E.vec_ok) {
             constexpr int GP = kSkCols * GSZ / 16, GE = 16 / GSZ;    // 16-byte pieces per row, elements per piece
             for (int q = threadIdx.x; q < kSkRows * GP; q += kThreads) {
@@ -220,34 +286,34 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
         }
         __syncthreads();                       // chunk c complete for every thread
         const int c0 = c * kSkCols;
-        unsigned char* gs = sm + s * kStage;
-        float* ms = reinterpret_cast<float*>(gs + kGBytes);
-        const float* os = reinterpret_cast<const float*>(gs + kGBytes + kMBytes);
-        // momentum: M <- mu M + G, back to global memory and kept for the product;
-        // 4 consecutive elements per thread, so a warp's 16-byte accesses are
+        unsigned char* gs = sm + s * S::kStage;
+        float* ms = reinterpret_cast<float*>(gs + S::kG);
+        const float* os = reinterpret_cast<const float*>(gs + S::kG + S::kM);
+        // momentum: M <- mu M + G, back to global memory; its tf32 high part
+        // replaces it in shared memory and the low part goes to mlo.  4
+        // consecutive elements per thread, so a warp's 16-byte accesses are
         // consecutive in shared memory
 #pragma unroll
         for (int it = 0; it < kSkRows * kSkCols / (4 * kThreads); ++it) {
             const int q = threadIdx.x + kThreads * it;
             const int rr = q / (kSkCols / 4), cc = (q % (kSkCols / 4)) * 4;
             const int i = row0 + rr, j = c0 + cc;
-            float g[4];
+            float g4[4];
             if (GSZ == 2) {
                 const uint2 u = *reinterpret_cast<const uint2*>(gs + (rr * kSkCols + cc) * 2);
                 using T = typename std::conditional<G_DT == DT_BF16, __nv_bfloat16, __half>::type;
-                g[0] = unpack_lo<T>(u.x); g[1] = unpack_hi<T>(u.x); g[2] = unpack_lo<T>(u.y); g[3] = unpack_hi<T>(u.y);
+                g4[0] = unpack_lo<T>(u.x); g4[1] = unpack_hi<T>(u.x); g4[2] = unpack_lo<T>(u.y); g4[3] = unpack_hi<T>(u.y);
             } else {
                 const float4 u = *reinterpret_cast<const float4*>(gs + (rr * kSkCols + cc) * 4);
-                g[0] = u.x; g[1] = u.y; g[2] = u.z; g[3] = u.w;
+                g4[0] = u.x; g4[1] = u.y; g4[2] = u.z; g4[3] = u.w;
             }
             float4* mp = reinterpret_cast<float4*>(ms + rr * kSkLd + cc);
             float4 m = *mp;
-            m.x = fmaf(p.mu, m.x, g[0]);      // zero outside the matrix
-            m.y = fmaf(p.mu, m.y, g[1]);
-            m.z = fmaf(p.mu, m.z, g[2]);
-            m.w = fmaf(p.mu, m.w, g[3]);
+            m.x = fmaf(p.mu, m.x, g4[0]);      // zero outside the matrix
+            m.y = fmaf(p.mu, m.y, g4[1]);
+            m.z = fmaf(p.mu, m.z, g4[2]);
+            m.w = fmaf(p.mu, m.w, g4[3]);
             bad |= !isfinite(m.x) || !isfinite(m.y) || !isfinite(m.z) || !isfinite(m.w);
-            *mp = m;
             if (i < E.rows && j < E.cols) {
                 float* dst = E.M + (long long)i * E.cols + j;
                 if (E.vec_ok) {
@@ -257,39 +323,49 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
                     for (int e = 0; e < 4 && j + e < E.cols; ++e) dst[e] = mv[e];
                 }
             }
+            uint4 h, l;
+            split_tf32(m.x, h.x, l.x);
+            split_tf32(m.y, h.y, l.y);
+            split_tf32(m.z, h.z, l.z);
+            split_tf32(m.w, h.w, l.w);
+            *reinterpret_cast<uint4*>(mp) = h;
+            *reinterpret_cast<uint4*>(mlo + rr * kSkLd + cc) = l;
+        }
+        for (int q = threadIdx.x; q < kSkCols * KT; q += kThreads) {
+            const int jj = q / KT, t = q % KT;
+            split_tf32(os[q], omh[jj * S::kOmLd + t], oml[jj * S::kOmLd + t]);
         }
         __syncthreads();
-        // Y[ty*RPT + r][4 tx + c] += sum_jj M[ty*RPT + r][jj] Omega[jj][4 tx + c]
-#pragma unroll 2
-        for (int jj = 0; jj < kSkCols; jj += 4) {
-            float4 o[4];
+        // Y[16 mt + .., n0 + ..] += M[rows, chunk] Omega[chunk, columns]
+        const uint32_t* mh = reinterpret_cast<const uint32_t*>(ms);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) o[q] = *reinterpret_cast<const float4*>(os + (jj + q) * KT + 4 * tx);
+        for (int kk = 0; kk < kSkCols; kk += 8) {
+            const int a0 = (16 * mt + g) * kSkLd + kk + q4;
+            const uint32_t ah[4] = {mh[a0], mh[a0 + 8 * kSkLd], mh[a0 + 4], mh[a0 + 8 * kSkLd + 4]};
+            const uint32_t al[4] = {mlo[a0], mlo[a0 + 8 * kSkLd], mlo[a0 + 4], mlo[a0 + 8 * kSkLd + 4]};
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const float4 mv = *reinterpret_cast<const float4*>(ms + (ty * RPT + r) * kSkLd + jj);
-                const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    acc[r][0] = fmaf(mm[q], o[q].x, acc[r][0]);
-                    acc[r][1] = fmaf(mm[q], o[q].y, acc[r][1]);
-                    acc[r][2] = fmaf(mm[q], o[q].z, acc[r][2]);
-                    acc[r][3] = fmaf(mm[q], o[q].w, acc[r][3]);
-                }
+            for (int t = 0; t < NT; ++t) {
+                const int b0 = (kk + q4) * S::kOmLd + n0 + 8 * t + g;
+                mma3_tf32(acc[t], ah, al, omh[b0], omh[b0 + 4 * S::kOmLd], oml[b0], oml[b0 + 4 * S::kOmLd]);
             }
         }
-        __syncthreads();                       // stage s free for chunk c + 2
+        __syncthreads();                       // stage s and the split buffers free for the next chunks
     }
     // Y to the workspace, and this block's rows' share of Y^T Y
     float* ys = reinterpret_cast<float*>(sm);  // [kSkRows][KT]
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        const int rr = ty * RPT + r, i = row0 + rr;
-        const float4 v = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-        *reinterpret_cast<float4*>(ys + rr * KT + 4 * tx) = v;      // zero for rows past the matrix
-        if (i < E.rows) *reinterpret_cast<float4*>(E.Y + (long long)i * KT + 4 * tx) = v;
+    for (int t = 0; t < NT; ++t) {
+        const int col = n0 + 8 * t + 2 * q4;
+        *reinterpret_cast<float2*>(ys + (16 * mt + g) * KT + col) = make_float2(acc[t][0], acc[t][1]);
+        *reinterpret_cast<float2*>(ys + (16 * mt + g + 8) * KT + col) = make_float2(acc[t][2], acc[t][3]);
     }
     __syncthreads();
+    for (int q = threadIdx.x; q < kSkRows * (KT / 4); q += kThreads) {
+        const int rr = q / (KT / 4), pc = q % (KT / 4), i = row0 + rr;   // zero for rows past the matrix
+        if (i < E.rows)
+            *reinterpret_cast<float4*>(E.Y + (long long)i * KT + 4 * pc) =
+                *reinterpret_cast<const float4*>(ys + rr * KT + 4 * pc);
+    }
     add_gram<KT>(ys, min(kSkRows, E.rows - row0), p.k, E.Gy);
     if (__syncthreads_or(bad) && threadIdx.x == 0) mark_bad(p, E);
 }
@@ -391,42 +467,56 @@ __global__ void __launch_bounds__(kThreads) lim_rowmul(const __grid_constant__ L
 // ---------------------------------------------------------------------------
 // 4. B^T = M^T Q (+ share of B B^T)
 // ---------------------------------------------------------------------------
-template <int KT>
-__host__ __device__ constexpr int project_stage_floats() { return kPjRows * kPjCols + kPjRows * KT; }
+// Shared memory of the projection: kPjStages stages of M rows [kPjRows][kPjLd]
+// (the block's columns) and Q rows [kPjRows][KT], then one buffer each of the
+// chunk's Q high and low tf32 parts [kPjRows][KT + 8].  The pitches (8 words
+// past a multiple of 32) make the fragment loads conflict-free.
+constexpr int kPjLd = kPjCols + 8;
 
 template <int KT>
-__global__ void __launch_bounds__(kThreads, 3) lim_project(const __grid_constant__ LimParams p) {
-    constexpr int kStage = project_stage_floats<KT>();
-    // register tile: JPT columns of M (rows of B^T) x 4 columns of Q per thread
-    constexpr int CG = KT / 4, JG = kThreads / CG, JPT = kPjCols / JG;
-    static_assert(JPT * JG == kPjCols && JPT % 4 == 0, "column tiling");
-    extern __shared__ __align__(16) float fsm[];
+struct ProjSmem {
+    static constexpr int kQLd = KT + 8;
+    static constexpr int kM = kPjRows * kPjLd * 4;
+    static constexpr int kStage = kM + kPjRows * KT * 4;
+    static constexpr int kQHi = kPjStages * kStage;
+    static constexpr int kQLo = kQHi + kPjRows * kQLd * 4;
+    static constexpr int kBytes = kQLo + kPjRows * kQLd * 4;
+};
+
+template <int KT>
+__global__ void __launch_bounds__(kThreads, KT == 32 ? 3 : 2) lim_project(const __grid_constant__ LimParams p) {
+    using S = ProjSmem<KT>;
+    constexpr int NT = KT / 8;                 // 8-column MMA tiles: a warp takes every column of Q
+    static_assert(kPjCols == 16 * (kThreads / 32), "one 16-column MMA tile of M per warp");
+    extern __shared__ __align__(16) unsigned char sm[];
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 2)];
     const int c0 = (blockIdx.x - E.t_proj) * kPjCols;
-    const int tt = threadIdx.x % CG, tj = threadIdx.x / CG;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q4 = lane & 3;
     const int nchunks = (E.rows + kPjRows - 1) / kPjRows;
-    float acc[JPT][4];
+    uint32_t* qh = reinterpret_cast<uint32_t*>(sm + S::kQHi);
+    uint32_t* ql = reinterpret_cast<uint32_t*>(sm + S::kQLo);
+    float acc[NT][4];
 #pragma unroll
-    for (int c = 0; c < JPT; ++c)
+    for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int h = 0; h < 4; ++h) acc[c][h] = 0.f;
+        for (int h = 0; h < 4; ++h) acc[t][h] = 0.f;
 
     // rows i0.. of M (this block's columns) and of Q into stage s
     auto issue = [&](int ch, int s) {
         const int i0 = ch * kPjRows;
-        float* ms = fsm + s * kStage;
-        float* qs = ms + kPjRows * kPjCols;
+        float* ms = reinterpret_cast<float*>(sm + s * S::kStage);
+        float* qs = reinterpret_cast<float*>(sm + s * S::kStage + S::kM);
         if (E.vec_ok) {
             constexpr int MP = kPjCols / 4;
             for (int q = threadIdx.x; q < kPjRows * MP; q += kThreads) {
                 const int rr = q / MP, pc = q % MP, i = i0 + rr, j = c0 + pc * 4;
                 const bool in = i < E.rows && j < E.cols;
-                cp_async16(ms + rr * kPjCols + pc * 4, E.M + (in ? (long long)i * E.cols + j : 0), in ? 16u : 0u);
+                cp_async16(ms + rr * kPjLd + pc * 4, E.M + (in ? (long long)i * E.cols + j : 0), in ? 16u : 0u);
             }
         } else {
             for (int q = threadIdx.x; q < kPjRows * kPjCols; q += kThreads) {
                 const int rr = q / kPjCols, cc = q % kPjCols, i = i0 + rr, j = c0 + cc;
-                ms[q] = (i < E.rows && j < E.cols) ? E.M[(long long)i * E.cols + j] : 0.f;
+                ms[rr * kPjLd + cc] = (i < E.rows && j < E.cols) ? E.M[(long long)i * E.cols + j] : 0.f;
             }
         }
         constexpr int QP = KT / 4;
@@ -445,35 +535,46 @@ __global__ void __launch_bounds__(kThreads, 3) lim_project(const __grid_constant
         else cp_async_commit();
         cp_async_wait<kPjStages - 1>();
         __syncthreads();
-        const float* ms = fsm + (ch % kPjStages) * kStage;
-        const float* qs = ms + kPjRows * kPjCols;
-#pragma unroll 4
-        for (int rr = 0; rr < kPjRows; ++rr) {
-            const float4 q4 = *reinterpret_cast<const float4*>(qs + rr * KT + 4 * tt);
-            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+        const float* ms = reinterpret_cast<const float*>(sm + (ch % kPjStages) * S::kStage);
+        const float* qs = reinterpret_cast<const float*>(sm + (ch % kPjStages) * S::kStage + S::kM);
+        for (int q = threadIdx.x; q < kPjRows * KT; q += kThreads) {
+            const int rr = q / KT, t = q % KT;
+            split_tf32(qs[q], qh[rr * S::kQLd + t], ql[rr * S::kQLd + t]);
+        }
+        __syncthreads();
+        // B^T[16 warp + .., :] += M[chunk, columns]^T Q[chunk, :]
 #pragma unroll
-            for (int c4 = 0; c4 < JPT / 4; ++c4) {
-                const float4 mv = *reinterpret_cast<const float4*>(ms + rr * kPjCols + tj * JPT + 4 * c4);
-                const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
+        for (int kk = 0; kk < kPjRows; kk += 8) {
+            const float* mr = ms + (kk + q4) * kPjLd + 16 * warp + g;
+            uint32_t ah[4], al[4];
+            split_tf32(mr[0], ah[0], al[0]);
+            split_tf32(mr[8], ah[1], al[1]);
+            split_tf32(mr[4 * kPjLd], ah[2], al[2]);
+            split_tf32(mr[4 * kPjLd + 8], ah[3], al[3]);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) acc[4 * c4 + e][h] = fmaf(mm[e], qv[h], acc[4 * c4 + e][h]);
+            for (int t = 0; t < NT; ++t) {
+                const int b0 = (kk + q4) * S::kQLd + 8 * t + g;
+                mma3_tf32(acc[t], ah, al, qh[b0], qh[b0 + 4 * S::kQLd], ql[b0], ql[b0 + 4 * S::kQLd]);
             }
         }
-        __syncthreads();                       // this stage is refilled next
+        __syncthreads();                       // this stage and the split buffers are refilled next
     }
     cp_async_wait<0>();
     // B^T to the workspace, and this block's columns' share of B B^T
-    float* bs = fsm;                           // [kPjCols][KT]
+    float* bs = reinterpret_cast<float*>(sm);  // [kPjCols][KT]
 #pragma unroll
-    for (int c = 0; c < JPT; ++c) {
-        const int cc = tj * JPT + c, j = c0 + cc;
-        const float4 v = make_float4(acc[c][0], acc[c][1], acc[c][2], acc[c][3]);
-        *reinterpret_cast<float4*>(bs + cc * KT + 4 * tt) = v;
-        if (j < E.cols) *reinterpret_cast<float4*>(E.Bt + (long long)j * KT + 4 * tt) = v;
+    for (int t = 0; t < NT; ++t) {
+        const int col = 8 * t + 2 * q4;
+        *reinterpret_cast<float2*>(bs + (16 * warp + g) * KT + col) = make_float2(acc[t][0], acc[t][1]);
+        *reinterpret_cast<float2*>(bs + (16 * warp + g + 8) * KT + col) = make_float2(acc[t][2], acc[t][3]);
     }
     __syncthreads();
+    for (int q = threadIdx.x; q < kPjCols * (KT / 4); q += kThreads) {
+        const int cc = q / (KT / 4), pc = q % (KT / 4), j = c0 + cc;
+        if (j < E.cols)
+            *reinterpret_cast<float4*>(E.Bt + (long long)j * KT + 4 * pc) =
+                *reinterpret_cast<const float4*>(bs + cc * KT + 4 * pc);
+    }
     add_gram<KT>(bs, min(kPjCols, E.cols - c0), p.k, E.Cg);
 }
 
@@ -593,141 +694,151 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
 // ---------------------------------------------------------------------------
 // 7. O = Z B and the weight update
 // ---------------------------------------------------------------------------
-template <int W_DT>
-__device__ __forceinline__ void load4_w(const void* base, long long idx, bool vec, int nvalid, float* v) {
-    if (vec) {
-        if (W_DT == DT_FP32) {
-            const float4 x = *reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
-            v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-        } else {
-            const uint2 x = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + idx);
-            using T = typename std::conditional<W_DT == DT_BF16, __nv_bfloat16, __half>::type;
-            v[0] = unpack_lo<T>(x.x); v[1] = unpack_hi<T>(x.x);
-            v[2] = unpack_lo<T>(x.y); v[3] = unpack_hi<T>(x.y);
-        }
-        return;
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) v[c] = c < nvalid ? ld_elem(base, idx + c, W_DT) : 0.f;
-}
-
-template <int W_DT>
-__device__ __forceinline__ void store4_w(void* base, long long idx, bool vec, int nvalid, const float* v) {
-    if (vec) {
-        if (W_DT == DT_FP32) {
-            *reinterpret_cast<float4*>(static_cast<float*>(base) + idx) = make_float4(v[0], v[1], v[2], v[3]);
-        } else {
-            using T = typename std::conditional<W_DT == DT_BF16, __nv_bfloat16, __half>::type;
-            *reinterpret_cast<uint2*>(static_cast<uint16_t*>(base) + idx) =
-                make_uint2(pack2<T>(v[0], v[1]), pack2<T>(v[2], v[3]));
-        }
-        return;
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-        if (c < nvalid) st_elem(base, idx + c, W_DT, v[c]);
-}
-
-// Shared memory of lim_update: Z rows [kUpRows][KT], B [KT][kBsLd] (the tile's
-// columns of B = (B^T)^T), the B^T tile as loaded [kUpCols][KT], and the
-// tile of W [kUpRows][kUpCols] in W's type.
-template <int KT>
-__host__ __device__ constexpr int update_smem_floats() { return kUpRows * KT + KT * kBsLd + kUpCols * KT; }
-
+// Shared memory of lim_update: Z rows [kUpRows][KT + 4] and the B^T rows of
+// the tile's columns [kUpCols][KT + 4] as loaded, each then replaced by its
+// tf32 high part with the low parts in two more such arrays, and the tile of W
+// [kUpRows][kUpCols + 8] in W's type.  The pitches make the fragment loads
+// and the epilogue's accesses to W conflict-free.
 template <int KT, int W_DT>
-__host__ __device__ constexpr int update_smem_bytes() {
-    return update_smem_floats<KT>() * 4 + kUpRows * kUpCols * g_size<W_DT>();
-}
+struct UpdSmem {
+    static constexpr int kLd = KT + 4;
+    static constexpr int kWLd = kUpCols + 8;
+    static constexpr int kArr = kUpRows * kLd * 4;
+    static constexpr int kZ = 0, kZlo = kArr, kBt = 2 * kArr, kBtlo = 3 * kArr, kW = 4 * kArr;
+    static constexpr int kBytes = kW + kUpRows * kWLd * g_size<W_DT>();
+    static_assert(kUpRows == kUpCols, "Z and B^T tiles share a shape");
+};
 
 template <int KT, int W_DT>
 __global__ void __launch_bounds__(kThreads, 2) lim_update(const __grid_constant__ LimParams p) {
+    using S = UpdSmem<KT, W_DT>;
     constexpr int WSZ = g_size<W_DT>();
-    extern __shared__ __align__(16) float fsm[];
-    float* Zs = fsm;                           // [kUpRows][KT]
-    float* Bs = Zs + kUpRows * KT;             // [KT][kBsLd]
-    float* Bts = Bs + KT * kBsLd;              // [kUpCols][KT]
-    unsigned char* Ws = reinterpret_cast<unsigned char*>(Bts + kUpCols * KT);   // [kUpRows][kUpCols]
+    constexpr int NT = kUpCols / 8;            // 8-column MMA tiles: a warp takes 16 rows x every column
+    static_assert(kUpRows == 16 * (kThreads / 32), "one 16-row MMA tile per warp");
+    extern __shared__ __align__(16) unsigned char sm[];
+    float* Zs = reinterpret_cast<float*>(sm + S::kZ);
+    float* Bts = reinterpret_cast<float*>(sm + S::kBt);
+    uint32_t* Zlo = reinterpret_cast<uint32_t*>(sm + S::kZlo);
+    uint32_t* Btlo = reinterpret_cast<uint32_t*>(sm + S::kBtlo);
+    unsigned char* Ws = sm + S::kW;
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 3)];
     const int tile = blockIdx.x - E.t_upd;
     const int tiles_c = (E.cols + kUpCols - 1) / kUpCols;
     const int row0 = (tile / tiles_c) * kUpRows, c0 = (tile % tiles_c) * kUpCols;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q4 = lane & 3;
     const bool skip = *E.bad != 0;
+    const bool wtile = E.vec_ok && !skip;      // W through shared memory (16-byte pieces)
     // every global read of the tile in one asynchronous group: Z rows, the
     // B^T rows of the tile's columns, and (aligned rows) the tile of W
     constexpr int ZP = KT / 4;
     for (int q = threadIdx.x; q < kUpRows * ZP; q += kThreads) {
         const int rr = q / ZP, pc = q % ZP, i = row0 + rr;
         const bool in = i < E.rows;
-        cp_async16(Zs + rr * KT + pc * 4, E.Y + (in ? (long long)i * KT + pc * 4 : 0), in ? 16u : 0u);
+        cp_async16(Zs + rr * S::kLd + pc * 4, E.Y + (in ? (long long)i * KT + pc * 4 : 0), in ? 16u : 0u);
     }
     for (int q = threadIdx.x; q < kUpCols * ZP; q += kThreads) {
         const int jj = q / ZP, pc = q % ZP, j = c0 + jj;
         const bool in = j < E.cols;
-        cp_async16(Bts + jj * KT + pc * 4, E.Bt + (in ? (long long)j * KT + pc * 4 : 0), in ? 16u : 0u);
+        cp_async16(Bts + jj * S::kLd + pc * 4, E.Bt + (in ? (long long)j * KT + pc * 4 : 0), in ? 16u : 0u);
     }
-    if (E.vec_ok && !skip) {
+    if (wtile) {
         constexpr int WP = kUpCols * WSZ / 16, WE = 16 / WSZ;   // 16-byte pieces per row, elements per piece
         for (int q = threadIdx.x; q < kUpRows * WP; q += kThreads) {
             const int rr = q / WP, pc = q % WP, i = row0 + rr, j = c0 + pc * WE;
             const bool in = i < E.rows && j < E.cols;
             const char* src = static_cast<const char*>(E.W) + (in ? ((long long)i * E.cols + j) * WSZ : 0);
-            cp_async16(Ws + (rr * kUpCols + pc * WE) * WSZ, src, in ? 16u : 0u);
+            cp_async16(Ws + (rr * S::kWLd + pc * WE) * WSZ, src, in ? 16u : 0u);
         }
     }
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
-    for (int q = threadIdx.x; q < kUpCols * KT; q += kThreads) {   // B = (B^T)^T, shared to shared
-        const int t = q % KT, jj = q / KT;
-        Bs[t * kBsLd + jj] = Bts[jj * KT + t];
+    const int kk8 = (p.k + 7) & ~7;            // columns of Z (and of B^T) past k are zero
+    for (int q = threadIdx.x; q < kUpRows * KT; q += kThreads) {
+        const int rr = q / KT, t = q % KT, o = rr * S::kLd + t;
+        if (t >= kk8) continue;
+        uint32_t h;
+        split_tf32(Zs[o], h, Zlo[o]);
+        Zs[o] = __uint_as_float(h);
+        split_tf32(Bts[o], h, Btlo[o]);
+        Bts[o] = __uint_as_float(h);
     }
     __syncthreads();
-    float o[16][4];
+    const uint32_t* Zh = reinterpret_cast<const uint32_t*>(Zs);
+    const uint32_t* Bth = reinterpret_cast<const uint32_t*>(Bts);
+    float o[NT][4];
 #pragma unroll
-    for (int r = 0; r < 16; ++r)
+    for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) o[r][c] = 0.f;
-    const int kk = (p.k + 3) & ~3;             // columns of Z past k are zero
+        for (int c = 0; c < 4; ++c) o[t][c] = 0.f;
 #pragma unroll 1
-    for (int t = 0; t < kk; t += 4) {
-        float4 b[4];
+    for (int kk = 0; kk < kk8; kk += 8) {
+        const int a0 = (16 * warp + g) * S::kLd + kk + q4;
+        const uint32_t ah[4] = {Zh[a0], Zh[a0 + 8 * S::kLd], Zh[a0 + 4], Zh[a0 + 8 * S::kLd + 4]};
+        const uint32_t al[4] = {Zlo[a0], Zlo[a0 + 8 * S::kLd], Zlo[a0 + 4], Zlo[a0 + 8 * S::kLd + 4]};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) b[q] = *reinterpret_cast<const float4*>(Bs + (t + q) * kBsLd + 4 * lane);
+        for (int t = 0; t < NT; ++t) {
+            // B (k x columns) = (B^T)^T: b0 = B^T[8 t + g][kk + q4]
+            const int b0 = (8 * t + g) * S::kLd + kk + q4;
+            mma3_tf32(o[t], ah, al, Bth[b0], Bth[b0 + 4], Btlo[b0], Btlo[b0 + 4]);
+        }
+    }
+    // epilogue: O (optional) and W <- W - eta (gamma O + lambda W); this
+    // thread holds rows 16 warp + g (+ 8), columns 8 t + 2 q4 (+ 1)
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const float4 z = *reinterpret_cast<const float4*>(Zs + (16 * warp + r) * KT + t);
-            const float zz[4] = {z.x, z.y, z.z, z.w};
+    for (int h = 0; h < 2; ++h) {
+        const int rr = 16 * warp + g + 8 * h, i = row0 + rr;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                o[r][0] = fmaf(zz[q], b[q].x, o[r][0]);
-                o[r][1] = fmaf(zz[q], b[q].y, o[r][1]);
-                o[r][2] = fmaf(zz[q], b[q].z, o[r][2]);
-                o[r][3] = fmaf(zz[q], b[q].w, o[r][3]);
+        for (int t = 0; t < NT; ++t) {
+            const int cc = 8 * t + 2 * q4, j = c0 + cc;
+            const float v0 = o[t][2 * h], v1 = o[t][2 * h + 1];
+            const bool in0 = i < E.rows && j < E.cols, in1 = i < E.rows && j + 1 < E.cols;
+            if (E.O_out) {
+                const long long idx = (long long)i * E.cols + j;
+                if (E.vec_ok && in0) *reinterpret_cast<float2*>(E.O_out + idx) = make_float2(v0, v1);
+                else {
+                    if (in0) E.O_out[idx] = v0;
+                    if (in1) E.O_out[idx + 1] = v1;
+                }
+            }
+            if (skip) continue;
+            if (wtile) {                       // in shared memory, stored below
+                unsigned char* wp = Ws + (rr * S::kWLd + cc) * WSZ;
+                if (W_DT == DT_FP32) {
+                    float2 w = *reinterpret_cast<float2*>(wp);
+                    w.x = w.x - p.eta * (E.gamma * v0 + p.lambda * w.x);
+                    w.y = w.y - p.eta * (E.gamma * v1 + p.lambda * w.y);
+                    *reinterpret_cast<float2*>(wp) = w;
+                } else {
+                    using T = typename std::conditional<W_DT == DT_BF16, __nv_bfloat16, __half>::type;
+                    const uint32_t u = *reinterpret_cast<const uint32_t*>(wp);
+                    float w0 = unpack_lo<T>(u), w1 = unpack_hi<T>(u);
+                    w0 = w0 - p.eta * (E.gamma * v0 + p.lambda * w0);
+                    w1 = w1 - p.eta * (E.gamma * v1 + p.lambda * w1);
+                    *reinterpret_cast<uint32_t*>(wp) = pack2<T>(w0, w1);
+                }
+            } else {
+                const long long idx = (long long)i * E.cols + j;
+                if (in0) {
+                    const float w0 = ld_elem(E.W, idx, W_DT);
+                    st_elem(E.W, idx, W_DT, w0 - p.eta * (E.gamma * v0 + p.lambda * w0));
+                }
+                if (in1) {
+                    const float w1 = ld_elem(E.W, idx + 1, W_DT);
+                    st_elem(E.W, idx + 1, W_DT, w1 - p.eta * (E.gamma * v1 + p.lambda * w1));
+                }
             }
         }
     }
-    const int j = c0 + 4 * lane;
-    if (j >= E.cols) return;
-    const int nvalid = min(4, E.cols - j);
-    const bool vec = E.vec_ok && nvalid == 4;
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        const int rr = 16 * warp + r, i = row0 + rr;
-        if (i >= E.rows) break;
-        const long long idx = (long long)i * E.cols + j;
-        if (E.O_out) {
-            if (vec) *reinterpret_cast<float4*>(E.O_out + idx) = make_float4(o[r][0], o[r][1], o[r][2], o[r][3]);
-            else
-                for (int c = 0; c < nvalid; ++c) E.O_out[idx + c] = o[r][c];
+    if (wtile) {                               // uniform over the block
+        __syncthreads();
+        constexpr int WP = kUpCols * WSZ / 16, WE = 16 / WSZ;
+        for (int q = threadIdx.x; q < kUpRows * WP; q += kThreads) {
+            const int rr = q / WP, pc = q % WP, i = row0 + rr, j = c0 + pc * WE;
+            if (i < E.rows && j < E.cols)       // cols % 8 == 0: a piece is wholly in or out
+                *reinterpret_cast<uint4*>(static_cast<char*>(E.W) + ((long long)i * E.cols + j) * WSZ) =
+                    *reinterpret_cast<const uint4*>(Ws + (rr * S::kWLd + pc * WE) * WSZ);
         }
-        if (skip) continue;
-        float w[4];
-        if (vec) load4_w<W_DT>(Ws, (long long)rr * kUpCols + 4 * lane, true, 4, w);   // staged
-        else load4_w<W_DT>(E.W, idx, false, nvalid, w);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) w[c] = w[c] - p.eta * (E.gamma * o[r][c] + p.lambda * w[c]);
-        store4_w<W_DT>(E.W, idx, vec, nvalid, w);
     }
 }
 
@@ -737,11 +848,11 @@ __global__ void __launch_bounds__(kThreads, 2) lim_update(const __grid_constant_
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 template <int KT, int G_DT>
-constexpr size_t sketch_smem() { return 2 * (size_t)sketch_stage_bytes<KT, G_DT>(); }
+constexpr size_t sketch_smem() { return (size_t)SketchSmem<KT, G_DT>::kBytes; }
 template <int KT>
-constexpr size_t project_smem() { return sizeof(float) * kPjStages * project_stage_floats<KT>(); }
+constexpr size_t project_smem() { return (size_t)ProjSmem<KT>::kBytes; }
 template <int KT, int W_DT>
-constexpr size_t update_smem() { return (size_t)update_smem_bytes<KT, W_DT>(); }
+constexpr size_t update_smem() { return (size_t)UpdSmem<KT, W_DT>::kBytes; }
 template <int KT>
 constexpr size_t chol_smem() { return sizeof(double) * (2 * KT * KT + KT) + sizeof(int) * KT; }
 template <int KT>
@@ -904,7 +1015,6 @@ muon_status limuon_step_batched(const muon_rsvd_param* params, int n, muon_dtype
         prm.k = k; prm.r = hp->rank;
         prm.mu = hp->mu; prm.eta = hp->eta; prm.lambda = hp->lambda;
         prm.d_status = d_status;
-        long long ts = 0, tr = 0, tp = 0, tu = 0;
         LaunchShape L = {};
         for (int i = 0; i < prm.n; ++i) {
             const muon_rsvd_param& q = params[b + i];
@@ -921,18 +1031,37 @@ muon_status limuon_step_batched(const muon_rsvd_param* params, int n, muon_dtype
             const uintptr_t al = reinterpret_cast<uintptr_t>(q.W) | reinterpret_cast<uintptr_t>(q.G) |
                                  reinterpret_cast<uintptr_t>(q.M) | reinterpret_cast<uintptr_t>(q.O_out);
             E.vec_ok = (al & 15) == 0 && q.cols % 8 == 0;
-            E.t_sketch = (int)ts; E.t_rows = (int)tr; E.t_proj = (int)tp; E.t_upd = (int)tu;
-            ts += (q.rows + kSkRows - 1) / kSkRows;
-            tr += (q.rows + kThreads - 1) / kThreads;
-            tp += (q.cols + kPjCols - 1) / kPjCols;
-            tu += (long long)((q.rows + kUpRows - 1) / kUpRows) * ((q.cols + kUpCols - 1) / kUpCols);
             L.elems += (double)q.rows * q.cols;
             L.rows_k += (double)q.rows * k;
             L.cols_k += (double)q.cols * k;
             L.rows_total += q.rows;
         }
-        if (ts > INT32_MAX || tr > INT32_MAX || tp > INT32_MAX || tu > INT32_MAX) return MUON_ERR_UNSUPPORTED;
-        L.sketch = (int)ts; L.rows = (int)tr; L.proj = (int)tp; L.upd = (int)tu;
+        // Each launch's grid in its own order of the matrices: a sketch block
+        // runs over its matrix's columns and a projection block over its rows,
+        // so those two put the longest first (stable: ties keep their order).
+        long long tot[4] = {0, 0, 0, 0};
+        for (int w = 0; w < 4; ++w) {
+            int idx[kLimMax];
+            for (int i = 0; i < prm.n; ++i) idx[i] = i;
+            if (w == 0 || w == 2)
+                std::stable_sort(idx, idx + prm.n, [&](int a, int b) {
+                    return w == 0 ? prm.e[a].cols > prm.e[b].cols : prm.e[a].rows > prm.e[b].rows;
+                });
+            for (int pos = 0; pos < prm.n; ++pos) {
+                LimEntry& E = prm.e[idx[pos]];
+                prm.ord[w][pos] = (unsigned char)idx[pos];
+                const long long first = tot[w];
+                if (w == 0) { E.t_sketch = (int)first; tot[w] += (E.rows + kSkRows - 1) / kSkRows; }
+                else if (w == 1) { E.t_rows = (int)first; tot[w] += (E.rows + kThreads - 1) / kThreads; }
+                else if (w == 2) { E.t_proj = (int)first; tot[w] += (E.cols + kPjCols - 1) / kPjCols; }
+                else {
+                    E.t_upd = (int)first;
+                    tot[w] += (long long)((E.rows + kUpRows - 1) / kUpRows) * ((E.cols + kUpCols - 1) / kUpCols);
+                }
+                if (tot[w] > INT32_MAX) return MUON_ERR_UNSUPPORTED;
+            }
+        }
+        L.sketch = (int)tot[0]; L.rows = (int)tot[1]; L.proj = (int)tot[2]; L.upd = (int)tot[3];
         if (KT == 32) {
             if (w_dtype == MUON_BF16) st = launch_all<32, DT_BF16>(prm, s, L);
             else if (w_dtype == MUON_FP16) st = launch_all<32, DT_FP16>(prm, s, L);
