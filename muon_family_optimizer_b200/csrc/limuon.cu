@@ -28,12 +28,14 @@
 //                  cp.async stages), tensor cores as in 1; each block adds its
 //                  columns' share of B B^T (fp64) to the matrix's k x k sum.
 //                  Reads M.
-//   5 lim_eig      per matrix (k x k): cyclic Jacobi on B B^T in fp64,
-//                  round-robin order (k/2 disjoint rotations per round), a
+//   5 lim_eig      per matrix (k x k): cyclic Jacobi on B B^T in fp64, padded
+//                  with zeros to KT = 32 or 64 indices, round-robin order
+//                  from a table (KT/2 disjoint rotations per round), a
 //                  rotation only while |C_pq| > 1e-15 sqrt(C_pp C_qq) (and
 //                  above 1e-16 of the trace: fp64 noise), stop after a sweep
 //                  without one; P from the r largest eigenpairs.
-//   6 lim_rowmul   Z = Q P in place.
+//   6 lim_rowmul   Z = Q P in place.  Q and Z are stored as tf32 high and low
+//                  parts (the operands of 4 and 7).
 //   7 lim_update   O = Z B on 128 x 128 tiles (tensor cores as in 1), fused
 //                  with the weight update (reads and writes W; O never stored
 //                  unless O_out is given).
@@ -55,12 +57,12 @@ namespace {
 constexpr int kLimMax = 128;      // matrices per launch
 constexpr int kThreads = 256;
 constexpr int kSmallThreads = 64; // per-matrix k x k kernels
-constexpr int kSkRows = 64;       // lim_sketch: rows per block
-constexpr int kSkCols = 64;       // lim_sketch: columns per chunk (two stages)
-constexpr int kSkLd = kSkCols + 4;   // padded row of a staged M chunk
-constexpr int kPjCols = 128;      // lim_project: columns per block
+constexpr int kSkRows = 128;      // lim_sketch: rows per block (one 16-row MMA tile per warp)
+constexpr int kSkCols = 32;       // lim_sketch: columns per chunk (two stages)
+constexpr int kPjCols = 128;      // lim_project: columns per block (one 16-column MMA tile per warp)
 constexpr int kPjRows = 32;       // lim_project: rows per chunk
 constexpr int kPjStages = 3;
+constexpr int kPjSegRows = 1024;  // lim_project: rows per block; taller matrices split into segments
 constexpr int kUpRows = 128;      // lim_update: tile rows
 constexpr int kUpCols = 128;      // lim_update: tile columns
 constexpr double kDrop = 1e-10;   // Cholesky pivot / squared column norm below which a column is dropped
@@ -71,8 +73,13 @@ constexpr int kMaxDevices = 64;    // devices whose kernel attributes are tracke
 
 struct LimEntry {
     void* W; const void* G; float* M; const float* Omega; float* O_out;
-    float* Y;        // rows x KT workspace: Y, then Q, then Z (in place)
-    float* Bt;       // cols x KT workspace: B^T
+    float* Y;        // rows x KT workspace: Y, then the tf32 high parts of Q, then of Z (in place)
+    float* Ylo;      // rows x KT workspace: the tf32 low parts of Q, then of Z
+    float* Bt;       // cols x KT workspace: the tf32 high parts of B^T
+    float* Btlo;     // cols x KT workspace: the tf32 low parts of B^T
+    float* Bpart;    // nseg x cols x KT workspace: the projection's per-segment partial B^T (nseg > 1)
+    int* pj_count;   // per 128-column block: segments finished (workspace, zeroed per call; nseg > 1)
+    int nseg;        // row segments of the projection
     double* Gy;      // KT x KT: Y^T Y, upper triangle summed by lim_sketch (zeroed per call)
     double* Cg;      // KT x KT: B B^T, upper triangle summed by lim_project (zeroed per call)
     double* K;       // KT x KT: R^-1 (lim_chol), then P (lim_eig)
@@ -155,10 +162,13 @@ __device__ __forceinline__ void add_gram(const float* X, int n, int k, double* d
 // b1 = (q + 4, g); C (16 x 8) c0, c1 = (g, 2q), (g, 2q + 1); c2, c3 = the same
 // columns of row g + 8.
 // ---------------------------------------------------------------------------
+// x rounded to the nearest tf32 value (ties away from zero): add half of the
+// dropped 13 bits' weight to the magnitude bits and clear them (integer ops,
+// full-rate pipes).  Finite values that round past the largest float become
+// infinite; infinities and NaN (whose bits could wrap) are only truncated.
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    const uint32_t u = __float_as_uint(x);
+    return ((u & 0x7f800000u) == 0x7f800000u ? u : u + 0x1000u) & 0xffffe000u;
 }
 
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
@@ -188,41 +198,72 @@ __device__ __forceinline__ void mma3_tf32(float (&d)[4], const uint32_t (&ah)[4]
 template <int G_DT>
 __host__ __device__ constexpr int g_size() { return G_DT == DT_FP32 ? 4 : 2; }
 
+// Swizzled rows of 32-bit words (a multiple of 32 per row): word c of row r
+// sits at c ^ 16 (r & 1), so a quarter-warp's 16-byte loads of two adjacent
+// rows at the same columns fall in different banks.  16-byte pieces stay whole.
+__device__ __forceinline__ int swz(int r, int c) { return c ^ ((r & 1) << 4); }
+
+// Tensor-core operand loads with the k index permuted inside each 16-wide
+// group: in k-step s (0, 1) of the group, the MMA's k = q and q + 4 take the
+// group's columns 4 q + 2 s and 4 q + 2 s + 1, the same for A and B, so one
+// 16-byte load gives a thread its A (or B) words for both k-steps.  (The
+// contraction runs over every column of the group either way.)
+struct Frag16 {
+    uint32_t h[4], l[4];   // the four words at columns 4 q .. 4 q + 3: high and low parts
+};
+
+__device__ __forceinline__ void ld_frag16(Frag16& f, const uint32_t* hi, const uint32_t* lo, int off) {
+    const uint4 a = *reinterpret_cast<const uint4*>(hi + off);
+    const uint4 b = *reinterpret_cast<const uint4*>(lo + off);
+    f.h[0] = a.x; f.h[1] = a.y; f.h[2] = a.z; f.h[3] = a.w;
+    f.l[0] = b.x; f.l[1] = b.y; f.l[2] = b.z; f.l[3] = b.w;
+}
+
+// d += A B over one 16-wide k group: ra / rb = the A rows g and g + 8, fb = the
+// B column g (all loaded by ld_frag16 at the group's columns 4 q ..).
+__device__ __forceinline__ void mma16(float (&d)[4], const Frag16& ra, const Frag16& rb, const Frag16& fb) {
+#pragma unroll
+    for (int st = 0; st < 2; ++st) {
+        const uint32_t ah[4] = {ra.h[2 * st], rb.h[2 * st], ra.h[2 * st + 1], rb.h[2 * st + 1]};
+        const uint32_t al[4] = {ra.l[2 * st], rb.l[2 * st], ra.l[2 * st + 1], rb.l[2 * st + 1]};
+        mma3_tf32(d, ah, al, fb.h[2 * st], fb.h[2 * st + 1], fb.l[2 * st], fb.l[2 * st + 1]);
+    }
+}
+
 // Shared memory of the sketch.  Two stages of raw chunks: G [kSkRows][kSkCols]
-// in its own type, M [kSkRows][kSkLd] fp32 (its tf32 high part after the
-// momentum phase, in place), Omega [kSkCols][KT] fp32.  One buffer each of the
-// chunk's M low part [kSkRows][kSkLd] and Omega's high and low parts
-// [kSkCols][KT + 8].  Row pitches 4 (M) and 8 (Omega) words past a multiple
-// of 32 make the fragment loads conflict-free.
+// in its own type, M [kSkRows][kSkCols] fp32 swizzled (its tf32 high part after
+// the momentum phase, in place), Omega [kSkCols][KT + 4] fp32 (the pitch makes
+// the transposing reads conflict-free).  One buffer each of the chunk's M low
+// part (as M) and of Omega^T's high and low parts [KT][kSkCols] swizzled.
 template <int KT, int G_DT>
 struct SketchSmem {
-    static constexpr int kOmLd = KT + 8;
+    static constexpr int kOmLd = KT + 4;
     static constexpr int kG = kSkRows * kSkCols * g_size<G_DT>();
-    static constexpr int kM = kSkRows * kSkLd * 4;
-    static constexpr int kOm = kSkCols * KT * 4;
+    static constexpr int kM = kSkRows * kSkCols * 4;
+    static constexpr int kOm = kSkCols * kOmLd * 4;
     static constexpr int kStage = kG + kM + kOm;
     static constexpr int kMlo = 2 * kStage;
-    static constexpr int kOmHi = kMlo + kSkRows * kSkLd * 4;
-    static constexpr int kOmLo = kOmHi + kSkCols * kOmLd * 4;
-    static constexpr int kBytes = kOmLo + kSkCols * kOmLd * 4;
+    static constexpr int kOtHi = kMlo + kSkRows * kSkCols * 4;
+    static constexpr int kOtLo = kOtHi + KT * kSkCols * 4;
+    static constexpr int kBytes = kOtLo + KT * kSkCols * 4;
+    static_assert(kStage % 16 == 0 && kSkCols == 32, "16-byte aligned stages; one swizzled 32-word row per chunk row");
 };
 
 template <int KT, int G_DT>
-__global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant__ LimParams p) {
+__global__ void __launch_bounds__(kThreads, KT == 32 ? 2 : 1) lim_sketch(const __grid_constant__ LimParams p) {
     using S = SketchSmem<KT, G_DT>;
     constexpr int GSZ = g_size<G_DT>();
-    constexpr int NT = KT / 16;                // 8-column MMA tiles per warp (a warp takes half of Y's columns)
-    static_assert(kSkRows == 64 && kThreads == 256, "four 16-row MMA tiles x two column halves");
+    constexpr int NT = KT / 8;                 // 8-column MMA tiles: a warp takes 16 rows x every column of Y
+    static_assert(kSkRows == 16 * (kThreads / 32), "one 16-row MMA tile per warp");
     extern __shared__ __align__(16) unsigned char sm[];
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 0)];
     const int row0 = (blockIdx.x - E.t_sketch) * kSkRows;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q4 = lane & 3;
-    const int mt = warp & 3, n0 = (warp >> 2) * (KT / 2);   // rows 16 mt.., columns n0.. of Y
     const int nchunks = (E.cols + kSkCols - 1) / kSkCols;
     const bool om_vec = (p.k & 3) == 0;       // Omega rows 16-byte aligned
     uint32_t* mlo = reinterpret_cast<uint32_t*>(sm + S::kMlo);
-    uint32_t* omh = reinterpret_cast<uint32_t*>(sm + S::kOmHi);
-    uint32_t* oml = reinterpret_cast<uint32_t*>(sm + S::kOmLo);
+    uint32_t* oth = reinterpret_cast<uint32_t*>(sm + S::kOtHi);
+    uint32_t* otl = reinterpret_cast<uint32_t*>(sm + S::kOtLo);
     float acc[NT][4];
 #pragma unroll
     for (int t = 0; t < NT; ++t)
@@ -248,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
             for (int q = threadIdx.x; q < kSkRows * MP; q += kThreads) {
                 const int rr = q / MP, pc = q % MP, i = row0 + rr, j = c0 + pc * 4;
                 const bool in = i < E.rows && j < E.cols;
-                cp_async16(ms + rr * kSkLd + pc * 4, E.M + (in ? (long long)i * E.cols + j : 0), in ? 16u : 0u);
+                cp_async16(ms + rr * kSkCols + swz(rr, pc * 4), E.M + (in ? (long long)i * E.cols + j : 0),
+                           in ? 16u : 0u);
             }
         } else {
             for (int q = threadIdx.x; q < kSkRows * kSkCols; q += kThreads) {
@@ -256,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
                 const bool in = i < E.rows && j < E.cols;
                 const long long idx = (long long)i * E.cols + j;
                 st_elem(gs, rr * kSkCols + cc, G_DT, in ? ld_elem(E.G, idx, G_DT) : 0.f);
-                ms[rr * kSkLd + cc] = in ? E.M[idx] : 0.f;
+                ms[rr * kSkCols + swz(rr, cc)] = in ? E.M[idx] : 0.f;
             }
         }
         if (om_vec) {
@@ -264,12 +306,13 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
             for (int q = threadIdx.x; q < kSkCols * OP; q += kThreads) {
                 const int jj = q / OP, pc = q % OP, j = c0 + jj;
                 const bool in = j < E.cols && pc * 4 < p.k;
-                cp_async16(os + jj * KT + pc * 4, E.Omega + (in ? (long long)j * p.k + pc * 4 : 0), in ? 16u : 0u);
+                cp_async16(os + jj * S::kOmLd + pc * 4, E.Omega + (in ? (long long)j * p.k + pc * 4 : 0),
+                           in ? 16u : 0u);
             }
         } else {
             for (int q = threadIdx.x; q < kSkCols * KT; q += kThreads) {
                 const int jj = q / KT, t = q % KT, j = c0 + jj;
-                os[q] = (j < E.cols && t < p.k) ? E.Omega[(long long)j * p.k + t] : 0.f;
+                os[jj * S::kOmLd + t] = (j < E.cols && t < p.k) ? E.Omega[(long long)j * p.k + t] : 0.f;
             }
         }
         cp_async_commit();
@@ -307,7 +350,8 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
                 const float4 u = *reinterpret_cast<const float4*>(gs + (rr * kSkCols + cc) * 4);
                 g4[0] = u.x; g4[1] = u.y; g4[2] = u.z; g4[3] = u.w;
             }
-            float4* mp = reinterpret_cast<float4*>(ms + rr * kSkLd + cc);
+            const int o = rr * kSkCols + swz(rr, cc);
+            float4* mp = reinterpret_cast<float4*>(ms + o);
             float4 m = *mp;
             m.x = fmaf(p.mu, m.x, g4[0]);      // zero outside the matrix
             m.y = fmaf(p.mu, m.y, g4[1]);
@@ -329,24 +373,35 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
             split_tf32(m.z, h.z, l.z);
             split_tf32(m.w, h.w, l.w);
             *reinterpret_cast<uint4*>(mp) = h;
-            *reinterpret_cast<uint4*>(mlo + rr * kSkLd + cc) = l;
+            *reinterpret_cast<uint4*>(mlo + o) = l;
         }
-        for (int q = threadIdx.x; q < kSkCols * KT; q += kThreads) {
-            const int jj = q / KT, t = q % KT;
-            split_tf32(os[q], omh[jj * S::kOmLd + t], oml[jj * S::kOmLd + t]);
+        // Omega^T high and low parts: a thread takes 4 consecutive columns t of one row jj
+        for (int q = threadIdx.x; q < kSkCols * (KT / 4); q += kThreads) {
+            const int jj = q % kSkCols, t0 = (q / kSkCols) * 4;
+            const float4 v = *reinterpret_cast<const float4*>(os + jj * S::kOmLd + t0);
+            const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int t = t0 + e, o = t * kSkCols + swz(t, jj);
+                split_tf32(vv[e], oth[o], otl[o]);
+            }
         }
         __syncthreads();
-        // Y[16 mt + .., n0 + ..] += M[rows, chunk] Omega[chunk, columns]
+        // Y[16 warp + .., :] += M[rows, chunk] Omega[chunk, :]
         const uint32_t* mh = reinterpret_cast<const uint32_t*>(ms);
+        const int ra = 16 * warp + g;          // rows ra and ra + 8 share a swizzle
 #pragma unroll
-        for (int kk = 0; kk < kSkCols; kk += 8) {
-            const int a0 = (16 * mt + g) * kSkLd + kk + q4;
-            const uint32_t ah[4] = {mh[a0], mh[a0 + 8 * kSkLd], mh[a0 + 4], mh[a0 + 8 * kSkLd + 4]};
-            const uint32_t al[4] = {mlo[a0], mlo[a0 + 8 * kSkLd], mlo[a0 + 4], mlo[a0 + 8 * kSkLd + 4]};
+        for (int kk = 0; kk < kSkCols; kk += 16) {
+            const int co = swz(ra, kk + 4 * q4);
+            Frag16 fa, fb;
+            ld_frag16(fa, mh, mlo, ra * kSkCols + co);
+            ld_frag16(fb, mh, mlo, (ra + 8) * kSkCols + co);
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                const int b0 = (kk + q4) * S::kOmLd + n0 + 8 * t + g;
-                mma3_tf32(acc[t], ah, al, omh[b0], omh[b0 + 4 * S::kOmLd], oml[b0], oml[b0 + 4 * S::kOmLd]);
+                const int n = 8 * t + g;
+                Frag16 fo;
+                ld_frag16(fo, oth, otl, n * kSkCols + swz(n, kk + 4 * q4));
+                mma16(acc[t], fa, fb, fo);
             }
         }
         __syncthreads();                       // stage s and the split buffers free for the next chunks
@@ -355,9 +410,9 @@ __global__ void __launch_bounds__(kThreads, 2) lim_sketch(const __grid_constant_
     float* ys = reinterpret_cast<float*>(sm);  // [kSkRows][KT]
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-        const int col = n0 + 8 * t + 2 * q4;
-        *reinterpret_cast<float2*>(ys + (16 * mt + g) * KT + col) = make_float2(acc[t][0], acc[t][1]);
-        *reinterpret_cast<float2*>(ys + (16 * mt + g + 8) * KT + col) = make_float2(acc[t][2], acc[t][3]);
+        const int col = 8 * t + 2 * q4;
+        *reinterpret_cast<float2*>(ys + (16 * warp + g) * KT + col) = make_float2(acc[t][0], acc[t][1]);
+        *reinterpret_cast<float2*>(ys + (16 * warp + g + 8) * KT + col) = make_float2(acc[t][2], acc[t][3]);
     }
     __syncthreads();
     for (int q = threadIdx.x; q < kSkRows * (KT / 4); q += kThreads) {
@@ -431,9 +486,12 @@ __global__ void __launch_bounds__(kSmallThreads) lim_chol(const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------
-// 3 / 6. rows of Y times the matrix's k x k factor K, in place (fp64 sums)
+// 3 / 6. rows times the matrix's k x k factor K, in place (fp64 sums): step 3
+//    reads Y and forms Q = Y R^-1, step 6 reads Q (high + low parts) and forms
+//    Z = Q P.  The result is stored as its tf32 high and low parts, the
+//    operands of the tensor-core products that read it.
 // ---------------------------------------------------------------------------
-template <int KT>
+template <int KT, bool FROM_SPLIT>
 __global__ void __launch_bounds__(kThreads) lim_rowmul(const __grid_constant__ LimParams p) {
     __shared__ double Ks[KT * KT];
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 1)];
@@ -442,11 +500,16 @@ __global__ void __launch_bounds__(kThreads) lim_rowmul(const __grid_constant__ L
     const int i = (blockIdx.x - E.t_rows) * kThreads + threadIdx.x;
     if (i >= E.rows) return;
     float* row = E.Y + (long long)i * KT;
+    float* rlo = E.Ylo + (long long)i * KT;
     float y[KT];
 #pragma unroll
     for (int t = 0; t < KT; t += 4) {
         const float4 v = *reinterpret_cast<const float4*>(row + t);
         y[t] = v.x; y[t + 1] = v.y; y[t + 2] = v.z; y[t + 3] = v.w;
+        if (FROM_SPLIT) {
+            const float4 w = *reinterpret_cast<const float4*>(rlo + t);
+            y[t] += w.x; y[t + 1] += w.y; y[t + 2] += w.z; y[t + 3] += w.w;
+        }
     }
     // four output columns at a time, stored as they are formed (the row was read whole)
 #pragma unroll 1
@@ -460,7 +523,13 @@ __global__ void __launch_bounds__(kThreads) lim_rowmul(const __grid_constant__ L
             s2 = fma(ya, Ks[a * KT + j + 2], s2);
             s3 = fma(ya, Ks[a * KT + j + 3], s3);
         }
-        *reinterpret_cast<float4*>(row + j) = make_float4((float)s0, (float)s1, (float)s2, (float)s3);
+        uint4 h, l;
+        split_tf32((float)s0, h.x, l.x);
+        split_tf32((float)s1, h.y, l.y);
+        split_tf32((float)s2, h.z, l.z);
+        split_tf32((float)s3, h.w, l.w);
+        *reinterpret_cast<uint4*>(row + j) = h;
+        *reinterpret_cast<uint4*>(rlo + j) = l;
     }
 }
 
@@ -468,62 +537,70 @@ __global__ void __launch_bounds__(kThreads) lim_rowmul(const __grid_constant__ L
 // 4. B^T = M^T Q (+ share of B B^T)
 // ---------------------------------------------------------------------------
 // Shared memory of the projection: kPjStages stages of M rows [kPjRows][kPjLd]
-// (the block's columns) and Q rows [kPjRows][KT], then one buffer each of the
-// chunk's Q high and low tf32 parts [kPjRows][KT + 8].  The pitches (8 words
-// past a multiple of 32) make the fragment loads conflict-free.
+// (the block's columns) and of Q's high and low parts [kPjRows][KT + 8].  The
+// pitches (8 words past a multiple of 32) make the fragment loads
+// conflict-free.
 constexpr int kPjLd = kPjCols + 8;
 
 template <int KT>
 struct ProjSmem {
     static constexpr int kQLd = KT + 8;
     static constexpr int kM = kPjRows * kPjLd * 4;
-    static constexpr int kStage = kM + kPjRows * KT * 4;
-    static constexpr int kQHi = kPjStages * kStage;
-    static constexpr int kQLo = kQHi + kPjRows * kQLd * 4;
-    static constexpr int kBytes = kQLo + kPjRows * kQLd * 4;
+    static constexpr int kQ = kPjRows * kQLd * 4;
+    static constexpr int kStage = kM + 2 * kQ;
+    static constexpr int kBytes = kPjStages * kStage;
+    static_assert(kStage % 16 == 0, "16-byte aligned stages");
 };
 
+// Block b of the projection: column block cb of its matrix and row segment
+// seg (rows seg * kPjSegRows ..).  A matrix with more rows than one segment
+// has each segment's partial B^T written to Bpart; the segment that finishes
+// a column block last (counted in pj_count) adds the partials in segment
+// order and finishes the block: the same sums in the same order on every run.
 template <int KT>
-__global__ void __launch_bounds__(kThreads, KT == 32 ? 3 : 2) lim_project(const __grid_constant__ LimParams p) {
+__global__ void __launch_bounds__(kThreads, 2) lim_project(const __grid_constant__ LimParams p) {
     using S = ProjSmem<KT>;
     constexpr int NT = KT / 8;                 // 8-column MMA tiles: a warp takes every column of Q
     static_assert(kPjCols == 16 * (kThreads / 32), "one 16-column MMA tile of M per warp");
     extern __shared__ __align__(16) unsigned char sm[];
+    __shared__ int last;
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 2)];
-    const int c0 = (blockIdx.x - E.t_proj) * kPjCols;
+    const int local = blockIdx.x - E.t_proj, cb = local / E.nseg, seg = local % E.nseg;
+    const int c0 = cb * kPjCols;
+    const int r_begin = seg * kPjSegRows, r_end = min(E.rows, r_begin + kPjSegRows);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q4 = lane & 3;
-    const int nchunks = (E.rows + kPjRows - 1) / kPjRows;
-    uint32_t* qh = reinterpret_cast<uint32_t*>(sm + S::kQHi);
-    uint32_t* ql = reinterpret_cast<uint32_t*>(sm + S::kQLo);
+    const int nchunks = (r_end - r_begin + kPjRows - 1) / kPjRows;
     float acc[NT][4];
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
         for (int h = 0; h < 4; ++h) acc[t][h] = 0.f;
 
-    // rows i0.. of M (this block's columns) and of Q into stage s
+    // rows i0.. of M (this block's columns) and of Q's two parts into stage s
     auto issue = [&](int ch, int s) {
-        const int i0 = ch * kPjRows;
+        const int i0 = r_begin + ch * kPjRows;
         float* ms = reinterpret_cast<float*>(sm + s * S::kStage);
-        float* qs = reinterpret_cast<float*>(sm + s * S::kStage + S::kM);
+        float* qh = reinterpret_cast<float*>(sm + s * S::kStage + S::kM);
+        float* ql = reinterpret_cast<float*>(sm + s * S::kStage + S::kM + S::kQ);
         if (E.vec_ok) {
             constexpr int MP = kPjCols / 4;
             for (int q = threadIdx.x; q < kPjRows * MP; q += kThreads) {
                 const int rr = q / MP, pc = q % MP, i = i0 + rr, j = c0 + pc * 4;
-                const bool in = i < E.rows && j < E.cols;
+                const bool in = i < r_end && j < E.cols;
                 cp_async16(ms + rr * kPjLd + pc * 4, E.M + (in ? (long long)i * E.cols + j : 0), in ? 16u : 0u);
             }
         } else {
             for (int q = threadIdx.x; q < kPjRows * kPjCols; q += kThreads) {
                 const int rr = q / kPjCols, cc = q % kPjCols, i = i0 + rr, j = c0 + cc;
-                ms[rr * kPjLd + cc] = (i < E.rows && j < E.cols) ? E.M[(long long)i * E.cols + j] : 0.f;
+                ms[rr * kPjLd + cc] = (i < r_end && j < E.cols) ? E.M[(long long)i * E.cols + j] : 0.f;
             }
         }
         constexpr int QP = KT / 4;
-        for (int q = threadIdx.x; q < kPjRows * QP; q += kThreads) {
-            const int rr = q / QP, pc = q % QP, i = i0 + rr;
-            const bool in = i < E.rows;
-            cp_async16(qs + rr * KT + pc * 4, E.Y + (in ? (long long)i * KT + pc * 4 : 0), in ? 16u : 0u);
+        for (int q = threadIdx.x; q < 2 * kPjRows * QP; q += kThreads) {
+            const int part = q / (kPjRows * QP), r = q % (kPjRows * QP), rr = r / QP, pc = r % QP, i = i0 + rr;
+            const bool in = i < r_end;
+            const float* src = (part ? E.Ylo : E.Y) + (in ? (long long)i * KT + pc * 4 : 0);
+            cp_async16((part ? ql : qh) + rr * S::kQLd + pc * 4, src, in ? 16u : 0u);
         }
         cp_async_commit();
     };
@@ -536,12 +613,8 @@ __global__ void __launch_bounds__(kThreads, KT == 32 ? 3 : 2) lim_project(const 
         cp_async_wait<kPjStages - 1>();
         __syncthreads();
         const float* ms = reinterpret_cast<const float*>(sm + (ch % kPjStages) * S::kStage);
-        const float* qs = reinterpret_cast<const float*>(sm + (ch % kPjStages) * S::kStage + S::kM);
-        for (int q = threadIdx.x; q < kPjRows * KT; q += kThreads) {
-            const int rr = q / KT, t = q % KT;
-            split_tf32(qs[q], qh[rr * S::kQLd + t], ql[rr * S::kQLd + t]);
-        }
-        __syncthreads();
+        const uint32_t* qh = reinterpret_cast<const uint32_t*>(sm + (ch % kPjStages) * S::kStage + S::kM);
+        const uint32_t* ql = reinterpret_cast<const uint32_t*>(sm + (ch % kPjStages) * S::kStage + S::kM + S::kQ);
         // B^T[16 warp + .., :] += M[chunk, columns]^T Q[chunk, :]
 #pragma unroll
         for (int kk = 0; kk < kPjRows; kk += 8) {
@@ -557,10 +630,9 @@ __global__ void __launch_bounds__(kThreads, KT == 32 ? 3 : 2) lim_project(const 
                 mma3_tf32(acc[t], ah, al, qh[b0], qh[b0 + 4 * S::kQLd], ql[b0], ql[b0 + 4 * S::kQLd]);
             }
         }
-        __syncthreads();                       // this stage and the split buffers are refilled next
+        __syncthreads();                       // this stage is refilled next
     }
     cp_async_wait<0>();
-    // B^T to the workspace, and this block's columns' share of B B^T
     float* bs = reinterpret_cast<float*>(sm);  // [kPjCols][KT]
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
@@ -569,11 +641,45 @@ __global__ void __launch_bounds__(kThreads, KT == 32 ? 3 : 2) lim_project(const 
         *reinterpret_cast<float2*>(bs + (16 * warp + g + 8) * KT + col) = make_float2(acc[t][2], acc[t][3]);
     }
     __syncthreads();
+    if (E.nseg > 1) {                          // uniform over the block
+        float* part = E.Bpart + ((long long)seg * E.cols + c0) * KT;
+        for (int q = threadIdx.x; q < kPjCols * (KT / 4); q += kThreads) {
+            const int cc = q / (KT / 4), pc = q % (KT / 4);
+            if (c0 + cc < E.cols)
+                *reinterpret_cast<float4*>(part + cc * KT + 4 * pc) = *reinterpret_cast<const float4*>(bs + cc * KT + 4 * pc);
+        }
+        __threadfence();                       // this segment's partial visible before it is counted
+        __syncthreads();
+        if (threadIdx.x == 0) last = atomicAdd(E.pj_count + cb, 1) == E.nseg - 1;
+        __syncthreads();
+        if (!last) return;
+        __threadfence();                       // the other segments' partials, counted before ours
+        for (int q = threadIdx.x; q < kPjCols * (KT / 4); q += kThreads) {
+            const int cc = q / (KT / 4), pc = q % (KT / 4);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c0 + cc < E.cols)
+                for (int sg = 0; sg < E.nseg; ++sg) {
+                    const float4 w = __ldcg(reinterpret_cast<const float4*>(
+                        E.Bpart + ((long long)sg * E.cols + c0 + cc) * KT + 4 * pc));
+                    v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+                }
+            *reinterpret_cast<float4*>(bs + cc * KT + 4 * pc) = v;
+        }
+        __syncthreads();
+    }
+    // B^T (high and low parts) to the workspace, and this block's columns' share of B B^T
     for (int q = threadIdx.x; q < kPjCols * (KT / 4); q += kThreads) {
         const int cc = q / (KT / 4), pc = q % (KT / 4), j = c0 + cc;
-        if (j < E.cols)
-            *reinterpret_cast<float4*>(E.Bt + (long long)j * KT + 4 * pc) =
-                *reinterpret_cast<const float4*>(bs + cc * KT + 4 * pc);
+        if (j < E.cols) {
+            const float4 v = *reinterpret_cast<const float4*>(bs + cc * KT + 4 * pc);
+            uint4 h, l;
+            split_tf32(v.x, h.x, l.x);
+            split_tf32(v.y, h.y, l.y);
+            split_tf32(v.z, h.z, l.z);
+            split_tf32(v.w, h.w, l.w);
+            *reinterpret_cast<uint4*>(E.Bt + (long long)j * KT + 4 * pc) = h;
+            *reinterpret_cast<uint4*>(E.Btlo + (long long)j * KT + 4 * pc) = l;
+        }
     }
     add_gram<KT>(bs, min(kPjCols, E.cols - c0), p.k, E.Cg);
 }
@@ -588,25 +694,36 @@ __global__ void __launch_bounds__(kThreads, KT == 32 ? 3 : 2) lim_project(const 
 template <int KT>
 __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimParams p) {
     constexpr int LD = KT + 1;          // padded rows: a column of C spreads over the banks
+    constexpr int NP = KT / 2, NR = KT - 1;   // pairs per round, rounds per sweep (on all KT indices)
     extern __shared__ __align__(16) double dsm[];
     double* C = dsm;                    // [KT][LD]
     double* Ev = dsm + KT * LD;         // [KT][LD] eigenvectors (columns)
-    double* cs = Ev + KT * LD;          // [KT/2] cosines
-    double* sn = cs + KT / 2;           // [KT/2] sines
-    double* lam = sn + KT / 2;          // [KT] eigenvalues
-    int* pp = reinterpret_cast<int*>(lam + KT);   // [KT/2]
-    int* pq = pp + KT / 2;                         // [KT/2]
+    double* cs = Ev + KT * LD;          // [NP] cosines
+    double* sn = cs + NP;               // [NP] sines
+    double* lam = sn + NP;              // [KT] eigenvalues
+    unsigned char* pa = reinterpret_cast<unsigned char*>(lam + KT);   // [NR][NP] pair tables
+    unsigned char* pb = pa + NR * NP;
     __shared__ int rotated, nonfinite;
     const LimEntry& E = p.e[blockIdx.x];
-    const int k = p.k, ke = k + (k & 1), n = ke - 1, np = ke / 2;
+    const int k = p.k;
     if (threadIdx.x == 0) nonfinite = 0;
     __syncthreads();
+    // C padded to KT x KT with zeros: indices >= k never rotate (their couplings are 0)
     for (int idx = threadIdx.x; idx < KT * KT; idx += blockDim.x) {
         const int a = idx / KT, b = idx % KT;
         const double v = (a < k && b < k) ? (a <= b ? E.Cg[a * KT + b] : E.Cg[b * KT + a]) : 0.0;
         if (!isfinite(v)) nonfinite = 1;
         C[a * LD + b] = v;
         Ev[a * LD + b] = a == b ? 1.0 : 0.0;
+    }
+    // round-robin schedule: in round rd, pair 0 is (NR, rd) and pair i is
+    // ((rd + i) mod NR, (rd - i) mod NR); every index pair meets once a sweep
+    for (int idx = threadIdx.x; idx < NR * NP; idx += blockDim.x) {
+        const int rd = idx / NP, i = idx % NP;
+        int a = i == 0 ? NR : (rd + i) % NR, b = i == 0 ? rd : (rd - i + NR) % NR;
+        if (a > b) { const int t = a; a = b; b = t; }
+        pa[idx] = (unsigned char)a;
+        pb[idx] = (unsigned char)b;
     }
     __syncthreads();
     if (nonfinite || *E.bad) {          // no factor for a marked matrix: its W is kept
@@ -620,31 +737,37 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
     double tr = 0.0;
     for (int a = 0; a < k; ++a) tr += fabs(C[a * LD + a]);
     const double floor_abs = kRotTol * 0.1 * tr;
-    for (int sweep = 0; sweep < kMaxSweeps && n > 0; ++sweep) {
+    for (int sweep = 0; sweep < kMaxSweeps; ++sweep) {
         if (threadIdx.x == 0) rotated = 0;
         __syncthreads();
-        for (int rd = 0; rd < n; ++rd) {
-            if (threadIdx.x < np) {
-                const int i = threadIdx.x;
-                int a = i == 0 ? n : (rd + i) % n, b = i == 0 ? rd : (rd - i + n) % n;
-                if (a > b) { const int t = a; a = b; b = t; }
+        for (int rd = 0; rd < NR; ++rd) {
+            const unsigned char* ra = pa + rd * NP;
+            const unsigned char* rb = pb + rd * NP;
+            if (threadIdx.x < NP) {
+                const int i = threadIdx.x, a = ra[i], b = rb[i];
                 const double apq = C[a * LD + b], app = C[a * LD + a], aqq = C[b * LD + b];
                 double c = 1.0, s = 0.0;
-                if (fabs(apq) > kRotTol * sqrt(fabs(app * aqq)) && fabs(apq) > floor_abs) {
-                    const double tau = (aqq - app) / (2.0 * apq);
-                    const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
-                    c = 1.0 / sqrt(1.0 + t * t);
+                if (apq * apq > kRotTol * kRotTol * fabs(app * aqq) && fabs(apq) > floor_abs) {
+                    // the textbook rotation t = sign(tau) / (|tau| + sqrt(1 + tau^2)),
+                    // tau = d / (2 apq), d = aqq - app, multiplied through by 2 |apq|:
+                    // one square root, one division and one reciprocal square root
+                    const double d = aqq - app;
+                    const double t = (d >= 0.0 ? 2.0 : -2.0) * apq / (fabs(d) + sqrt(d * d + 4.0 * apq * apq));
+                    c = rsqrt(1.0 + t * t);
                     s = t * c;
                     rotated = 1;
                 }
-                pp[i] = a; pq[i] = b; cs[i] = c; sn[i] = s;
+                cs[i] = c; sn[i] = s;
             }
             __syncthreads();
-            for (int idx = threadIdx.x; idx < np * np; idx += blockDim.x) {   // C <- J^T C J, block by block
-                const int i = idx / np, j = idx % np;
+#pragma unroll
+            for (int it = 0; it < (NP * NP + kThreads - 1) / kThreads; ++it) {   // C <- J^T C J, block by block
+                const int idx = threadIdx.x + it * kThreads;
+                if (idx >= NP * NP) break;
+                const int i = idx / NP, j = idx % NP;
                 const double c1 = cs[i], s1 = sn[i], c2 = cs[j], s2 = sn[j];
                 if (s1 == 0.0 && s2 == 0.0) continue;
-                const int a1 = pp[i], b1 = pq[i], a2 = pp[j], b2 = pq[j];
+                const int a1 = ra[i], b1 = rb[i], a2 = ra[j], b2 = rb[j];
                 const double x = C[a1 * LD + a2], y = C[a1 * LD + b2], z = C[b1 * LD + a2], w = C[b1 * LD + b2];
                 const double r0 = c1 * x - s1 * z, r1 = c1 * y - s1 * w;   // rows a1, b1 rotated
                 const double r2 = s1 * x + c1 * z, r3 = s1 * y + c1 * w;
@@ -653,13 +776,17 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
                 C[b1 * LD + a2] = c2 * r2 - s2 * r3;
                 C[b1 * LD + b2] = s2 * r2 + c2 * r3;
             }
-            for (int idx = threadIdx.x; idx < ke * np; idx += blockDim.x) {   // E <- E J
-                const int row = idx / np, i = idx % np;
+#pragma unroll
+            for (int it = 0; it < (KT * NP + kThreads - 1) / kThreads; ++it) {   // E <- E J
+                const int idx = threadIdx.x + it * kThreads;
+                if (idx >= KT * NP) break;
+                const int row = idx / NP, i = idx % NP;
                 const double c = cs[i], s = sn[i];
                 if (s == 0.0) continue;
-                const double u = Ev[row * LD + pp[i]], v = Ev[row * LD + pq[i]];
-                Ev[row * LD + pp[i]] = c * u - s * v;
-                Ev[row * LD + pq[i]] = s * u + c * v;
+                const int a = ra[i], b = rb[i];
+                const double u = Ev[row * LD + a], v = Ev[row * LD + b];
+                Ev[row * LD + a] = c * u - s * v;
+                Ev[row * LD + b] = s * u + c * v;
             }
             __syncthreads();
         }
@@ -694,150 +821,132 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
 // ---------------------------------------------------------------------------
 // 7. O = Z B and the weight update
 // ---------------------------------------------------------------------------
-// Shared memory of lim_update: Z rows [kUpRows][KT + 4] and the B^T rows of
-// the tile's columns [kUpCols][KT + 4] as loaded, each then replaced by its
-// tf32 high part with the low parts in two more such arrays, and the tile of W
-// [kUpRows][kUpCols + 8] in W's type.  The pitches make the fragment loads
-// and the epilogue's accesses to W conflict-free.
-template <int KT, int W_DT>
+// Shared memory of lim_update: the high and low parts of Z's rows and of the
+// B^T rows of the tile's columns, [kUpRows][KT] each, swizzled.  After the
+// product the same bytes hold the tile of O, [kUpRows][kUpCols] fp32 with
+// 8-word groups XOR-swizzled by row (conflict-free fragment stores), which the
+// epilogue reads 8 consecutive columns at a time next to W's 16-byte pieces.
+template <int KT>
 struct UpdSmem {
-    static constexpr int kLd = KT + 4;
-    static constexpr int kWLd = kUpCols + 8;
-    static constexpr int kArr = kUpRows * kLd * 4;
-    static constexpr int kZ = 0, kZlo = kArr, kBt = 2 * kArr, kBtlo = 3 * kArr, kW = 4 * kArr;
-    static constexpr int kBytes = kW + kUpRows * kWLd * g_size<W_DT>();
-    static_assert(kUpRows == kUpCols, "Z and B^T tiles share a shape");
+    static constexpr int kArr = kUpRows * KT * 4;
+    static constexpr int kZh = 0, kZl = kArr, kBh = 2 * kArr, kBl = 3 * kArr;
+    static constexpr int kO = kUpRows * kUpCols * 4;
+    static constexpr int kBytes = 4 * kArr > kO ? 4 * kArr : kO;
+    static_assert(kUpRows == kUpCols && KT % 32 == 0, "Z and B^T tiles share a shape; swizzled 32-word rows");
 };
+
+// word offset of O[r][c] in the staged tile
+__device__ __forceinline__ int o_off(int r, int c) { return r * kUpCols + (c ^ ((r & 7) << 3)); }
 
 template <int KT, int W_DT>
 __global__ void __launch_bounds__(kThreads, 2) lim_update(const __grid_constant__ LimParams p) {
-    using S = UpdSmem<KT, W_DT>;
-    constexpr int WSZ = g_size<W_DT>();
+    using S = UpdSmem<KT>;
     constexpr int NT = kUpCols / 8;            // 8-column MMA tiles: a warp takes 16 rows x every column
+    constexpr int ZP = KT / 4;                 // 16-byte pieces per row of Z / B^T
     static_assert(kUpRows == 16 * (kThreads / 32), "one 16-row MMA tile per warp");
     extern __shared__ __align__(16) unsigned char sm[];
-    float* Zs = reinterpret_cast<float*>(sm + S::kZ);
-    float* Bts = reinterpret_cast<float*>(sm + S::kBt);
-    uint32_t* Zlo = reinterpret_cast<uint32_t*>(sm + S::kZlo);
-    uint32_t* Btlo = reinterpret_cast<uint32_t*>(sm + S::kBtlo);
-    unsigned char* Ws = sm + S::kW;
+    const uint32_t* Zh = reinterpret_cast<const uint32_t*>(sm + S::kZh);
+    const uint32_t* Zl = reinterpret_cast<const uint32_t*>(sm + S::kZl);
+    const uint32_t* Bh = reinterpret_cast<const uint32_t*>(sm + S::kBh);
+    const uint32_t* Bl = reinterpret_cast<const uint32_t*>(sm + S::kBl);
+    float* Os = reinterpret_cast<float*>(sm);
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 3)];
     const int tile = blockIdx.x - E.t_upd;
     const int tiles_c = (E.cols + kUpCols - 1) / kUpCols;
     const int row0 = (tile / tiles_c) * kUpRows, c0 = (tile % tiles_c) * kUpCols;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q4 = lane & 3;
     const bool skip = *E.bad != 0;
-    const bool wtile = E.vec_ok && !skip;      // W through shared memory (16-byte pieces)
-    // every global read of the tile in one asynchronous group: Z rows, the
-    // B^T rows of the tile's columns, and (aligned rows) the tile of W
-    constexpr int ZP = KT / 4;
-    for (int q = threadIdx.x; q < kUpRows * ZP; q += kThreads) {
-        const int rr = q / ZP, pc = q % ZP, i = row0 + rr;
-        const bool in = i < E.rows;
-        cp_async16(Zs + rr * S::kLd + pc * 4, E.Y + (in ? (long long)i * KT + pc * 4 : 0), in ? 16u : 0u);
-    }
-    for (int q = threadIdx.x; q < kUpCols * ZP; q += kThreads) {
-        const int jj = q / ZP, pc = q % ZP, j = c0 + jj;
-        const bool in = j < E.cols;
-        cp_async16(Bts + jj * S::kLd + pc * 4, E.Bt + (in ? (long long)j * KT + pc * 4 : 0), in ? 16u : 0u);
-    }
-    if (wtile) {
-        constexpr int WP = kUpCols * WSZ / 16, WE = 16 / WSZ;   // 16-byte pieces per row, elements per piece
-        for (int q = threadIdx.x; q < kUpRows * WP; q += kThreads) {
-            const int rr = q / WP, pc = q % WP, i = row0 + rr, j = c0 + pc * WE;
-            const bool in = i < E.rows && j < E.cols;
-            const char* src = static_cast<const char*>(E.W) + (in ? ((long long)i * E.cols + j) * WSZ : 0);
-            cp_async16(Ws + (rr * S::kWLd + pc * WE) * WSZ, src, in ? 16u : 0u);
-        }
+    // the two parts of Z's rows and of the tile's B^T rows, one asynchronous group
+    for (int q = threadIdx.x; q < 4 * kUpRows * ZP; q += kThreads) {
+        const int arr = q / (kUpRows * ZP), r = q % (kUpRows * ZP), rr = r / ZP, pc = r % ZP;
+        const int idx = arr < 2 ? row0 + rr : c0 + rr, lim = arr < 2 ? E.rows : E.cols;
+        const bool in = idx < lim;
+        const float* base = arr == 0 ? E.Y : arr == 1 ? E.Ylo : arr == 2 ? E.Bt : E.Btlo;
+        cp_async16(sm + arr * S::kArr + (rr * KT + swz(rr, pc * 4)) * 4, base + (in ? (long long)idx * KT + pc * 4 : 0),
+                   in ? 16u : 0u);
     }
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
-    const int kk8 = (p.k + 7) & ~7;            // columns of Z (and of B^T) past k are zero
-    for (int q = threadIdx.x; q < kUpRows * KT; q += kThreads) {
-        const int rr = q / KT, t = q % KT, o = rr * S::kLd + t;
-        if (t >= kk8) continue;
-        uint32_t h;
-        split_tf32(Zs[o], h, Zlo[o]);
-        Zs[o] = __uint_as_float(h);
-        split_tf32(Bts[o], h, Btlo[o]);
-        Bts[o] = __uint_as_float(h);
-    }
-    __syncthreads();
-    const uint32_t* Zh = reinterpret_cast<const uint32_t*>(Zs);
-    const uint32_t* Bth = reinterpret_cast<const uint32_t*>(Bts);
     float o[NT][4];
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
         for (int c = 0; c < 4; ++c) o[t][c] = 0.f;
+    const int kk16 = (p.k + 15) & ~15;         // columns of Z (and of B^T) past k are zero
+    const int ra = 16 * warp + g;              // rows ra and ra + 8 share a swizzle
 #pragma unroll 1
-    for (int kk = 0; kk < kk8; kk += 8) {
-        const int a0 = (16 * warp + g) * S::kLd + kk + q4;
-        const uint32_t ah[4] = {Zh[a0], Zh[a0 + 8 * S::kLd], Zh[a0 + 4], Zh[a0 + 8 * S::kLd + 4]};
-        const uint32_t al[4] = {Zlo[a0], Zlo[a0 + 8 * S::kLd], Zlo[a0 + 4], Zlo[a0 + 8 * S::kLd + 4]};
+    for (int kk = 0; kk < kk16; kk += 16) {
+        const int co = swz(ra, kk + 4 * q4);
+        Frag16 fa, fb;
+        ld_frag16(fa, Zh, Zl, ra * KT + co);
+        ld_frag16(fb, Zh, Zl, (ra + 8) * KT + co);
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-            // B (k x columns) = (B^T)^T: b0 = B^T[8 t + g][kk + q4]
-            const int b0 = (8 * t + g) * S::kLd + kk + q4;
-            mma3_tf32(o[t], ah, al, Bth[b0], Bth[b0 + 4], Btlo[b0], Btlo[b0 + 4]);
+            // B (k x columns) = (B^T)^T: column n of B is row n of the B^T tile
+            const int n = 8 * t + g;
+            Frag16 fo;
+            ld_frag16(fo, Bh, Bl, n * KT + swz(n, kk + 4 * q4));
+            mma16(o[t], fa, fb, fo);
         }
     }
-    // epilogue: O (optional) and W <- W - eta (gamma O + lambda W); this
-    // thread holds rows 16 warp + g (+ 8), columns 8 t + 2 q4 (+ 1)
+    __syncthreads();                           // Z and B^T no longer read: the tile of O replaces them
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int rr = 16 * warp + g + 8 * h, i = row0 + rr;
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const int cc = 8 * t + 2 * q4, j = c0 + cc;
-            const float v0 = o[t][2 * h], v1 = o[t][2 * h + 1];
-            const bool in0 = i < E.rows && j < E.cols, in1 = i < E.rows && j + 1 < E.cols;
-            if (E.O_out) {
-                const long long idx = (long long)i * E.cols + j;
-                if (E.vec_ok && in0) *reinterpret_cast<float2*>(E.O_out + idx) = make_float2(v0, v1);
-                else {
-                    if (in0) E.O_out[idx] = v0;
-                    if (in1) E.O_out[idx + 1] = v1;
-                }
-            }
-            if (skip) continue;
-            if (wtile) {                       // in shared memory, stored below
-                unsigned char* wp = Ws + (rr * S::kWLd + cc) * WSZ;
-                if (W_DT == DT_FP32) {
-                    float2 w = *reinterpret_cast<float2*>(wp);
-                    w.x = w.x - p.eta * (E.gamma * v0 + p.lambda * w.x);
-                    w.y = w.y - p.eta * (E.gamma * v1 + p.lambda * w.y);
-                    *reinterpret_cast<float2*>(wp) = w;
-                } else {
-                    using T = typename std::conditional<W_DT == DT_BF16, __nv_bfloat16, __half>::type;
-                    const uint32_t u = *reinterpret_cast<const uint32_t*>(wp);
-                    float w0 = unpack_lo<T>(u), w1 = unpack_hi<T>(u);
-                    w0 = w0 - p.eta * (E.gamma * v0 + p.lambda * w0);
-                    w1 = w1 - p.eta * (E.gamma * v1 + p.lambda * w1);
-                    *reinterpret_cast<uint32_t*>(wp) = pack2<T>(w0, w1);
-                }
+    for (int t = 0; t < NT; ++t) {
+        const int cc = 8 * t + 2 * q4;
+        *reinterpret_cast<float2*>(Os + o_off(ra, cc)) = make_float2(o[t][0], o[t][1]);
+        *reinterpret_cast<float2*>(Os + o_off(ra + 8, cc)) = make_float2(o[t][2], o[t][3]);
+    }
+    __syncthreads();
+    // epilogue, 8 consecutive columns per item: O (optional) and
+    // W <- W - eta (gamma O + lambda W), 16-byte pieces of W where aligned
+    for (int q = threadIdx.x; q < kUpRows * (kUpCols / 8); q += kThreads) {
+        const int rr = q / (kUpCols / 8), c8 = (q % (kUpCols / 8)) * 8, i = row0 + rr, j = c0 + c8;
+        if (i >= E.rows || j >= E.cols) continue;
+        const float4 a = *reinterpret_cast<const float4*>(Os + o_off(rr, c8));
+        const float4 b = *reinterpret_cast<const float4*>(Os + o_off(rr, c8) + 4);
+        const float ov[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        const long long idx = (long long)i * E.cols + j;
+        const int nv = min(8, E.cols - j);
+        if (E.O_out) {
+            if (E.vec_ok) {                    // cols % 8 == 0: the item is whole
+                *reinterpret_cast<float4*>(E.O_out + idx) = a;
+                *reinterpret_cast<float4*>(E.O_out + idx + 4) = b;
             } else {
-                const long long idx = (long long)i * E.cols + j;
-                if (in0) {
-                    const float w0 = ld_elem(E.W, idx, W_DT);
-                    st_elem(E.W, idx, W_DT, w0 - p.eta * (E.gamma * v0 + p.lambda * w0));
-                }
-                if (in1) {
-                    const float w1 = ld_elem(E.W, idx + 1, W_DT);
-                    st_elem(E.W, idx + 1, W_DT, w1 - p.eta * (E.gamma * v1 + p.lambda * w1));
-                }
+                for (int e = 0; e < nv; ++e) E.O_out[idx + e] = ov[e];
             }
         }
-    }
-    if (wtile) {                               // uniform over the block
-        __syncthreads();
-        constexpr int WP = kUpCols * WSZ / 16, WE = 16 / WSZ;
-        for (int q = threadIdx.x; q < kUpRows * WP; q += kThreads) {
-            const int rr = q / WP, pc = q % WP, i = row0 + rr, j = c0 + pc * WE;
-            if (i < E.rows && j < E.cols)       // cols % 8 == 0: a piece is wholly in or out
-                *reinterpret_cast<uint4*>(static_cast<char*>(E.W) + ((long long)i * E.cols + j) * WSZ) =
-                    *reinterpret_cast<const uint4*>(Ws + (rr * S::kWLd + pc * WE) * WSZ);
+        if (skip) continue;
+        if (E.vec_ok && W_DT != DT_FP32) {
+            using T = typename std::conditional<W_DT == DT_BF16, __nv_bfloat16, __half>::type;
+            uint4* wp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(E.W) + idx);
+            const uint4 u = *wp;
+            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+            uint32_t r[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float w0 = unpack_lo<T>(uw[e]), w1 = unpack_hi<T>(uw[e]);
+                w0 = w0 - p.eta * (E.gamma * ov[2 * e] + p.lambda * w0);
+                w1 = w1 - p.eta * (E.gamma * ov[2 * e + 1] + p.lambda * w1);
+                r[e] = pack2<T>(w0, w1);
+            }
+            *wp = make_uint4(r[0], r[1], r[2], r[3]);
+        } else if (E.vec_ok) {
+            float4* wp = reinterpret_cast<float4*>(static_cast<float*>(E.W) + idx);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float4 w = wp[hh];
+                w.x = w.x - p.eta * (E.gamma * ov[4 * hh] + p.lambda * w.x);
+                w.y = w.y - p.eta * (E.gamma * ov[4 * hh + 1] + p.lambda * w.y);
+                w.z = w.z - p.eta * (E.gamma * ov[4 * hh + 2] + p.lambda * w.z);
+                w.w = w.w - p.eta * (E.gamma * ov[4 * hh + 3] + p.lambda * w.w);
+                wp[hh] = w;
+            }
+        } else {
+            for (int e = 0; e < nv; ++e) {
+                const float w = ld_elem(E.W, idx + e, W_DT);
+                st_elem(E.W, idx + e, W_DT, w - p.eta * (E.gamma * ov[e] + p.lambda * w));
+            }
         }
     }
 }
@@ -852,14 +961,16 @@ constexpr size_t sketch_smem() { return (size_t)SketchSmem<KT, G_DT>::kBytes; }
 template <int KT>
 constexpr size_t project_smem() { return (size_t)ProjSmem<KT>::kBytes; }
 template <int KT, int W_DT>
-constexpr size_t update_smem() { return (size_t)UpdSmem<KT, W_DT>::kBytes; }
+constexpr size_t update_smem() { return (size_t)UpdSmem<KT>::kBytes; }
 template <int KT>
 constexpr size_t chol_smem() { return sizeof(double) * (2 * KT * KT + KT) + sizeof(int) * KT; }
 template <int KT>
-constexpr size_t eig_smem() { return sizeof(double) * (2 * KT * (KT + 1) + KT / 2 * 2 + KT) + sizeof(int) * KT; }
+constexpr size_t eig_smem() { return sizeof(double) * (2 * KT * (KT + 1) + KT / 2 * 2 + KT) + 2 * (KT - 1) * (KT / 2); }
 
-static_assert(sketch_smem<64, DT_FP32>() >= sizeof(float) * kSkRows * 64, "sketch Y staging fits a stage");
+static_assert(sketch_smem<64, DT_FP32>() >= sizeof(float) * kSkRows * 64, "sketch Y staging fits");
 static_assert(project_smem<64>() >= sizeof(float) * kPjCols * 64, "projection B^T staging fits the stages");
+static_assert(sketch_smem<64, DT_FP32>() <= 227 * 1024 && update_smem<64, DT_FP32>() <= 227 * 1024,
+              "shared memory per block");
 
 template <typename K>
 cudaError_t allow_smem(K kernel, size_t bytes) {
@@ -901,27 +1012,35 @@ muon_status launch_all(LimParams& prm, cudaStream_t s, const LaunchShape& L) {
     trace_begin(MUON_KERNEL_RSVD_SMALL, 2.0 * kk, s);                                // Gram read, R^-1 written
     lim_chol<KT><<<prm.n, kSmallThreads, chol_smem<KT>(), s>>>(prm);
     trace_end(s);
-    trace_begin(MUON_KERNEL_RSVD_SMALL, 8.0 * L.rows_total * KT + kk, s);           // Y read and written
-    lim_rowmul<KT><<<L.rows, kThreads, 0, s>>>(prm);
+    trace_begin(MUON_KERNEL_RSVD_SMALL, 12.0 * L.rows_total * KT + kk, s);          // Y read, Q's parts written
+    lim_rowmul<KT, false><<<L.rows, kThreads, 0, s>>>(prm);
     trace_end(s);
-    trace_begin(MUON_KERNEL_RSVD, L.elems * 4.0 + 4.0 * (L.rows_k + L.cols_k), s);  // M, Q read; B^T written
+    trace_begin(MUON_KERNEL_RSVD, L.elems * 4.0 + 8.0 * (L.rows_k + L.cols_k), s);  // M, Q read; B^T written
     lim_project<KT><<<L.proj, kThreads, project_smem<KT>(), s>>>(prm);
     trace_end(s);
     trace_begin(MUON_KERNEL_RSVD_SMALL, 2.0 * kk, s);                                // Gram read, P written
     lim_eig<KT><<<prm.n, kThreads, eig_smem<KT>(), s>>>(prm);
     trace_end(s);
-    trace_begin(MUON_KERNEL_RSVD_SMALL, 8.0 * L.rows_total * KT + kk, s);           // Q read, Z written
-    lim_rowmul<KT><<<L.rows, kThreads, 0, s>>>(prm);
+    trace_begin(MUON_KERNEL_RSVD_SMALL, 16.0 * L.rows_total * KT + kk, s);          // Q's parts read, Z's written
+    lim_rowmul<KT, true><<<L.rows, kThreads, 0, s>>>(prm);
     trace_end(s);
-    trace_begin(MUON_KERNEL_RSVD, L.elems * 2.0 * wsz + 4.0 * (L.rows_k + L.cols_k), s);   // W read and written
+    trace_begin(MUON_KERNEL_RSVD, L.elems * 2.0 * wsz + 8.0 * (L.rows_k + L.cols_k), s);   // W read and written
     lim_update<KT, W_DT><<<L.upd, kThreads, update_smem<KT, W_DT>(), s>>>(prm);
     trace_end(s);
     (void)k;
     return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
+int proj_segments(int rows) { return (rows + kPjSegRows - 1) / kPjSegRows; }
+int proj_col_blocks(int cols) { return (cols + kPjCols - 1) / kPjCols; }
+
+// Per matrix: Y and its low parts (rows x KT each), B^T and its low parts
+// (cols x KT each), and with more than one projection segment the partial B^T
+// of every segment (nseg x cols x KT).
 size_t matrix_ws(int rows, int cols, int KT) {
-    return align256(sizeof(float) * (size_t)rows * KT) + align256(sizeof(float) * (size_t)cols * KT);
+    const int nseg = proj_segments(rows);
+    return 2 * align256(sizeof(float) * (size_t)rows * KT) + 2 * align256(sizeof(float) * (size_t)cols * KT) +
+           (nseg > 1 ? align256(sizeof(float) * (size_t)nseg * cols * KT) : 0);
 }
 
 int kt_for(int k) { return k <= 32 ? 32 : 64; }
@@ -945,17 +1064,22 @@ muon_status check_shapes(const muon_rsvd_param* params, int n) {
     return MUON_OK;
 }
 
-// Workspace: the per-matrix flags, then the k x k sums that start at zero
-// (Y^T Y, B B^T), then the k x k factors, then per matrix Y and B^T.
+// Workspace: the per-matrix flags, the projection's per-column-block segment
+// counters, then the k x k sums (all these start at zero: Y^T Y, B B^T), then
+// the k x k factors, then the per-matrix arrays.
 struct WsLayout {
-    size_t flags, zero_bytes, gy, cg, kf, mats, total;
+    size_t flags, counts, zero_bytes, gy, cg, kf, mats, total;
 };
 
 WsLayout ws_layout(const muon_rsvd_param* params, int n, int KT) {
     WsLayout L;
     const size_t kk = sizeof(double) * (size_t)KT * KT * n;
+    size_t ncount = 0;
+    for (int i = 0; i < n; ++i)
+        if (proj_segments(params[i].rows) > 1) ncount += proj_col_blocks(params[i].cols);
     L.flags = 0;
-    L.gy = align256(sizeof(int) * (size_t)n);
+    L.counts = align256(sizeof(int) * (size_t)n);
+    L.gy = L.counts + (ncount ? align256(sizeof(int) * ncount) : 0);
     L.cg = L.gy + align256(kk);
     L.zero_bytes = L.cg + align256(kk);
     L.kf = L.zero_bytes;
@@ -1002,6 +1126,7 @@ muon_status limuon_step_batched(const muon_rsvd_param* params, int n, muon_dtype
     // flags and the two Gram sums start at zero
     if (cudaMemsetAsync(ws, 0, W.zero_bytes, s) != cudaSuccess) return MUON_ERR_CUDA;
     int* bad = reinterpret_cast<int*>(ws + W.flags);
+    int* counts = reinterpret_cast<int*>(ws + W.counts);
     double* gy = reinterpret_cast<double*>(ws + W.gy);
     double* cg = reinterpret_cast<double*>(ws + W.cg);
     double* kf = reinterpret_cast<double*>(ws + W.kf);
@@ -1025,8 +1150,19 @@ muon_status limuon_step_batched(const muon_rsvd_param* params, int n, muon_dtype
             E.bad = bad + b + i;
             const size_t kk = (size_t)KT * KT * (b + i);
             E.Gy = gy + kk; E.Cg = cg + kk; E.K = kf + kk;
+            const size_t yb = align256(sizeof(float) * (size_t)q.rows * KT);
+            const size_t bb = align256(sizeof(float) * (size_t)q.cols * KT);
             E.Y = reinterpret_cast<float*>(cur);
-            E.Bt = reinterpret_cast<float*>(cur + align256(sizeof(float) * (size_t)q.rows * KT));
+            E.Ylo = reinterpret_cast<float*>(cur + yb);
+            E.Bt = reinterpret_cast<float*>(cur + 2 * yb);
+            E.Btlo = reinterpret_cast<float*>(cur + 2 * yb + bb);
+            E.nseg = proj_segments(q.rows);
+            E.Bpart = E.nseg > 1 ? reinterpret_cast<float*>(cur + 2 * yb + 2 * bb) : nullptr;
+            E.pj_count = nullptr;
+            if (E.nseg > 1) {
+                E.pj_count = counts;
+                counts += proj_col_blocks(q.cols);
+            }
             cur += matrix_ws(q.rows, q.cols, KT);
             const uintptr_t al = reinterpret_cast<uintptr_t>(q.W) | reinterpret_cast<uintptr_t>(q.G) |
                                  reinterpret_cast<uintptr_t>(q.M) | reinterpret_cast<uintptr_t>(q.O_out);
@@ -1053,7 +1189,7 @@ muon_status limuon_step_batched(const muon_rsvd_param* params, int n, muon_dtype
                 const long long first = tot[w];
                 if (w == 0) { E.t_sketch = (int)first; tot[w] += (E.rows + kSkRows - 1) / kSkRows; }
                 else if (w == 1) { E.t_rows = (int)first; tot[w] += (E.rows + kThreads - 1) / kThreads; }
-                else if (w == 2) { E.t_proj = (int)first; tot[w] += (E.cols + kPjCols - 1) / kPjCols; }
+                else if (w == 2) { E.t_proj = (int)first; tot[w] += (long long)proj_col_blocks(E.cols) * E.nseg; }
                 else {
                     E.t_upd = (int)first;
                     tot[w] += (long long)((E.rows + kUpRows - 1) / kUpRows) * ((E.cols + kUpCols - 1) / kUpCols);

@@ -236,11 +236,17 @@ def test_limuon_argument_checks(lib):
     size = ctypes.c_size_t(0)
     assert L.limuon_workspace_size(one, 1, ctypes.byref(good), ctypes.byref(size)) == mo.OK
     # the per-matrix flag, three k x k fp64 matrices (Y^T Y, B B^T, the factor) on 32 columns,
-    # then Y (4 x 32 floats) and B^T (8 x 32 floats), each region 256-byte aligned
-    assert size.value == 256 + 3 * 32 * 32 * 8 + 512 + 1024
+    # then Y and its low parts (4 x 32 floats each) and B^T and its low parts (8 x 32 floats
+    # each), each region 256-byte aligned
+    assert size.value == 256 + 3 * 32 * 32 * 8 + 2 * 512 + 2 * 1024
     big = mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 40, 8)
     assert L.limuon_workspace_size(one, 1, ctypes.byref(big), ctypes.byref(size)) == mo.OK
-    assert size.value == 256 + 3 * 64 * 64 * 8 + 1024 + 2048   # k = 48 runs on 64 columns
+    assert size.value == 256 + 3 * 64 * 64 * 8 + 2 * 1024 + 2 * 2048   # k = 48 runs on 64 columns
+    # 2500 rows: three projection segments of at most 1024 rows, so one segment counter for the
+    # single 128-column block and the three partial B^T (3 x 8 x 32 floats)
+    tall = (mo.RsvdParam * 1)(mo.RsvdParam(2500, 8, p, p, p, p, float("nan"), None))
+    assert L.limuon_workspace_size(tall, 1, ctypes.byref(good), ctypes.byref(size)) == mo.OK
+    assert size.value == 256 + 256 + 3 * 32 * 32 * 8 + 2 * 2500 * 32 * 4 + 2 * 1024 + 3 * 1024
     too_big = mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 60, 5)
     assert L.limuon_workspace_size(one, 1, ctypes.byref(too_big), ctypes.byref(size)) == mo.ERR_UNSUPPORTED
     for bad in (mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 0, 4), mo.RsvdHParams(0.95, 0.02, 0.0, 1.0, 4, -1),

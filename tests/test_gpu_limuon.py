@@ -18,7 +18,9 @@ hyper-parameters the GPU computes with.  Tolerances:
          within O's tolerance
 Plus: k = 48 (64-column kernels), r above the rank (partial isometry), a zero
 momentum (O = 0), a non-finite gradient element, 130 parameters (two launches),
-and the 72-matrix GPT-2-small set at full size, one matrix per shape group.
+matrices taller than one projection segment (1024 rows; ragged segments and
+column blocks), and the 72-matrix GPT-2-small set at full size, one matrix per
+shape group.
 """
 import numpy as np
 import pytest
@@ -115,6 +117,19 @@ def _check_step(params, w_dtype, hp, t):
 def test_limuon_two_steps_vs_oracle(w_dtype):
     hp = _hp(16, 16)
     params = _params(SHAPES, w_dtype, 32, 16)
+    for t in range(2):
+        _check_step(params, w_dtype, hp, t)
+
+
+TALL = [(2100, 136), (1500, 36), (1025, 64)]
+
+
+@pytest.mark.parametrize("w_dtype", [torch.bfloat16, torch.float32])
+def test_limuon_tall_matrices_segmented_projection(w_dtype):
+    # more than 1024 rows: the projection runs each 128-column block as row
+    # segments whose partial B^T are added by the segment that finishes last
+    hp = _hp(16, 16)
+    params = _params(TALL, w_dtype, 32, 16, seed=11)
     for t in range(2):
         _check_step(params, w_dtype, hp, t)
 
