@@ -502,7 +502,6 @@ def run_model_route(args, w):
 # LiMuon: rank r, oversampling p (k = r + p columns of the test matrix)
 LIMUON_HP = dict(mu=0.95, eta=0.02, gamma=1.0, rank=16, oversample=16, **{"lambda": 0.0})
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 flops at the 1965 MHz maximum SM clock
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 LIMUON_KERNELS = ["lim_sketch", "lim_chol", "lim_rowmul_q", "lim_project", "lim_eig", "lim_rowmul_z", "lim_update"]
 
 
@@ -622,17 +621,25 @@ def run_limuon_route(args, w):
     by, fl = limuon_kernel_work(shapes, k)
     pk, src = peaks()
     kernels = {}
+    # The sketch, projection and update products run on tensor cores in tf32, three MMAs per
+    # product (split operands): their arithmetic floor is 3 x flops at the tf32 dense peak, taken
+    # as the bf16 peak x 1.1 / 2.25 (the nominal tf32 / bf16 ratio).  The row transforms are fp64
+    # sums on CUDA cores; the Cholesky and eigen steps are latency-bound k x k work.
+    tf32_peak = pk["bf16_tflops"] * 1.1 / 2.25
+    tc_kernels = (0, 3, 6)
     for i, name in enumerate(LIMUON_KERNELS[:per]):
         t = kms[i] / 1e3
         kernels[name] = {"us": kms[i] * 1e3, "GB/s": by[i] / t / 1e9, "TFLOP/s": fl[i] / t / 1e12,
-                         "hbm_frac": by[i] / t / 1e9 / pk["hbm_gbs"], "alu_frac": fl[i] / t / 1e12 / FP32_ALU_TFLOPS}
+                         "hbm_frac": by[i] / t / 1e9 / pk["hbm_gbs"]}
+        if i in tc_kernels:
+            kernels[name]["tf32_frac"] = 3.0 * fl[i] / t / 1e12 / tf32_peak
     top = max(range(per), key=lambda i: kms[i])
     t_top = kms[top] / 1e3
     # the binding roof of the dominant kernel: the larger of its memory and arithmetic times
-    if fl[top] / (FP32_ALU_TFLOPS * 1e12) > by[top] / (pk["hbm_gbs"] * 1e9):
-        roof = {"bound": "alu", "achieved": fl[top] / t_top / 1e12, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-                "frac": fl[top] / t_top / 1e12 / FP32_ALU_TFLOPS, "traffic": None,
-                "peak_source": "fp32 FMA units x 1965 MHz maximum SM clock (derived)"}
+    if top in tc_kernels and 3.0 * fl[top] / (tf32_peak * 1e12) > by[top] / (pk["hbm_gbs"] * 1e9):
+        roof = {"bound": "tensor", "achieved": 3.0 * fl[top] / t_top / 1e12, "peak": tf32_peak, "unit": "TFLOP/s",
+                "frac": 3.0 * fl[top] / t_top / 1e12 / tf32_peak, "traffic": None,
+                "peak_source": f"{src} bf16 peak x 1.1 / 2.25 (tf32), three MMAs per product"}
     else:
         roof = {"bound": "hbm", "achieved": by[top] / t_top / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": by[top] / t_top / 1e9 / pk["hbm_gbs"], "traffic": None, "peak_source": f"{src} (copy)"}
