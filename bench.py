@@ -502,6 +502,11 @@ def run_model_route(args, w):
 # LiMuon: rank r, oversampling p (k = r + p columns of the test matrix)
 LIMUON_HP = dict(mu=0.95, eta=0.02, gamma=1.0, rank=16, oversample=16, **{"lambda": 0.0})
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 flops at the 1965 MHz maximum SM clock
+def tf32_tflops(pk):
+    """Dense tf32 tensor peak: the bf16 peak times the nominal tf32 / bf16 ratio (1.1 / 2.25)."""
+    return pk["bf16_tflops"] * 1.1 / 2.25
+
+
 LIMUON_KERNELS = ["lim_sketch", "lim_chol", "lim_rowmul_q", "lim_project", "lim_eig", "lim_rowmul_z", "lim_update"]
 
 
@@ -625,7 +630,7 @@ def run_limuon_route(args, w):
     # product (split operands): their arithmetic floor is 3 x flops at the tf32 dense peak, taken
     # as the bf16 peak x 1.1 / 2.25 (the nominal tf32 / bf16 ratio).  The row transforms are fp64
     # sums on CUDA cores; the Cholesky and eigen steps are latency-bound k x k work.
-    tf32_peak = pk["bf16_tflops"] * 1.1 / 2.25
+    tf32_peak = tf32_tflops(pk)
     tc_kernels = (0, 3, 6)
     for i, name in enumerate(LIMUON_KERNELS[:per]):
         t = kms[i] / 1e3
