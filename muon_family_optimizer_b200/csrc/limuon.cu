@@ -14,11 +14,12 @@
 //     O = Q P B,   P = E_r L_r^{-1/2} E_r^T      (k x k)
 // and Q = Y R^-1 with Y^T Y = R^T R (Cholesky QR).  Every pass over an l x s
 // array streams; everything per matrix touches only k x k data:
-//   1 lim_sketch   M <- mu M + G and Y = M Omega, 64-row blocks over 64-column
-//                  chunks double-buffered in shared memory (cp.async), the
-//                  product on tensor cores (tf32 x 3, fp32 accuracy); each
-//                  block adds its rows' share of the Gram Y^T Y (fp64) to the
-//                  matrix's k x k sum.  Reads G and M, writes M.
+//   1 lim_sketch   M <- mu M + G and Y = M Omega, 128-row blocks over
+//                  32-column chunks double-buffered in shared memory
+//                  (cp.async), the product on tensor cores (warp-level MMA,
+//                  tf32 x 3, fp32 accuracy); each block adds its rows' share
+//                  of the Gram Y^T Y (fp64) to the matrix's k x k sum.  Reads
+//                  G and M, writes M.
 //   2 lim_chol     per matrix (k x k): Cholesky of Y^T Y in fp64 (a column whose
 //                  pivot falls to 1e-10 of its squared norm lies in the span of
 //                  the previous ones and is dropped: its Q column is zero), R^-1.
@@ -36,9 +37,10 @@
 //                  without one; P from the r largest eigenpairs.
 //   6 lim_rowmul   Z = Q P in place.  Q and Z are stored as tf32 high and low
 //                  parts (the operands of 4 and 7).
-//   7 lim_update   O = Z B on 128 x 128 tiles (tensor cores as in 1), fused
-//                  with the weight update (reads and writes W; O never stored
-//                  unless O_out is given).
+//   7 lim_update   O = Z B on 128 x 128 tiles with tcgen05 (kind::tf32,
+//                  accumulator in tensor memory, tf32 x 3), fused with the
+//                  weight update (reads and writes W, staged in shared memory
+//                  while the MMAs run; O never stored unless O_out is given).
 // The sketch and the projection order their blocks longest first.
 // A non-finite momentum element or k x k factor marks its matrix: its W is
 // kept and MUON_FLAG_NONFINITE raised.
@@ -63,8 +65,8 @@ constexpr int kPjCols = 128;      // lim_project: columns per block (one 16-colu
 constexpr int kPjRows = 32;       // lim_project: rows per chunk
 constexpr int kPjStages = 3;
 constexpr int kPjSegRows = 1024;  // lim_project: rows per block; taller matrices split into segments
-constexpr int kUpRows = 128;      // lim_update: tile rows
-constexpr int kUpCols = 128;      // lim_update: tile columns
+constexpr int kUpRows = 128;      // lim_update: tile rows (the MMA's M)
+constexpr int kUpCols = 128;      // lim_update: tile columns (the MMA's N)
 constexpr double kDrop = 1e-10;   // Cholesky pivot / squared column norm below which a column is dropped
 constexpr double kTau2 = 1e-10;   // (singular value / largest)^2 at or below which it counts as zero
 constexpr double kRotTol = 1e-15; // Jacobi: rotate while |C_pq| > kRotTol sqrt(C_pp C_qq)
@@ -148,15 +150,17 @@ __device__ __forceinline__ void add_gram(const float* X, int n, int k, double* d
 
 // ---------------------------------------------------------------------------
 // Tensor-core products with fp32 accuracy.  The three products with k columns
-// (Y = M Omega, B^T = M^T Q, O = Z B) run on mma.sync m16n8k8 in tf32 with
-// each operand split as x = hi + lo (hi = x rounded to tf32, lo = the
-// remainder rounded to tf32) and the product summed as hi*lo + lo*hi + hi*hi
-// into fp32 accumulators ("3xTF32"): the dropped lo*lo term and the rounding
-// of lo are below 2^-21 of |a b| per product, under the fp32 accumulation's
-// own rounding for sums of a few hundred terms or more.  At 2 k flops per
-// element these products are below the HBM ridge once on tensor cores; the
-// legacy warp-level MMA gives that rate with the fragments in registers,
-// next to the fused momentum, Gram and weight-update code.
+// (Y = M Omega, B^T = M^T Q, O = Z B) run in tf32 with each operand split as
+// x = hi + lo (hi = x rounded to tf32, lo = the remainder rounded to tf32) and
+// the product summed as hi*lo + lo*hi + hi*hi into fp32 accumulators
+// ("3xTF32"): the dropped lo*lo term and the rounding of lo are below 2^-21 of
+// |a b| per product, under the fp32 accumulation's own rounding for sums of a
+// few hundred terms or more.  At 2 k flops per element these products are
+// below the HBM ridge once on tensor cores.  The update, a 128 x 128 x k
+// product per tile, runs on tcgen05 (kind::tf32) with the accumulator in
+// tensor memory; the sketch and the projection, whose contraction runs over a
+// whole row or column of the matrix next to per-element momentum work, use
+// the warp-level MMA with the fragments in registers.
 // Fragments of m16n8k8 (g = lane / 4, q = lane % 4): A (16 x 8) a0 = (g, q),
 // a1 = (g + 8, q), a2 = (g, q + 4), a3 = (g + 8, q + 4); B (8 x 8) b0 = (q, g),
 // b1 = (q + 4, g); C (16 x 8) c0, c1 = (g, 2q), (g, 2q + 1); c2, c3 = the same
@@ -190,6 +194,31 @@ __device__ __forceinline__ void mma3_tf32(float (&d)[4], const uint32_t (&ah)[4]
     mma_tf32(d, ah, bl0, bl1);
     mma_tf32(d, al, bh0, bh1);
     mma_tf32(d, ah, bh0, bh1);
+}
+
+// tcgen05 in tf32 (kind::tf32, fp32 accumulators in tensor memory), one CTA.
+// Instruction descriptor: fp32 accumulate, A and B tf32, K-major unless the
+// operand is MN-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_tf32(int a_mn, int b_mn, int M, int N) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Byte offset of the 16-byte piece `pc` (4 words) of row r in a K-major
+// 128-byte-swizzled operand of `rows` rows and KT words per row: KT / 32
+// atoms of [rows][128 bytes], piece (pc % 8) of a row at (pc % 8) ^ (r % 8).
+__device__ __forceinline__ int sw128_piece(int r, int pc, int rows) {
+    return (pc >> 3) * rows * 128 + r * 128 + (((pc & 7) ^ (r & 7)) << 4);
 }
 
 // ---------------------------------------------------------------------------
@@ -821,133 +850,172 @@ __global__ void __launch_bounds__(kThreads) lim_eig(const __grid_constant__ LimP
 // ---------------------------------------------------------------------------
 // 7. O = Z B and the weight update
 // ---------------------------------------------------------------------------
-// Shared memory of lim_update: the high and low parts of Z's rows and of the
-// B^T rows of the tile's columns, [kUpRows][KT] each, swizzled.  After the
-// product the same bytes hold the tile of O, [kUpRows][kUpCols] fp32 with
-// 8-word groups XOR-swizzled by row (conflict-free fragment stores), which the
-// epilogue reads 8 consecutive columns at a time next to W's 16-byte pieces.
-template <int KT>
+// Shared memory of lim_update (1024-byte aligned): the high and low parts of
+// Z's rows [kUpRows] and of the B^T rows of the tile's columns [kUpCols], each
+// K-major with KT words per row in 128-byte swizzled atoms; then the tile of W
+// [kUpRows] rows of kUpCols elements plus 16 bytes (rows 16 bytes apart in the
+// banks: the epilogue's row-per-lane accesses are conflict-free).
+template <int KT, int W_DT>
 struct UpdSmem {
-    static constexpr int kArr = kUpRows * KT * 4;
-    static constexpr int kZh = 0, kZl = kArr, kBh = 2 * kArr, kBl = 3 * kArr;
-    static constexpr int kO = kUpRows * kUpCols * 4;
-    static constexpr int kBytes = 4 * kArr > kO ? 4 * kArr : kO;
-    static_assert(kUpRows == kUpCols && KT % 32 == 0, "Z and B^T tiles share a shape; swizzled 32-word rows");
+    static constexpr int kA = kUpRows * KT * 4, kB = kUpCols * KT * 4;
+    static constexpr int kAh = 0, kAl = kA, kBh = 2 * kA, kBl = 2 * kA + kB, kW = 2 * kA + 2 * kB;
+    static constexpr int kWRow = kUpCols * g_size<W_DT>() + 16;
+    static constexpr int kBytes = kW + kUpRows * kWRow + 1024;   // + the alignment slack
+    static_assert(KT % 32 == 0, "whole 128-byte atoms");
 };
 
-// word offset of O[r][c] in the staged tile
-__device__ __forceinline__ int o_off(int r, int c) { return r * kUpCols + (c ^ ((r & 7) << 3)); }
-
+// 7. O = Z B on a 128 x 128 tile: one thread issues the tf32 MMAs (K = 8
+// each, three per k-step for the split parts) while the tile of W streams into
+// shared memory; eight warps read the fp32 accumulator from tensor memory (a
+// lane quadrant and half of the columns each) and write W row-wise, 16-byte
+// pieces where aligned.
 template <int KT, int W_DT>
 __global__ void __launch_bounds__(kThreads, 2) lim_update(const __grid_constant__ LimParams p) {
-    using S = UpdSmem<KT>;
-    constexpr int NT = kUpCols / 8;            // 8-column MMA tiles: a warp takes 16 rows x every column
+    using S = UpdSmem<KT, W_DT>;
+    constexpr int WSZ = g_size<W_DT>();
     constexpr int ZP = KT / 4;                 // 16-byte pieces per row of Z / B^T
-    static_assert(kUpRows == 16 * (kThreads / 32), "one 16-row MMA tile per warp");
-    extern __shared__ __align__(16) unsigned char sm[];
-    const uint32_t* Zh = reinterpret_cast<const uint32_t*>(sm + S::kZh);
-    const uint32_t* Zl = reinterpret_cast<const uint32_t*>(sm + S::kZl);
-    const uint32_t* Bh = reinterpret_cast<const uint32_t*>(sm + S::kBh);
-    const uint32_t* Bl = reinterpret_cast<const uint32_t*>(sm + S::kBl);
-    float* Os = reinterpret_cast<float*>(sm);
+    constexpr uint32_t kTmemCols = kUpCols;
+    extern __shared__ uint8_t sm_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
     const LimEntry& E = p.e[find_entry(p, blockIdx.x, 3)];
     const int tile = blockIdx.x - E.t_upd;
     const int tiles_c = (E.cols + kUpCols - 1) / kUpCols;
     const int row0 = (tile / tiles_c) * kUpRows, c0 = (tile % tiles_c) * kUpCols;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q4 = lane & 3;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool skip = *E.bad != 0;
-    // the two parts of Z's rows and of the tile's B^T rows, one asynchronous group
-    for (int q = threadIdx.x; q < 4 * kUpRows * ZP; q += kThreads) {
-        const int arr = q / (kUpRows * ZP), r = q % (kUpRows * ZP), rr = r / ZP, pc = r % ZP;
-        const int idx = arr < 2 ? row0 + rr : c0 + rr, lim = arr < 2 ? E.rows : E.cols;
-        const bool in = idx < lim;
-        const float* base = arr == 0 ? E.Y : arr == 1 ? E.Ylo : arr == 2 ? E.Bt : E.Btlo;
-        cp_async16(sm + arr * S::kArr + (rr * KT + swz(rr, pc * 4)) * 4, base + (in ? (long long)idx * KT + pc * 4 : 0),
-                   in ? 16u : 0u);
+    const bool wtile = E.vec_ok && !skip;      // W through shared memory (16-byte pieces)
+    if (threadIdx.x == 0) {
+        mbar_init(&done_bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    // the two parts of Z's rows and of the tile's B^T rows, swizzled for the MMA
+    for (int q = threadIdx.x; q < 2 * (kUpRows + kUpCols) * ZP; q += kThreads) {
+        const int part = q / ((kUpRows + kUpCols) * ZP), r0 = q % ((kUpRows + kUpCols) * ZP);
+        const bool is_a = r0 < kUpRows * ZP;
+        const int r = (is_a ? r0 : r0 - kUpRows * ZP) / ZP, pc = (is_a ? r0 : r0 - kUpRows * ZP) % ZP;
+        const int idx = is_a ? row0 + r : c0 + r;
+        const bool in = idx < (is_a ? E.rows : E.cols);
+        const float* base = is_a ? (part ? E.Ylo : E.Y) : (part ? E.Btlo : E.Bt);
+        const int off = (is_a ? (part ? S::kAl : S::kAh) : (part ? S::kBl : S::kBh)) +
+                        sw128_piece(r, pc, is_a ? kUpRows : kUpCols);
+        cp_async16(sm + off, base + (in ? (long long)idx * KT + pc * 4 : 0), in ? 16u : 0u);
     }
     cp_async_commit();
-    cp_async_wait<0>();
+    if (wtile) {                               // its own group: waited for after the MMAs are issued
+        constexpr int WP = kUpCols * WSZ / 16, WE = 16 / WSZ;   // 16-byte pieces per row, elements per piece
+        for (int q = threadIdx.x; q < kUpRows * WP; q += kThreads) {
+            const int rr = q / WP, pc = q % WP, i = row0 + rr, j = c0 + pc * WE;
+            const bool in = i < E.rows && j < E.cols;
+            const char* src = static_cast<const char*>(E.W) + (in ? ((long long)i * E.cols + j) * WSZ : 0);
+            cp_async16(sm + S::kW + rr * S::kWRow + pc * 16, src, in ? 16u : 0u);
+        }
+    }
+    cp_async_commit();
+    cp_async_wait<1>();                        // the operands (the W tile may still be in flight)
+    fence_proxy_async_smem();                  // the copies, visible to the tensor cores
+    tc_fence_before();
     __syncthreads();
-    float o[NT][4];
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) o[t][c] = 0.f;
-    const int kk16 = (p.k + 15) & ~15;         // columns of Z (and of B^T) past k are zero
-    const int ra = 16 * warp + g;              // rows ra and ra + 8 share a swizzle
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    if (threadIdx.x == 0) {
+        constexpr uint32_t idesc = idesc_tf32(0, 0, kUpRows, kUpCols);
+        const uint32_t base = smem_u32(sm);
+        const int nks = (p.k + 7) / 8;         // columns of Z (and of B^T) past k are zero
+        for (int ks = 0; ks < nks; ++ks) {
+            const uint32_t ao = (ks >> 2) * (kUpRows * 128) + (ks & 3) * 32;
+            const uint32_t bo = (ks >> 2) * (kUpCols * 128) + (ks & 3) * 32;
+            const uint64_t ah = smem_desc_sw128(base + S::kAh + ao, 16, 1024);
+            const uint64_t al = smem_desc_sw128(base + S::kAl + ao, 16, 1024);
+            const uint64_t bh = smem_desc_sw128(base + S::kBh + bo, 16, 1024);
+            const uint64_t bl = smem_desc_sw128(base + S::kBl + bo, 16, 1024);
+            tc_mma_tf32(tmem, ah, bl, idesc, ks > 0 ? 1u : 0u);   // small terms first
+            tc_mma_tf32(tmem, al, bh, idesc, 1u);
+            tc_mma_tf32(tmem, ah, bh, idesc, 1u);
+        }
+        tc_commit(&done_bar);
+    }
+    __syncwarp();
+    cp_async_wait<0>();                        // this thread's pieces of the W tile
+    __syncthreads();                           // everyone's
+    if (mbar_wait(&done_bar, 0, &abort_flag, p.d_status)) {
+        tc_fence_after();
+        // epilogue: warp w reads lanes 32 (w % 4).. (rows) and columns 64 (w / 4)..
+        const int q = warp & 3, h = warp >> 2, rr = 32 * q + lane, i = row0 + rr;
 #pragma unroll 1
-    for (int kk = 0; kk < kk16; kk += 16) {
-        const int co = swz(ra, kk + 4 * q4);
-        Frag16 fa, fb;
-        ld_frag16(fa, Zh, Zl, ra * KT + co);
-        ld_frag16(fb, Zh, Zl, (ra + 8) * KT + co);
+        for (int ch = 0; ch < 2; ++ch) {
+            const int cc = 64 * h + 32 * ch, j0 = c0 + cc;
+            float v[32];
+            tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)cc, v);   // whole warp
+            if (i >= E.rows || j0 >= E.cols) continue;
+            const long long idx = (long long)i * E.cols + j0;
+            const int nv = min(32, E.cols - j0);
+            if (E.O_out) {
+                if (E.vec_ok) {                // cols % 8 == 0: 8-column pieces are whole
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            // B (k x columns) = (B^T)^T: column n of B is row n of the B^T tile
-            const int n = 8 * t + g;
-            Frag16 fo;
-            ld_frag16(fo, Bh, Bl, n * KT + swz(n, kk + 4 * q4));
-            mma16(o[t], fa, fb, fo);
-        }
-    }
-    __syncthreads();                           // Z and B^T no longer read: the tile of O replaces them
+                    for (int e = 0; e < 32; e += 4)
+                        if (e < nv)
+                            *reinterpret_cast<float4*>(E.O_out + idx + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                } else {
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-        const int cc = 8 * t + 2 * q4;
-        *reinterpret_cast<float2*>(Os + o_off(ra, cc)) = make_float2(o[t][0], o[t][1]);
-        *reinterpret_cast<float2*>(Os + o_off(ra + 8, cc)) = make_float2(o[t][2], o[t][3]);
-    }
-    __syncthreads();
-    // epilogue, 8 consecutive columns per item: O (optional) and
-    // W <- W - eta (gamma O + lambda W), 16-byte pieces of W where aligned
-    for (int q = threadIdx.x; q < kUpRows * (kUpCols / 8); q += kThreads) {
-        const int rr = q / (kUpCols / 8), c8 = (q % (kUpCols / 8)) * 8, i = row0 + rr, j = c0 + c8;
-        if (i >= E.rows || j >= E.cols) continue;
-        const float4 a = *reinterpret_cast<const float4*>(Os + o_off(rr, c8));
-        const float4 b = *reinterpret_cast<const float4*>(Os + o_off(rr, c8) + 4);
-        const float ov[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        const long long idx = (long long)i * E.cols + j;
-        const int nv = min(8, E.cols - j);
-        if (E.O_out) {
-            if (E.vec_ok) {                    // cols % 8 == 0: the item is whole
-                *reinterpret_cast<float4*>(E.O_out + idx) = a;
-                *reinterpret_cast<float4*>(E.O_out + idx + 4) = b;
+                    for (int e = 0; e < 32; ++e)
+                        if (e < nv) E.O_out[idx + e] = v[e];
+                }
+            }
+            if (skip) continue;
+            const uint8_t* ws = sm + S::kW + rr * S::kWRow + cc * WSZ;    // this row's staged W
+            if (E.vec_ok && W_DT != DT_FP32) {
+                using T = typename std::conditional<W_DT == DT_BF16, __nv_bfloat16, __half>::type;
+                uint4* wp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(E.W) + idx);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (8 * u >= nv) continue;
+                    const uint4 x = reinterpret_cast<const uint4*>(ws)[u];
+                    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+                    uint32_t r[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float w0 = unpack_lo<T>(xw[e]), w1 = unpack_hi<T>(xw[e]);
+                        w0 = w0 - p.eta * (E.gamma * v[8 * u + 2 * e] + p.lambda * w0);
+                        w1 = w1 - p.eta * (E.gamma * v[8 * u + 2 * e + 1] + p.lambda * w1);
+                        r[e] = pack2<T>(w0, w1);
+                    }
+                    wp[u] = make_uint4(r[0], r[1], r[2], r[3]);
+                }
+            } else if (E.vec_ok) {
+                float4* wp = reinterpret_cast<float4*>(static_cast<float*>(E.W) + idx);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (4 * u >= nv) continue;
+                    float4 w = reinterpret_cast<const float4*>(ws)[u];
+                    w.x = w.x - p.eta * (E.gamma * v[4 * u] + p.lambda * w.x);
+                    w.y = w.y - p.eta * (E.gamma * v[4 * u + 1] + p.lambda * w.y);
+                    w.z = w.z - p.eta * (E.gamma * v[4 * u + 2] + p.lambda * w.z);
+                    w.w = w.w - p.eta * (E.gamma * v[4 * u + 3] + p.lambda * w.w);
+                    wp[u] = w;
+                }
             } else {
-                for (int e = 0; e < nv; ++e) E.O_out[idx + e] = ov[e];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    if (e >= nv) continue;
+                    const float w = ld_elem(E.W, idx + e, W_DT);
+                    st_elem(E.W, idx + e, W_DT, w - p.eta * (E.gamma * v[e] + p.lambda * w));
+                }
             }
         }
-        if (skip) continue;
-        if (E.vec_ok && W_DT != DT_FP32) {
-            using T = typename std::conditional<W_DT == DT_BF16, __nv_bfloat16, __half>::type;
-            uint4* wp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(E.W) + idx);
-            const uint4 u = *wp;
-            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-            uint32_t r[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float w0 = unpack_lo<T>(uw[e]), w1 = unpack_hi<T>(uw[e]);
-                w0 = w0 - p.eta * (E.gamma * ov[2 * e] + p.lambda * w0);
-                w1 = w1 - p.eta * (E.gamma * ov[2 * e + 1] + p.lambda * w1);
-                r[e] = pack2<T>(w0, w1);
-            }
-            *wp = make_uint4(r[0], r[1], r[2], r[3]);
-        } else if (E.vec_ok) {
-            float4* wp = reinterpret_cast<float4*>(static_cast<float*>(E.W) + idx);
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float4 w = wp[hh];
-                w.x = w.x - p.eta * (E.gamma * ov[4 * hh] + p.lambda * w.x);
-                w.y = w.y - p.eta * (E.gamma * ov[4 * hh + 1] + p.lambda * w.y);
-                w.z = w.z - p.eta * (E.gamma * ov[4 * hh + 2] + p.lambda * w.z);
-                w.w = w.w - p.eta * (E.gamma * ov[4 * hh + 3] + p.lambda * w.w);
-                wp[hh] = w;
-            }
-        } else {
-            for (int e = 0; e < nv; ++e) {
-                const float w = ld_elem(E.W, idx + e, W_DT);
-                st_elem(E.W, idx + e, W_DT, w - p.eta * (E.gamma * ov[e] + p.lambda * w));
-            }
-        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -961,7 +1029,7 @@ constexpr size_t sketch_smem() { return (size_t)SketchSmem<KT, G_DT>::kBytes; }
 template <int KT>
 constexpr size_t project_smem() { return (size_t)ProjSmem<KT>::kBytes; }
 template <int KT, int W_DT>
-constexpr size_t update_smem() { return (size_t)UpdSmem<KT>::kBytes; }
+constexpr size_t update_smem() { return (size_t)UpdSmem<KT, W_DT>::kBytes; }
 template <int KT>
 constexpr size_t chol_smem() { return sizeof(double) * (2 * KT * KT + KT) + sizeof(int) * KT; }
 template <int KT>
