@@ -248,14 +248,16 @@ __device__ __forceinline__ void ld_frag16(Frag16& f, const uint32_t* hi, const u
     f.l[0] = b.x; f.l[1] = b.y; f.l[2] = b.z; f.l[3] = b.w;
 }
 
-// d += A B over one 16-wide k group: ra / rb = the A rows g and g + 8, fb = the
-// B column g (all loaded by ld_frag16 at the group's columns 4 q ..).
-__device__ __forceinline__ void mma16(float (&d)[4], const Frag16& ra, const Frag16& rb, const Frag16& fb) {
+// d0 += A B over k-step 0 and d1 += A B over k-step 1 of one 16-wide k group
+// (two accumulators: independent MMA chains): ra / rb = the A rows g and
+// g + 8, fb = the B column g (all loaded by ld_frag16 at the group's columns 4 q ..).
+__device__ __forceinline__ void mma16(float (&d0)[4], float (&d1)[4], const Frag16& ra, const Frag16& rb,
+                                      const Frag16& fb) {
 #pragma unroll
     for (int st = 0; st < 2; ++st) {
         const uint32_t ah[4] = {ra.h[2 * st], rb.h[2 * st], ra.h[2 * st + 1], rb.h[2 * st + 1]};
         const uint32_t al[4] = {ra.l[2 * st], rb.l[2 * st], ra.l[2 * st + 1], rb.l[2 * st + 1]};
-        mma3_tf32(d, ah, al, fb.h[2 * st], fb.h[2 * st + 1], fb.l[2 * st], fb.l[2 * st + 1]);
+        mma3_tf32(st ? d1 : d0, ah, al, fb.h[2 * st], fb.h[2 * st + 1], fb.l[2 * st], fb.l[2 * st + 1]);
     }
 }
 
@@ -293,11 +295,13 @@ __global__ void __launch_bounds__(kThreads, KT == 32 ? 2 : 1) lim_sketch(const _
     uint32_t* mlo = reinterpret_cast<uint32_t*>(sm + S::kMlo);
     uint32_t* oth = reinterpret_cast<uint32_t*>(sm + S::kOtHi);
     uint32_t* otl = reinterpret_cast<uint32_t*>(sm + S::kOtLo);
-    float acc[NT][4];
+    float acc[2][NT][4];                      // the two k-steps of a group: independent chains
 #pragma unroll
-    for (int t = 0; t < NT; ++t)
+    for (int e = 0; e < 2; ++e)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[t][c] = 0.f;
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[e][t][c] = 0.f;
     bool bad = false;
 
     // Chunk c (columns c*kSkCols..) of G, M and Omega into stage s; zeros outside.
@@ -430,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, KT == 32 ? 2 : 1) lim_sketch(const _
                 const int n = 8 * t + g;
                 Frag16 fo;
                 ld_frag16(fo, oth, otl, n * kSkCols + swz(n, kk + 4 * q4));
-                mma16(acc[t], fa, fb, fo);
+                mma16(acc[0][t], acc[1][t], fa, fb, fo);
             }
         }
         __syncthreads();                       // stage s and the split buffers free for the next chunks
@@ -440,8 +444,10 @@ __global__ void __launch_bounds__(kThreads, KT == 32 ? 2 : 1) lim_sketch(const _
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
         const int col = 8 * t + 2 * q4;
-        *reinterpret_cast<float2*>(ys + (16 * warp + g) * KT + col) = make_float2(acc[t][0], acc[t][1]);
-        *reinterpret_cast<float2*>(ys + (16 * warp + g + 8) * KT + col) = make_float2(acc[t][2], acc[t][3]);
+        *reinterpret_cast<float2*>(ys + (16 * warp + g) * KT + col) =
+            make_float2(acc[0][t][0] + acc[1][t][0], acc[0][t][1] + acc[1][t][1]);
+        *reinterpret_cast<float2*>(ys + (16 * warp + g + 8) * KT + col) =
+            make_float2(acc[0][t][2] + acc[1][t][2], acc[0][t][3] + acc[1][t][3]);
     }
     __syncthreads();
     for (int q = threadIdx.x; q < kSkRows * (KT / 4); q += kThreads) {
@@ -599,11 +605,15 @@ __global__ void __launch_bounds__(kThreads, 2) lim_project(const __grid_constant
     const int r_begin = seg * kPjSegRows, r_end = min(E.rows, r_begin + kPjSegRows);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q4 = lane & 3;
     const int nchunks = (r_end - r_begin + kPjRows - 1) / kPjRows;
-    float acc[NT][4];
+    // two accumulator sets, for the even and the odd k-steps: twice as many
+    // independent MMA chains (each k-step is three dependent MMAs per tile)
+    float acc[2][NT][4];
 #pragma unroll
-    for (int t = 0; t < NT; ++t)
+    for (int e = 0; e < 2; ++e)
 #pragma unroll
-        for (int h = 0; h < 4; ++h) acc[t][h] = 0.f;
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int h = 0; h < 4; ++h) acc[e][t][h] = 0.f;
 
     // rows i0.. of M (this block's columns) and of Q's two parts into stage s
     auto issue = [&](int ch, int s) {
@@ -656,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 2) lim_project(const __grid_constant
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 const int b0 = (kk + q4) * S::kQLd + 8 * t + g;
-                mma3_tf32(acc[t], ah, al, qh[b0], qh[b0 + 4 * S::kQLd], ql[b0], ql[b0 + 4 * S::kQLd]);
+                mma3_tf32(acc[(kk >> 3) & 1][t], ah, al, qh[b0], qh[b0 + 4 * S::kQLd], ql[b0], ql[b0 + 4 * S::kQLd]);
             }
         }
         __syncthreads();                       // this stage is refilled next
@@ -666,8 +676,10 @@ __global__ void __launch_bounds__(kThreads, 2) lim_project(const __grid_constant
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
         const int col = 8 * t + 2 * q4;
-        *reinterpret_cast<float2*>(bs + (16 * warp + g) * KT + col) = make_float2(acc[t][0], acc[t][1]);
-        *reinterpret_cast<float2*>(bs + (16 * warp + g + 8) * KT + col) = make_float2(acc[t][2], acc[t][3]);
+        *reinterpret_cast<float2*>(bs + (16 * warp + g) * KT + col) =
+            make_float2(acc[0][t][0] + acc[1][t][0], acc[0][t][1] + acc[1][t][1]);
+        *reinterpret_cast<float2*>(bs + (16 * warp + g + 8) * KT + col) =
+            make_float2(acc[0][t][2] + acc[1][t][2], acc[0][t][3] + acc[1][t][3]);
     }
     __syncthreads();
     if (E.nseg > 1) {                          // uniform over the block
