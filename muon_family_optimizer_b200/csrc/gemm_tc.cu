@@ -50,18 +50,25 @@ constexpr int kEpiThreads = 32 * kEpiWarps;
 
 // Per-CTA configuration.  PAIR: two CTAs share each MMA (cta_group::2): the
 // pair computes a 256 x BN tile, each CTA loads its 128 rows of A and BN/2 of B.
-template <int BN, bool PAIR, bool B_MN, bool FIN>
+// S1: a symmetric product on CTA pairs whose diagonal tiles need no
+// cross-warp symmetrisation (every problem a product of one operand with
+// itself): each epilogue warp stages its two boxes one after the other in one
+// box, and the 64 KB this frees hold a sixth pipeline stage.  The operand
+// stream is latency-bound per SM, so the k-loop runs in proportion to the
+// stages in flight.
+template <int BN, bool PAIR, bool B_MN, bool FIN, bool S1 = false>
 struct Cfg {
-    // symmetric products on CTA pairs stage a whole 128 x 256 output (16 boxes);
-    // the final step keeps two 32 x 32 blocks of the target per epilogue warp
+    // symmetric products on CTA pairs stage a whole 128 x 256 output (16 boxes,
+    // or 8 with S1); the final step keeps two 32 x 32 blocks of the target per
+    // epilogue warp
     static constexpr bool kSymPair = PAIR && !B_MN;
-    static constexpr int kStages = FIN ? (PAIR ? 4 : 3) : kSymPair ? 5 : ((PAIR || BN == 128) ? 6 : 4);
+    static constexpr int kStages = FIN ? (PAIR ? 4 : 3) : kSymPair ? (S1 ? 6 : 5) : ((PAIR || BN == 128) ? 6 : 4);
     static constexpr int kABytes = BM * BK * 2;
     static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * BK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kTmemCols = 2 * BN;
     static constexpr int kStgBytes = 32 * 64 * 2;              // one 32 x 64 16-bit box
-    static constexpr int kBoxes = kSymPair ? 16 : kEpiWarps;   // staging boxes
+    static constexpr int kBoxes = (kSymPair && !S1) ? 16 : kEpiWarps;   // staging boxes
     static constexpr int kFinBlock = 32 * 32 * 4;               // one 32 x 32 block of the target (up to fp32)
     static constexpr int kStgRegion = FIN ? kEpiWarps * 2 * kFinBlock : kBoxes * kStgBytes;
     static constexpr int kStgOffset = kStages * kStageBytes;
@@ -496,11 +503,12 @@ __device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int cb0, 
 // of an optimizer step); without it the operand layouts of every k-block are
 // compile-time or per-problem symmetric-storage decisions only, which keeps
 // the single MMA-issuing thread's work per instruction minimal.
-template <int BN, bool B_MN, bool PAIR, bool FIN, bool TRX, typename T>
+template <int BN, bool B_MN, bool PAIR, bool FIN, bool TRX, typename T, bool S1 = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
     static_assert(!PAIR || BN == 256, "CTA pairs compute 256 x 256 tiles");
     static_assert(!FIN || B_MN, "the final step is an update product");
-    using C = Cfg<BN, PAIR, B_MN, FIN>;
+    static_assert(!S1 || (PAIR && !B_MN), "one staging box per warp: symmetric products on pairs");
+    using C = Cfg<BN, PAIR, B_MN, FIN, S1>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
@@ -819,6 +827,68 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     __syncwarp();
                 }
                 const uint32_t tcol = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN + 2 * half * 64);
+                if constexpr (S1) {
+                    // one box per warp, the two 64-column boxes in turn (the product's
+                    // diagonal blocks are exactly symmetric as formed: nothing to fix)
+                    uint8_t* box = stg_base + (quad + 4 * half) * C::kStgBytes;
+                    const bool rows_ok = row0 + quad * 32 < P.M;
+                    const bool lower = diag_pair && rank == 1 && half == 0;   // below the diagonal
+                    const bool store = rows_ok && !lower;
+                    if (have0) {
+                        sym_chunk<T>(E, gi, gjb, sc, tcol, box, lane, 0, c0);
+                        sym_chunk<T>(E, gi, gjb + 32, sc, tcol + 32, box, lane, 4, c1);
+                        if (!have1) {          // the accumulator has been read
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+                            released = true;
+                        }
+                        if (store) {
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_3d(&P.mapD, box, gjb, row0 + quad * 32, m);
+                                bulk_commit();
+                            }
+                            stg_busy = true;
+                        }
+                        if (mirror && rows_ok) {
+                            __syncwarp();
+                            mirror_box<T>(E, m, row0 + quad * 32, gjb, P.M, P.N, box, lane);
+                        }
+                    }
+                    if (have1) {
+                        if (stg_busy) {        // the box is reused: the first store has read it
+                            if (lane == 0) bulk_wait_read0();
+                        }
+                        __syncwarp();
+                        sym_chunk<T>(E, gi, gjb + 64, sc, tcol + 64, box, lane, 0, c2);
+                        sym_chunk<T>(E, gi, gjb + 96, sc, tcol + 96, box, lane, 4, c3);
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+                        released = true;
+                        if (store) {
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_3d(&P.mapD, box, gjb + 64, row0 + quad * 32, m);
+                                bulk_commit();
+                            }
+                            stg_busy = true;
+                        }
+                        if (mirror && rows_ok) {
+                            __syncwarp();
+                            mirror_box<T>(E, m, row0 + quad * 32, gjb + 64, P.M, P.N, box, lane);
+                        }
+                    }
+                    if (!dead && !released) {  // no column of this warp's half inside the matrix
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+                        released = true;
+                    }
+                } else {
                 uint8_t* box0 = stg_base + (quad + 4 * (2 * half)) * C::kStgBytes;
                 uint8_t* box1 = stg_base + (quad + 4 * (2 * half + 1)) * C::kStgBytes;
                 if (have0) {
@@ -864,6 +934,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     if (have0) mirror_box<T>(E, m, row0 + quad * 32, gjb, P.M, P.N, box0, lane);
                     if (have1) mirror_box<T>(E, m, row0 + quad * 32, gjb + 64, P.M, P.N, box1, lane);
                 }
+                }   // S1
             } else {
 #pragma unroll 1
             for (int pr = 0; pr < kPairs; ++pr) {
@@ -987,10 +1058,10 @@ static bool encode_map(CUtensorMap* map, int dt, const void* base, long long inn
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool B_MN, bool PAIR, bool FIN, bool TRX, typename T>
+template <int BN, bool B_MN, bool PAIR, bool FIN, bool TRX, typename T, bool S1 = false>
 static cudaError_t launch_one(const TcParams& prm, int grid, cudaStream_t stream) {
-    using C = Cfg<BN, PAIR, B_MN, FIN>;
-    auto kern = tc_gemm_kernel<BN, B_MN, PAIR, FIN, TRX, T>;
+    using C = Cfg<BN, PAIR, B_MN, FIN, S1>;
+    auto kern = tc_gemm_kernel<BN, B_MN, PAIR, FIN, TRX, T, S1>;
     static thread_local int configured_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1108,12 +1179,16 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
     trace_begin(sym ? MUON_KERNEL_SYM : MUON_KERNEL_UPD, work, stream);
     cudaError_t e;
     const bool final_step = ops[0].epi.fin != FIN_STORE;
-    bool any_tr = false;
-    for (int i = 0; i < nops; ++i) any_tr |= ops[i].a_tr || ops[i].b_tr;
+    bool any_tr = false, one_operand = sym != 0;
+    for (int i = 0; i < nops; ++i) {
+        any_tr |= ops[i].a_tr || ops[i].b_tr;
+        one_operand &= prm.prob[i].same_ab != 0;   // diagonal tiles exactly symmetric as formed
+    }
     // one instantiation per product kind, CTA-pair mode, operand layouts and element type
 #define MUON_TC_LAUNCH(TRX, T)                                                                         \
     do {                                                                                               \
-        if (sym) e = pair ? launch_one<256, false, true, false, TRX, T>(prm, grid, stream)             \
+        if (sym) e = pair ? (one_operand ? launch_one<256, false, true, false, TRX, T, true>(prm, grid, stream) \
+                                         : launch_one<256, false, true, false, TRX, T>(prm, grid, stream))     \
                           : launch_one<128, false, false, false, TRX, T>(prm, grid, stream);           \
         else if (final_step) e = pair ? launch_one<256, true, true, true, TRX, T>(prm, grid, stream)   \
                                : launch_one<256, true, false, true, TRX, T>(prm, grid, stream);        \
