@@ -43,6 +43,7 @@ namespace muon {
 namespace tc {
 
 constexpr int BM = 128;
+constexpr int kWideMinK = 1024;   // update products on 256 x 512 tiles from this depth
 constexpr int BK = 64;    // 64 16-bit elements = one 128-byte swizzle row
 constexpr int kEpiWarps = 8;    // two per tensor-memory lane quadrant, each takes half the columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -62,11 +63,15 @@ struct Cfg {
     // or 8 with S1); the final step keeps two 32 x 32 blocks of the target per
     // epilogue warp
     static constexpr bool kSymPair = PAIR && !B_MN;
-    static constexpr int kStages = FIN ? (PAIR ? 4 : 3) : kSymPair ? (S1 ? 6 : 5) : ((PAIR || BN == 128) ? 6 : 4);
+    // BN = 512 (update products on pairs): two N = 256 MMAs per k-slice into all
+    // 512 tensor-memory columns, one accumulator buffer
+    static constexpr bool kWide = BN == 512;
+    static constexpr int kStages = FIN ? (PAIR ? 4 : 3) : kSymPair ? (S1 ? 6 : 5) : kWide ? 4 : ((PAIR || BN == 128) ? 6 : 4);
     static constexpr int kABytes = BM * BK * 2;
     static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * BK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kTmemCols = 2 * BN;
+    static constexpr int kNumBuf = kWide ? 1 : 2;            // accumulator buffers
+    static constexpr int kTmemCols = kNumBuf * BN;
     static constexpr int kStgBytes = 32 * 64 * 2;              // one 32 x 64 16-bit box
     static constexpr int kBoxes = (kSymPair && !S1) ? 16 : kEpiWarps;   // staging boxes
     static constexpr int kFinBlock = 32 * 32 * 4;               // one 32 x 32 block of the target (up to fp32)
@@ -505,7 +510,9 @@ __device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int cb0, 
 // the single MMA-issuing thread's work per instruction minimal.
 template <int BN, bool B_MN, bool PAIR, bool FIN, bool TRX, typename T, bool S1 = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
-    static_assert(!PAIR || BN == 256, "CTA pairs compute 256 x 256 tiles");
+    static_assert(!PAIR || BN == 256 || (BN == 512 && B_MN && !FIN && !TRX),
+                  "CTA pairs compute 256 x 256 tiles, or 256 x 512 update tiles without transposed reads");
+    static_assert(PAIR || BN <= 256, "one CTA computes 128 x 128 or 128 x 256 tiles");
     static_assert(!FIN || B_MN, "the final step is an update product");
     static_assert(!S1 || (PAIR && !B_MN), "one staging box per warp: symmetric products on pairs");
     using C = Cfg<BN, PAIR, B_MN, FIN, S1>;
@@ -582,6 +589,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 const int bcol0 = tj * BN + (int)rank * kBCols;
                 auto chunks = [&](int c0) { return chunks_of(P.N, c0); };
                 const int nchunk = B_MN ? chunks(bcol0) : kBCols / 64;
+                // wide update tiles: MMA h (0, 1) covers the tile's columns 256 h..; this
+                // CTA supplies 128 of them (256 h + 128 rank..), as two 64-column chunks
+                auto wide_col = [&](int r, int c) { return tj * BN + 256 * (c >> 1) + 128 * r + 64 * (c & 1); };
                 // A diagonal tile of a product whose operands are one matrix (X X^T,
                 // S S) needs the same rows as A and as B: one panel serves both.
                 const bool one_panel = !B_MN && P.same_ab && ti == tj;
@@ -593,6 +603,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     bytes = B_MN ? (b_kmaj ? 2 * (C::kABytes + C::kBBytes)
                                            : 2 * C::kABytes + (chunks(tj * BN) + chunks(tj * BN + kBCols)) * 64 * BK * 2)
                                  : 2 * (C::kABytes + (one_panel ? 0 : C::kBBytes));
+                    if constexpr (C::kWide) {
+                        int n = 0;
+                        for (int r = 0; r < 2; ++r)
+                            for (int c = 0; c < 4; ++c) n += wide_col(r, c) < P.N ? 1 : 0;
+                        bytes = 2 * C::kABytes + n * 64 * BK * 2;
+                    }
                 }
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, d_status)) break;
@@ -619,6 +635,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     }
                     if (b_kmaj) {
                         load(&P.mapB, sb, kb * BK, bcol0);
+                    } else if (B_MN && C::kWide) {
+                        for (int c = 0; c < 4; ++c) {
+                            const int col = wide_col((int)rank, c);
+                            if (col < P.N) load(&P.mapB, sb + c * (64 * BK * 2), col, kb * BK);
+                        }
                     } else if (B_MN) {
                         for (int c = 0; c < nchunk; ++c) load(&P.mapB, sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK);
                     } else if (one_panel) {
@@ -655,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc0 = make_idesc_f16(IsBf16<T>::value ? 1 : 0, 0, C::kRows, BN);
+            constexpr uint32_t idesc0 = make_idesc_f16(IsBf16<T>::value ? 1 : 0, 0, C::kRows, C::kWide ? 256 : BN);
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
@@ -665,8 +686,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 decode_tile(p, t, pi, m, ti, tj);
                 const TcProblem& P = p.prob[pi];
                 const int nkb = (P.K + BK - 1) / BK;
-                const int buf = it & 1;
-                const uint32_t tphase = (it >> 1) & 1;
+                const int buf = it % C::kNumBuf;
+                const uint32_t tphase = (it / C::kNumBuf) & 1;
                 if (!mbar_wait(&tempty_bar[buf], tphase ^ 1, abort_flag, d_status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
@@ -693,6 +714,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                                : smem_desc_sw128(sb + k * 32, 16, 1024);
                         if (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
                         else tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+                        if constexpr (C::kWide) {   // the tile's columns 256..511: this CTA's chunks 2, 3
+                            const uint64_t bd1 = smem_desc_sw128(sb + 2 * (64 * BK * 2) + k * 2048, 64 * BK * 2, 1024);
+                            tc_mma_f16_pair(d_tmem + 256, ad, bd1, idesc, (kb | k) != 0 ? 1u : 0u);
+                        }
                     }
                     if (PAIR) {   // release the stage in both CTAs
                         tc_commit_pair(smem_u32(&empty_bar[stage]));
@@ -740,8 +765,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             decode_tile(p, t, pi, m, ti, tj);
             const TcProblem& P = p.prob[pi];
             const Epilogue& E = P.epi;
-            const int buf = it & 1;
-            const uint32_t tphase = (it >> 1) & 1;
+            const int buf = it % C::kNumBuf;
+            const uint32_t tphase = (it / C::kNumBuf) & 1;
             const int row0 = ti * C::kRows + (int)rank * BM;   // first output row of this CTA
             const int gi = row0 + row;
             const int col0 = tj * BN + half * (BN / 2);
@@ -1102,7 +1127,18 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         const char* v = getenv("MUON_CTA_PAIRS");
         return !(v && strcmp(v, "0") == 0);
     }();
-    const int BN = (sym && !pair) ? 128 : 256;
+    // Update products on pairs with K >= kWideMinK in every problem and no
+    // transposed reads run on 256 x 512 tiles: 25% fewer operand bytes per flop
+    // (the operand stream per SM bounds these products) for an epilogue that no
+    // longer overlaps the next tile's MMAs (one accumulator in all 512 columns).
+    // MUON_WIDE_UPDATES=0 keeps 256 x 256 tiles.
+    static const bool wide_ok = [] {
+        const char* v = getenv("MUON_WIDE_UPDATES");
+        return !(v && strcmp(v, "0") == 0);
+    }();
+    bool wide = wide_ok && pair && !sym && ops[0].epi.fin == FIN_STORE;
+    for (int i = 0; i < nops; ++i) wide = wide && ops[i].K >= kWideMinK && !ops[i].a_tr && !ops[i].b_tr;
+    const int BN = (sym && !pair) ? 128 : wide ? 512 : 256;
     const int rows_per_tile = pair ? 2 * BM : BM;
     // the final-step staging boxes overlap the store boxes: one kind per launch
     for (int i = 1; i < nops; ++i)
@@ -1192,6 +1228,7 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
                           : launch_one<128, false, false, false, TRX, T>(prm, grid, stream);           \
         else if (final_step) e = pair ? launch_one<256, true, true, true, TRX, T>(prm, grid, stream)   \
                                : launch_one<256, true, false, true, TRX, T>(prm, grid, stream);        \
+        else if (wide) e = launch_one<512, true, true, false, false, T>(prm, grid, stream);            \
         else e = pair ? launch_one<256, true, true, false, TRX, T>(prm, grid, stream)                  \
                       : launch_one<256, true, false, false, TRX, T>(prm, grid, stream);                \
     } while (0)
