@@ -510,8 +510,8 @@ __device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int cb0, 
 // the single MMA-issuing thread's work per instruction minimal.
 template <int BN, bool B_MN, bool PAIR, bool FIN, bool TRX, typename T, bool S1 = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
-    static_assert(!PAIR || BN == 256 || (BN == 512 && B_MN && !FIN && !TRX),
-                  "CTA pairs compute 256 x 256 tiles, or 256 x 512 update tiles without transposed reads");
+    static_assert(!PAIR || BN == 256 || (BN == 512 && B_MN && !FIN),
+                  "CTA pairs compute 256 x 256 tiles, or 256 x 512 update tiles");
     static_assert(PAIR || BN <= 256, "one CTA computes 128 x 128 or 128 x 256 tiles");
     static_assert(!FIN || B_MN, "the final step is an update product");
     static_assert(!S1 || (PAIR && !B_MN), "one staging box per warp: symmetric products on pairs");
@@ -604,10 +604,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                            : 2 * C::kABytes + (chunks(tj * BN) + chunks(tj * BN + kBCols)) * 64 * BK * 2)
                                  : 2 * (C::kABytes + (one_panel ? 0 : C::kBBytes));
                     if constexpr (C::kWide) {
+                        // 64-column panel chunks, or (X stored transposed) 128-row K-major boxes
                         int n = 0;
                         for (int r = 0; r < 2; ++r)
-                            for (int c = 0; c < 4; ++c) n += wide_col(r, c) < P.N ? 1 : 0;
-                        bytes = 2 * C::kABytes + n * 64 * BK * 2;
+                            for (int c = 0; c < 4; ++c)
+                                n += (b_kmaj ? (c & 1) == 0 : true) && wide_col(r, c) < P.N ? 1 : 0;
+                        bytes = 2 * C::kABytes + n * (b_kmaj ? 128 : 64) * BK * 2;
                     }
                 }
                 for (int kb = 0; kb < nkb; ++kb) {
@@ -633,7 +635,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     } else {
                         load(&P.mapA, sa, kb * BK, rows0);
                     }
-                    if (b_kmaj) {
+                    if (b_kmaj && C::kWide) {
+                        // this CTA's 128 rows of X for each half of the tile, K-major
+                        for (int h = 0; h < 2; ++h) {
+                            const int row = wide_col((int)rank, 2 * h);
+                            if (row < P.N) load(&P.mapB, sb + h * (128 * BK * 2), kb * BK, row);
+                        }
+                    } else if (b_kmaj) {
                         load(&P.mapB, sb, kb * BK, bcol0);
                     } else if (B_MN && C::kWide) {
                         for (int c = 0; c < 4; ++c) {
@@ -714,8 +722,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                                : smem_desc_sw128(sb + k * 32, 16, 1024);
                         if (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
                         else tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
-                        if constexpr (C::kWide) {   // the tile's columns 256..511: this CTA's chunks 2, 3
-                            const uint64_t bd1 = smem_desc_sw128(sb + 2 * (64 * BK * 2) + k * 2048, 64 * BK * 2, 1024);
+                        if constexpr (C::kWide) {   // the tile's columns 256..511: the second 16 KB of B
+                            const uint64_t bd1 = bm ? smem_desc_sw128(sb + 16384 + k * 2048, 64 * BK * 2, 1024)
+                                                    : smem_desc_sw128(sb + 16384 + k * 32, 16, 1024);
                             tc_mma_f16_pair(d_tmem + 256, ad, bd1, idesc, (kb | k) != 0 ? 1u : 0u);
                         }
                     }
@@ -1127,8 +1136,8 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         const char* v = getenv("MUON_CTA_PAIRS");
         return !(v && strcmp(v, "0") == 0);
     }();
-    // Update products on pairs with K >= kWideMinK in every problem and no
-    // transposed reads run on 256 x 512 tiles: 25% fewer operand bytes per flop
+    // Update products on pairs with K >= kWideMinK in every problem run on
+    // 256 x 512 tiles: 25% fewer operand bytes per flop
     // (the operand stream per SM bounds these products) for an epilogue that no
     // longer overlaps the next tile's MMAs (one accumulator in all 512 columns).
     // MUON_WIDE_UPDATES=0 keeps 256 x 256 tiles.
@@ -1137,7 +1146,7 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         return !(v && strcmp(v, "0") == 0);
     }();
     bool wide = wide_ok && pair && !sym && ops[0].epi.fin == FIN_STORE;
-    for (int i = 0; i < nops; ++i) wide = wide && ops[i].K >= kWideMinK && !ops[i].a_tr && !ops[i].b_tr;
+    for (int i = 0; i < nops; ++i) wide = wide && ops[i].K >= kWideMinK;
     const int BN = (sym && !pair) ? 128 : wide ? 512 : 256;
     const int rows_per_tile = pair ? 2 * BM : BM;
     // the final-step staging boxes overlap the store boxes: one kind per launch
@@ -1182,8 +1191,10 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
                                                    o.count, o.ldb, o.strideB, 64, BK))
                 return MUON_ERR_CUDA;
         } else if (o.b_tr) {
-            // X stored N x K (K contiguous); boxes of BK (K) x the CTA's N columns
-            if (!encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK, pair ? BN / 2 : BN))
+            // X stored N x K (K contiguous); boxes of BK (K) x the CTA's N columns (128 of
+            // them per half of a 256 x 512 tile)
+            if (!encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK,
+                            BN == 512 ? 128 : (pair ? BN / 2 : BN)))
                 return MUON_ERR_CUDA;
         } else {
             // X panel: K rows x N (N contiguous); boxes of 64 (N) x BK (K)
@@ -1228,7 +1239,7 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
                           : launch_one<128, false, false, false, TRX, T>(prm, grid, stream);           \
         else if (final_step) e = pair ? launch_one<256, true, true, true, TRX, T>(prm, grid, stream)   \
                                : launch_one<256, true, false, true, TRX, T>(prm, grid, stream);        \
-        else if (wide) e = launch_one<512, true, true, false, false, T>(prm, grid, stream);            \
+        else if (wide) e = launch_one<512, true, true, false, TRX, T>(prm, grid, stream);              \
         else e = pair ? launch_one<256, true, true, false, TRX, T>(prm, grid, stream)                  \
                       : launch_one<256, true, false, false, TRX, T>(prm, grid, stream);                \
     } while (0)
