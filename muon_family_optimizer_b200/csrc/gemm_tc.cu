@@ -66,7 +66,7 @@ struct Cfg {
     // BN = 512 (update products on pairs): two N = 256 MMAs per k-slice into all
     // 512 tensor-memory columns, one accumulator buffer
     static constexpr bool kWide = BN == 512;
-    static constexpr int kStages = FIN ? (PAIR ? 4 : 3) : kSymPair ? (S1 ? 6 : 5) : kWide ? 4 : ((PAIR || BN == 128) ? 6 : 4);
+    static constexpr int kStages = FIN ? (PAIR ? 4 : 3) : kWide ? 4 : kSymPair ? (S1 ? 6 : 5) : ((PAIR || BN == 128) ? 6 : 4);
     static constexpr int kABytes = BM * BK * 2;
     static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * BK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
@@ -95,6 +95,7 @@ struct TcProblem {
     int tiles_m, tiles_n, tiles_per_mat, sym, a_sym, b_sym, band;
     int a_tr, b_tr;      // operands stored transposed in full (see GemmOp)
     int same_ab;         // A and B are one operand: a diagonal tile loads one panel for both
+    int wide;            // symmetric on 256 x 512 tiles: row tile ti spans 512-column tiles ti / 2 ..
     long long tile_begin;
     Epilogue epi;
 };
@@ -115,7 +116,12 @@ __device__ __forceinline__ void decode_tile(const TcParams& p, long long t, int&
     long long local = t - P.tile_begin;
     m = (int)(local / P.tiles_per_mat);
     int r = (int)(local - (long long)m * P.tiles_per_mat);
-    if (P.sym) {
+    if (P.sym && P.wide) {
+        int i = 0;
+        while (r >= P.tiles_n - (i >> 1)) { r -= P.tiles_n - (i >> 1); ++i; }
+        ti = i;
+        tj = (i >> 1) + r;
+    } else if (P.sym) {
         int nt = P.tiles_m, i = 0;
         while (r >= nt - i) { r -= nt - i; ++i; }
         ti = i;
@@ -510,8 +516,8 @@ __device__ __forceinline__ void fix_lower(uint8_t* stg_base, int quad, int cb0, 
 // the single MMA-issuing thread's work per instruction minimal.
 template <int BN, bool B_MN, bool PAIR, bool FIN, bool TRX, typename T, bool S1 = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
-    static_assert(!PAIR || BN == 256 || (BN == 512 && B_MN && !FIN),
-                  "CTA pairs compute 256 x 256 tiles, or 256 x 512 update tiles");
+    static_assert(!PAIR || BN == 256 || (BN == 512 && !FIN && (B_MN || S1)),
+                  "CTA pairs compute 256 x 256 tiles, or 256 x 512 update / one-operand symmetric tiles");
     static_assert(PAIR || BN <= 256, "one CTA computes 128 x 128 or 128 x 256 tiles");
     static_assert(!FIN || B_MN, "the final step is an update product");
     static_assert(!S1 || (PAIR && !B_MN), "one staging box per warp: symmetric products on pairs");
@@ -594,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 auto wide_col = [&](int r, int c) { return tj * BN + 256 * (c >> 1) + 128 * r + 64 * (c & 1); };
                 // A diagonal tile of a product whose operands are one matrix (X X^T,
                 // S S) needs the same rows as A and as B: one panel serves both.
-                const bool one_panel = !B_MN && P.same_ab && ti == tj;
+                const bool one_panel = !C::kWide && !B_MN && P.same_ab && ti == tj;
                 // an update product whose X is stored transposed loads whole K-major boxes
                 const bool b_kmaj = B_MN && TRX && P.b_tr;
                 uint32_t bytes = C::kABytes + (B_MN ? (b_kmaj ? C::kBBytes : nchunk * 64 * BK * 2)
@@ -604,12 +610,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                            : 2 * C::kABytes + (chunks(tj * BN) + chunks(tj * BN + kBCols)) * 64 * BK * 2)
                                  : 2 * (C::kABytes + (one_panel ? 0 : C::kBBytes));
                     if constexpr (C::kWide) {
-                        // 64-column panel chunks, or (X stored transposed) 128-row K-major boxes
+                        // 64-column panel chunks, or 128-row units (K-major boxes of X stored
+                        // transposed; symmetric products: B rows, or two transposed chunks)
+                        const bool rows128 = b_kmaj || !B_MN;
                         int n = 0;
                         for (int r = 0; r < 2; ++r)
                             for (int c = 0; c < 4; ++c)
-                                n += (b_kmaj ? (c & 1) == 0 : true) && wide_col(r, c) < P.N ? 1 : 0;
-                        bytes = 2 * C::kABytes + n * (b_kmaj ? 128 : 64) * BK * 2;
+                                n += (rows128 ? (c & 1) == 0 : true) && wide_col(r, c) < P.N ? 1 : 0;
+                        bytes = 2 * C::kABytes + n * (rows128 ? 128 : 64) * BK * 2;
                     }
                 }
                 for (int kb = 0; kb < nkb; ++kb) {
@@ -650,6 +658,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                         }
                     } else if (B_MN) {
                         for (int c = 0; c < nchunk; ++c) load(&P.mapB, sb + c * (64 * BK * 2), bcol0 + c * 64, kb * BK);
+                    } else if (C::kWide) {
+                        // symmetric, 256 x 512: for each half of the tile this CTA's 128 B rows
+                        // (the half's own transposed-read rule for a stored symmetric operand)
+                        for (int h = 0; h < 2; ++h) {
+                            const int row = wide_col((int)rank, 2 * h);
+                            if (row >= P.N) continue;
+                            const bool bth = (TRX && P.b_tr) || (P.b_sym && (kb >> 1) < 2 * (2 * tj + h));
+                            if (bth) {
+                                load(&P.mapBt, sb + h * 16384, row, kb * BK);
+                                load(&P.mapBt, sb + h * 16384 + 64 * BK * 2, row + 64, kb * BK);
+                            } else {
+                                load(&P.mapB, sb + h * 16384, kb * BK, row);
+                            }
+                        }
                     } else if (one_panel) {
                         // B is the A panel just loaded
                     } else if (bt) {
@@ -699,16 +721,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 if (!mbar_wait(&tempty_bar[buf], tphase ^ 1, abort_flag, d_status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
-                const bool one_panel = !B_MN && P.same_ab && ti == tj;   // B read from the A panel
+                const bool one_panel = !C::kWide && !B_MN && P.same_ab && ti == tj;   // B read from the A panel
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, abort_flag, d_status)) { ok = false; break; }
                     tc_fence_after();
                     // A block read transposed; B block MN-major (an update product's X panel
                     // always, unless stored transposed in full)
                     const bool at = (TRX && P.a_tr) || (P.a_sym && (kb >> 1) < (PAIR ? 2 * ti : ti));
+                    const int tjb = C::kWide && !B_MN ? 2 * tj : tj;   // 256-column tile of the (first) MMA
                     const bool bm = B_MN ? !(TRX && P.b_tr)
-                                         : ((TRX && P.b_tr) || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tj : tj)));
+                                         : ((TRX && P.b_tr) || (P.b_sym && (kb >> 1) < (PAIR ? 2 * tjb : tjb)));
+                    const bool bm1 = B_MN ? bm : ((TRX && P.b_tr) || (P.b_sym && (kb >> 1) < 2 * (tjb + 1)));
                     const uint32_t idesc = idesc0 | (at ? 1u << 15 : 0u) | (bm ? 1u << 16 : 0u);
+                    const uint32_t idesc1 = idesc0 | (at ? 1u << 15 : 0u) | (bm1 ? 1u << 16 : 0u);
+                    (void)idesc1;
                     const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t sb = one_panel ? sa : sa + C::kABytes;
 #pragma unroll
@@ -723,9 +749,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                         if (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
                         else tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
                         if constexpr (C::kWide) {   // the tile's columns 256..511: the second 16 KB of B
-                            const uint64_t bd1 = bm ? smem_desc_sw128(sb + 16384 + k * 2048, 64 * BK * 2, 1024)
-                                                    : smem_desc_sw128(sb + 16384 + k * 32, 16, 1024);
-                            tc_mma_f16_pair(d_tmem + 256, ad, bd1, idesc, (kb | k) != 0 ? 1u : 0u);
+                            const uint64_t bd1 = bm1 ? smem_desc_sw128(sb + 16384 + k * 2048, 64 * BK * 2, 1024)
+                                                     : smem_desc_sw128(sb + 16384 + k * 32, 16, 1024);
+                            tc_mma_f16_pair(d_tmem + 256, ad, bd1, idesc1, (kb | k) != 0 ? 1u : 0u);
                         }
                     }
                     if (PAIR) {   // release the stage in both CTAs
@@ -850,6 +876,61 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 // warps holding the first block right of the diagonal (bj = bi + 1),
                 // straight from the registers that fill their staging boxes.  The
                 // accumulator buffer is handed back as soon as it has been read.
+                if constexpr (C::kWide) {
+                    // 256 x 512 tile of a product of one operand with itself: this warp's
+                    // half of the columns is the 256 x 256 tile (ti, tjh); its four 64-column
+                    // boxes in turn through one staging box.  A 128-block (bi, bj) is stored
+                    // when bj >= bi (on or above the diagonal; the part of the tile left of
+                    // the diagonal is computed and dropped), and mirrored below the
+                    // diagonal when it is the first block right of it (band).
+                    const int tjh = 2 * tj + half;
+                    const int bi = 2 * ti + (int)rank;
+                    const bool rows_ok = row0 + quad * 32 < P.M;
+                    uint8_t* box = stg_base + (quad + 4 * half) * C::kStgBytes;
+#pragma unroll 1
+                    for (int b = 0; b < 4; ++b) {
+                        const int bj = 2 * tjh + (b >> 1), gj = 256 * tjh + 64 * b;
+                        if (dead || bj < bi || gj >= P.N) continue;   // warp-uniform
+                        if (stg_busy) {
+                            if (lane == 0) bulk_wait_read0();
+                            __syncwarp();
+                        }
+                        uint4 ca[4] = {}, cb[4] = {};
+                        if (has_cin) {
+                            if (b == 0) {
+                                for (int q = 0; q < 4; ++q) { ca[q] = c0[q]; cb[q] = c1[q]; }
+                            } else if (b == 1) {
+                                for (int q = 0; q < 4; ++q) { ca[q] = c2[q]; cb[q] = c3[q]; }
+                            } else {
+                                cin_fetch<T>(E, m, gi, gj, P.M, P.N, ca);
+                                cin_fetch<T>(E, m, gi, gj + 32, P.M, P.N, cb);
+                            }
+                        }
+                        const uint32_t tc = tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                            (uint32_t)(buf * BN + half * 256 + 64 * b);
+                        sym_chunk<T>(E, gi, gj, sc, tc, box, lane, 0, ca);
+                        sym_chunk<T>(E, gi, gj + 32, sc, tc + 32, box, lane, 4, cb);
+                        if (rows_ok) {
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_3d(&P.mapD, box, gj, row0 + quad * 32, m);
+                                bulk_commit();
+                            }
+                            stg_busy = true;
+                            if (P.band && bj == bi + 1) {
+                                __syncwarp();
+                                mirror_box<T>(E, m, row0 + quad * 32, gj, P.M, P.N, box, lane);
+                            }
+                        }
+                    }
+                    if (!dead) {               // every column this warp needs has been read
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+                        released = true;
+                    }
+                } else {
                 const bool diag_pair = ti == tj;
                 const int bi = 2 * ti + (int)rank, bj = 2 * tj + half;
                 const bool mirror = P.band && bj == bi + 1;
@@ -969,6 +1050,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     if (have1) mirror_box<T>(E, m, row0 + quad * 32, gjb + 64, P.M, P.N, box1, lane);
                 }
                 }   // S1
+                }   // kWide
             } else {
 #pragma unroll 1
             for (int pr = 0; pr < kPairs; ++pr) {
@@ -1147,7 +1229,21 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
     }();
     bool wide = wide_ok && pair && !sym && ops[0].epi.fin == FIN_STORE;
     for (int i = 0; i < nops; ++i) wide = wide && ops[i].K >= kWideMinK;
-    const int BN = (sym && !pair) ? 128 : wide ? 512 : 256;
+    // Symmetric products of one operand with itself (X X^T, S S) with s >= kWideMinK
+    // in every problem run on 256 x 512 tiles too: row tile ti spans the 512-column
+    // tiles from ti / 2, the blocks left of the diagonal computed and dropped.
+    // MUON_WIDE_SYMMETRIC=0 keeps them on 256 x 256 tiles.
+    static const bool wide_sym_ok = [] {
+        const char* v = getenv("MUON_WIDE_SYMMETRIC");
+        return !(v && strcmp(v, "0") == 0);
+    }();
+    bool wide_sym = wide_sym_ok && pair && sym != 0;
+    for (int i = 0; i < nops; ++i) {
+        const GemmOp& o = ops[i];
+        wide_sym = wide_sym && o.N >= kWideMinK && o.A == o.B && o.lda == o.ldb && o.strideA == o.strideB &&
+                   o.a_sym == o.b_sym && o.a_tr == o.b_tr;
+    }
+    const int BN = (sym && !pair) ? 128 : (wide || wide_sym) ? 512 : 256;
     const int rows_per_tile = pair ? 2 * BM : BM;
     // the final-step staging boxes overlap the store boxes: one kind per launch
     for (int i = 1; i < nops; ++i)
@@ -1165,7 +1261,13 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
         P.count = o.count; P.M = o.M; P.N = o.N; P.K = o.K; P.sym = sym;
         P.tiles_m = (o.M + rows_per_tile - 1) / rows_per_tile;
         P.tiles_n = (o.N + BN - 1) / BN;
-        P.tiles_per_mat = sym ? P.tiles_m * (P.tiles_m + 1) / 2 : P.tiles_m * P.tiles_n;
+        P.wide = wide_sym ? 1 : 0;
+        if (wide_sym) {
+            P.tiles_per_mat = 0;
+            for (int ti = 0; ti < P.tiles_m; ++ti) P.tiles_per_mat += P.tiles_n - ti / 2;
+        } else {
+            P.tiles_per_mat = sym ? P.tiles_m * (P.tiles_m + 1) / 2 : P.tiles_m * P.tiles_n;
+        }
         P.tile_begin = tiles;
         tiles += (long long)P.tiles_per_mat * o.count;
         P.epi = o.epi;
@@ -1184,8 +1286,10 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
                                                o.lda, o.strideA, 64, BK))
             return MUON_ERR_CUDA;
         if (sym) {
-            // each CTA of a pair loads half of the tile's B rows
-            if (!o.b_tr && !encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK, pair ? BN / 2 : BN))
+            // each CTA of a pair loads half of the tile's B rows (128 of them for each
+            // 256-column half of a 256 x 512 tile)
+            if (!o.b_tr && !encode_map(&P.mapB, dt, o.B, o.K, o.N, o.count, o.ldb, o.strideB, BK,
+                                       pair ? (BN == 512 ? 128 : BN / 2) : BN))
                 return MUON_ERR_CUDA;
             if ((o.b_sym || o.b_tr) && !encode_map(&P.mapBt, dt, o.B, o.b_tr ? o.N : o.K, o.b_tr ? o.K : o.N,
                                                    o.count, o.ldb, o.strideB, 64, BK))
@@ -1234,7 +1338,8 @@ muon_status tc_run(const GemmOp* ops, int nops, int dt, const FinalCtx& fc, cons
     // one instantiation per product kind, CTA-pair mode, operand layouts and element type
 #define MUON_TC_LAUNCH(TRX, T)                                                                         \
     do {                                                                                               \
-        if (sym) e = pair ? (one_operand ? launch_one<256, false, true, false, TRX, T, true>(prm, grid, stream) \
+        if (sym && wide_sym) e = launch_one<512, false, true, false, TRX, T, true>(prm, grid, stream); \
+        else if (sym) e = pair ? (one_operand ? launch_one<256, false, true, false, TRX, T, true>(prm, grid, stream) \
                                          : launch_one<256, false, true, false, TRX, T>(prm, grid, stream))     \
                           : launch_one<128, false, false, false, TRX, T>(prm, grid, stream);           \
         else if (final_step) e = pair ? launch_one<256, true, true, true, TRX, T>(prm, grid, stream)   \

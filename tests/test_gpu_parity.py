@@ -58,7 +58,7 @@ def test_ns_polar_fp32_tiny():
 
 @pytest.mark.parametrize("dt", ["bf16", "fp16"])
 @pytest.mark.parametrize("shape", [(128, 256), (200, 328), (328, 200), (256, 256), (37, 1000),
-                                   (1, 64), (64, 1), (3, 5), (130, 130)])
+                                   (1, 64), (64, 1), (3, 5), (130, 130), (1100, 1300), (1300, 1100)])
 def test_ns_polar_16bit_vs_oracle(dt, shape):
     X = syn.gaussian(shape, 11 + shape[0], "cpu").to(DT[dt]).cuda()
     out, st = run_polar("direct", X, [QUINTIC] * 5)
@@ -67,11 +67,17 @@ def test_ns_polar_16bit_vs_oracle(dt, shape):
     assert rel_fro(f64(out), ref) <= 3e-2
 
 
-@pytest.mark.parametrize("coeff", [(1.0, 0.0, 0.0), (0.0, 1.0, 0.0), (0.0, 0.0, 1.0), (0.5, -0.25, 0.125)])
-def test_single_step_products(coeff):
+@pytest.mark.parametrize("shape", [(200, 456), (1100, 1300), (1300, 1100)])
+@pytest.mark.parametrize("coeff", [(1.0, 0.0, 0.0), (0.0, 1.0, 0.0), (0.0, 0.0, 1e4), (0.5, -0.25, 1250.0)])
+def test_single_step_products(coeff, shape):
     # isolates the three products of one step: (1,0,0) the copy and scaling,
-    # (0,1,0) X X^T X, (0,0,1) (X X^T)^2 X
-    X = syn.gaussian((200, 456), 5, "cpu").to(torch.bfloat16).cuda()
+    # (0,1,0) X X^T X, (0,0,c) (X X^T)^2 X; s >= 1024 takes the 256 x 512
+    # tiles for the symmetric products too, with ragged edges.  A bfloat16
+    # input is iterated in fp16: with c = 1 the entries of B' = (X X^T)^2 of a
+    # normalised 1100 x 1300 matrix are below 2e-6, in fp16's subnormal range,
+    # where the fp16-rounded computation itself is 12% off; c = 1e4 keeps B' in
+    # the normal range (fp16-rounded computation: 5e-4 off).
+    X = syn.gaussian(shape, 5, "cpu").to(torch.bfloat16).cuda()
     out, st = run_polar("direct", X, [coeff])
     assert st == 0
     ref = oracle.orthogonalise(f64(X), [coeff])

@@ -30,7 +30,7 @@ from muon_family_optimizer_b200 import synthetic as syn  # noqa: E402
 
 pytestmark = pytest.mark.gpu
 
-CASES = [(768, 768), (768, 3072), (700, 1000), (3072, 768), (1100, 1100)]
+CASES = [(768, 768), (768, 3072), (700, 1000), (3072, 768), (1100, 1100), (1100, 2600), (2600, 1100)]
 
 
 def _align(x, a=1024):
