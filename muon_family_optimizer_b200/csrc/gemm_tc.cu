@@ -43,7 +43,7 @@ namespace muon {
 namespace tc {
 
 constexpr int BM = 128;
-constexpr int kWideMinK = 1024;   // update products on 256 x 512 tiles from this depth
+constexpr int kWideMinK = 1024;   // 256 x 512 tiles from this depth (update) or size (symmetric)
 constexpr int BK = 64;    // 64 16-bit elements = one 128-byte swizzle row
 constexpr int kEpiWarps = 8;    // two per tensor-memory lane quadrant, each takes half the columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -63,7 +63,8 @@ struct Cfg {
     // or 8 with S1); the final step keeps two 32 x 32 blocks of the target per
     // epilogue warp
     static constexpr bool kSymPair = PAIR && !B_MN;
-    // BN = 512 (update products on pairs): two N = 256 MMAs per k-slice into all
+    // BN = 512 (update products, and symmetric products of one operand with
+    // itself, on pairs): two N = 256 MMAs per k-slice into all
     // 512 tensor-memory columns, one accumulator buffer
     static constexpr bool kWide = BN == 512;
     static constexpr int kStages = FIN ? (PAIR ? 4 : 3) : kWide ? 4 : kSymPair ? (S1 ? 6 : 5) : ((PAIR || BN == 128) ? 6 : 4);
