@@ -70,13 +70,29 @@ def parse():
     return ap.parse_args()
 
 
-def peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
+def peaks(path=None):
+    """Roofline denominators: the measured figures of MEASURED_PEAKS.json where it has them
+    (positive numbers under the keys of FALLBACK_PEAKS), the fallback figures otherwise."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    out = dict(FALLBACK_PEAKS)
+    if not os.path.exists(p):
+        return out, "fallback"
+    try:
         with open(p) as fh:
             d = json.load(fh)
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+    except (OSError, ValueError):
+        return out, "fallback (MEASURED_PEAKS.json unreadable)"
+    found = []
+    for k in FALLBACK_PEAKS:
+        v = d.get(k) if isinstance(d, dict) else None
+        if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+            out[k] = float(v)
+            found.append(k)
+    if not found:
+        return out, "fallback (MEASURED_PEAKS.json has none of the peaks)"
+    if len(found) < len(FALLBACK_PEAKS):
+        return out, "measured (" + ", ".join(found) + "; fallback for the rest)"
+    return out, "measured"
 
 
 # Sources whose change invalidates a recorded DRAM-traffic figure, per kernel.

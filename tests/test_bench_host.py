@@ -115,3 +115,25 @@ def test_recorded_traffic_scales_a_layer_slice_by_elements(tmp_path, monkeypatch
     b, src = bench.recorded_traffic("tc_upd", "llama3_8b", 5, elements=32 * 218103808)
     assert b == 32000.0 and "scaled" in src
     assert bench.recorded_traffic("tc_upd", "llama3_8b", 5, elements=218103808)[0] == 1000.0
+
+
+def test_peaks_from_measured_file_and_fallbacks(tmp_path):
+    # the generated file: every key measured
+    p = tmp_path / "MEASURED_PEAKS.json"
+    p.write_text(json.dumps({"hbm_gbs": 6530.6, "bf16_tflops": 1670.9, "bf16_tflops_sustained": 1410.8,
+                             "clocks": {"sm": 1965}}))
+    pk, src = bench.peaks(str(p))
+    assert src == "measured"
+    assert pk == {"hbm_gbs": 6530.6, "bf16_tflops": 1670.9, "bf16_tflops_sustained": 1410.8}
+    # a key missing: that one from the fallback figures, and the source says so
+    p.write_text(json.dumps({"hbm_gbs": 6530.6, "bf16_tflops": 1670.9}))
+    pk, src = bench.peaks(str(p))
+    assert pk["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+    assert pk["hbm_gbs"] == 6530.6 and src.startswith("measured (")
+    # nothing usable, unreadable, or absent: the fallback figures
+    for text in (json.dumps({"hbm_gbs": "fast", "bf16_tflops": -1}), "{not json", json.dumps([1, 2])):
+        p.write_text(text)
+        pk, src = bench.peaks(str(p))
+        assert pk == bench.FALLBACK_PEAKS and src.startswith("fallback")
+    pk, src = bench.peaks(str(tmp_path / "absent.json"))
+    assert pk == bench.FALLBACK_PEAKS and src == "fallback"
